@@ -1,0 +1,204 @@
+/*
+ * nvfp4.h -- C ABI of libnvfp4.so: NVFP4 (e2m1 values, 16-element blocks, ue4m3 block
+ * scales) quantization and block-scaled FP4 GEMMs for NVIDIA B200 (sm_100a).
+ *
+ * Sources, cited by page title and section:
+ *   [TRT] TensorRT-LLM NVFP4LinearMethod.create_weights (linear.py:871-915)
+ *   [FV]  FastVideo PR #1350 "Add NVFP4QAT linear layer", code-review thread (_global_sf)
+ *   [FI3] flashinfer PR #1774 "Masked batch nvfp4 quantization"
+ *   [FI5] flashinfer docs flashinfer.gemm.mm_nvfp4_svdquant (signature, Parameters)
+ *   [NVF] NVIDIA/Fuser PR #5737 "Benchmark for nvfp4 scaled mm" (module tree, forward)
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Pointers are CUDA device pointers owned by the caller unless stated otherwise.
+ *    Sizes are element counts.  bf16 tensors are passed as `const void*`.
+ *  - Tensors are dense and row-major.  Packed FP4 tensors are uint8 [rows, k/2] with two
+ *    e2m1 codes per byte: byte i of a row holds element 2i in its low nibble and element
+ *    2i+1 in its high nibble.  e2m1 magnitudes are {0, .5, 1, 1.5, 2, 3, 4, 6}; bit 3
+ *    is the sign.
+ *  - A block-scale buffer holds one ue4m3 byte per 16-element block along k, in the
+ *    128x4 swizzled layout [TRT, FI5 a_sf]: nvfp4_scale_bytes(rows, k) bytes, a
+ *    sequence of 512-byte chunks, one per (128-row tile, 4-block group) with the group
+ *    index fastest; the scale of row r, block c is at chunk byte
+ *    (r % 32) * 16 + ((r % 128) / 32) * 4 + c % 4.  Padding entries (rows >= rows or
+ *    blocks >= k/16) are written as 0 by the dense quantizer.
+ *  - The global scale is gsf = 448*6 / amax with amax = max|x| (NaN counted as 0,
+ *    +-Inf as FLT_MAX, clamped below at 1e-12) [FV, TRT input_scale].  The GEMM factor
+ *    is alpha = amax_a * amax_b / (448*6)^2 [TRT alpha].  Both are fp32 DEVICE values,
+ *    so every call is stream-ordered and capturable in a CUDA graph.
+ *  - Every call launches on `stream` (a cudaStream_t; NULL is the legacy default
+ *    stream), never synchronizes the host, and allocates nothing per call.  The first
+ *    call on a device (and, for the global-scale reductions, the first on a stream)
+ *    allocates a small library-owned workspace with cudaMalloc; make that first call
+ *    before capturing the stream into a CUDA graph.
+ *  - Arguments are validated before anything is launched: a call that returns an
+ *    error has written nothing.
+ *  - Return value: NVFP4_OK or one of the NVFP4_ERR_* codes below.
+ */
+#ifndef NVFP4_H
+#define NVFP4_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NVFP4_API __attribute__((visibility("default")))
+#else
+#define NVFP4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *nvfp4_stream_t;
+
+enum nvfp4_status {
+  NVFP4_OK = 0,
+  NVFP4_ERR_INVALID_ARGUMENT = 1, /* null/misaligned pointer, unsupported size or rank */
+  NVFP4_ERR_UNSUPPORTED_DEVICE = 2, /* the current device is not compute capability 10.0 */
+  NVFP4_ERR_CUDA = 3,             /* a CUDA runtime/driver call or a launch failed */
+  NVFP4_ERR_DEVICE_TIMEOUT = 4,   /* a bounded device-side wait gave up (see nvfp4_device_status) */
+  NVFP4_ERR_OUT_OF_MEMORY = 5     /* the one-time workspace allocation failed */
+};
+
+/* Human-readable name of a status code (static string, never NULL). */
+NVFP4_API const char *nvfp4_status_string(int status);
+
+/*
+ * Bytes of a block-scale buffer for `rows` rows of `k` elements:
+ * pad_up(rows, 128) * pad_up(k / 16, 4) = ceil(rows/128)*128 * ceil(k/64)*4
+ * [TRT create_weights weight_scale padding; FI5 a_sf numel].  Returns -1 when
+ * rows < 0 or k is negative or not a multiple of 16.  Host-only, never fails otherwise.
+ */
+NVFP4_API int64_t nvfp4_scale_bytes(int64_t rows, int64_t k);
+
+/*
+ * Global scale of a bf16 tensor [FV _global_sf; TRT input_scale and alpha].
+ *   x_bf16     [numel] bf16, 16-byte aligned.  numel >= 0 (0 gives amax = 1e-12).
+ *   amax_out   nullable; receives the clamped amax (fp32 [1]).
+ *   gsf_out    required; receives 448*6/amax (fp32 [1]).
+ *   other_amax nullable; the amax of the GEMM's other operand (fp32 [1]).  When given,
+ *   alpha_out  (required then) receives amax * other_amax / (448*6)^2 (fp32 [1]).
+ * One kernel launch; all outputs are written by its last block.
+ */
+NVFP4_API int nvfp4_global_scale(const void *x_bf16, int64_t numel, float *amax_out, float *gsf_out,
+                       const float *other_amax, float *alpha_out, nvfp4_stream_t stream);
+
+/*
+ * Per-item global scale over the valid rows of a batch [FI3 per-item global_scale;
+ * the domain of each item's amax is its rows r < mask[i]].
+ *   x_bf16   [b, m, k] bf16, or [b, m, 2k] when silu_mul != 0 (gate | up halves), in
+ *            which case amax is taken over h = bf16(silu(gate) * up).  16-byte aligned.
+ *   mask     nullable int32 [b]: valid rows per item (values clamped to [0, m]); NULL
+ *            means every row.
+ *   amax_out nullable fp32 [b]; gsf_out required fp32 [b].
+ * Requires k % 8 == 0 and b <= 4096.
+ */
+NVFP4_API int nvfp4_global_scale_batched(const void *x_bf16, int64_t b, int64_t m, int64_t k,
+                               const int32_t *mask, int silu_mul, float *amax_out,
+                               float *gsf_out, nvfp4_stream_t stream);
+
+/*
+ * Dense NVFP4 quantize [TRT create_weights; FI3 fp4_quantize(x, global_scale, 16, ...)].
+ *   x_bf16 [m, k] bf16, 16-byte aligned; k % 16 == 0, m >= 0.
+ *   gsf    fp32 [1] device: the global scale 448*6/amax.
+ *   q_out  uint8 [m, k/2] packed e2m1 (4-byte aligned).
+ *   sf_out uint8 [nvfp4_scale_bytes(m, k)] ue4m3 scales, swizzled; padding entries 0.
+ * Per 16-element block: s = ue4m3_rn_satfinite((max|x| / 6) * gsf); each element is
+ * encoded as e2m1_rn_satfinite(x * (s == 0 ? 0 : gsf / s)).
+ */
+NVFP4_API int nvfp4_quantize(const void *x_bf16, int64_t m, int64_t k, const float *gsf,
+                   uint8_t *q_out, uint8_t *sf_out, nvfp4_stream_t stream);
+
+/*
+ * Masked batched quantize [FI3 nvfp4_batched_quantize(..., mask)].
+ *   x_bf16 [b, m, k] bf16; mask nullable int32 [b] (NULL: all rows); gsf fp32 [b].
+ *   q_out  uint8 [b, m, k/2]; sf_out uint8 [b][nvfp4_scale_bytes(m, k)].
+ * Item i is quantized as nvfp4_quantize on its rows r < mask[i] with gsf[i].  Rows at
+ * or beyond mask[i] and their scale entries are NOT written (they keep whatever the
+ * caller left there).  With mask == NULL, the padding rows' scale entries are zeroed.
+ */
+NVFP4_API int nvfp4_quantize_masked_batched(const void *x_bf16, int64_t b, int64_t m, int64_t k,
+                                  const int32_t *mask, const float *gsf, uint8_t *q_out,
+                                  uint8_t *sf_out, nvfp4_stream_t stream);
+
+/*
+ * SiLU-and-mul fused quantize [FI3 silu_and_mul_fp4_batched_quantize; the
+ * "2*hidden -> hidden" mapping, k_by_2 % 2 == 0 check].
+ *   x_bf16 [b, m, 2k] bf16: gate = x[..., :k], up = x[..., k:].
+ *   k      the OUTPUT width; k % 16 == 0.
+ *   mask, gsf, q_out [b, m, k/2], sf_out [b][nvfp4_scale_bytes(m, k)] as in
+ *   nvfp4_quantize_masked_batched.
+ * h = bf16(silu(gate) * up) with silu(g) = g / (1 + exp(-g)), where exp is the
+ * library's specified fp32 exponential (Cody-Waite reduction, degree-7 Taylor
+ * polynomial, exact 2^n scaling); h is then quantized as above.
+ */
+NVFP4_API int nvfp4_silu_mul_quantize_batched(const void *x_bf16, int64_t b, int64_t m, int64_t k,
+                                    const int32_t *mask, const float *gsf, uint8_t *q_out,
+                                    uint8_t *sf_out, nvfp4_stream_t stream);
+
+/*
+ * Dense block-scaled FP4 GEMM  out = bf16(alpha * (a @ b^T) [+ bias])
+ * [FI5 mm_nvfp4_svdquant without the low-rank term; NVF f16a_nvfp4weight_scaled_mm
+ * output [M, N] bf16; TRT weight [out, in/2]].
+ *   a     uint8 [m, k/2] packed e2m1 (row-major, K contiguous), 16-byte aligned.
+ *   b     uint8 [n, k/2] packed e2m1 (the weight, [out_features, in_features/2]).
+ *   a_sf  uint8 [nvfp4_scale_bytes(m, k)], b_sf uint8 [nvfp4_scale_bytes(n, k)],
+ *         16-byte aligned.
+ *   alpha fp32 [1] device scalar.
+ *   bias  nullable bf16 [n] (added after the alpha scaling, not scaled).
+ *   out   bf16 [m, n], 16-byte aligned; n % 8 == 0.
+ *   k % 64 == 0 (one 64-element MMA step and a full 4-block scale group), k > 0.
+ * Accumulation is fp32 in tensor memory (tcgen05 block-scaled MMA).
+ */
+NVFP4_API int nvfp4_gemm(const uint8_t *a, const uint8_t *b, const uint8_t *a_sf, const uint8_t *b_sf,
+               const float *alpha, const void *bias_bf16, void *out_bf16, int64_t m, int64_t n,
+               int64_t k, nvfp4_stream_t stream);
+
+/*
+ * Masked grouped GEMM for MoE experts [FI3: inputs for grouped_gemm_nt_masked; NVF
+ * routed_experts GroupedLinear].  For every expert e and row i < mask[e]:
+ *   out[e, i, :] = bf16(alpha[e] * a[e, i, :] @ b[e]^T)
+ *   a     uint8 [E, mmax, k/2]; a_sf uint8 [E][nvfp4_scale_bytes(mmax, k)]
+ *   b     uint8 [E, n, k/2];    b_sf uint8 [E][nvfp4_scale_bytes(n, k)]
+ *   mask  int32 [E] device (values clamped to [0, mmax]); alpha fp32 [E] device.
+ *   out   bf16 [E, mmax, n]; rows i >= mask[e] are not written.
+ * Constraints as nvfp4_gemm.  Empty rows cost no tensor-core work: the device-side
+ * scheduler walks only the row tiles below each expert's mask.
+ */
+NVFP4_API int nvfp4_grouped_gemm_masked(const uint8_t *a, const uint8_t *b, const uint8_t *a_sf,
+                              const uint8_t *b_sf, const int32_t *mask, const float *alpha,
+                              void *out_bf16, int64_t E, int64_t mmax, int64_t n, int64_t k,
+                              nvfp4_stream_t stream);
+
+/*
+ * Low-rank-corrected GEMM (SVDQuant) [FI5 mm_nvfp4_svdquant]:
+ *   out = bf16(alpha * (a @ b^T + d @ l1^T) [+ bias])
+ * i.e. the FP4 K-loop and then a bf16 MMA of d @ l1^T into the same fp32 accumulator,
+ * with the epilogue alpha * acc + bias; l1 is the LoRA-up weight pre-divided by alpha.
+ *   d     bf16 [m, r] contiguous, 16-byte aligned (LoRA-down output).
+ *   l1    bf16 [n, r] contiguous, 16-byte aligned.
+ *   r     rank: a positive multiple of 32, at most 256.
+ *   Other arguments and constraints as nvfp4_gemm.
+ */
+NVFP4_API int nvfp4_gemm_lowrank_bias(const uint8_t *a, const uint8_t *b, const uint8_t *a_sf,
+                            const uint8_t *b_sf, const float *alpha, const void *d_bf16,
+                            const void *l1_bf16, int64_t r, const void *bias_bf16,
+                            void *out_bf16, int64_t m, int64_t n, int64_t k,
+                            nvfp4_stream_t stream);
+
+/*
+ * Device-side status word of the current device.  GEMM kernels bound every wait; a
+ * wait that runs out records NVFP4_ERR_DEVICE_TIMEOUT here and the kernel returns
+ * without hanging the GPU.  Synchronizes the device, then stores the word in
+ * *status_out and, when clear != 0, resets it to NVFP4_OK.
+ */
+NVFP4_API int nvfp4_device_status(int *status_out, int clear);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_H */

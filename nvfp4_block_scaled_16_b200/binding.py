@@ -1,0 +1,224 @@
+"""ctypes binding of libnvfp4.so (argument marshalling only).
+
+Every function takes PyTorch CUDA tensors (or None for nullable arguments), passes their
+device pointers and the current stream to the C entry point of the same name, and raises
+:class:`NVFP4Error` on a non-zero status.  Outputs the caller does not provide are
+allocated with ``torch.empty`` on the input's device.
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB = None
+
+EXPORTED_SYMBOLS = (
+    "nvfp4_status_string",
+    "nvfp4_scale_bytes",
+    "nvfp4_global_scale",
+    "nvfp4_global_scale_batched",
+    "nvfp4_quantize",
+    "nvfp4_quantize_masked_batched",
+    "nvfp4_silu_mul_quantize_batched",
+    "nvfp4_gemm",
+    "nvfp4_grouped_gemm_masked",
+    "nvfp4_gemm_lowrank_bias",
+    "nvfp4_device_status",
+)
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_INT = ctypes.c_int
+
+_SIGNATURES = {
+    "nvfp4_status_string": (ctypes.c_char_p, [_INT]),
+    "nvfp4_scale_bytes": (_I64, [_I64, _I64]),
+    "nvfp4_global_scale": (_INT, [_P, _I64, _P, _P, _P, _P, _P]),
+    "nvfp4_global_scale_batched": (_INT, [_P, _I64, _I64, _I64, _P, _INT, _P, _P, _P]),
+    "nvfp4_quantize": (_INT, [_P, _I64, _I64, _P, _P, _P, _P]),
+    "nvfp4_quantize_masked_batched": (_INT, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P]),
+    "nvfp4_silu_mul_quantize_batched": (_INT, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P]),
+    "nvfp4_gemm": (_INT, [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
+    "nvfp4_grouped_gemm_masked": (_INT, [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P]),
+    "nvfp4_gemm_lowrank_bias": (_INT, [_P, _P, _P, _P, _P, _P, _P, _I64, _P, _P, _I64, _I64, _I64, _P]),
+    "nvfp4_device_status": (_INT, [ctypes.POINTER(_INT), _INT]),
+}
+
+
+class NVFP4Error(RuntimeError):
+    def __init__(self, fn, status):
+        self.status = status
+        super().__init__(f"{fn} failed: {nvfp4_status_string(status)} ({status})")
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, "libnvfp4.so")
+
+
+def load_library():
+    """Load libnvfp4.so (built in-tree by ``python -m nvfp4_block_scaled_16_b200.build``)."""
+    global _LIB
+    if _LIB is None:
+        path = library_path()
+        if not os.path.exists(path):
+            raise ImportError(f"{path} is missing; build it with `python -m nvfp4_block_scaled_16_b200.build`")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = lib
+    return _LIB
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"expected a torch.Tensor, got {type(t)}")
+    if not t.is_cuda:
+        raise ValueError("tensor must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(fn, status):
+    if status != 0:
+        raise NVFP4Error(fn, status)
+
+
+def _device_of(*ts):
+    for t in ts:
+        if isinstance(t, torch.Tensor):
+            return t.device
+    return torch.device("cuda", torch.cuda.current_device())
+
+
+def nvfp4_status_string(status: int) -> str:
+    return load_library().nvfp4_status_string(int(status)).decode()
+
+
+def nvfp4_scale_bytes(rows: int, k: int) -> int:
+    return int(load_library().nvfp4_scale_bytes(int(rows), int(k)))
+
+
+def nvfp4_global_scale(x, amax_out=None, gsf_out=None, other_amax=None, alpha_out=None, stream=None):
+    """amax/gsf (and alpha when ``other_amax`` is given) of a bf16 tensor; fp32 [1] outputs."""
+    dev = x.device
+    amax_out = torch.empty(1, dtype=torch.float32, device=dev) if amax_out is None else amax_out
+    gsf_out = torch.empty(1, dtype=torch.float32, device=dev) if gsf_out is None else gsf_out
+    if other_amax is not None and alpha_out is None:
+        alpha_out = torch.empty(1, dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        st = load_library().nvfp4_global_scale(_ptr(x), x.numel(), _ptr(amax_out), _ptr(gsf_out),
+                                               _ptr(other_amax), _ptr(alpha_out), _stream(stream))
+    _check("nvfp4_global_scale", st)
+    return amax_out, gsf_out, alpha_out
+
+
+def nvfp4_global_scale_batched(x, mask=None, silu_mul=False, amax_out=None, gsf_out=None, stream=None):
+    """Per-item amax/gsf over valid rows of x [b, m, k] (or [b, m, 2k] with silu_mul)."""
+    b, m, w = x.shape
+    k = w // 2 if silu_mul else w
+    amax_out = torch.empty(b, dtype=torch.float32, device=x.device) if amax_out is None else amax_out
+    gsf_out = torch.empty(b, dtype=torch.float32, device=x.device) if gsf_out is None else gsf_out
+    with torch.cuda.device(x.device):
+        st = load_library().nvfp4_global_scale_batched(_ptr(x), b, m, k, _ptr(mask), int(bool(silu_mul)),
+                                                       _ptr(amax_out), _ptr(gsf_out), _stream(stream))
+    _check("nvfp4_global_scale_batched", st)
+    return amax_out, gsf_out
+
+
+def nvfp4_quantize(x, gsf, q_out=None, sf_out=None, stream=None):
+    """x [m, k] bf16 -> (q [m, k/2] uint8, sf [scale_bytes(m, k)] uint8)."""
+    m, k = x.shape
+    q_out = torch.empty((m, k // 2), dtype=torch.uint8, device=x.device) if q_out is None else q_out
+    if sf_out is None:
+        sf_out = torch.empty(max(nvfp4_scale_bytes(m, k), 0), dtype=torch.uint8, device=x.device)
+    with torch.cuda.device(x.device):
+        st = load_library().nvfp4_quantize(_ptr(x), m, k, _ptr(gsf), _ptr(q_out), _ptr(sf_out), _stream(stream))
+    _check("nvfp4_quantize", st)
+    return q_out, sf_out
+
+
+def _batched_outputs(x, b, m, k, q_out, sf_out):
+    q_out = torch.empty((b, m, k // 2), dtype=torch.uint8, device=x.device) if q_out is None else q_out
+    if sf_out is None:
+        sf_out = torch.empty((b, max(nvfp4_scale_bytes(m, k), 0)), dtype=torch.uint8, device=x.device)
+    return q_out, sf_out
+
+
+def nvfp4_quantize_masked_batched(x, gsf, mask=None, q_out=None, sf_out=None, stream=None):
+    """x [b, m, k] bf16, gsf [b], mask [b] int32 or None -> (q [b, m, k/2], sf [b, scale_bytes(m, k)])."""
+    b, m, k = x.shape
+    q_out, sf_out = _batched_outputs(x, b, m, k, q_out, sf_out)
+    with torch.cuda.device(x.device):
+        st = load_library().nvfp4_quantize_masked_batched(_ptr(x), b, m, k, _ptr(mask), _ptr(gsf), _ptr(q_out),
+                                                          _ptr(sf_out), _stream(stream))
+    _check("nvfp4_quantize_masked_batched", st)
+    return q_out, sf_out
+
+
+def nvfp4_silu_mul_quantize_batched(x, gsf, mask=None, q_out=None, sf_out=None, stream=None):
+    """x [b, m, 2k] bf16 (gate | up) -> quantized h = bf16(silu(gate) * up): (q [b, m, k/2], sf)."""
+    b, m, w = x.shape
+    k = w // 2
+    q_out, sf_out = _batched_outputs(x, b, m, k, q_out, sf_out)
+    with torch.cuda.device(x.device):
+        st = load_library().nvfp4_silu_mul_quantize_batched(_ptr(x), b, m, k, _ptr(mask), _ptr(gsf), _ptr(q_out),
+                                                            _ptr(sf_out), _stream(stream))
+    _check("nvfp4_silu_mul_quantize_batched", st)
+    return q_out, sf_out
+
+
+def nvfp4_gemm(a, b, a_sf, b_sf, alpha, bias=None, out=None, stream=None):
+    """a [m, k/2], b [n, k/2] packed e2m1 -> out [m, n] bf16 = alpha * a @ b^T (+ bias)."""
+    m, kh = a.shape
+    n = b.shape[0]
+    out = torch.empty((m, n), dtype=torch.bfloat16, device=a.device) if out is None else out
+    with torch.cuda.device(a.device):
+        st = load_library().nvfp4_gemm(_ptr(a), _ptr(b), _ptr(a_sf), _ptr(b_sf), _ptr(alpha), _ptr(bias), _ptr(out),
+                                       m, n, 2 * kh, _stream(stream))
+    _check("nvfp4_gemm", st)
+    return out
+
+
+def nvfp4_grouped_gemm_masked(a, b, a_sf, b_sf, mask, alpha, out=None, stream=None):
+    """a [E, mmax, k/2], b [E, n, k/2] -> out [E, mmax, n] bf16 (rows >= mask[e] not written)."""
+    E, mmax, kh = a.shape
+    n = b.shape[1]
+    out = torch.empty((E, mmax, n), dtype=torch.bfloat16, device=a.device) if out is None else out
+    with torch.cuda.device(a.device):
+        st = load_library().nvfp4_grouped_gemm_masked(_ptr(a), _ptr(b), _ptr(a_sf), _ptr(b_sf), _ptr(mask),
+                                                      _ptr(alpha), _ptr(out), E, mmax, n, 2 * kh, _stream(stream))
+    _check("nvfp4_grouped_gemm_masked", st)
+    return out
+
+
+def nvfp4_gemm_lowrank_bias(a, b, a_sf, b_sf, alpha, d, l1, bias=None, out=None, stream=None):
+    """out [m, n] bf16 = alpha * (a @ b^T + d @ l1^T) (+ bias); d [m, r], l1 [n, r] bf16."""
+    m, kh = a.shape
+    n = b.shape[0]
+    r = d.shape[1]
+    out = torch.empty((m, n), dtype=torch.bfloat16, device=a.device) if out is None else out
+    with torch.cuda.device(a.device):
+        st = load_library().nvfp4_gemm_lowrank_bias(_ptr(a), _ptr(b), _ptr(a_sf), _ptr(b_sf), _ptr(alpha), _ptr(d),
+                                                    _ptr(l1), r, _ptr(bias), _ptr(out), m, n, 2 * kh,
+                                                    _stream(stream))
+    _check("nvfp4_gemm_lowrank_bias", st)
+    return out
+
+
+def nvfp4_device_status(clear: bool = True) -> int:
+    """Synchronize the device and return (optionally clearing) its status word."""
+    v = _INT(0)
+    st = load_library().nvfp4_device_status(ctypes.byref(v), int(bool(clear)))
+    _check("nvfp4_device_status", st)
+    return v.value

@@ -1,0 +1,143 @@
+// context.cu -- per-device state, per-stream reduction scratch, status codes.
+#include <map>
+#include <mutex>
+#include <utility>
+
+#include "common.cuh"
+
+namespace nvfp4 {
+namespace {
+
+std::mutex g_mu;
+DeviceInfo g_dev[64];
+std::map<std::pair<int, cudaStream_t>, uint32_t*> g_ws;
+
+}  // namespace
+
+int current_device(DeviceInfo* out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return NVFP4_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (d.device < 0) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return NVFP4_ERR_CUDA;
+    }
+    if (major != 10 || minor != 0) return NVFP4_ERR_UNSUPPORTED_DEVICE;
+    int* status = nullptr;
+    if (cudaMalloc(&status, sizeof(int)) != cudaSuccess) {
+      cudaGetLastError();
+      return NVFP4_ERR_OUT_OF_MEMORY;
+    }
+    if (cudaMemset(status, 0, sizeof(int)) != cudaSuccess) {
+      cudaGetLastError();
+      cudaFree(status);
+      return NVFP4_ERR_CUDA;
+    }
+    d.status = status;
+    d.sm_count = sms;
+    d.device = dev;
+  }
+  *out = d;
+  return NVFP4_OK;
+}
+
+int stream_workspace(cudaStream_t stream, uint32_t** out) {
+  DeviceInfo info;
+  int st = current_device(&info);
+  if (st != NVFP4_OK) return st;
+  std::lock_guard<std::mutex> lock(g_mu);
+  auto key = std::make_pair(info.device, stream);
+  auto it = g_ws.find(key);
+  if (it != g_ws.end()) {
+    *out = it->second;
+    return NVFP4_OK;
+  }
+  uint32_t* ws = nullptr;
+  const size_t bytes = sizeof(uint32_t) * (1 + kMaxItems);
+  if (cudaMalloc(&ws, bytes) != cudaSuccess) {
+    cudaGetLastError();
+    return NVFP4_ERR_OUT_OF_MEMORY;
+  }
+  if (cudaMemset(ws, 0, bytes) != cudaSuccess) {
+    cudaGetLastError();
+    cudaFree(ws);
+    return NVFP4_ERR_CUDA;
+  }
+  g_ws[key] = ws;
+  *out = ws;
+  return NVFP4_OK;
+}
+
+int launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+}  // namespace nvfp4
+
+extern "C" {
+
+const char* nvfp4_status_string(int status) {
+  switch (status) {
+    case NVFP4_OK: return "NVFP4_OK";
+    case NVFP4_ERR_INVALID_ARGUMENT: return "NVFP4_ERR_INVALID_ARGUMENT";
+    case NVFP4_ERR_UNSUPPORTED_DEVICE: return "NVFP4_ERR_UNSUPPORTED_DEVICE";
+    case NVFP4_ERR_CUDA: return "NVFP4_ERR_CUDA";
+    case NVFP4_ERR_DEVICE_TIMEOUT: return "NVFP4_ERR_DEVICE_TIMEOUT";
+    case NVFP4_ERR_OUT_OF_MEMORY: return "NVFP4_ERR_OUT_OF_MEMORY";
+    default: return "NVFP4_ERR_UNKNOWN";
+  }
+}
+
+int64_t nvfp4_scale_bytes(int64_t rows, int64_t k) {
+  if (rows < 0 || k < 0 || k % 16 != 0) return -1;
+  const int64_t rp = (rows + 127) / 128 * 128;
+  const int64_t cp = (k / 16 + 3) / 4 * 4;
+  return rp * cp;
+}
+
+int nvfp4_device_status(int* status_out, int clear) {
+  if (!status_out) return NVFP4_ERR_INVALID_ARGUMENT;
+  nvfp4::DeviceInfo info;
+  int st = nvfp4::current_device(&info);
+  if (st != NVFP4_OK) return st;
+  if (cudaDeviceSynchronize() != cudaSuccess) {
+    cudaGetLastError();
+    return NVFP4_ERR_CUDA;
+  }
+  int v = 0;
+  if (cudaMemcpy(&v, info.status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return NVFP4_ERR_CUDA;
+  }
+  if (clear && cudaMemset(info.status, 0, sizeof(int)) != cudaSuccess) {
+    cudaGetLastError();
+    return NVFP4_ERR_CUDA;
+  }
+  *status_out = v;
+  return NVFP4_OK;
+}
+
+}  // extern "C"

@@ -4,9 +4,11 @@ This module holds only random-number recipes and the bf16 rounding of the drawn
 values; it contains none of the quantization or GEMM arithmetic, and it imports
 neither the oracle nor the CUDA library.
 
-Recipe (one stream per tensor): ``numpy.random.default_rng([seed, tensor_id])``,
-values drawn in fp32 and rounded to bf16 with round-to-nearest-even; bf16 tensors are
-returned as ``uint16`` bit patterns.  Seed 0 everywhere unless a caller says otherwise.
+Recipe: a tensor is drawn in chunks of 2^24 values, chunk c from its own stream
+``numpy.random.default_rng([seed, tensor_id, c])`` (chunks are generated in parallel
+threads); values are drawn in fp32 and rounded to bf16 with round-to-nearest-even; bf16
+tensors are returned as ``uint16`` bit patterns.  Small per-tensor draws (masks, l1) use
+``default_rng([seed, tensor_id])``.  Seed 0 everywhere unless a caller says otherwise.
 
 Workload shapes (NVFP4 linear-layer inference):
   * pr1_linear      x [128, 256] ~ N(0,1), W [256, 256] ~ N(0, 0.02)
@@ -37,9 +39,13 @@ def rng(seed: int, tensor_id: int) -> np.random.Generator:
 def f32_to_bf16_bits(a) -> np.ndarray:
     """Round fp32 values to bf16 (nearest, ties to even); returns uint16 bits."""
     a = np.ascontiguousarray(a, dtype=np.float32)
-    u = a.view(np.uint32).astype(np.uint64)
-    lsb = (u >> np.uint64(16)) & np.uint64(1)
-    r = ((u + np.uint64(0x7FFF) + lsb) >> np.uint64(16)).astype(np.uint16)
+    u = a.view(np.uint32)
+    # uint32 arithmetic: only NaN bit patterns can wrap around, and they are replaced below
+    t = (u >> np.uint32(16)) & np.uint32(1)
+    t += np.uint32(0x7FFF)
+    t += u
+    t >>= np.uint32(16)
+    r = t.astype(np.uint16)
     nan = np.isnan(a)
     if nan.any():
         r[nan] = np.uint16(0x7FC0)
@@ -51,34 +57,43 @@ def bf16_bits_to_f32(u) -> np.ndarray:
     return (u.astype(np.uint32) << np.uint32(16)).view(np.float32)
 
 
-def normal_bf16(shape, std=1.0, seed=0, tensor_id=TID["x"], chunk=1 << 24) -> np.ndarray:
-    """N(0, std^2) drawn in fp32 and rounded to bf16, generated in chunks."""
-    g = rng(seed, tensor_id)
+CHUNK = 1 << 24
+
+
+def _chunked(shape, fill):
+    """Fill a flat uint16 array chunk by chunk; chunk c gets its own generator."""
     n = int(np.prod(shape))
     out = np.empty(n, np.uint16)
-    for s in range(0, n, chunk):
-        e = min(n, s + chunk)
-        v = g.standard_normal(e - s, dtype=np.float32)
+    starts = list(range(0, n, CHUNK))
+    if len(starts) <= 1:
+        for c, s in enumerate(starts):
+            fill(c, out[s:min(n, s + CHUNK)])
+    else:
+        from concurrent.futures import ThreadPoolExecutor
+        import os
+        with ThreadPoolExecutor(max_workers=min(32, os.cpu_count() or 1)) as ex:
+            list(ex.map(lambda cs: fill(cs[0], out[cs[1]:min(n, cs[1] + CHUNK)]), enumerate(starts)))
+    return out.reshape(shape)
+
+
+def normal_bf16(shape, std=1.0, seed=0, tensor_id=TID["x"]) -> np.ndarray:
+    """N(0, std^2) drawn in fp32 and rounded to bf16."""
+    def fill(c, dst):
+        v = np.random.default_rng([int(seed), int(tensor_id), c]).standard_normal(dst.size, dtype=np.float32)
         if std != 1.0:
             v *= np.float32(std)
-        out[s:e] = f32_to_bf16_bits(v)
-    return out.reshape(shape)
+        dst[:] = f32_to_bf16_bits(v)
+    return _chunked(shape, fill)
 
 
-def normal_with_outliers_bf16(shape, p=0.001, factor=50.0, seed=0, tensor_id=TID["x"],
-                              chunk=1 << 24) -> np.ndarray:
+def normal_with_outliers_bf16(shape, p=0.001, factor=50.0, seed=0, tensor_id=TID["x"]) -> np.ndarray:
     """N(0,1) with Bernoulli(p) positions multiplied by ``factor`` before bf16 rounding."""
-    g = rng(seed, tensor_id)
-    go = rng(seed, TID["outlier"])
-    n = int(np.prod(shape))
-    out = np.empty(n, np.uint16)
-    for s in range(0, n, chunk):
-        e = min(n, s + chunk)
-        v = g.standard_normal(e - s, dtype=np.float32)
-        hit = go.random(e - s, dtype=np.float32) < np.float32(p)
+    def fill(c, dst):
+        v = np.random.default_rng([int(seed), int(tensor_id), c]).standard_normal(dst.size, dtype=np.float32)
+        hit = np.random.default_rng([int(seed), TID["outlier"], c]).random(dst.size, dtype=np.float32) < np.float32(p)
         v[hit] *= np.float32(factor)
-        out[s:e] = f32_to_bf16_bits(v)
-    return out.reshape(shape)
+        dst[:] = f32_to_bf16_bits(v)
+    return _chunked(shape, fill)
 
 
 def masks_uniform(count, mmax, seed=0, tensor_id=TID["mask"]) -> np.ndarray:

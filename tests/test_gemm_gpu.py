@@ -1,0 +1,222 @@
+"""GPU parity of the tcgen05 block-scaled FP4 GEMMs against the oracle's fp64 reference
+on the dequantized operands, within |out - ref| <= 1e-2*|ref| + 1e-3*max|ref|.
+
+Operands are quantized by the oracle, so these tests pin the GEMM alone: the packing
+(low nibble = lower K index), the 128x4 scale layout read straight into tensor memory,
+the accumulator layout and the epilogue.  Sizes span several 128 x 256 tiles with ragged
+M, N and K tails; the full-size cases check sampled outputs."""
+import numpy as np
+import pytest
+import torch
+
+import nvfp4_block_scaled_16_b200 as nv
+import nvfp4_synth as S
+from tests.helpers import (assert_gemm_close, bf16_to_f64, dev_bf16, dev_f32, dev_i32, dev_u8, host)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from nvfp4_block_scaled_16_b200 import build
+    build.build()
+    nv.load_library()
+    yield
+
+
+@pytest.fixture(autouse=True)
+def _status_clean():
+    yield
+    assert nv.nvfp4_device_status(clear=True) == 0, "a device-side wait timed out"
+
+
+def quantized(oracle, x):
+    amax, gsf = oracle.global_scale(x)
+    q, sf = oracle.quantize(x, gsf)
+    return q, sf, amax
+
+
+def operands(oracle, m, n, k, seed=0, std_b=0.02):
+    xa = S.normal_bf16((m, k), 1.0, seed, S.TID["x"])
+    xb = S.normal_bf16((n, k), std_b, seed, S.TID["w"])
+    qa, sfa, amax_a = quantized(oracle, xa)
+    qb, sfb, amax_b = quantized(oracle, xb)
+    alpha = np.float32(oracle.alpha(float(amax_a), float(amax_b)))
+    return qa, sfa, qb, sfb, alpha
+
+
+def run_gemm(qa, sfa, qb, sfb, alpha, bias=None):
+    return nv.nvfp4_gemm(dev_u8(qa), dev_u8(qb), dev_u8(sfa), dev_u8(sfb), dev_f32(alpha),
+                         None if bias is None else dev_bf16(bias))
+
+
+def test_unit_scales_integer_codes_bit_exact(oracle):
+    # All scales 1.0 and alpha 1: every product is a multiple of 1/4 with |sum| small, so
+    # the fp32 accumulation is exact and the bf16 output must equal the exact result
+    # rounded once.
+    for m, n, k in [(128, 256, 256), (128, 256, 64), (256, 512, 128)]:
+        g = np.random.default_rng(m + n + k)
+        ca = g.integers(0, 16, size=(m, k)).astype(np.uint8)
+        cb = g.integers(0, 16, size=(n, k)).astype(np.uint8)
+        qa = (ca[:, 0::2] | (ca[:, 1::2] << 4)).astype(np.uint8)
+        qb = (cb[:, 0::2] | (cb[:, 1::2] << 4)).astype(np.uint8)
+        sfa = np.full(nv.nvfp4_scale_bytes(m, k), 0x38, np.uint8)
+        sfb = np.full(nv.nvfp4_scale_bytes(n, k), 0x38, np.uint8)
+        ref = oracle.gemm_ref(qa, qb, sfa, sfb, 1.0, m, n, k)
+        out = run_gemm(qa, sfa, qb, sfb, np.float32(1.0))
+        expect = S.f32_to_bf16_bits(ref.astype(np.float32))
+        assert (host(out) == expect).all(), np.argwhere(host(out) != expect)[:5]
+
+
+def test_pr1_linear(oracle):
+    d = S.pr1_linear()
+    qa, sfa, amax_a = quantized(oracle, d["x"])
+    qb, sfb, amax_b = quantized(oracle, d["w"])
+    alpha = np.float32(oracle.alpha(float(amax_a), float(amax_b)))
+    out = run_gemm(qa, sfa, qb, sfb, alpha)
+    ref = oracle.gemm_ref(qa, qb, sfa, sfb, alpha, 128, 256, 256)
+    assert_gemm_close(bf16_to_f64(out), ref, "pr1 linear 128x256x256")
+
+
+@pytest.mark.parametrize("m,n,k", [(128, 256, 256), (200, 264, 320), (300, 520, 1024), (1, 8, 64),
+                                   (129, 256, 64), (384, 768, 576)])
+def test_gemm_ragged(oracle, m, n, k):
+    qa, sfa, qb, sfb, alpha = operands(oracle, m, n, k, seed=m + n + k)
+    ref = oracle.gemm_ref(qa, qb, sfa, sfb, alpha, m, n, k)
+    out = run_gemm(qa, sfa, qb, sfb, alpha)
+    assert_gemm_close(bf16_to_f64(out), ref, f"gemm {m}x{n}x{k}")
+
+
+def test_gemm_bias_and_output_bounds(oracle):
+    m, n, k = 200, 264, 320
+    qa, sfa, qb, sfb, alpha = operands(oracle, m, n, k, seed=5)
+    bias = S.normal_bf16((n,), 0.1, 5, S.TID["bias"])
+    ref = oracle.gemm_ref(qa, qb, sfa, sfb, alpha, m, n, k, bias=bias)
+    # write into the middle of a larger sentinel buffer: nothing outside [m, n] may change
+    big = torch.full((m * n + 64,), 7.0, dtype=torch.bfloat16, device="cuda")
+    out = big[32:32 + m * n].view(m, n)
+    nv.nvfp4_gemm(dev_u8(qa), dev_u8(qb), dev_u8(sfa), dev_u8(sfb), dev_f32(alpha), dev_bf16(bias), out)
+    assert_gemm_close(bf16_to_f64(out), ref, "gemm + bias")
+    assert (big[:32] == 7.0).all() and (big[32 + m * n:] == 7.0).all()
+
+
+@pytest.mark.parametrize("r", [32, 64, 96, 128])
+def test_lowrank_bias(oracle, r):
+    m, n, k = 200, 264, 320
+    qa, sfa, qb, sfb, alpha = operands(oracle, m, n, k, seed=r)
+    d = S.normal_bf16((m, r), 1.0, r, S.TID["d"])
+    l1 = S.f32_to_bf16_bits(S.rng(r, S.TID["l1"]).standard_normal((n, r), dtype=np.float32)
+                            * np.float32(0.01) / alpha)
+    bias = S.normal_bf16((n,), 0.1, r, S.TID["bias"])
+    ref = oracle.gemm_ref(qa, qb, sfa, sfb, alpha, m, n, k, d=d, l1=l1, bias=bias)
+    out = nv.nvfp4_gemm_lowrank_bias(dev_u8(qa), dev_u8(qb), dev_u8(sfa), dev_u8(sfb), dev_f32(alpha),
+                                     dev_bf16(d), dev_bf16(l1), dev_bf16(bias))
+    assert_gemm_close(bf16_to_f64(out), ref, f"lowrank r={r}")
+
+
+def test_lowrank_special_cases(oracle):
+    m, n, k, r = 128, 256, 256, 64
+    qa, sfa, qb, sfb, alpha = operands(oracle, m, n, k, seed=9)
+    d = S.normal_bf16((m, r), 1.0, 9, S.TID["d"])
+    l1 = S.normal_bf16((n, r), 0.5, 9, S.TID["l1"])
+    bias = S.normal_bf16((n,), 0.1, 9, S.TID["bias"])
+    # a == 0: only the bf16 low-rank product and the bias remain
+    qz = np.zeros_like(qa)
+    ref = oracle.gemm_ref(qz, qb, sfa, sfb, alpha, m, n, k, d=d, l1=l1, bias=bias)
+    out = nv.nvfp4_gemm_lowrank_bias(dev_u8(qz), dev_u8(qb), dev_u8(sfa), dev_u8(sfb), dev_f32(alpha),
+                                     dev_bf16(d), dev_bf16(l1), dev_bf16(bias))
+    assert_gemm_close(bf16_to_f64(out), ref, "lowrank with a = 0")
+    # d == 0: identical to the plain GEMM with bias
+    dz = np.zeros_like(d)
+    out_lr = nv.nvfp4_gemm_lowrank_bias(dev_u8(qa), dev_u8(qb), dev_u8(sfa), dev_u8(sfb), dev_f32(alpha),
+                                        dev_bf16(dz), dev_bf16(l1), dev_bf16(bias))
+    out_plain = run_gemm(qa, sfa, qb, sfb, alpha, bias)
+    assert (host(out_lr) == host(out_plain)).all()
+
+
+@pytest.mark.parametrize("E,mmax,n,k,mask", [
+    (4, 300, 264, 320, [0, 300, 77, 129]),
+    (3, 128, 256, 256, [128, 1, 0]),
+    (2, 64, 512, 128, [64, 64]),
+])
+def test_grouped_masked(oracle, E, mmax, n, k, mask):
+    mask = np.array(mask, np.int32)
+    a = S.normal_bf16((E, mmax, k), 1.0, E, S.TID["x"])
+    w = S.normal_bf16((E, n, k), 0.02, E, S.TID["w"])
+    amax_a, ga = oracle.global_scale_batched(a, mask)
+    amax_w, gw = oracle.global_scale_batched(w, None)
+    qa, sfa = oracle.quantize_masked_batched(a, ga, mask)
+    qw, sfw = oracle.quantize_masked_batched(w, gw, None)
+    alphas = np.array([oracle.alpha(float(x), float(y)) for x, y in zip(amax_a, amax_w)], np.float32)
+    ref = oracle.grouped_gemm_ref(qa, qw, sfa, sfw, mask, alphas, E, mmax, n, k)
+    out = torch.full((E, mmax, n), -3.0, dtype=torch.bfloat16, device="cuda")
+    nv.nvfp4_grouped_gemm_masked(dev_u8(qa), dev_u8(qw), dev_u8(sfa), dev_u8(sfw), dev_i32(mask),
+                                 dev_f32(alphas), out)
+    o = bf16_to_f64(out)
+    for e in range(E):
+        v = int(mask[e])
+        if v:
+            assert_gemm_close(o[e, :v], ref[e, :v], f"expert {e}")
+        assert (o[e, v:] == -3.0).all(), f"expert {e}: rows beyond the mask were written"
+
+
+# ---- full sizes, sampled outputs ------------------------------------------------------------
+
+def sample_positions(m, n, count, seed):
+    g = S.rng(seed, S.TID["sample"])
+    ii = g.integers(0, m, count)
+    jj = g.integers(0, n, count)
+    # always include the corners of the ragged edges
+    ii[:4] = [0, m - 1, 0, m - 1]
+    jj[:4] = [0, n - 1, n - 1, 0]
+    return ii, jj
+
+
+def test_swiglu_gate_up_full_size_sampled(oracle):
+    # [8192 x 5120] @ [16384 x 5120]^T, the large dense GEMM of the SwiGLU block
+    m, n, k = 8192, 16384, 5120
+    qa, sfa, qb, sfb, alpha = operands(oracle, m, n, k, seed=0)
+    out = host(run_gemm(qa, sfa, qb, sfb, alpha))
+    ii, jj = sample_positions(m, n, 2048, 1)
+    ref = oracle.gemm_ref_sampled(qa, qb, sfa, sfb, alpha, k, ii, jj)
+    got = S.bf16_bits_to_f32(out[ii, jj]).astype(np.float64)
+    assert_gemm_close(got, ref, "gate/up 8192x16384x5120 (sampled)")
+
+
+@pytest.mark.parametrize("r", [32, 64, 128])
+def test_lowrank_full_size(oracle, r):
+    d = S.lowrank(r=r)
+    m, k, n = 4096, 3072, 3072
+    qa, sfa, amax_a = quantized(oracle, d["x"])
+    qb, sfb, amax_b = quantized(oracle, d["w"])
+    alpha = np.float32(oracle.alpha(float(amax_a), float(amax_b)))
+    l1 = S.f32_to_bf16_bits(d["l1_f32"] / alpha)
+    out = host(nv.nvfp4_gemm_lowrank_bias(dev_u8(qa), dev_u8(qb), dev_u8(sfa), dev_u8(sfb), dev_f32(alpha),
+                                          dev_bf16(d["d"]), dev_bf16(l1), dev_bf16(d["bias"])))
+    ii, jj = sample_positions(m, n, 4096, r)
+    ref = oracle.gemm_ref_sampled(qa, qb, sfa, sfb, alpha, k, ii, jj, d=d["d"], l1=l1, bias=d["bias"])
+    assert_gemm_close(S.bf16_bits_to_f32(out[ii, jj]).astype(np.float64), ref, f"lowrank full r={r}")
+
+
+def test_grouped_full_size_sampled(oracle):
+    d = S.grouped_moe()
+    E, mmax, k, n = 16, 2048, 5120, 8192
+    mask = d["mask"]
+    amax_a, ga = oracle.global_scale_batched(d["a"], mask)
+    amax_w, gw = oracle.global_scale_batched(d["w"], None)
+    qa, sfa = oracle.quantize_masked_batched(d["a"], ga, mask)
+    qw, sfw = oracle.quantize_masked_batched(d["w"], gw, None)
+    alphas = np.array([oracle.alpha(float(x), float(y)) for x, y in zip(amax_a, amax_w)], np.float32)
+    out = torch.full((E, mmax, n), -3.0, dtype=torch.bfloat16, device="cuda")
+    nv.nvfp4_grouped_gemm_masked(dev_u8(qa), dev_u8(qw), dev_u8(sfa), dev_u8(sfw), dev_i32(mask),
+                                 dev_f32(alphas), out)
+    o = host(out)
+    for e in range(E):
+        v = int(mask[e])
+        if v:
+            ii, jj = sample_positions(v, n, 256, e)
+            ref = oracle.gemm_ref_sampled(qa[e], qw[e], sfa[e], sfw[e], alphas[e], k, ii, jj)
+            assert_gemm_close(S.bf16_bits_to_f32(o[e, ii, jj]).astype(np.float64), ref, f"expert {e}")
+        if v < mmax:
+            tail = o[e, v:]
+            assert (tail == S.f32_to_bf16_bits(np.float32([-3.0]))[0]).all()

@@ -1,0 +1,116 @@
+"""Host-only checks of the C-ABI library: it builds, loads, exports every symbol that
+include/nvfp4.h declares, and rejects invalid arguments before touching the GPU.
+None of these call a kernel."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import nvfp4_block_scaled_16_b200 as nv
+from nvfp4_block_scaled_16_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+INVALID = 1
+
+
+def declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names.update(re.findall(r"^NVFP4_API\s+[\w\s\*]+?\b(nvfp4_\w+)\s*\(", text, flags=re.M))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from nvfp4_block_scaled_16_b200 import build
+    build.build()
+    return nv.load_library()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    decl = declared_symbols()
+    assert decl, "no declarations found"
+    assert decl == set(binding.EXPORTED_SYMBOLS) | (decl - set(binding.EXPORTED_SYMBOLS))
+    handle = ctypes.CDLL(nv.library_path())
+    for name in sorted(decl):
+        assert hasattr(handle, name), f"{name} declared in include/ but not exported"
+    for name in binding.EXPORTED_SYMBOLS:
+        assert name in decl, f"{name} bound in Python but not declared in include/"
+
+
+@pytest.mark.parametrize("rows,k,expect", [(128, 256, 2048), (8192, 8192, 4194304), (129, 16, 1024),
+                                           (0, 64, 0), (200, 80, 2048), (5, 8, -1), (-1, 16, -1)])
+def test_scale_bytes(lib, rows, k, expect):
+    assert nv.nvfp4_scale_bytes(rows, k) == expect
+
+
+def test_status_strings(lib):
+    assert nv.nvfp4_status_string(0) == "NVFP4_OK"
+    assert nv.nvfp4_status_string(1) == "NVFP4_ERR_INVALID_ARGUMENT"
+    assert nv.nvfp4_status_string(4) == "NVFP4_ERR_DEVICE_TIMEOUT"
+    assert nv.nvfp4_status_string(99) == "NVFP4_ERR_UNKNOWN"
+
+
+P = ctypes.c_void_p
+A16 = P(1 << 20)      # 16-byte aligned fake address, never dereferenced by validation
+A1 = P((1 << 20) + 1)  # misaligned
+
+
+@pytest.mark.parametrize("args", [
+    (A16, 4, 32, P(0), A16, A16, None),      # null gsf
+    (A1, 4, 32, A16, A16, A16, None),        # misaligned x
+    (A16, 4, 24, A16, A16, A16, None),       # k % 16 != 0
+    (A16, -1, 32, A16, A16, A16, None),      # negative m
+])
+def test_quantize_rejects_invalid(lib, args):
+    assert lib.nvfp4_quantize(*args) == INVALID
+
+
+def test_quantize_empty_is_noop(lib):
+    # m == 0 or k == 0: nothing to do, no device needed
+    assert lib.nvfp4_quantize(None, 0, 32, None, None, None, None) == 0
+    assert lib.nvfp4_quantize_masked_batched(None, 0, 4, 32, None, None, None, None, None) == 0
+
+
+def test_silu_rejects_odd_width(lib):
+    assert lib.nvfp4_silu_mul_quantize_batched(A16, 1, 4, 40, None, A16, A16, A16, None) == INVALID
+
+
+@pytest.mark.parametrize("m,n,k", [(128, 256, 96), (128, 250, 256), (128, 256, 0)])
+def test_gemm_rejects_bad_shapes(lib, m, n, k):
+    assert lib.nvfp4_gemm(A16, A16, A16, A16, A16, None, A16, m, n, k, None) == INVALID
+
+
+def test_gemm_rejects_null_and_misaligned(lib):
+    assert lib.nvfp4_gemm(A16, P(0), A16, A16, A16, None, A16, 128, 256, 256, None) == INVALID
+    assert lib.nvfp4_gemm(A16, A16, A1, A16, A16, None, A16, 128, 256, 256, None) == INVALID
+    assert lib.nvfp4_gemm(A16, A16, A16, A16, A16, A1, A16, 128, 256, 256, None) == INVALID
+
+
+@pytest.mark.parametrize("r", [0, 16, 48, 288, -32])
+def test_lowrank_rejects_bad_rank(lib, r):
+    assert lib.nvfp4_gemm_lowrank_bias(A16, A16, A16, A16, A16, A16, A16, r, None, A16, 128, 256, 256, None) == INVALID
+
+
+def test_grouped_requires_mask(lib):
+    assert lib.nvfp4_grouped_gemm_masked(A16, A16, A16, A16, None, A16, A16, 2, 128, 256, 256, None) == INVALID
+    assert lib.nvfp4_grouped_gemm_masked(A16, A16, A16, A16, A16, A16, A16, 2000, 128, 256, 256, None) == INVALID
+
+
+def test_global_scale_argument_checks(lib):
+    assert lib.nvfp4_global_scale(A16, 16, None, None, None, None, None) == INVALID          # gsf required
+    assert lib.nvfp4_global_scale(A16, 16, None, A16, A16, None, None) == INVALID           # alpha_out required
+    assert lib.nvfp4_global_scale(A1, 16, None, A16, None, None, None) == INVALID            # misaligned
+    assert lib.nvfp4_global_scale_batched(A16, 5000, 4, 16, None, 0, None, A16, None) == INVALID
+
+
+def test_valid_call_without_gpu_fails_loudly(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    # valid arguments reach the device query, which must report an error (no fallback)
+    st = lib.nvfp4_quantize(A16, 4, 32, A16, A16, A16, None)
+    assert st != 0
