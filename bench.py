@@ -1,0 +1,838 @@
+"""Benchmark of the NVFP4 linear-layer hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl nvfp4|reference]
+                    [--workload swiglu_block|quant_dense|quant_masked|quant_silu|grouped_moe|lowrank|pr1_linear]
+                    [--rank-lr R]
+
+Default workload: the dense NVFP4 SwiGLU shared-expert block, M = 8192 tokens, hidden
+5120, intermediate 8192.  One step is the whole hot path over one batch:
+    global amax of x (dynamic activation scale; also yields the gate/up alpha)
+    -> quantize x [8192, 5120]
+    -> gate/up GEMM [8192 x 5120] @ [16384 x 5120]^T  (bf16 out, [gate | up])
+    -> SiLU-and-mul fused quantize [8192, 16384] -> [8192, 8192] (calibrated static scale)
+    -> down GEMM [8192 x 8192] @ [5120 x 8192]^T  (bf16 out)
+Weights are quantized once before timing (offline weight quantization), and the static
+activation scale of h is calibrated once, as a deployed layer would.
+
+Timing: the step is captured once into a CUDA graph with a CUDA event node before and
+after every kernel; W warm-up replays, then K timed replays bracketed by a barrier and a
+device synchronize.  L2 is flushed (a 512 MB write) before every replay, outside the
+events; the step time is the device time between the first and the last event.  The value is whole-job throughput (sum over
+ranks of the work / the max over ranks of the device time).  With N > 1 every rank runs
+its own independent batch (data parallel, no collective on the data path): weak scaling.
+
+``--impl reference`` times the CPU oracle (the plain C reference implementation) on a
+bounded sample of the same workload on this machine's host cores.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import nvfp4_synth as S  # noqa: E402
+
+METRIC = "NVFP4 GEMM TFLOPS (% of FP4 peak); quantize HBM GB/s (% of HBM peak)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP4_OVER_BF16 = 4.0          # nominal dense ratio 9 PFLOP/s / 2.25 PFLOP/s
+L2_FLUSH_BYTES = 512 << 20
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def file_sha(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel source is unchanged."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(f"{kernel}@{workload}")
+    if not e:
+        return None
+    src = os.path.join(ROOT, e["source"])
+    if not os.path.exists(src) or file_sha(src) != e["source_sha"]:
+        return None
+    return e["bytes_per_launch"]
+
+
+# ---------------------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------------------
+
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, v):
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.item()
+
+
+def sum_over_ranks(world, v):
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return t.item()
+
+
+# ---------------------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"nvfp4_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu), "-lms", "20"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self, busy_only=True):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            p = [x.strip() for x in line.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                rows.append((float(p[1]), float(p[2]), float(p[3]) if p[3] not in ("[N/A]", "N/A") else 0.0, p[4:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        pmax = max(r[2] for r in rows)
+        loaded = [r for r in rows if r[2] >= 0.5 * pmax] if busy_only else rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[3][1:]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows), "samples_under_load": len(loaded),
+                "power_w_max": pmax}
+
+
+# ---------------------------------------------------------------------------------------
+# workloads (GPU)
+# ---------------------------------------------------------------------------------------
+
+def to_dev_bf16(bits):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def quantize_weight(nv, w):
+    """Offline weight quantization with the library: global scale, then block quantize."""
+    amax, gsf, _ = nv.nvfp4_global_scale(w)
+    q, sf = nv.nvfp4_quantize(w, gsf)
+    return q, sf, amax
+
+
+class Workload:
+    name = ""
+    unit = "TFLOP/s"
+    dominant = ""
+
+    def launches(self):
+        """List of (kernel name, callable) making up one step on the current stream."""
+        raise NotImplementedError
+
+    def work(self):
+        """Algorithmic work per step in the metric's unit base (FLOP or bytes)."""
+        raise NotImplementedError
+
+
+class SwigluBlock(Workload):
+    name = "swiglu_block"
+    unit = "TFLOP/s"
+    dominant = "gemm_gate_up"
+
+    def __init__(self, nv, seed=0):
+        import torch
+        self.nv = nv
+        self.M, self.H, self.I = 8192, 5120, 8192
+        d = S.swiglu_block(self.M, self.H, self.I, seed)
+        self.x_host = d["x"]
+        self.x = to_dev_bf16(d["x"])
+        self.wgu_q, self.wgu_sf, self.amax_wgu = quantize_weight(nv, to_dev_bf16(d["w_gate_up"]))
+        self.wd_q, self.wd_sf, self.amax_wd = quantize_weight(nv, to_dev_bf16(d["w_down"]))
+        dev = self.x.device
+        self.amax_x = torch.empty(1, dtype=torch.float32, device=dev)
+        self.gsf_x = torch.empty(1, dtype=torch.float32, device=dev)
+        self.alpha1 = torch.empty(1, dtype=torch.float32, device=dev)
+        self.xq = torch.empty((self.M, self.H // 2), dtype=torch.uint8, device=dev)
+        self.xsf = torch.empty(nv.nvfp4_scale_bytes(self.M, self.H), dtype=torch.uint8, device=dev)
+        self.gu = torch.empty((self.M, 2 * self.I), dtype=torch.bfloat16, device=dev)
+        self.hq = torch.empty((1, self.M, self.I // 2), dtype=torch.uint8, device=dev)
+        self.hsf = torch.empty((1, nv.nvfp4_scale_bytes(self.M, self.I)), dtype=torch.uint8, device=dev)
+        self.y = torch.empty((self.M, self.H), dtype=torch.bfloat16, device=dev)
+        # calibration pass: static scale of h = silu(gate) * up and the down-projection alpha
+        for _, fn in self.launches()[:3]:
+            fn()
+        amax_h, self.gsf_h = nv.nvfp4_global_scale_batched(self.gu.view(1, self.M, 2 * self.I), None, silu_mul=True)
+        a_h = np.float32(amax_h.item())
+        a_w = np.float32(self.amax_wd.item())
+        self.alpha2 = torch.tensor([np.float32(a_h * a_w) / np.float32(7225344.0)], dtype=torch.float32, device=dev)
+        torch.cuda.synchronize()
+
+    def launches(self):
+        nv = self
+        lib = self.nv
+        return [
+            ("global_scale_x", lambda: lib.nvfp4_global_scale(nv.x, nv.amax_x, nv.gsf_x, nv.amax_wgu, nv.alpha1)),
+            ("quantize_x", lambda: lib.nvfp4_quantize(nv.x, nv.gsf_x, nv.xq, nv.xsf)),
+            ("gemm_gate_up", lambda: lib.nvfp4_gemm(nv.xq, nv.wgu_q, nv.xsf, nv.wgu_sf, nv.alpha1, None, nv.gu)),
+            ("silu_mul_quantize", lambda: lib.nvfp4_silu_mul_quantize_batched(
+                nv.gu.view(1, nv.M, 2 * nv.I), nv.gsf_h, None, nv.hq, nv.hsf)),
+            ("gemm_down", lambda: lib.nvfp4_gemm(nv.hq.view(nv.M, nv.I // 2), nv.wd_q, nv.hsf.view(-1), nv.wd_sf,
+                                                 nv.alpha2, None, nv.y)),
+        ]
+
+    def work(self):
+        return 2.0 * self.M * self.H * (2 * self.I) + 2.0 * self.M * self.I * self.H
+
+    def kernel_work(self):
+        M, H, I = self.M, self.H, self.I
+        return {
+            "global_scale_x": (2.0 * M * H, "GB/s"),
+            "quantize_x": (2.5625 * M * H, "GB/s"),
+            "gemm_gate_up": (2.0 * M * H * 2 * I, "TFLOP/s"),
+            "silu_mul_quantize": (4.5625 * M * I, "GB/s"),
+            "gemm_down": (2.0 * M * I * H, "TFLOP/s"),
+        }
+
+    def e2e_io(self):
+        """(host input, device input, device output) of the end-to-end measurement."""
+        return self.x_host, self.x, self.y
+
+    def config(self):
+        return {"workload": "dense NVFP4 SwiGLU shared-expert block: tokens M=8192, hidden K=5120, "
+                            "intermediate 8192; gate/up [8192x5120]@[16384x5120]^T, silu*mul requantize, "
+                            "down [8192x8192]@[5120x8192]^T; x~N(0,1), W~N(0,0.02)",
+                "tokens": self.M, "hidden": self.H, "intermediate": self.I,
+                "l2": "flushed between steps (512 MB write, outside the timed events)"}
+
+
+class QuantDense(Workload):
+    name = "quant_dense"
+    unit = "GB/s"
+    dominant = "quantize"
+
+    def __init__(self, nv, seed=0):
+        import torch
+        self.nv = nv
+        self.m = self.k = 8192
+        self.x_host = S.quant_dense(self.m, self.k, seed)["x"]
+        self.x = to_dev_bf16(self.x_host)
+        self.amax = torch.empty(1, dtype=torch.float32, device="cuda")
+        self.gsf = torch.empty(1, dtype=torch.float32, device="cuda")
+        self.q = torch.empty((self.m, self.k // 2), dtype=torch.uint8, device="cuda")
+        self.sf = torch.empty(nv.nvfp4_scale_bytes(self.m, self.k), dtype=torch.uint8, device="cuda")
+
+    def launches(self):
+        lib, s = self.nv, self
+        return [("global_scale", lambda: lib.nvfp4_global_scale(s.x, s.amax, s.gsf)),
+                ("quantize", lambda: lib.nvfp4_quantize(s.x, s.gsf, s.q, s.sf))]
+
+    def work(self):
+        return 2.5625 * self.m * self.k
+
+    def kernel_work(self):
+        return {"global_scale": (2.0 * self.m * self.k, "GB/s"), "quantize": (2.5625 * self.m * self.k, "GB/s")}
+
+    def e2e_io(self):
+        return self.x_host, self.x, self.q
+
+    def config(self):
+        return {"workload": "quantize bf16 [8192,8192] ~N(0,1) with 0.1% outliers x50 (amax + quantize)",
+                "l2": "flushed between steps"}
+
+
+class QuantMasked(Workload):
+    unit = "GB/s"
+    dominant = "quantize_masked"
+
+    def __init__(self, nv, silu, seed=0):
+        import torch
+        self.nv, self.silu = nv, silu
+        self.name = "quant_silu" if silu else "quant_masked"
+        self.dominant = "silu_mul_quantize" if silu else "quantize_masked"
+        self.b, self.m, self.k = 8, 4096, 7168
+        d = S.quant_silu(self.b, self.m, self.k, seed) if silu else S.quant_masked(self.b, self.m, self.k, seed)
+        self.x_host = d["x"]
+        self.x = to_dev_bf16(d["x"])
+        self.mask_host = d["mask"]
+        self.mask = torch.from_numpy(d["mask"]).cuda()
+        _, self.gsf = nv.nvfp4_global_scale_batched(self.x, self.mask, silu_mul=silu)
+        self.q = torch.empty((self.b, self.m, self.k // 2), dtype=torch.uint8, device="cuda")
+        self.sf = torch.empty((self.b, nv.nvfp4_scale_bytes(self.m, self.k)), dtype=torch.uint8, device="cuda")
+        torch.cuda.synchronize()
+
+    def launches(self):
+        lib, s = self.nv, self
+        fn = lib.nvfp4_silu_mul_quantize_batched if self.silu else lib.nvfp4_quantize_masked_batched
+        return [(self.dominant, lambda: fn(s.x, s.gsf, s.mask, s.q, s.sf))]
+
+    def work(self):
+        per_row = (4 * self.k + self.k // 2 + self.k // 16) if self.silu else (2 * self.k + self.k // 2 + self.k // 16)
+        return float(per_row * int(self.mask_host.sum()))
+
+    def kernel_work(self):
+        return {self.dominant: (self.work(), "GB/s")}
+
+    def e2e_io(self):
+        return self.x_host, self.x, self.q
+
+    def config(self):
+        w = "[8,4096,2*7168] silu(gate)*up fused" if self.silu else "[8,4096,7168]"
+        return {"workload": f"masked batched quantize {w}, valid rows per item U[0,4096] (sum {int(self.mask_host.sum())})",
+                "l2": "flushed between steps"}
+
+
+class GroupedMoE(Workload):
+    name = "grouped_moe"
+    unit = "TFLOP/s"
+    dominant = "grouped_gemm"
+
+    def __init__(self, nv, seed=0):
+        import torch
+        self.nv = nv
+        self.E, self.mmax, self.k, self.n = 16, 2048, 5120, 8192
+        d = S.grouped_moe(self.E, self.mmax, self.k, self.n, 512, seed)
+        self.mask_host = d["mask"]
+        self.mask = torch.from_numpy(d["mask"]).cuda()
+        a = to_dev_bf16(d["a"])
+        w = to_dev_bf16(d["w"])
+        amax_a, ga = nv.nvfp4_global_scale_batched(a, self.mask)
+        amax_w, gw = nv.nvfp4_global_scale_batched(w, None)
+        self.aq, self.asf = nv.nvfp4_quantize_masked_batched(a, ga, self.mask)
+        self.wq, self.wsf = nv.nvfp4_quantize_masked_batched(w, gw, None)
+        al = (amax_a.cpu().numpy().astype(np.float32) * amax_w.cpu().numpy().astype(np.float32)) / np.float32(7225344.0)
+        self.alpha = torch.from_numpy(al.astype(np.float32)).cuda()
+        self.out = torch.empty((self.E, self.mmax, self.n), dtype=torch.bfloat16, device="cuda")
+        self.a_host = d["a"]
+        del a, w
+        torch.cuda.synchronize()
+
+    def launches(self):
+        lib, s = self.nv, self
+        return [("grouped_gemm", lambda: lib.nvfp4_grouped_gemm_masked(s.aq, s.wq, s.asf, s.wsf, s.mask, s.alpha,
+                                                                        s.out))]
+
+    def work(self):
+        return 2.0 * int(self.mask_host.sum()) * self.n * self.k
+
+    def kernel_work(self):
+        return {"grouped_gemm": (self.work(), "TFLOP/s")}
+
+    def e2e_io(self):
+        return None
+
+    def config(self):
+        return {"workload": f"masked grouped NVFP4 GEMM E=16 Mmax=2048 K=5120 N=8192, valid rows "
+                            f"min(Poisson(512),2048) (sum {int(self.mask_host.sum())})",
+                "l2": "flushed between steps"}
+
+
+class LowRank(Workload):
+    name = "lowrank"
+    unit = "TFLOP/s"
+    dominant = "gemm_lowrank"
+
+    def __init__(self, nv, r=64, seed=0):
+        import torch
+        self.nv, self.r = nv, r
+        self.m, self.k, self.n = 4096, 3072, 3072
+        d = S.lowrank(self.m, self.k, self.n, r, seed)
+        x = to_dev_bf16(d["x"])
+        amax_x, gsf_x, _ = nv.nvfp4_global_scale(x)
+        self.xq, self.xsf = nv.nvfp4_quantize(x, gsf_x)
+        self.wq, self.wsf, amax_w = quantize_weight(nv, to_dev_bf16(d["w"]))
+        alpha = np.float32(np.float32(amax_x.item()) * np.float32(amax_w.item())) / np.float32(7225344.0)
+        self.alpha = torch.tensor([alpha], dtype=torch.float32, device="cuda")
+        self.d = to_dev_bf16(d["d"])
+        self.l1 = to_dev_bf16(S.f32_to_bf16_bits(d["l1_f32"] / alpha))
+        self.bias = to_dev_bf16(d["bias"])
+        self.out = torch.empty((self.m, self.n), dtype=torch.bfloat16, device="cuda")
+        torch.cuda.synchronize()
+
+    def launches(self):
+        lib, s = self.nv, self
+        return [("gemm_lowrank", lambda: lib.nvfp4_gemm_lowrank_bias(s.xq, s.wq, s.xsf, s.wsf, s.alpha, s.d, s.l1,
+                                                                      s.bias, s.out))]
+
+    def work(self):
+        return 2.0 * self.m * self.n * self.k + 2.0 * self.m * self.n * self.r
+
+    def kernel_work(self):
+        return {"gemm_lowrank": (self.work(), "TFLOP/s")}
+
+    def e2e_io(self):
+        return None
+
+    def config(self):
+        return {"workload": f"low-rank-corrected NVFP4 GEMM M=4096 K=3072 N=3072 r={self.r} + bias",
+                "l2": "flushed between steps"}
+
+
+class PR1Linear(Workload):
+    name = "pr1_linear"
+    unit = "TFLOP/s"
+    dominant = "gemm"
+
+    def __init__(self, nv, seed=0):
+        import torch
+        self.nv = nv
+        d = S.pr1_linear(seed)
+        self.x = to_dev_bf16(d["x"])
+        self.wq, self.wsf, self.amax_w = quantize_weight(nv, to_dev_bf16(d["w"]))
+        self.amax = torch.empty(1, dtype=torch.float32, device="cuda")
+        self.gsf = torch.empty(1, dtype=torch.float32, device="cuda")
+        self.alpha = torch.empty(1, dtype=torch.float32, device="cuda")
+        self.xq = torch.empty((128, 128), dtype=torch.uint8, device="cuda")
+        self.xsf = torch.empty(nv.nvfp4_scale_bytes(128, 256), dtype=torch.uint8, device="cuda")
+        self.out = torch.empty((128, 256), dtype=torch.bfloat16, device="cuda")
+        self.x_host = d["x"]
+
+    def launches(self):
+        lib, s = self.nv, self
+        return [("global_scale", lambda: lib.nvfp4_global_scale(s.x, s.amax, s.gsf, s.amax_w, s.alpha)),
+                ("quantize", lambda: lib.nvfp4_quantize(s.x, s.gsf, s.xq, s.xsf)),
+                ("gemm", lambda: lib.nvfp4_gemm(s.xq, s.wq, s.xsf, s.wsf, s.alpha, None, s.out))]
+
+    def work(self):
+        return 2.0 * 128 * 256 * 256
+
+    def kernel_work(self):
+        return {"gemm": (self.work(), "TFLOP/s")}
+
+    def e2e_io(self):
+        return self.x_host, self.x, self.out
+
+    def config(self):
+        return {"workload": "single NVFP4 linear x[128,256] W[256,256] (latency-bound)", "l2": "flushed between steps"}
+
+
+def make_workload(name, nv, rank_lr):
+    if name == "swiglu_block":
+        return SwigluBlock(nv)
+    if name == "quant_dense":
+        return QuantDense(nv)
+    if name == "quant_masked":
+        return QuantMasked(nv, False)
+    if name == "quant_silu":
+        return QuantMasked(nv, True)
+    if name == "grouped_moe":
+        return GroupedMoE(nv)
+    if name == "lowrank":
+        return LowRank(nv, rank_lr)
+    if name == "pr1_linear":
+        return PR1Linear(nv)
+    raise SystemExit(f"unknown workload {name}")
+
+
+def scale(v, unit):
+    return v / 1e12 if unit == "TFLOP/s" else v / 1e9
+
+
+# ---------------------------------------------------------------------------------------
+# CPU oracle timing (reference arm and cpu_baseline)
+# ---------------------------------------------------------------------------------------
+
+class OracleSample:
+    """The CPU oracle on a bounded sample of a workload: ``setup()`` prepares (and
+    quantizes, offline) the weights once; each ``step()`` runs the sample's hot path and
+    returns its work in the metric's unit base and the seconds it took."""
+
+    def __init__(self, workload, rows=None):
+        import oracle as O
+        self.O = O
+        self.workload = workload
+        self.threads = O.get_threads()
+        self.unit = "GB/s" if workload.startswith("quant") else "TFLOP/s"
+        w = workload
+        if w == "swiglu_block":
+            self.rows = rows or 4
+            d = S.swiglu_block(8192, 5120, 8192, 0)
+            self.x = d["x"][:self.rows].copy()
+            self.wgu, self.wd = d["w_gate_up"], d["w_down"]
+            self.H, self.I = 5120, 8192
+            self.sample = f"{self.rows} of 8192 token rows through the whole block (amax, quantize, gate/up GEMM, " \
+                          f"SiLU-mul quantize, down GEMM)"
+        elif w == "pr1_linear":
+            self.rows = 128
+            d = S.pr1_linear(0)
+            self.x, self.w = d["x"], d["w"]
+            self.sample = "the whole 128x256x256 linear (amax, quantize, GEMM)"
+        elif w in ("quant_dense", "quant_masked", "quant_silu"):
+            self.rows = rows or 256
+            if w == "quant_dense":
+                self.x = S.quant_dense(8192, 8192, 0)["x"][:self.rows].copy()
+            else:
+                k = 7168
+                self.x = S.normal_bf16((1, self.rows, 2 * k if w == "quant_silu" else k), 1.0, 0, S.TID["x"])
+            self.sample = f"{self.rows} valid rows"
+        elif w in ("grouped_moe", "lowrank"):
+            self.rows = rows or 2
+            self.m, self.k, self.n = (self.rows, 5120, 8192) if w == "grouped_moe" else (self.rows, 3072, 3072)
+            self.x = S.normal_bf16((self.m, self.k), 1.0, 0, S.TID["x"])
+            self.w = S.normal_bf16((self.n, self.k), 0.02, 0, S.TID["w"])
+            self.sample = f"{self.m} rows x N={self.n} x K={self.k}"
+        else:
+            raise SystemExit(f"no oracle sample for {w}")
+        self._setup()
+
+    def _setup(self):
+        O = self.O
+        if self.workload == "swiglu_block":
+            self.aw, gw = O.global_scale(self.wgu)
+            self.qw, self.sfw = O.quantize(self.wgu, gw)
+            self.ad, gd = O.global_scale(self.wd)
+            self.qd, self.sfd = O.quantize(self.wd, gd)
+        elif self.workload in ("pr1_linear", "grouped_moe", "lowrank"):
+            self.aw, gw = O.global_scale(self.w)
+            self.qw, self.sfw = O.quantize(self.w, gw)
+
+    def step(self):
+        O = self.O
+        w = self.workload
+        t0 = time.perf_counter()
+        if w == "swiglu_block":
+            rows, H, I = self.rows, self.H, self.I
+            ax, gx = O.global_scale(self.x)
+            qx, sfx = O.quantize(self.x, gx)
+            gu = O.gemm_ref(qx, self.qw, sfx, self.sfw, O.alpha(float(ax), float(self.aw)), rows, 2 * I, H)
+            gu_bits = S.f32_to_bf16_bits(gu.astype(np.float32)).reshape(1, rows, 2 * I)
+            ah, gh = O.global_scale_batched(gu_bits, None, silu_mul=True)
+            hq, hsf = O.silu_mul_quantize_batched(gu_bits, gh)
+            O.gemm_ref(hq[0], self.qd, hsf[0], self.sfd, O.alpha(float(ah[0]), float(self.ad)), rows, H, I)
+            work = 2.0 * rows * H * 2 * I + 2.0 * rows * I * H
+        elif w == "pr1_linear":
+            ax, gx = O.global_scale(self.x)
+            qx, sfx = O.quantize(self.x, gx)
+            O.gemm_ref(qx, self.qw, sfx, self.sfw, O.alpha(float(ax), float(self.aw)), 128, 256, 256)
+            work = 2.0 * 128 * 256 * 256
+        elif w == "quant_dense":
+            a, g = O.global_scale(self.x)
+            O.quantize(self.x, g)
+            work = 2.5625 * self.x.size
+        elif w in ("quant_masked", "quant_silu"):
+            silu = w == "quant_silu"
+            _, gs = O.global_scale_batched(self.x, None, silu_mul=silu)
+            (O.silu_mul_quantize_batched if silu else O.quantize_masked_batched)(self.x, gs)
+            work = (32704.0 if silu else 18368.0) * self.rows
+        else:
+            ax, gx = O.global_scale(self.x)
+            qx, sfx = O.quantize(self.x, gx)
+            O.gemm_ref(qx, self.qw, sfx, self.sfw, O.alpha(float(ax), float(self.aw)), self.m, self.n, self.k)
+            work = 2.0 * self.m * self.n * self.k
+        return work, time.perf_counter() - t0
+
+    def measure(self, steps):
+        work = secs = 0.0
+        for _ in range(steps):
+            w, dt = self.step()
+            work += w
+            secs += dt
+        return scale(work / secs, self.unit), secs
+
+
+# ---------------------------------------------------------------------------------------
+# main
+# ---------------------------------------------------------------------------------------
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return       # the oracle runs on rank 0 only; the other ranks exit without work
+    wl = args.workload
+    rows = 1 if wl == "swiglu_block" else None
+    o = OracleSample(wl, rows)
+    o.measure(min(args.warmup, 1))
+    t0 = time.perf_counter()
+    value, secs = o.measure(args.steps)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": o.unit, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / max(args.steps, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (plain C oracle)",
+            "data": "synthetic", "config": {"workload": wl},
+            "cpu_baseline": {"value": value, "unit": o.unit, "cores": o.threads, "kind": "oracle",
+                             "sample": o.sample + " per step"},
+            "e2e": {"value": value, "unit": o.unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "wall_s": round(time.perf_counter() - t0, 2)}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="nvfp4", choices=["nvfp4", "reference"])
+    ap.add_argument("--workload", default="swiglu_block",
+                    choices=["swiglu_block", "quant_dense", "quant_masked", "quant_silu", "grouped_moe", "lowrank",
+                             "pr1_linear"])
+    ap.add_argument("--rank-lr", type=int, default=64)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, world, rank)
+        return
+
+    import torch
+    import nvfp4_block_scaled_16_b200 as nv
+    world, rank, local = dist_setup(args.gpus)
+    nv.load_library()
+    wl = make_workload(args.workload, nv, args.rank_lr)
+    launches = wl.launches()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.Stream()
+
+    def step(evs=None):
+        for i, (_, fn) in enumerate(launches):
+            if evs is not None:
+                evs[i].record()
+            fn()
+        if evs is not None:
+            evs[len(launches)].record()
+
+    # One eager pass on the launch stream (allocates the library's per-stream scratch),
+    # then the step is captured once into a CUDA graph with an external event node
+    # around every kernel, so host launch overhead never appears inside the timed
+    # kernels.  Should the driver refuse timing on graph event nodes, every kernel is
+    # captured into its own graph and timed by events recorded around its replay.
+    with torch.cuda.stream(stream):
+        step()
+    torch.cuda.synchronize()
+
+    def replay_all(graphs):
+        for g in graphs:
+            g.replay()
+
+    events = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(launches) + 1)]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step(events)
+    torch.cuda.synchronize()
+    timing_mode = "event nodes inside one CUDA graph per step"
+
+    def run_step_graph():
+        graph.replay()
+        stream.synchronize()
+        return [events[i].elapsed_time(events[i + 1]) for i in range(len(launches))] + \
+               [events[0].elapsed_time(events[-1])]
+
+    run_step = run_step_graph
+    try:
+        with torch.cuda.stream(stream):
+            run_step()
+    except Exception:                                      # noqa: BLE001
+        torch.cuda.synchronize()
+        graphs = []
+        for _, fn in launches:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                fn()
+            graphs.append(g)
+        outer = [torch.cuda.Event(enable_timing=True) for _ in range(len(launches) + 1)]
+        timing_mode = "one CUDA graph per kernel, events around each replay"
+
+        def run_step_split():
+            for i, g in enumerate(graphs):
+                outer[i].record()
+                g.replay()
+            outer[-1].record()
+            stream.synchronize()
+            return [outer[i].elapsed_time(outer[i + 1]) for i in range(len(launches))] + \
+                   [outer[0].elapsed_time(outer[-1])]
+
+        run_step = run_step_split
+        graph = None
+
+        def replay_step():
+            replay_all(graphs)
+    else:
+        def replay_step():
+            graph.replay()
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            flush.zero_()
+            replay_step()
+    torch.cuda.synchronize()
+    if nv.nvfp4_device_status(clear=True) != 0:
+        raise SystemExit("device-side timeout during warm-up")
+
+    samples = []
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        t_wall = time.perf_counter()
+        with torch.cuda.stream(stream):
+            for s in range(args.steps):
+                flush.zero_()
+                samples.append(run_step())
+        torch.cuda.synchronize()
+        t_wall = time.perf_counter() - t_wall
+    barrier(world)
+    status = nv.nvfp4_device_status(clear=True)
+    if status != 0:
+        raise SystemExit(f"device-side timeout in the timed region (status {status})")
+
+    per_kernel = {name: [smp[i] for smp in samples] for i, (name, _) in enumerate(launches)}
+    step_ms = [smp[-1] for smp in samples]
+    total_ms = sum(step_ms)
+    total_ms_max = max_over_ranks(world, total_ms)
+    work_all = sum_over_ranks(world, wl.work() * args.steps)
+    value = scale(work_all / (total_ms_max * 1e-3), wl.unit)
+    ms_per_step = total_ms_max / args.steps
+
+    peaks, peak_kind = load_peaks()
+    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    hbm_peak = peaks["hbm_gbs"]
+    parts = {}
+    for name, (w, unit) in wl.kernel_work().items():
+        ms = statistics.mean(per_kernel[name])
+        ach = scale(w / (ms * 1e-3), unit)
+        peak = fp4_peak if unit == "TFLOP/s" else hbm_peak
+        parts[name] = {"ms": round(ms, 5), "achieved": round(ach, 2), "unit": unit,
+                       "frac": round(ach / peak, 4)}
+
+    dom = wl.dominant
+    w, unit = wl.kernel_work()[dom]
+    dom_ms = statistics.mean(per_kernel[dom])
+    achieved = scale(w / (dom_ms * 1e-3), unit)
+    peak = fp4_peak if unit == "TFLOP/s" else hbm_peak
+    kernel_name = "nvfp4_gemm_kernel" if unit == "TFLOP/s" else "quantize_kernel"
+    traffic = recorded_traffic(kernel_name, f"{wl.name}:{dom}")
+    roofline = {"bound": "tensor" if unit == "TFLOP/s" else "hbm", "achieved": round(achieved, 2),
+                "peak": round(peak, 1), "unit": unit, "frac": round(achieved / peak, 4), "traffic": traffic,
+                "kernel": dom, "peak_source": f"{peak_kind}: " + (
+                    f"bf16 burst {peaks['bf16_tflops']} TFLOP/s x {FP4_OVER_BF16} (nominal FP4/BF16 dense ratio)"
+                    if unit == "TFLOP/s" else f"HBM copy {peaks['hbm_gbs']} GB/s")}
+
+    e2e = None
+    if not args.no_e2e and wl.e2e_io() is not None:
+        x_host_bits, x_dev, y_dev = wl.e2e_io()
+        x_pinned = torch.from_numpy(np.ascontiguousarray(x_host_bits).view(np.int16)).view(x_dev.dtype).pin_memory()
+        y_pinned = torch.empty(y_dev.shape, dtype=y_dev.dtype).pin_memory()
+        e_start = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        e_end = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        with torch.cuda.stream(stream):
+            for s in range(args.steps + args.warmup):
+                flush.zero_()
+                i = s - args.warmup
+                if i >= 0:
+                    e_start[i].record()
+                x_dev.copy_(x_pinned, non_blocking=True)
+                replay_step()
+                y_pinned.copy_(y_dev, non_blocking=True)
+                if i >= 0:
+                    e_end[i].record()
+        torch.cuda.synchronize()
+        e2e_ms = sum(a.elapsed_time(b) for a, b in zip(e_start, e_end))
+        e2e_ms = max_over_ranks(world, e2e_ms)
+        e2e_val = scale(sum_over_ranks(world, wl.work() * args.steps) / (e2e_ms * 1e-3), wl.unit)
+        e2e = {"value": round(e2e_val, 3), "unit": wl.unit, "h2d_bytes_per_step": int(x_pinned.numel() * x_pinned.element_size()),
+               "d2h_bytes_per_step": int(y_pinned.numel() * y_pinned.element_size()), "ms_per_step": round(e2e_ms / args.steps, 4)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        o = OracleSample(wl.name)
+        v, secs = o.measure(1)
+        cpu = {"value": v, "unit": wl.unit, "cores": o.threads, "kind": "oracle", "sample": o.sample,
+               "seconds": round(secs, 2)}
+
+    if rank == 0:
+        clk = clocks.summary()
+        line = {"metric": METRIC, "value": round(value, 3), "unit": wl.unit, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "e2m1 x e2m1 (ue4m3 block scales) -> f32 accumulate",
+                "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights)", "config": wl.config(),
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": len(launches) * args.steps, "parts": parts,
+                "clocks": {"sm_mhz": clk.get("sm_mhz"), "sm_max_mhz": clk.get("sm_max_mhz"),
+                           "reasons": clk.get("reasons")},
+                "wall_s_timed_region": round(t_wall, 4), "timing": timing_mode}
+        if world > 1:
+            line["config"]["parallelism"] = f"dp{world} (independent batch per GPU, no collective)"
+        print(json.dumps(line), flush=True)
+
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

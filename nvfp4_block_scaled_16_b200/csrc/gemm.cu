@@ -11,24 +11,30 @@
 // NVFP4LinearMethod.create_weights (weight [out, in/2], alpha); flashinfer PR #1774
 // "Masked batch nvfp4 quantization" (masked per-expert operands for the grouped GEMM).
 //
-// Kernel structure (one CTA per SM, persistent over output tiles of 128 x 256):
-//   warp 0      TMA producer: 2-D/3-D tiled loads of the packed operands (128-byte
-//               swizzle, one 128-byte K row = 256 FP4 values per stage) and 1-D bulk
-//               copies of the scale chunks, which are contiguous 512-byte blocks in the
-//               128x4 layout, into a 4-stage shared-memory ring.
-//   warp 1      TMEM allocator + MMA issuer (one thread): moves the stage's scale chunks
-//               to tensor memory with tcgen05.cp (32x128b, replicated to the 4 lane
-//               quarters) and issues tcgen05.mma kind::mxf4nvf4 (K = 64, ue4m3 scales per
-//               16 values) into an fp32 accumulator in TMEM; the low-rank term follows
-//               as kind::f16 (bf16) MMAs into the same accumulator.
-//   warps 2-5   epilogue: tcgen05.ld of the accumulator (each warp owns its 32-lane TMEM
-//               quarter = 32 rows), alpha * acc + bias, bf16 stores.
+// Kernel structure.  CTA pairs (clusters of 2 on one TPC) are persistent over output
+// tiles of 256 x 256.  Each CTA of a pair owns 128 rows of the A tile and 128 rows (one
+// half of N) of the B tile; the leader CTA issues tcgen05.mma.cta_group::2 (M = 256,
+// N = 256, K = 64, kind::mxf4nvf4 with ue4m3 scales per 16 values) for both, so each
+// SM streams only its own operand halves through shared memory.  Each CTA's tensor
+// memory holds the scales of its own 128 A rows and of all 256 B rows of the tile.
+//   warp 0      TMA producer (both CTAs): tiled loads (cta_group::2 form, no multicast)
+//               of the packed operands (128-byte swizzle, one 128-byte K row = 256 FP4
+//               values per stage) and of the scale chunks (each 128-row x 4-block group
+//               of the 128x4 layout is one contiguous 512-byte chunk); all loads of both
+//               CTAs complete on the leader's stage barrier.  5-stage ring.
+//   warp 1      TMEM allocator (both CTAs) and MMA issuer (leader, one thread): per
+//               K-step one tcgen05.cp (32x128b, replicated to the 4 lane quarters) of the
+//               SFA chunk and two of the SFB chunks, each CTA from its own shared memory
+//               into its own tensor memory, then the MMA; the low-rank term follows as kind::f16 (bf16) MMAs into the same
+//               accumulator.  Commits are multicast to both CTAs.
+//   warps 2-5   epilogue (both CTAs): tcgen05.ld of the CTA's 128 x 256 fp32 accumulator
+//               (each warp owns its 32-lane TMEM quarter), alpha * acc + bias, bf16 stores.
 // Two accumulators of 256 columns share TMEM columns [192, 256): the epilogue drains that
 // overlap first and releases the accumulator, so the next tile's MMAs overlap the rest of
 // the epilogue.  Scale factors use columns [448, 496).
 // Every mbarrier wait is bounded (about one second of global time); a wait that runs out
-// records NVFP4_ERR_DEVICE_TIMEOUT in the device status word and the whole CTA unwinds
-// without hanging the GPU.
+// records NVFP4_ERR_DEVICE_TIMEOUT in the device status word and the CTA unwinds without
+// hanging the GPU.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -36,47 +42,69 @@
 namespace nvfp4 {
 namespace {
 
-constexpr int kBM = 128;                 // output tile rows (MMA M)
-constexpr int kBN = 256;                 // output tile columns (MMA N)
+constexpr int kBM = 128;                 // A rows per CTA (MMA M = 256 per pair)
+constexpr int kBN = 256;                 // MMA N per pair tile
+constexpr int kBNHalf = 128;             // B rows per CTA
+constexpr int kTileM = 2 * kBM;          // output tile rows per pair
 constexpr int kStageK = 256;             // FP4 values of K per stage (128 bytes per row)
 constexpr int kStageBytesRow = kStageK / 2;
-constexpr int kStages = 4;
-constexpr int kABytes = kBM * kStageBytesRow;     // 16 KB
-constexpr int kBBytes = kBN * kStageBytesRow;     // 32 KB
-constexpr int kSfaBytes = 4 * 512;                // 4 K-steps x one 512-byte chunk
-constexpr int kSfbBytes = 2 * 4 * 512;            // two 128-row halves x 4 K-steps
-constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;  // 55296 = 54 KB
+constexpr int kStages = 5;
+constexpr int kABytes = kBM * kStageBytesRow;        // 16 KB
+constexpr int kBBytes = kBNHalf * kStageBytesRow;    // 16 KB
+constexpr int kSfaBytes = 4 * 512;                   // 4 K-steps x one 512-byte chunk
+constexpr int kSfbBytes = 2 * 4 * 512;               // both 128-row halves of the N tile
+constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;  // 38 KB
+constexpr uint32_t kFp4TxBytes = 2u * kStageBytes;              // both CTAs
+constexpr uint32_t kLrTxBytes = 2u * (kABytes + kBBytes);
 constexpr int kMaxExperts = 1024;
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccOverlapCol = 192;          // accumulator 1 starts here
-constexpr uint32_t kSfCol = 448;                  // SFA: +0..15, SFB: +16..47
+constexpr uint32_t kSfaCol = 448;                 // SFA: 448 + 4j, SFB: 464 + 8j (+4 upper half)
+constexpr uint32_t kSfbCol = 464;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
 
 // smem layout after the stage ring
 struct __align__(8) Control {
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
-  uint64_t acc_full;
-  uint64_t acc_empty;
+  uint64_t full[kStages];     // leader: all loads of a stage (both CTAs) landed
+  uint64_t empty[kStages];    // both: the stage's MMAs completed (multicast commit)
+  uint64_t acc_full;          // both: the tile's accumulator is complete (multicast commit)
+  uint64_t acc_empty;         // leader: the epilogues of both CTAs drained the overlap
   uint32_t tmem_base;
   int32_t abort;
-  int32_t prefix[kMaxExperts + 1];   // grouped: prefix sums of tiles per expert
+  int32_t prefix[kMaxExperts + 1];   // grouped: prefix sums of pair tiles per expert
 };
 constexpr int kSmemBytes = kStages * kStageBytes + sizeof(Control) + 1024;
 
 // Instruction descriptors (tcgen05 "instruction descriptor" bit fields).
 //   kind::mxf4nvf4: A/B format E2M1 (1) at bits 7..9 / 10..12, both K-major, N>>3 at
 //   bits 17..22, ue4m3 scale format (0) at bit 23, M>>4 at bits 24..28, scale ids 0.
-constexpr uint32_t kIdescFp4 = (1u << 7) | (1u << 10) | (uint32_t(kBN >> 3) << 17) | (uint32_t(kBM >> 4) << 24);
+constexpr uint32_t kIdescFp4 = (1u << 7) | (1u << 10) | (uint32_t(kBN >> 3) << 17) | (uint32_t(kTileM >> 4) << 24);
 //   kind::f16: fp32 accumulator (1) at bits 4..5, A/B bf16 (1), K-major, N, M as above.
 constexpr uint32_t kIdescBf16 =
-    (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kBN >> 3) << 17) | (uint32_t(kBM >> 4) << 24);
+    (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kBN >> 3) << 17) | (uint32_t(kTileM >> 4) << 24);
 
 // ---- PTX wrappers ---------------------------------------------------------------------------
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Shared::cluster address of the same smem variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(const void* p, uint32_t rank) {
+  uint32_t out;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(smem_u32(p)), "r"(rank));
+  return out;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 __device__ __forceinline__ uint64_t global_ns() {
@@ -89,8 +117,9 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
 }
 
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+// Arrive on a barrier given by its shared::cluster address (possibly in the peer CTA).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
@@ -102,7 +131,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(smem_u32(bar)), "r"(parity)
@@ -129,26 +158,22 @@ __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile 
   }
 }
 
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1) {
+// Tiled TMA loads into this CTA's shared memory, completing on the barrier at the
+// shared::cluster address `bar` (the leader's; the .cta_group::2 form allows either CTA
+// of the pair).
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint32_t bar, int c0, int c1) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
-      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
       : "memory");
 }
 
-__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
-                                            int c2) {
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint32_t bar, int c0, int c1, int c2) {
   asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
       "[%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
-}
-
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-               ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
-               : "memory");
 }
 
 __device__ __forceinline__ void prefetch_map(const CUtensorMap* map) {
@@ -170,8 +195,10 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t addr) { return smem_de
 // One 512-byte scale chunk as 32 rows x 16 bytes: 8-row core matrices 128 bytes apart.
 __device__ __forceinline__ uint64_t sf_desc(uint32_t addr) { return smem_desc(addr, 0, 128, 0); }
 
+// Copies a 512-byte scale chunk at the same smem address of both CTAs into 4 TMEM columns
+// (all 128 lanes) of both CTAs.
 __device__ __forceinline__ void tc_copy_sf(uint32_t tmem_col_addr, uint64_t desc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(tmem_col_addr), "l"(desc) : "memory");
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(tmem_col_addr), "l"(desc) : "memory");
 }
 
 __device__ __forceinline__ void mma_fp4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t sfa, uint32_t sfb,
@@ -179,7 +206,7 @@ __device__ __forceinline__ void mma_fp4(uint32_t d_tmem, uint64_t a_desc, uint64
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
       ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(kIdescFp4), "r"(accumulate), "r"(sfa), "r"(sfb)
       : "memory");
 }
@@ -188,14 +215,19 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint6
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
       ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(kIdescBf16), "r"(accumulate)
       : "memory");
 }
 
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
+// Arrives on the barrier at the same smem offset in both CTAs once every prior
+// tcgen05 operation of this thread has completed.
+__device__ __forceinline__ void mma_commit_both(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(static_cast<uint16_t>(3))
+      : "memory");
 }
 
 // 32 lanes x 64 consecutive fp32 columns: thread i of the warp gets lane (quarter*32 + i).
@@ -227,26 +259,21 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // ---- problem description ----------------------------------------------------------------------
 
 struct GemmParams {
-  const uint8_t* a_sf;     // expert 0
-  const uint8_t* b_sf;
-  int64_t a_sf_stride;     // bytes between experts
-  int64_t b_sf_stride;
-  const float* alpha;      // [1] or [E]
+  const float* alpha;         // [1] or [E]
   const __nv_bfloat16* bias;  // nullable [n]
-  __nv_bfloat16* out;      // [E, mmax, n] (E = 1 for dense)
-  const int32_t* mask;     // grouped only
+  __nv_bfloat16* out;         // [E, mmax, n] (E = 1 for dense)
+  const int32_t* mask;        // grouped only
   int* status;
-  int32_t m;               // rows per expert (mmax)
+  int32_t m;                  // rows per expert (mmax)
   int32_t n;
   int32_t k;
   int32_t experts;
-  int32_t rank;            // low-rank r (0 = none)
-  int32_t n_tiles;
-  int32_t m_tiles;         // dense: ceil(m / 128)
-  int32_t k_stages;        // ceil(k / 256)
-  int32_t k_steps;         // k / 64
-  int32_t sf_groups;       // ceil(k / 64): 512-byte chunks per 128-row tile
-  int32_t sf_row_tiles_b;  // ceil(n / 128)
+  int32_t rank;               // low-rank r (0 = none)
+  int32_t n_tiles;            // ceil(n / 256)
+  int32_t m_tiles;            // dense: ceil(m / 256)
+  int32_t k_stages;           // ceil(k / 256)
+  int32_t k_steps;            // k / 64
+  int32_t sf_groups;          // k / 64: 512-byte chunks per 128-row tile
 };
 
 struct TileCoord {
@@ -276,19 +303,25 @@ __device__ __forceinline__ bool tile_coord(const GemmParams& p, const Control& c
   }
 }
 
+struct Maps {
+  CUtensorMap a, b, sfa, sfb, d, l1;
+};
+
 // ---- the kernel ---------------------------------------------------------------------------------
 
 template <bool kGrouped, bool kLowRank>
-__global__ void __launch_bounds__(kThreads, 1)
-    nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
-                      const __grid_constant__ CUtensorMap map_d, const __grid_constant__ CUtensorMap map_l1,
-                      const GemmParams p) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    nvfp4_gemm_kernel(const __grid_constant__ Maps maps, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Control& ctl = *reinterpret_cast<Control*>(smem + kStages * kStageBytes);
   volatile int32_t* abort = &ctl.abort;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();           // 0 = leader of the pair
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1;
+  const int pairs = gridDim.x >> 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -296,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ctl.empty[s], 1);
     }
     mbar_init(&ctl.acc_full, 1);
-    mbar_init(&ctl.acc_empty, 4);
+    mbar_init(&ctl.acc_empty, 8);     // 4 epilogue warps in each CTA of the pair
     ctl.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -306,78 +339,84 @@ __global__ void __launch_bounds__(kThreads, 1)
       ctl.prefix[0] = 0;
       for (int e = 0; e < p.experts; ++e) {
         const int valid = min(max(p.mask[e], 0), p.m);
-        acc += (valid + kBM - 1) / kBM * p.n_tiles;
+        acc += (valid + kTileM - 1) / kTileM * p.n_tiles;
         ctl.prefix[e + 1] = acc;
       }
     }
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&ctl.tmem_base)),
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&ctl.tmem_base)),
                  "r"(kTmemCols)
                  : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync();      // the leader's barriers are initialized before the peer signals them
   tc_fence_after();
   const uint32_t tmem = ctl.tmem_base;
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      prefetch_map(&map_a);
-      prefetch_map(&map_b);
+      prefetch_map(&maps.a);
+      prefetch_map(&maps.b);
+      prefetch_map(&maps.sfa);
+      prefetch_map(&maps.sfb);
       if constexpr (kLowRank) {
-        prefetch_map(&map_d);
-        prefetch_map(&map_l1);
+        prefetch_map(&maps.d);
+        prefetch_map(&maps.l1);
       }
       const int lr_stages = kLowRank ? (p.rank + 63) / 64 : 0;
       uint32_t it = 0;
       bool ok = true;
       TileCoord t;
-      for (int tile = blockIdx.x; ok && tile_coord<kGrouped>(p, ctl, tile, t); tile += gridDim.x) {
-        const uint8_t* a_sf = p.a_sf + t.expert * p.a_sf_stride;
-        const uint8_t* b_sf = p.b_sf + t.expert * p.b_sf_stride;
+      for (int tile = pair; ok && tile_coord<kGrouped>(p, ctl, tile, t); tile += pairs) {
+        const int a_row = t.m_tile * kTileM + static_cast<int>(rank) * kBM;
+        const int b_row = t.n_tile * kBN + static_cast<int>(rank) * kBNHalf;
+        // scale chunk rows (128 bytes each, 4 per chunk) of this CTA's 128-row tiles
+        const int sfa_row0 = ((2 * t.m_tile + static_cast<int>(rank)) * p.sf_groups) * 4;
+        const int sfb_row0 = ((2 * t.n_tile) * p.sf_groups) * 4;      // both halves of the N tile
+        const int sfb_row1 = sfb_row0 + p.sf_groups * 4;
         for (int ks = 0; ks < p.k_stages + lr_stages; ++ks, ++it) {
           const uint32_t s = it % kStages, round = it / kStages;
           if (round > 0 && !(ok = mbar_wait(&ctl.empty[s], (round - 1) & 1, abort, p.status))) break;
           uint8_t* st = smem + s * kStageBytes;
+          const uint32_t full_bar = map_to_rank(&ctl.full[s], 0);
           if (ks < p.k_stages) {
-            const int nks = min(4, p.k_steps - 4 * ks);
-            const int halves = min(2, p.sf_row_tiles_b - 2 * t.n_tile);
-            mbar_arrive_expect_tx(&ctl.full[s], kABytes + kBBytes + nks * 512 * (1 + halves));
+            if (leader) mbar_arrive_expect_tx(&ctl.full[s], kFp4TxBytes);
             if constexpr (kGrouped) {
-              tma_load_3d(st, &map_a, &ctl.full[s], ks * kStageBytesRow, t.m_tile * kBM, t.expert);
-              tma_load_3d(st + kABytes, &map_b, &ctl.full[s], ks * kStageBytesRow, t.n_tile * kBN, t.expert);
+              tma_load_3d(st, &maps.a, full_bar, ks * kStageBytesRow, a_row, t.expert);
+              tma_load_3d(st + kABytes, &maps.b, full_bar, ks * kStageBytesRow, b_row, t.expert);
+              tma_load_3d(st + kABytes + kBBytes, &maps.sfa, full_bar, 0, sfa_row0 + 16 * ks, t.expert);
+              tma_load_3d(st + kABytes + kBBytes + kSfaBytes, &maps.sfb, full_bar, 0, sfb_row0 + 16 * ks, t.expert);
+              tma_load_3d(st + kABytes + kBBytes + kSfaBytes + kSfaBytes, &maps.sfb, full_bar, 0, sfb_row1 + 16 * ks,
+                          t.expert);
             } else {
-              tma_load_2d(st, &map_a, &ctl.full[s], ks * kStageBytesRow, t.m_tile * kBM);
-              tma_load_2d(st + kABytes, &map_b, &ctl.full[s], ks * kStageBytesRow, t.n_tile * kBN);
-            }
-            const int64_t chunk_a = static_cast<int64_t>(t.m_tile) * p.sf_groups + 4 * ks;
-            bulk_load(st + kABytes + kBBytes, a_sf + chunk_a * 512, nks * 512, &ctl.full[s]);
-            for (int h = 0; h < halves; ++h) {
-              const int64_t chunk_b = static_cast<int64_t>(2 * t.n_tile + h) * p.sf_groups + 4 * ks;
-              bulk_load(st + kABytes + kBBytes + kSfaBytes + h * 4 * 512, b_sf + chunk_b * 512, nks * 512,
-                        &ctl.full[s]);
+              tma_load_2d(st, &maps.a, full_bar, ks * kStageBytesRow, a_row);
+              tma_load_2d(st + kABytes, &maps.b, full_bar, ks * kStageBytesRow, b_row);
+              tma_load_2d(st + kABytes + kBBytes, &maps.sfa, full_bar, 0, sfa_row0 + 16 * ks);
+              tma_load_2d(st + kABytes + kBBytes + kSfaBytes, &maps.sfb, full_bar, 0, sfb_row0 + 16 * ks);
+              tma_load_2d(st + kABytes + kBBytes + kSfaBytes + kSfaBytes, &maps.sfb, full_bar, 0, sfb_row1 + 16 * ks);
             }
           } else if constexpr (kLowRank) {
             const int c = ks - p.k_stages;
-            mbar_arrive_expect_tx(&ctl.full[s], kABytes + kBBytes);
-            tma_load_2d(st, &map_d, &ctl.full[s], c * 64, t.m_tile * kBM);
-            tma_load_2d(st + kABytes, &map_l1, &ctl.full[s], c * 64, t.n_tile * kBN);
+            if (leader) mbar_arrive_expect_tx(&ctl.full[s], kLrTxBytes);
+            tma_load_2d(st, &maps.d, full_bar, c * 64, a_row);
+            tma_load_2d(st + kABytes, &maps.l1, full_bar, c * 64, b_row);
           }
         }
       }
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // ------------------------------------------------------------------ MMA issuer (leader)
+    if (leader && lane == 0) {
       const int lr_stages = kLowRank ? (p.rank + 63) / 64 : 0;
       uint32_t it = 0, tcount = 0;
       bool ok = true;
       TileCoord t;
-      for (int tile = blockIdx.x; ok && tile_coord<kGrouped>(p, ctl, tile, t); tile += gridDim.x, ++tcount) {
+      for (int tile = pair; ok && tile_coord<kGrouped>(p, ctl, tile, t); tile += pairs, ++tcount) {
         const uint32_t acc = tmem + ((tcount & 1) ? kAccOverlapCol : 0u);
         if (tcount > 0) {
           if (!(ok = mbar_wait(&ctl.acc_empty, (tcount - 1) & 1, abort, p.status))) break;
@@ -393,13 +432,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t sfa_s = st + kABytes + kBBytes;
             const uint32_t sfb_s = sfa_s + kSfaBytes;
             for (int j = 0; j < nks; ++j) {
-              tc_copy_sf(tmem + kSfCol + 4 * j, sf_desc(sfa_s + 512 * j));
-              tc_copy_sf(tmem + kSfCol + 16 + 8 * j, sf_desc(sfb_s + 512 * j));
-              tc_copy_sf(tmem + kSfCol + 16 + 8 * j + 4, sf_desc(sfb_s + 4 * 512 + 512 * j));
-            }
-            for (int j = 0; j < nks; ++j) {
-              mma_fp4(acc, operand_desc(st + 32 * j), operand_desc(st + kABytes + 32 * j), tmem + kSfCol + 4 * j,
-                      tmem + kSfCol + 16 + 8 * j, (ks > 0 || j > 0) ? 1u : 0u);
+              tc_copy_sf(tmem + kSfaCol + 4 * j, sf_desc(sfa_s + 512 * j));
+              tc_copy_sf(tmem + kSfbCol + 8 * j, sf_desc(sfb_s + 512 * j));
+              tc_copy_sf(tmem + kSfbCol + 8 * j + 4, sf_desc(sfb_s + kSfaBytes + 512 * j));
+              mma_fp4(acc, operand_desc(st + 32 * j), operand_desc(st + kABytes + 32 * j), tmem + kSfaCol + 4 * j,
+                      tmem + kSfbCol + 8 * j, (ks > 0 || j > 0) ? 1u : 0u);
             }
           } else if constexpr (kLowRank) {
             const int c = ks - p.k_stages;
@@ -407,30 +444,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < steps; ++j)
               mma_bf16(acc, operand_desc(st + 32 * j), operand_desc(st + kABytes + 32 * j), 1u);
           }
-          mma_commit(&ctl.empty[s]);
+          mma_commit_both(&ctl.empty[s]);
         }
         if (!ok) break;
-        mma_commit(&ctl.acc_full);
-      }
-      if (!ok) {
-        // Unwinding: wait (bounded) for this thread's MMAs to finish before TMEM is freed.
-        mma_commit(&ctl.acc_empty);
+        mma_commit_both(&ctl.acc_full);
       }
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------------ epilogue
+    // ------------------------------------------------------------------ epilogue (both CTAs)
     const int quarter = warp & 3;              // TMEM lane quarter this warp may access
     const int row_in_tile = quarter * 32 + lane;
+    const uint32_t acc_empty_leader = map_to_rank(&ctl.acc_empty, 0);
     uint32_t tcount = 0;
     TileCoord t;
-    for (int tile = blockIdx.x; tile_coord<kGrouped>(p, ctl, tile, t); tile += gridDim.x, ++tcount) {
+    for (int tile = pair; tile_coord<kGrouped>(p, ctl, tile, t); tile += pairs, ++tcount) {
       if (!mbar_wait(&ctl.acc_full, tcount & 1, abort, p.status)) break;
       tc_fence_after();
       const uint32_t buf = tcount & 1;
       const uint32_t col0 = buf ? kAccOverlapCol : 0u;
       const float alpha = __ldg(p.alpha + t.expert);
-      const int row = t.m_tile * kBM + row_in_tile;
+      const int row = t.m_tile * kTileM + static_cast<int>(rank) * kBM + row_in_tile;
       const bool row_ok = row < t.valid_rows;
       __nv_bfloat16* out_row = p.out + (static_cast<int64_t>(t.expert) * p.m + row) * p.n;
       for (int i = 0; i < 4; ++i) {
@@ -441,7 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (i == 0) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&ctl.acc_empty);
+          if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
         }
         const int col_base = t.n_tile * kBN + sub * 64;
         if (row_ok) {
@@ -480,48 +514,60 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---------------------------------------------------------------- teardown
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
-    if (*abort) {
-      // The issuer committed a final arrival on acc_empty when it unwound; give the
-      // outstanding MMAs a bounded time to finish before the columns are released.
-      const uint64_t t0 = global_ns();
-      while (global_ns() - t0 < 2000000ull) {
-      }
+  if (*abort) {
+    // Unwinding after a timed-out wait: give outstanding tensor-core and TMA operations a
+    // bounded time to drain before the tensor memory and the CTA's smem are released.
+    const uint64_t t0 = global_ns();
+    while (global_ns() - t0 < 2000000ull) {
     }
+  }
+  cluster_sync();      // no CTA leaves while its peer may still signal its barriers
+  if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
   }
 }
 
 // ---- host side ------------------------------------------------------------------------------------
 
 int make_map(CUtensorMap* map, CUtensorMapDataType dtype, uint32_t rank, const void* base, const uint64_t* dims,
-             const uint64_t* strides_bytes, const uint32_t* box) {
+             const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swizzle) {
   EncodeTiledFn encode = encode_tiled_fn();
   if (!encode) return NVFP4_ERR_CUDA;
   uint32_t elem_strides[3] = {1, 1, 1};
   CUresult r = encode(map, dtype, rank, const_cast<void*>(base), dims, strides_bytes, box, elem_strides,
-                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_INVALID_ARGUMENT;
 }
 
 // Packed FP4 operand [experts, rows, k/2] as a tiled uint8 tensor with boxes of 128 bytes
-// (one stage of K) by box_rows rows.
-int make_operand_map(CUtensorMap* map, const uint8_t* base, int64_t experts, int64_t rows, int64_t k,
-                     uint32_t box_rows, bool grouped) {
+// (one stage of K) by 128 rows, 128-byte swizzle.
+int make_operand_map(CUtensorMap* map, const uint8_t* base, int64_t experts, int64_t rows, int64_t k, bool grouped) {
   const uint64_t dims[3] = {static_cast<uint64_t>(k / 2), static_cast<uint64_t>(rows), static_cast<uint64_t>(experts)};
   const uint64_t strides[2] = {static_cast<uint64_t>(k / 2), static_cast<uint64_t>(rows * (k / 2))};
-  const uint32_t box[3] = {kStageBytesRow, box_rows, 1};
-  return make_map(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, grouped ? 3 : 2, base, dims, strides, box);
+  const uint32_t box[3] = {kStageBytesRow, 128, 1};
+  return make_map(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, grouped ? 3 : 2, base, dims, strides, box,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-// bf16 low-rank operand [rows, r] with boxes of 64 values (128 bytes) by box_rows rows.
-int make_lowrank_map(CUtensorMap* map, const void* base, int64_t rows, int64_t r, uint32_t box_rows) {
+// Scale buffer [experts][nvfp4_scale_bytes(rows, k)] viewed as rows of 128 bytes; a box
+// of 16 rows is 4 consecutive 512-byte chunks (one stage of K for one 128-row tile).
+int make_scale_map(CUtensorMap* map, const uint8_t* base, int64_t experts, int64_t rows, int64_t k, bool grouped) {
+  const int64_t bytes = nvfp4_scale_bytes(rows, k);
+  const uint64_t dims[3] = {128, static_cast<uint64_t>(bytes / 128), static_cast<uint64_t>(experts)};
+  const uint64_t strides[2] = {128, static_cast<uint64_t>(bytes)};
+  const uint32_t box[3] = {128, 16, 1};
+  return make_map(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, grouped ? 3 : 2, base, dims, strides, box,
+                  CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+// bf16 low-rank operand [rows, r] with boxes of 64 values (128 bytes) by 128 rows.
+int make_lowrank_map(CUtensorMap* map, const void* base, int64_t rows, int64_t r) {
   const uint64_t dims[2] = {static_cast<uint64_t>(r), static_cast<uint64_t>(rows)};
   const uint64_t strides[1] = {static_cast<uint64_t>(r * 2)};
-  const uint32_t box[2] = {64, box_rows};
-  return make_map(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box);
+  const uint32_t box[2] = {64, 128};
+  return make_map(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 template <bool kGrouped, bool kLowRank>
@@ -543,21 +589,18 @@ int launch_gemm(const uint8_t* a, const uint8_t* b, const uint8_t* a_sf, const u
   int st = current_device(&info);
   if (st != NVFP4_OK) return st;
 
-  CUtensorMap map_a, map_b, map_d, map_l1;
-  memset(&map_d, 0, sizeof(map_d));
-  memset(&map_l1, 0, sizeof(map_l1));
-  if ((st = make_operand_map(&map_a, a, E, m, k, kBM, kGrouped)) != NVFP4_OK) return st;
-  if ((st = make_operand_map(&map_b, b, E, n, k, kBN, kGrouped)) != NVFP4_OK) return st;
+  Maps maps;
+  memset(&maps, 0, sizeof(maps));
+  if ((st = make_operand_map(&maps.a, a, E, m, k, kGrouped)) != NVFP4_OK) return st;
+  if ((st = make_operand_map(&maps.b, b, E, n, k, kGrouped)) != NVFP4_OK) return st;
+  if ((st = make_scale_map(&maps.sfa, a_sf, E, m, k, kGrouped)) != NVFP4_OK) return st;
+  if ((st = make_scale_map(&maps.sfb, b_sf, E, n, k, kGrouped)) != NVFP4_OK) return st;
   if (kLowRank) {
-    if ((st = make_lowrank_map(&map_d, d, m, r, kBM)) != NVFP4_OK) return st;
-    if ((st = make_lowrank_map(&map_l1, l1, n, r, kBN)) != NVFP4_OK) return st;
+    if ((st = make_lowrank_map(&maps.d, d, m, r)) != NVFP4_OK) return st;
+    if ((st = make_lowrank_map(&maps.l1, l1, n, r)) != NVFP4_OK) return st;
   }
 
   GemmParams p;
-  p.a_sf = a_sf;
-  p.b_sf = b_sf;
-  p.a_sf_stride = nvfp4_scale_bytes(m, k);
-  p.b_sf_stride = nvfp4_scale_bytes(n, k);
   p.alpha = alpha;
   p.bias = static_cast<const __nv_bfloat16*>(bias);
   p.out = static_cast<__nv_bfloat16*>(out);
@@ -569,25 +612,37 @@ int launch_gemm(const uint8_t* a, const uint8_t* b, const uint8_t* a_sf, const u
   p.experts = static_cast<int32_t>(E);
   p.rank = static_cast<int32_t>(r);
   p.n_tiles = static_cast<int32_t>((n + kBN - 1) / kBN);
-  p.m_tiles = static_cast<int32_t>((m + kBM - 1) / kBM);
+  p.m_tiles = static_cast<int32_t>((m + kTileM - 1) / kTileM);
   p.k_stages = static_cast<int32_t>((k + kStageK - 1) / kStageK);
   p.k_steps = static_cast<int32_t>(k / 64);
   p.sf_groups = static_cast<int32_t>(k / 64);
-  p.sf_row_tiles_b = static_cast<int32_t>((n + 127) / 128);
 
   auto kernel = nvfp4_gemm_kernel<kGrouped, kLowRank>;
-  static bool attr_set = false;
-  if (!attr_set) {
+  // One-time set-up per kernel instantiation: the dynamic shared memory opt-in and the
+  // number of 2-CTA clusters that fit on the device at once (the persistent grid size).
+  static int max_clusters = 0;
+  if (max_clusters == 0) {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess) {
       cudaGetLastError();
       return NVFP4_ERR_CUDA;
     }
-    attr_set = true;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(info.sm_count / 2 * 2);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg) != cudaSuccess || clusters <= 0) {
+      cudaGetLastError();
+      clusters = info.sm_count / 2;
+    }
+    max_clusters = clusters;
   }
-  int64_t tiles = kGrouped ? static_cast<int64_t>(E) * p.m_tiles * p.n_tiles : static_cast<int64_t>(p.m_tiles) * p.n_tiles;
+  const int64_t tiles = kGrouped ? static_cast<int64_t>(E) * p.m_tiles * p.n_tiles
+                                 : static_cast<int64_t>(p.m_tiles) * p.n_tiles;
   if (tiles >= (int64_t(1) << 31)) return NVFP4_ERR_INVALID_ARGUMENT;
-  const int grid = static_cast<int>(tiles < info.sm_count ? tiles : info.sm_count);
-  kernel<<<grid, kThreads, kSmemBytes, stream>>>(map_a, map_b, map_d, map_l1, p);
+  const int64_t max_pairs = max_clusters;
+  const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
+  kernel<<<2 * pairs, kThreads, kSmemBytes, stream>>>(maps, p);
   return launch_status();
 }
 
