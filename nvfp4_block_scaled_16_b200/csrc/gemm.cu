@@ -90,6 +90,15 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// True in exactly one lane of a converged warp.  tcgen05 and TMA instructions are issued
+// from a converged warp through this election: issuing them from a lone lane of a
+// diverged warp serializes the tensor pipe.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile("{\n\t.reg .pred q;\n\telect.sync _|q, 0xffffffff;\n\tselp.u32 %0, 1, 0, q;\n\t}" : "=r"(pred));
+  return pred != 0;
+}
+
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
@@ -358,7 +367,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    // The whole warp runs the loop; one elected lane issues each stage's loads.
+    if (elect_one()) {
       prefetch_map(&maps.a);
       prefetch_map(&maps.b);
       prefetch_map(&maps.sfa);
@@ -367,22 +377,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         prefetch_map(&maps.d);
         prefetch_map(&maps.l1);
       }
-      const int lr_stages = kLowRank ? (p.rank + 63) / 64 : 0;
-      uint32_t it = 0;
-      bool ok = true;
-      TileCoord t;
-      for (int tile = pair; ok && tile_coord<kGrouped>(p, ctl, tile, t); tile += pairs) {
-        const int a_row = t.m_tile * kTileM + static_cast<int>(rank) * kBM;
-        const int b_row = t.n_tile * kBN + static_cast<int>(rank) * kBNHalf;
-        // scale chunk rows (128 bytes each, 4 per chunk) of this CTA's 128-row tiles
-        const int sfa_row0 = ((2 * t.m_tile + static_cast<int>(rank)) * p.sf_groups) * 4;
-        const int sfb_row0 = ((2 * t.n_tile) * p.sf_groups) * 4;      // both halves of the N tile
-        const int sfb_row1 = sfb_row0 + p.sf_groups * 4;
-        for (int ks = 0; ks < p.k_stages + lr_stages; ++ks, ++it) {
-          const uint32_t s = it % kStages, round = it / kStages;
-          if (round > 0 && !(ok = mbar_wait(&ctl.empty[s], (round - 1) & 1, abort, p.status))) break;
-          uint8_t* st = smem + s * kStageBytes;
-          const uint32_t full_bar = map_to_rank(&ctl.full[s], 0);
+    }
+    __syncwarp();
+    const int lr_stages = kLowRank ? (p.rank + 63) / 64 : 0;
+    uint32_t it = 0;
+    bool ok = true;
+    TileCoord t;
+    for (int tile = pair; ok && tile_coord<kGrouped>(p, ctl, tile, t); tile += pairs) {
+      const int a_row = t.m_tile * kTileM + static_cast<int>(rank) * kBM;
+      const int b_row = t.n_tile * kBN + static_cast<int>(rank) * kBNHalf;
+      // scale chunk rows (128 bytes each, 4 per chunk): this CTA's 128 A rows, both B halves
+      const int sfa_row0 = ((2 * t.m_tile + static_cast<int>(rank)) * p.sf_groups) * 4;
+      const int sfb_row0 = ((2 * t.n_tile) * p.sf_groups) * 4;
+      const int sfb_row1 = sfb_row0 + p.sf_groups * 4;
+      for (int ks = 0; ks < p.k_stages + lr_stages; ++ks, ++it) {
+        const uint32_t s = it % kStages, round = it / kStages;
+        if (round > 0 && !(ok = mbar_wait(&ctl.empty[s], (round - 1) & 1, abort, p.status))) break;
+        uint8_t* st = smem + s * kStageBytes;
+        const uint32_t full_bar = map_to_rank(&ctl.full[s], 0);
+        if (elect_one()) {
           if (ks < p.k_stages) {
             if (leader) mbar_arrive_expect_tx(&ctl.full[s], kFp4TxBytes);
             if constexpr (kGrouped) {
@@ -406,12 +419,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tma_load_2d(st + kABytes, &maps.l1, full_bar, c * 64, b_row);
           }
         }
+        __syncwarp();
       }
     }
-    __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer (leader)
-    if (leader && lane == 0) {
+    // The whole warp runs the loop; one elected lane issues each batch of tcgen05 ops.
+    if (leader) {
       const int lr_stages = kLowRank ? (p.rank + 63) / 64 : 0;
       uint32_t it = 0, tcount = 0;
       bool ok = true;
@@ -427,27 +441,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (!(ok = mbar_wait(&ctl.full[s], (it / kStages) & 1, abort, p.status))) break;
           tc_fence_after();
           const uint32_t st = smem_u32(smem + s * kStageBytes);
-          if (ks < p.k_stages) {
-            const int nks = min(4, p.k_steps - 4 * ks);
-            const uint32_t sfa_s = st + kABytes + kBBytes;
-            const uint32_t sfb_s = sfa_s + kSfaBytes;
-            for (int j = 0; j < nks; ++j) {
-              tc_copy_sf(tmem + kSfaCol + 4 * j, sf_desc(sfa_s + 512 * j));
-              tc_copy_sf(tmem + kSfbCol + 8 * j, sf_desc(sfb_s + 512 * j));
-              tc_copy_sf(tmem + kSfbCol + 8 * j + 4, sf_desc(sfb_s + kSfaBytes + 512 * j));
-              mma_fp4(acc, operand_desc(st + 32 * j), operand_desc(st + kABytes + 32 * j), tmem + kSfaCol + 4 * j,
-                      tmem + kSfbCol + 8 * j, (ks > 0 || j > 0) ? 1u : 0u);
+          if (elect_one()) {
+            if (ks < p.k_stages) {
+              const int nks = min(4, p.k_steps - 4 * ks);
+              const uint32_t sfa_s = st + kABytes + kBBytes;
+              const uint32_t sfb_s = sfa_s + kSfaBytes;
+              for (int j = 0; j < nks; ++j) {
+                tc_copy_sf(tmem + kSfaCol + 4 * j, sf_desc(sfa_s + 512 * j));
+                tc_copy_sf(tmem + kSfbCol + 8 * j, sf_desc(sfb_s + 512 * j));
+                tc_copy_sf(tmem + kSfbCol + 8 * j + 4, sf_desc(sfb_s + kSfaBytes + 512 * j));
+                mma_fp4(acc, operand_desc(st + 32 * j), operand_desc(st + kABytes + 32 * j), tmem + kSfaCol + 4 * j,
+                        tmem + kSfbCol + 8 * j, (ks > 0 || j > 0) ? 1u : 0u);
+              }
+            } else if constexpr (kLowRank) {
+              const int c = ks - p.k_stages;
+              const int steps = min(4, (p.rank - 64 * c) / 16);
+              for (int j = 0; j < steps; ++j)
+                mma_bf16(acc, operand_desc(st + 32 * j), operand_desc(st + kABytes + 32 * j), 1u);
             }
-          } else if constexpr (kLowRank) {
-            const int c = ks - p.k_stages;
-            const int steps = min(4, (p.rank - 64 * c) / 16);
-            for (int j = 0; j < steps; ++j)
-              mma_bf16(acc, operand_desc(st + 32 * j), operand_desc(st + kABytes + 32 * j), 1u);
+            mma_commit_both(&ctl.empty[s]);
           }
-          mma_commit_both(&ctl.empty[s]);
+          __syncwarp();
         }
         if (!ok) break;
-        mma_commit_both(&ctl.acc_full);
+        if (elect_one()) mma_commit_both(&ctl.acc_full);
+        __syncwarp();
       }
     }
     __syncwarp();
