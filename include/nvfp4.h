@@ -101,6 +101,27 @@ NVFP4_API int nvfp4_global_scale_batched(const void *x_bf16, int64_t b, int64_t 
                                float *gsf_out, nvfp4_stream_t stream);
 
 /*
+ * Non-allocating variant of nvfp4_global_scale_batched (same arguments, same results).
+ * The pages have no counterpart of this entry point; it exists for callers that cannot
+ * let the library call cudaMalloc: code being captured into a CUDA graph, hosts whose
+ * device memory belongs to their own allocator or is fixed at start-up, and paths that
+ * must not risk the implicit synchronization an allocation can cause.  Its reduction
+ * scratch is a fixed device array inside the library (4100 bytes, held by every GPU that
+ * loads the library until the process exits) instead of the per-stream workspace.
+ *   b must be at most 1024; larger b returns NVFP4_ERR_INVALID_ARGUMENT before anything
+ *   is launched.
+ *   The first call on each device looks up the array's device address (no allocation);
+ *   make that first call before capturing the stream into a CUDA graph.
+ *   Every call clears and uses the same array: calls that overlap on the GPU (concurrent
+ *   streams, or concurrently running graphs) race with each other and must be ordered by
+ *   the caller.  Calls on one stream are ordered and safe.
+ * Calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+NVFP4_API int nvfp4_global_scale_batched_noalloc(const void *x_bf16, int64_t b, int64_t m, int64_t k,
+                                                 const int32_t *mask, int silu_mul, float *amax_out,
+                                                 float *gsf_out, nvfp4_stream_t stream);
+
+/*
  * Dense NVFP4 quantize [TRT create_weights; FI3 fp4_quantize(x, global_scale, 16, ...)].
  *   x_bf16 [m, k] bf16, 16-byte aligned; k % 16 == 0, m >= 0.
  *   gsf    fp32 [1] device: the global scale 448*6/amax.

@@ -17,6 +17,7 @@ from .binding import (  # noqa: F401
     nvfp4_status_string,
     nvfp4_global_scale,
     nvfp4_global_scale_batched,
+    nvfp4_global_scale_batched_noalloc,
     nvfp4_quantize,
     nvfp4_quantize_masked_batched,
     nvfp4_silu_mul_quantize_batched,

@@ -18,6 +18,7 @@ EXPORTED_SYMBOLS = (
     "nvfp4_scale_bytes",
     "nvfp4_global_scale",
     "nvfp4_global_scale_batched",
+    "nvfp4_global_scale_batched_noalloc",
     "nvfp4_quantize",
     "nvfp4_quantize_masked_batched",
     "nvfp4_silu_mul_quantize_batched",
@@ -36,6 +37,7 @@ _SIGNATURES = {
     "nvfp4_scale_bytes": (_I64, [_I64, _I64]),
     "nvfp4_global_scale": (_INT, [_P, _I64, _P, _P, _P, _P, _P]),
     "nvfp4_global_scale_batched": (_INT, [_P, _I64, _I64, _I64, _P, _INT, _P, _P, _P]),
+    "nvfp4_global_scale_batched_noalloc": (_INT, [_P, _I64, _I64, _I64, _P, _INT, _P, _P, _P]),
     "nvfp4_quantize": (_INT, [_P, _I64, _I64, _P, _P, _P, _P]),
     "nvfp4_quantize_masked_batched": (_INT, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P]),
     "nvfp4_silu_mul_quantize_batched": (_INT, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P]),
@@ -133,6 +135,18 @@ def nvfp4_global_scale_batched(x, mask=None, silu_mul=False, amax_out=None, gsf_
         st = load_library().nvfp4_global_scale_batched(_ptr(x), b, m, k, _ptr(mask), int(bool(silu_mul)),
                                                        _ptr(amax_out), _ptr(gsf_out), _stream(stream))
     _check("nvfp4_global_scale_batched", st)
+    return amax_out, gsf_out
+
+
+def nvfp4_global_scale_batched_noalloc(x, mask, silu_mul, amax_out, gsf_out, stream=None):
+    """nvfp4_global_scale_batched with library-internal fixed scratch: nothing is allocated,
+    so the outputs must be passed in (fp32 [b] each; amax_out may be None)."""
+    b, m, w = x.shape
+    k = w // 2 if silu_mul else w
+    with torch.cuda.device(x.device):
+        st = load_library().nvfp4_global_scale_batched_noalloc(_ptr(x), b, m, k, _ptr(mask), int(bool(silu_mul)),
+                                                               _ptr(amax_out), _ptr(gsf_out), _stream(stream))
+    _check("nvfp4_global_scale_batched_noalloc", st)
     return amax_out, gsf_out
 
 

@@ -18,6 +18,7 @@
 // warp) and one scale byte at its swizzled position.  Conversions use the sm_100a
 // round-to-nearest-even, saturate-to-finite cvt instructions.
 #include <cfloat>
+#include <mutex>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -457,3 +458,95 @@ int nvfp4_silu_mul_quantize_batched(const void* x_bf16, int64_t b, int64_t m, in
 }
 
 }  // extern "C"
+
+// ---- non-allocating variant of the batched global scale ------------------------------------
+//
+// Some callers cannot let the library call cudaMalloc: code that is being captured into a
+// CUDA graph (allocation is not a capturable operation), hosts whose device memory is
+// owned by their own allocator or fixed at start-up (inference servers with a pre-sized
+// pool, embedded deployments), and latency-critical paths that must not risk the implicit
+// device synchronization cudaMalloc can cause.  nvfp4_global_scale_batched_noalloc serves
+// them: its reduction scratch is the file-scope device array below instead of the lazily
+// allocated per-stream workspace, so the call allocates nothing, ever.
+namespace nvfp4 {
+namespace {
+
+constexpr int kNoAllocMaxItems = 1024;
+// word 0: ticket counter; words 1..kNoAllocMaxItems: per-item amax bits.  Every GPU that
+// loads this library holds it until the process exits.
+static __device__ __align__(256) uint32_t g_noalloc_scratch[1 + kNoAllocMaxItems];
+
+std::mutex g_noalloc_mu;
+uint32_t* g_noalloc_ptr[64] = {};   // device address of g_noalloc_scratch, per device
+int g_noalloc_sms[64] = {};
+
+// Once per device, with that device current: look up the array's device address (host
+// code cannot use the symbol itself) and the SM count.  Allocates nothing.
+int noalloc_setup(int* dev_out, uint32_t** ptr_out, int* sms_out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return NVFP4_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return NVFP4_ERR_CUDA;
+    }
+    if (major != 10 || minor != 0) return NVFP4_ERR_UNSUPPORTED_DEVICE;
+    uint32_t* ptr = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&ptr), g_noalloc_scratch) != cudaSuccess || ptr == nullptr) {
+      cudaGetLastError();
+      return NVFP4_ERR_CUDA;
+    }
+    g_noalloc_sms[dev] = sms;
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *dev_out = dev;
+  *ptr_out = g_noalloc_ptr[dev];
+  *sms_out = g_noalloc_sms[dev];
+  return NVFP4_OK;
+}
+
+}  // namespace
+}  // namespace nvfp4
+
+extern "C" int nvfp4_global_scale_batched_noalloc(const void* x_bf16, int64_t b, int64_t m, int64_t k,
+                                                  const int32_t* mask, int silu_mul, float* amax_out,
+                                                  float* gsf_out, nvfp4_stream_t stream) {
+  using namespace nvfp4;
+  if (b < 0 || m < 0 || k < 0 || k % 8 != 0 || b > kNoAllocMaxItems || m > (1 << 30) || k > (1 << 30))
+    return NVFP4_ERR_INVALID_ARGUMENT;
+  if (b == 0) return NVFP4_OK;
+  if (!gsf_out || (m > 0 && k > 0 && !x_bf16)) return NVFP4_ERR_INVALID_ARGUMENT;
+  if ((x_bf16 && !aligned(x_bf16, 16)) || !aligned(gsf_out, 4) || (amax_out && !aligned(amax_out, 4)) ||
+      (mask && !aligned(mask, 4)))
+    return NVFP4_ERR_INVALID_ARGUMENT;
+  int dev = -1, sms = 0;
+  uint32_t* scratch = nullptr;
+  int st = noalloc_setup(&dev, &scratch, &sms);
+  if (st != NVFP4_OK) return st;
+  // The array keeps whatever the previous call left: the counter and the used amax words
+  // must start at zero.
+  if (cudaMemsetAsync(scratch, 0, sizeof(uint32_t) * (1 + b), stream) != cudaSuccess) {
+    cudaGetLastError();
+    return NVFP4_ERR_CUDA;
+  }
+  const int64_t nvec = m * (k / 8);
+  int64_t gx = (nvec + kThreads * 4 - 1) / (kThreads * 4);
+  const int64_t cap = (sms * 8 + b - 1) / b;
+  gx = gx < 1 ? 1 : (gx > cap ? cap : gx);
+  dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(b));
+  const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
+  if (silu_mul)
+    amax_batched_kernel<true><<<grid, kThreads, 0, stream>>>(x, static_cast<int32_t>(m), static_cast<int32_t>(k), mask,
+                                                             scratch, amax_out, gsf_out);
+  else
+    amax_batched_kernel<false><<<grid, kThreads, 0, stream>>>(x, static_cast<int32_t>(m), static_cast<int32_t>(k), mask,
+                                                              scratch, amax_out, gsf_out);
+  return launch_status();
+}
