@@ -114,6 +114,76 @@ __device__ __forceinline__ float silu_mul_bf16(float g, float u) {
   return __bfloat162float(__float2bfloat16_rn(p));
 }
 
+// ---- the same arithmetic on pairs of values with packed f32x2 instructions -----------------
+// Each lane of fma/mul/add.rn.f32x2 is one correctly rounded fp32 operation, so the pair
+// functions return exactly what the scalar ones return.
+
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unpack2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t splat2(float v) { return pack2(v, v); }
+
+// exp_specified of a pair.  The input is clamped to [-104, 89], which leaves every result
+// unchanged (e^x overflows to +inf for x > 88.73 and rounds to 0 for x <= -104), and 2^n
+// is applied as two exact power-of-two multiplications 2^(n/2) * 2^(n - n/2): both halves
+// are normal numbers for n in [-150, 128], so only the last multiplication can round --
+// the same single rounding as the three-way scaling of exp_specified.  NaN stays NaN.
+__device__ __forceinline__ void exp_specified2(float x0, float x1, float& e0, float& e1) {
+  const float c0 = fmaxf(fminf(x0, 89.0f), -104.0f);
+  const float c1 = fmaxf(fminf(x1, 89.0f), -104.0f);
+  const uint64_t x = pack2(c0, c1);
+  float t0, t1;
+  unpack2(mul2(x, splat2(0x1.715476p+0f)), t0, t1);
+  const float n0 = rintf(t0), n1 = rintf(t1);
+  const uint64_t n = pack2(n0, n1);
+  uint64_t r = fma2(n, splat2(-0x1.62e4p-1f), x);
+  r = fma2(n, splat2(-0x1.7f7d1cp-20f), r);
+  uint64_t p = splat2(0x1.a01a02p-13f);
+  p = fma2(p, r, splat2(0x1.6c16c2p-10f));
+  p = fma2(p, r, splat2(0x1.111112p-7f));
+  p = fma2(p, r, splat2(0x1.555556p-5f));
+  p = fma2(p, r, splat2(0x1.555556p-3f));
+  p = fma2(p, r, splat2(0x1.0p-1f));
+  p = fma2(p, r, splat2(1.0f));
+  p = fma2(p, r, splat2(1.0f));
+  const int i0 = static_cast<int>(n0), i1 = static_cast<int>(n1);
+  const int h0 = i0 / 2, h1 = i1 / 2;
+  p = mul2(p, pack2(pow2_int(h0), pow2_int(h1)));
+  p = mul2(p, pack2(pow2_int(i0 - h0), pow2_int(i1 - h1)));
+  unpack2(p, e0, e1);
+  if (x0 != x0) e0 = x0;
+  if (x1 != x1) e1 = x1;
+}
+
+// silu_mul_bf16 of a pair: h = bf16((g / (1 + exp(-g))) * u), as fp32 values.
+__device__ __forceinline__ void silu_mul_bf16_2(float g0, float g1, float u0, float u1, float& h0, float& h1) {
+  float e0, e1;
+  exp_specified2(-g0, -g1, e0, e1);
+  const float s0 = __fdiv_rn(g0, __fadd_rn(1.0f, e0));
+  const float s1 = __fdiv_rn(g1, __fadd_rn(1.0f, e1));
+  float p0, p1;
+  unpack2(mul2(pack2(s0, s1), pack2(u0, u1)), p0, p1);
+  uint32_t b2;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(b2) : "f"(p1), "f"(p0));   // p0 -> low half
+  h0 = __uint_as_float(b2 << 16);
+  h1 = __uint_as_float(b2 & 0xffff0000u);
+}
+
 // ---- one 16-element block ------------------------------------------------------------------
 
 struct QBlock {
@@ -130,13 +200,12 @@ __device__ __forceinline__ QBlock quantize16(const float* v, float gsf) {
   b.s8 = ue4m3_encode(s32);
   const float sd = e4m3_decode(b.s8);
   const float inv = sd == 0.0f ? 0.0f : __fdiv_rn(gsf, sd);
-  float t[8];
+  const uint64_t inv2 = pack2(inv, inv);
+  float t[16];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) t[i] = __fmul_rn(v[i], inv);
+  for (int i = 0; i < 16; i += 2) unpack2(mul2(pack2(v[i], v[i + 1]), inv2), t[i], t[i + 1]);
   b.lo = e2m1x8(t);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) t[i] = __fmul_rn(v[8 + i], inv);
-  b.hi = e2m1x8(t);
+  b.hi = e2m1x8(t + 8);
   return b;
 }
 
@@ -220,7 +289,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantParams p)
         unpack_bf16x8(raw[u][2], up);
         unpack_bf16x8(raw[u][3], up + 8);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = silu_mul_bf16(v[i], up[i]);
+        for (int i = 0; i < 16; i += 2) silu_mul_bf16_2(v[i], v[i + 1], up[i], up[i + 1], v[i], v[i + 1]);
       }
       const QBlock b = quantize16(v, gsf);
       *reinterpret_cast<uint2*>(q + static_cast<int64_t>(r) * (p.k / 2) + c * 8) = make_uint2(b.lo, b.hi);
