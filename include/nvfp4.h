@@ -211,6 +211,53 @@ NVFP4_API int nvfp4_gemm_lowrank_bias(const uint8_t *a, const uint8_t *b, const 
                             nvfp4_stream_t stream);
 
 /*
+ * Gate/up projection with SiLU * up and NVFP4 quantization in the GEMM epilogue (the
+ * SwiGLU block's first half) [NVF module tree: NVFP4InferenceSwiGLU gate_proj / up_proj;
+ * FI3 silu_and_mul_fp4_batched_quantize, the quantizer it replaces]:
+ *   g = bf16(alpha_gate * (a @ b_gate^T)),  u = bf16(alpha_up * (a @ b_up^T)),
+ *   h = bf16(silu(g) * u),  (q_out, sf_out) = NVFP4 quantization of h with gsf_h.
+ * Each of g, u, h and the quantized output is rounded exactly as by nvfp4_gemm (no
+ * bias) followed by nvfp4_silu_mul_quantize_batched on [g | u], so the result equals
+ * that two-call sequence on the same accumulator values; the bf16 g and u never
+ * reach memory.
+ *   a          uint8 [m, k/2] packed e2m1; a_sf [nvfp4_scale_bytes(m, k)].
+ *   b_gate     uint8 [n, k/2] (gate_proj weight); b_gate_sf [nvfp4_scale_bytes(n, k)].
+ *   b_up       uint8 [n, k/2] (up_proj weight);   b_up_sf   [nvfp4_scale_bytes(n, k)].
+ *              A concatenated [2n, k/2] gate/up weight quantized as one tensor is passed
+ *              as b_gate = w, b_up = w + n*k/2, b_up_sf = w_sf + nvfp4_scale_bytes(n, k)
+ *              and the same alpha twice.
+ *   alpha_gate, alpha_up  fp32 [1] device scalars.
+ *   gsf_h      fp32 [1] device scalar: the global scale of h (448*6 / amax(h), taken
+ *              from calibration because amax(h) is not known before the GEMM).
+ *   q_out      uint8 [m, n/2]; sf_out uint8 [nvfp4_scale_bytes(m, n)]; padding rows
+ *              m <= r < pad_up(m, 128) of sf_out are written as 0.
+ *   n % 128 == 0 (n is the width of h); k % 64 == 0; 16-byte aligned buffers.
+ */
+NVFP4_API int nvfp4_gemm_silu_mul_quantize(const uint8_t *a, const uint8_t *b_gate, const uint8_t *b_up,
+                                 const uint8_t *a_sf, const uint8_t *b_gate_sf,
+                                 const uint8_t *b_up_sf, const float *alpha_gate,
+                                 const float *alpha_up, const float *gsf_h, uint8_t *q_out,
+                                 uint8_t *sf_out, int64_t m, int64_t n, int64_t k,
+                                 nvfp4_stream_t stream);
+
+/*
+ * Masked grouped form for the routed experts [NVF NVFP4InferenceGroupedSwiGLU; FI3
+ * masked silu_and_mul quantize]: for every expert e and row i < mask[e], the computation
+ * of nvfp4_gemm_silu_mul_quantize with a[e], b_gate[e], b_up[e], alpha_gate[e],
+ * alpha_up[e] and gsf_h[e].
+ *   a [E, mmax, k/2]; a_sf [E][nvfp4_scale_bytes(mmax, k)].
+ *   b_gate, b_up [E, n, k/2]; b_gate_sf, b_up_sf [E][nvfp4_scale_bytes(n, k)].
+ *   mask int32 [E]; alpha_gate, alpha_up, gsf_h fp32 [E] (device).
+ *   q_out [E, mmax, n/2]; sf_out [E][nvfp4_scale_bytes(mmax, n)].  Rows i >= mask[e]
+ *   (codes and scale entries) are not written, as in nvfp4_silu_mul_quantize_batched.
+ */
+NVFP4_API int nvfp4_grouped_gemm_silu_mul_quantize_masked(
+    const uint8_t *a, const uint8_t *b_gate, const uint8_t *b_up, const uint8_t *a_sf,
+    const uint8_t *b_gate_sf, const uint8_t *b_up_sf, const int32_t *mask, const float *alpha_gate,
+    const float *alpha_up, const float *gsf_h, uint8_t *q_out, uint8_t *sf_out, int64_t E, int64_t mmax,
+    int64_t n, int64_t k, nvfp4_stream_t stream);
+
+/*
  * Device-side status word of the current device.  GEMM kernels bound every wait; a
  * wait that runs out records NVFP4_ERR_DEVICE_TIMEOUT here and the kernel returns
  * without hanging the GPU.  Synchronizes the device, then stores the word in

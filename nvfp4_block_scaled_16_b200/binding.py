@@ -25,6 +25,8 @@ EXPORTED_SYMBOLS = (
     "nvfp4_gemm",
     "nvfp4_grouped_gemm_masked",
     "nvfp4_gemm_lowrank_bias",
+    "nvfp4_gemm_silu_mul_quantize",
+    "nvfp4_grouped_gemm_silu_mul_quantize_masked",
     "nvfp4_device_status",
 )
 
@@ -44,6 +46,8 @@ _SIGNATURES = {
     "nvfp4_gemm": (_INT, [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "nvfp4_grouped_gemm_masked": (_INT, [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P]),
     "nvfp4_gemm_lowrank_bias": (_INT, [_P, _P, _P, _P, _P, _P, _P, _I64, _P, _P, _I64, _I64, _I64, _P]),
+    "nvfp4_gemm_silu_mul_quantize": (_INT, [_P] * 11 + [_I64, _I64, _I64, _P]),
+    "nvfp4_grouped_gemm_silu_mul_quantize_masked": (_INT, [_P] * 12 + [_I64, _I64, _I64, _I64, _P]),
     "nvfp4_device_status": (_INT, [ctypes.POINTER(_INT), _INT]),
 }
 
@@ -228,6 +232,47 @@ def nvfp4_gemm_lowrank_bias(a, b, a_sf, b_sf, alpha, d, l1, bias=None, out=None,
                                                     _stream(stream))
     _check("nvfp4_gemm_lowrank_bias", st)
     return out
+
+
+def nvfp4_gemm_silu_mul_quantize(a, b_gate, b_up, a_sf, b_gate_sf, b_up_sf, alpha_gate, alpha_up, gsf_h,
+                                 q_out=None, sf_out=None, stream=None):
+    """h = bf16(silu(bf16(alpha_gate * a @ b_gate^T)) * bf16(alpha_up * a @ b_up^T)) quantized with gsf_h.
+
+    a [m, k/2], b_gate / b_up [n, k/2] -> (q_out [m, n/2] uint8, sf_out [nvfp4_scale_bytes(m, n)] uint8).
+    """
+    m, kh = a.shape
+    n = b_gate.shape[0]
+    if q_out is None:
+        q_out = torch.empty((m, n // 2), dtype=torch.uint8, device=a.device)
+    if sf_out is None:
+        sf_out = torch.empty((nvfp4_scale_bytes(m, n),), dtype=torch.uint8, device=a.device)
+    with torch.cuda.device(a.device):
+        st = load_library().nvfp4_gemm_silu_mul_quantize(
+            _ptr(a), _ptr(b_gate), _ptr(b_up), _ptr(a_sf), _ptr(b_gate_sf), _ptr(b_up_sf), _ptr(alpha_gate),
+            _ptr(alpha_up), _ptr(gsf_h), _ptr(q_out), _ptr(sf_out), m, n, 2 * kh, _stream(stream))
+    _check("nvfp4_gemm_silu_mul_quantize", st)
+    return q_out, sf_out
+
+
+def nvfp4_grouped_gemm_silu_mul_quantize_masked(a, b_gate, b_up, a_sf, b_gate_sf, b_up_sf, mask, alpha_gate,
+                                                alpha_up, gsf_h, q_out=None, sf_out=None, stream=None):
+    """Per expert e, rows < mask[e]: nvfp4_gemm_silu_mul_quantize of a[e] with b_gate[e], b_up[e].
+
+    a [E, mmax, k/2], b_gate / b_up [E, n, k/2] -> (q_out [E, mmax, n/2], sf_out [E, nvfp4_scale_bytes(mmax, n)]).
+    """
+    E, mmax, kh = a.shape
+    n = b_gate.shape[1]
+    if q_out is None:
+        q_out = torch.empty((E, mmax, n // 2), dtype=torch.uint8, device=a.device)
+    if sf_out is None:
+        sf_out = torch.empty((E, nvfp4_scale_bytes(mmax, n)), dtype=torch.uint8, device=a.device)
+    with torch.cuda.device(a.device):
+        st = load_library().nvfp4_grouped_gemm_silu_mul_quantize_masked(
+            _ptr(a), _ptr(b_gate), _ptr(b_up), _ptr(a_sf), _ptr(b_gate_sf), _ptr(b_up_sf), _ptr(mask),
+            _ptr(alpha_gate), _ptr(alpha_up), _ptr(gsf_h), _ptr(q_out), _ptr(sf_out), E, mmax, n, 2 * kh,
+            _stream(stream))
+    _check("nvfp4_grouped_gemm_silu_mul_quantize_masked", st)
+    return q_out, sf_out
 
 
 def nvfp4_device_status(clear: bool = True) -> int:

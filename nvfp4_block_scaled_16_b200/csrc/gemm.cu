@@ -3,13 +3,19 @@
 //   nvfp4_gemm                 out = bf16(alpha * a @ b^T [+ bias])
 //   nvfp4_gemm_lowrank_bias    out = bf16(alpha * (a @ b^T + d @ l1^T) [+ bias])
 //   nvfp4_grouped_gemm_masked  out[e, i] = bf16(alpha[e] * a[e, i] @ b[e]^T), i < mask[e]
+//   nvfp4_gemm_silu_mul_quantize (and its masked grouped form)
+//                              g = bf16(alpha_gate * a @ b_gate^T), u = bf16(alpha_up * a @ b_up^T),
+//                              h = bf16(silu(g) * u) quantized to NVFP4 in the epilogue
 //
 // Sources (page title, section): flashinfer docs mm_nvfp4_svdquant (signature,
 // Parameters: packed (m, k/2) and (n, k/2) operands, 128x4-swizzled ue4m3 scales,
 // alpha device scalar, rank-r bf16 correction issued as a second MMA into the same
 // accumulator after the FP4 K-loop, epilogue alpha*acc + bias); TensorRT-LLM
 // NVFP4LinearMethod.create_weights (weight [out, in/2], alpha); flashinfer PR #1774
-// "Masked batch nvfp4 quantization" (masked per-expert operands for the grouped GEMM).
+// "Masked batch nvfp4 quantization" (masked per-expert operands for the grouped GEMM, and
+// the silu_and_mul quantizer whose input is the gate/up projection's output); the Llama4
+// MoE description on the same pages (routed experts: gate/up projection, SiLU * up, down
+// projection).
 //
 // Kernel structure.  CTA pairs (clusters of 2 on one TPC) are persistent over output
 // tiles of 256 x 256.  Each CTA of a pair owns 128 rows of the A tile and 128 rows (one
@@ -29,15 +35,25 @@
 //               accumulator.  Commits are multicast to both CTAs.
 //   warps 2-5   epilogue (both CTAs): tcgen05.ld of the CTA's 128 x 256 fp32 accumulator
 //               (each warp owns its 32-lane TMEM quarter), alpha * acc + bias, bf16 stores.
+//               The SiLU * up epilogue uses warps 2-9: two per lane quarter, one per half
+//               of the tile's 128 h columns.
 // Two accumulators of 256 columns share TMEM columns [192, 256): the epilogue drains that
 // overlap first and releases the accumulator, so the next tile's MMAs overlap the rest of
 // the epilogue.  Scale factors use columns [448, 496).
+// SiLU * up epilogue: the B half of CTA 0 is 128 rows of the gate weight and the B half of
+// CTA 1 the same 128 rows of the up weight, so accumulator columns [0, 128) hold g and
+// [128, 256) hold u for 128 columns of h.  Each thread owns one row: it rounds g and u to
+// bf16 exactly as the bf16 epilogue would, forms h, and quantizes each 16-value block with
+// the caller's global scale (64 code bytes and 8 scale bytes per row and tile).  Every
+// epilogue warp loads all its accumulator columns before any arithmetic and releases the
+// accumulator right after, so the next tile's MMAs overlap the whole SiLU and quantization.
 // Every mbarrier wait is bounded (about one second of global time); a wait that runs out
 // records NVFP4_ERR_DEVICE_TIMEOUT in the device status word and the CTA unwinds without
 // hanging the GPU.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
+#include "nvfp4_math.cuh"
 
 namespace nvfp4 {
 namespace {
@@ -57,7 +73,12 @@ constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;  // 38 KB
 constexpr uint32_t kFp4TxBytes = 2u * kStageBytes;              // both CTAs
 constexpr uint32_t kLrTxBytes = 2u * (kABytes + kBBytes);
 constexpr int kMaxExperts = 1024;
-constexpr int kThreads = 192;
+// Warps: 0 TMA producer, 1 MMA issuer, then the epilogue warps (two per TMEM lane quarter
+// for the SiLU * up epilogue, whose arithmetic needs more warps to hide its latency).
+template <bool kSwiGLU>
+constexpr int kEpiWarps = kSwiGLU ? 8 : 4;
+template <bool kSwiGLU>
+constexpr int kThreads = 64 + 32 * kEpiWarps<kSwiGLU>;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccOverlapCol = 192;          // accumulator 1 starts here
 constexpr uint32_t kSfaCol = 448;                 // SFA: 448 + 4j, SFB: 464 + 8j (+4 upper half)
@@ -256,7 +277,25 @@ __device__ __forceinline__ void tmem_load_64(uint32_t taddr, uint32_t* v) {
         "=r"(v[48]), "=r"(v[49]), "=r"(v[50]), "=r"(v[51]), "=r"(v[52]), "=r"(v[53]), "=r"(v[54]), "=r"(v[55]),
         "=r"(v[56]), "=r"(v[57]), "=r"(v[58]), "=r"(v[59]), "=r"(v[60]), "=r"(v[61]), "=r"(v[62]), "=r"(v[63])
       : "r"(taddr));
+}
+
+// Waits for this thread's tcgen05.ld results; the empty asm statements after the wait
+// redefine the registers, so no use of them can be scheduled before it.
+template <int N>
+__device__ __forceinline__ void tmem_wait_ld(uint32_t* v) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(v[i]));
+}
+
+// bf16(alpha * a), bf16(alpha * b) as fp32 values: the rounding of the bf16 epilogue.
+__device__ __forceinline__ void scale_round_bf16_2(float alpha, uint32_t a, uint32_t b, float& ra, float& rb) {
+  float pa, pb;
+  unpack2(mul2(pack2(__uint_as_float(a), __uint_as_float(b)), splat2(alpha)), pa, pb);
+  uint32_t w;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w) : "f"(pb), "f"(pa));   // pa -> low half
+  ra = __uint_as_float(w << 16);
+  rb = __uint_as_float(w & 0xffff0000u);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -283,6 +322,13 @@ struct GemmParams {
   int32_t k_stages;           // ceil(k / 256)
   int32_t k_steps;            // k / 64
   int32_t sf_groups;          // k / 64: 512-byte chunks per 128-row tile
+  // SiLU * up epilogue (n is the width of h; b is the gate weight, b2 the up weight)
+  const float* alpha_up;      // [1] or [E]: alpha of the up projection (alpha: gate)
+  const float* gsf_h;         // [1] or [E]: global scale of h
+  uint8_t* q;                 // [E, mmax, n/2] packed codes of h
+  uint8_t* sf;                // [E][nvfp4_scale_bytes(mmax, n)] swizzled scales of h
+  int64_t sf_item_stride;     // nvfp4_scale_bytes(mmax, n)
+  int32_t rows_pad;           // pad_up(mmax, 128)
 };
 
 struct TileCoord {
@@ -314,12 +360,13 @@ __device__ __forceinline__ bool tile_coord(const GemmParams& p, const Control& c
 
 struct Maps {
   CUtensorMap a, b, sfa, sfb, d, l1;
+  CUtensorMap b2, sfb2;       // SiLU * up: the up weight and its scales
 };
 
 // ---- the kernel ---------------------------------------------------------------------------------
 
-template <bool kGrouped, bool kLowRank>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+template <bool kGrouped, bool kLowRank, bool kSwiGLU>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kSwiGLU>, 1)
     nvfp4_gemm_kernel(const __grid_constant__ Maps maps, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -338,7 +385,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(&ctl.empty[s], 1);
     }
     mbar_init(&ctl.acc_full, 1);
-    mbar_init(&ctl.acc_empty, 8);     // 4 epilogue warps in each CTA of the pair
+    mbar_init(&ctl.acc_empty, 2 * kEpiWarps<kSwiGLU>);   // every epilogue warp of both CTAs
     ctl.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -373,6 +420,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       prefetch_map(&maps.b);
       prefetch_map(&maps.sfa);
       prefetch_map(&maps.sfb);
+      if constexpr (kSwiGLU) {
+        prefetch_map(&maps.b2);
+        prefetch_map(&maps.sfb2);
+      }
       if constexpr (kLowRank) {
         prefetch_map(&maps.d);
         prefetch_map(&maps.l1);
@@ -385,11 +436,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     TileCoord t;
     for (int tile = pair; ok && tile_coord<kGrouped>(p, ctl, tile, t); tile += pairs) {
       const int a_row = t.m_tile * kTileM + static_cast<int>(rank) * kBM;
-      const int b_row = t.n_tile * kBN + static_cast<int>(rank) * kBNHalf;
+      // 128-row tiles of B in the two halves of the pair tile: adjacent tiles of b, or for
+      // the SiLU * up epilogue the same tile of the gate weight (b) and the up weight (b2)
+      const int b_tile0 = kSwiGLU ? t.n_tile : 2 * t.n_tile;
+      const int b_tile1 = kSwiGLU ? t.n_tile : 2 * t.n_tile + 1;
+      const int b_row = (rank ? b_tile1 : b_tile0) * kBNHalf;
+      const CUtensorMap* b_map = (kSwiGLU && rank) ? &maps.b2 : &maps.b;
+      const CUtensorMap* sfb1_map = kSwiGLU ? &maps.sfb2 : &maps.sfb;
       // scale chunk rows (128 bytes each, 4 per chunk): this CTA's 128 A rows, both B halves
       const int sfa_row0 = ((2 * t.m_tile + static_cast<int>(rank)) * p.sf_groups) * 4;
-      const int sfb_row0 = ((2 * t.n_tile) * p.sf_groups) * 4;
-      const int sfb_row1 = sfb_row0 + p.sf_groups * 4;
+      const int sfb_row0 = (b_tile0 * p.sf_groups) * 4;
+      const int sfb_row1 = (b_tile1 * p.sf_groups) * 4;
       for (int ks = 0; ks < p.k_stages + lr_stages; ++ks, ++it) {
         const uint32_t s = it % kStages, round = it / kStages;
         if (round > 0 && !(ok = mbar_wait(&ctl.empty[s], (round - 1) & 1, abort, p.status))) break;
@@ -400,17 +457,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (leader) mbar_arrive_expect_tx(&ctl.full[s], kFp4TxBytes);
             if constexpr (kGrouped) {
               tma_load_3d(st, &maps.a, full_bar, ks * kStageBytesRow, a_row, t.expert);
-              tma_load_3d(st + kABytes, &maps.b, full_bar, ks * kStageBytesRow, b_row, t.expert);
+              tma_load_3d(st + kABytes, b_map, full_bar, ks * kStageBytesRow, b_row, t.expert);
               tma_load_3d(st + kABytes + kBBytes, &maps.sfa, full_bar, 0, sfa_row0 + 16 * ks, t.expert);
               tma_load_3d(st + kABytes + kBBytes + kSfaBytes, &maps.sfb, full_bar, 0, sfb_row0 + 16 * ks, t.expert);
-              tma_load_3d(st + kABytes + kBBytes + kSfaBytes + kSfaBytes, &maps.sfb, full_bar, 0, sfb_row1 + 16 * ks,
+              tma_load_3d(st + kABytes + kBBytes + kSfaBytes + kSfaBytes, sfb1_map, full_bar, 0, sfb_row1 + 16 * ks,
                           t.expert);
             } else {
               tma_load_2d(st, &maps.a, full_bar, ks * kStageBytesRow, a_row);
-              tma_load_2d(st + kABytes, &maps.b, full_bar, ks * kStageBytesRow, b_row);
+              tma_load_2d(st + kABytes, b_map, full_bar, ks * kStageBytesRow, b_row);
               tma_load_2d(st + kABytes + kBBytes, &maps.sfa, full_bar, 0, sfa_row0 + 16 * ks);
               tma_load_2d(st + kABytes + kBBytes + kSfaBytes, &maps.sfb, full_bar, 0, sfb_row0 + 16 * ks);
-              tma_load_2d(st + kABytes + kBBytes + kSfaBytes + kSfaBytes, &maps.sfb, full_bar, 0, sfb_row1 + 16 * ks);
+              tma_load_2d(st + kABytes + kBBytes + kSfaBytes + kSfaBytes, sfb1_map, full_bar, 0, sfb_row1 + 16 * ks);
             }
           } else if constexpr (kLowRank) {
             const int c = ks - p.k_stages;
@@ -473,6 +530,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------------ epilogue (both CTAs)
     const int quarter = warp & 3;              // TMEM lane quarter this warp may access
     const int row_in_tile = quarter * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t acc_empty_leader = map_to_rank(&ctl.acc_empty, 0);
     uint32_t tcount = 0;
     TileCoord t;
@@ -484,44 +542,93 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const float alpha = __ldg(p.alpha + t.expert);
       const int row = t.m_tile * kTileM + static_cast<int>(rank) * kBM + row_in_tile;
       const bool row_ok = row < t.valid_rows;
-      __nv_bfloat16* out_row = p.out + (static_cast<int64_t>(t.expert) * p.m + row) * p.n;
-      for (int i = 0; i < 4; ++i) {
-        // accumulator 0 drains its last 64 columns first, accumulator 1 its first 64
-        const int sub = buf ? i : 3 - i;
-        uint32_t v[64];
-        tmem_load_64(tmem + col0 + sub * 64 + (static_cast<uint32_t>(quarter * 32) << 16), v);
-        if (i == 0) {
+      if constexpr (kSwiGLU) {
+        // h columns [128 n_tile, 128 n_tile + 128): g in accumulator columns [0, 128), u in
+        // [128, 256); this warp's half of them is loaded whole, then the accumulator released.
+        const float gsf = __ldg(p.gsf_h + t.expert);
+        const float alpha_u = __ldg(p.alpha_up + t.expert);
+        const bool pad_row = !kGrouped && row >= p.m && row < p.rows_pad;   // zero scales
+        uint8_t* q_row = p.q + (static_cast<int64_t>(t.expert) * p.m + row) * (p.n / 2) + t.n_tile * 64;
+        uint8_t* sf_e = p.sf + static_cast<int64_t>(t.expert) * p.sf_item_stride;
+        const uint32_t groups = static_cast<uint32_t>(p.n / 64);
+        {
+          const int half = (warp - 2) >> 2;        // warps 2-5: columns [0, 64), warps 6-9: [64, 128)
+          uint32_t g[64], u[64];
+          tmem_load_64(tmem + col0 + half * 64 + lane_base, g);
+          tmem_load_64(tmem + col0 + 128 + half * 64 + lane_base, u);
+          tmem_wait_ld<64>(g);
+          tmem_wait_ld<64>(u);
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
-        }
-        const int col_base = t.n_tile * kBN + sub * 64;
-        if (row_ok) {
+          const uint32_t c0 = static_cast<uint32_t>(t.n_tile * 8 + half * 4);   // first block column
+          if (row_ok) {
+            uint32_t codes[8];
+            uint32_t scales = 0;
 #pragma unroll
-          for (int g = 0; g < 8; ++g) {
-            const int col = col_base + 8 * g;
-            if (col < p.n) {
-              float f[8];
+            for (int blk = 0; blk < 4; ++blk) {
+              float h[16];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * g + e]);
-              if (p.bias) {
-                const uint4 bw = __ldg(reinterpret_cast<const uint4*>(p.bias + col));
-                const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  f[2 * e] = __fmaf_rn(alpha, f[2 * e], __uint_as_float(bb[e] << 16));
-                  f[2 * e + 1] = __fmaf_rn(alpha, f[2 * e + 1], __uint_as_float(bb[e] & 0xffff0000u));
-                }
-              } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) f[e] = __fmul_rn(alpha, f[e]);
+              for (int e = 0; e < 16; e += 2) {
+                float g0, g1, u0, u1;
+                scale_round_bf16_2(alpha, g[16 * blk + e], g[16 * blk + e + 1], g0, g1);
+                scale_round_bf16_2(alpha_u, u[16 * blk + e], u[16 * blk + e + 1], u0, u1);
+                silu_mul_bf16_2(g0, g1, u0, u1, h[e], h[e + 1]);
               }
-              uint4 o;
-              o.x = pack_bf16x2(f[0], f[1]);
-              o.y = pack_bf16x2(f[2], f[3]);
-              o.z = pack_bf16x2(f[4], f[5]);
-              o.w = pack_bf16x2(f[6], f[7]);
-              *reinterpret_cast<uint4*>(out_row + col) = o;
+              const QBlock qb = quantize16(h, gsf);
+              codes[2 * blk] = qb.lo;
+              codes[2 * blk + 1] = qb.hi;
+              scales |= qb.s8 << (8 * blk);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(q_row + half * 32);
+            dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+            dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+            *reinterpret_cast<uint32_t*>(sf_e + sf_offset(static_cast<uint32_t>(row), c0, groups)) = scales;
+          } else if (pad_row) {
+            *reinterpret_cast<uint32_t*>(sf_e + sf_offset(static_cast<uint32_t>(row), c0, groups)) = 0u;
+          }
+        }
+      } else {
+        __nv_bfloat16* out_row = p.out + (static_cast<int64_t>(t.expert) * p.m + row) * p.n;
+        for (int i = 0; i < 4; ++i) {
+          // accumulator 0 drains its last 64 columns first, accumulator 1 its first 64
+          const int sub = buf ? i : 3 - i;
+          uint32_t v[64];
+          tmem_load_64(tmem + col0 + sub * 64 + lane_base, v);
+          tmem_wait_ld<64>(v);
+          if (i == 0) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
+          }
+          const int col_base = t.n_tile * kBN + sub * 64;
+          if (row_ok) {
+#pragma unroll
+            for (int g = 0; g < 8; ++g) {
+              const int col = col_base + 8 * g;
+              if (col < p.n) {
+                float f[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * g + e]);
+                if (p.bias) {
+                  const uint4 bw = __ldg(reinterpret_cast<const uint4*>(p.bias + col));
+                  const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w};
+#pragma unroll
+                  for (int e = 0; e < 4; ++e) {
+                    f[2 * e] = __fmaf_rn(alpha, f[2 * e], __uint_as_float(bb[e] << 16));
+                    f[2 * e + 1] = __fmaf_rn(alpha, f[2 * e + 1], __uint_as_float(bb[e] & 0xffff0000u));
+                  }
+                } else {
+#pragma unroll
+                  for (int e = 0; e < 8; ++e) f[e] = __fmul_rn(alpha, f[e]);
+                }
+                uint4 o;
+                o.x = pack_bf16x2(f[0], f[1]);
+                o.y = pack_bf16x2(f[2], f[3]);
+                o.z = pack_bf16x2(f[4], f[5]);
+                o.w = pack_bf16x2(f[6], f[7]);
+                *reinterpret_cast<uint4*>(out_row + col) = o;
+              }
             }
           }
         }
@@ -588,20 +695,42 @@ int make_lowrank_map(CUtensorMap* map, const void* base, int64_t rows, int64_t r
   return make_map(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-template <bool kGrouped, bool kLowRank>
-int launch_gemm(const uint8_t* a, const uint8_t* b, const uint8_t* a_sf, const uint8_t* b_sf, const float* alpha,
-                const void* d, const void* l1, int64_t r, const void* bias, const int32_t* mask, void* out,
-                int64_t E, int64_t m, int64_t n, int64_t k, cudaStream_t stream) {
+// Operands of one call; unused members are null / zero.
+struct GemmArgs {
+  const uint8_t *a = nullptr, *b = nullptr, *a_sf = nullptr, *b_sf = nullptr;
+  const float* alpha = nullptr;
+  const void *d = nullptr, *l1 = nullptr;  // low-rank
+  int64_t r = 0;
+  const void* bias = nullptr;
+  const int32_t* mask = nullptr;           // grouped
+  void* out = nullptr;                     // bf16 output
+  const uint8_t *b2 = nullptr, *b2_sf = nullptr;  // SiLU * up: up weight (b: gate weight)
+  const float *alpha2 = nullptr, *gsf_h = nullptr;
+  uint8_t *q = nullptr, *sf = nullptr;
+  int64_t E = 1, m = 0, n = 0, k = 0;      // n: output width (the width of h for SiLU * up)
+};
+
+template <bool kGrouped, bool kLowRank, bool kSwiGLU>
+int launch_gemm(const GemmArgs& g, cudaStream_t stream) {
+  const int64_t E = g.E, m = g.m, n = g.n, k = g.k;
   if (E < 0 || m < 0 || n < 0 || k <= 0 || k % 64 != 0 || n % 8 != 0) return NVFP4_ERR_INVALID_ARGUMENT;
-  if (m > (1 << 30) || n > (1 << 30) || k > (1 << 30) || E > kMaxExperts) return NVFP4_ERR_INVALID_ARGUMENT;
-  if (kLowRank && (r <= 0 || r % 32 != 0 || r > 256)) return NVFP4_ERR_INVALID_ARGUMENT;
+  if (kSwiGLU && n % 128 != 0) return NVFP4_ERR_INVALID_ARGUMENT;
+  if (m > (1 << 30) || n > (1 << 29) || k > (1 << 30) || E > kMaxExperts) return NVFP4_ERR_INVALID_ARGUMENT;
+  if (kLowRank && (g.r <= 0 || g.r % 32 != 0 || g.r > 256)) return NVFP4_ERR_INVALID_ARGUMENT;
   if (E == 0 || m == 0 || n == 0) return NVFP4_OK;
-  if (!a || !b || !a_sf || !b_sf || !alpha || !out) return NVFP4_ERR_INVALID_ARGUMENT;
-  if (!aligned(a, 16) || !aligned(b, 16) || !aligned(a_sf, 16) || !aligned(b_sf, 16) || !aligned(out, 16) ||
-      !aligned(alpha, 4) || (bias && !aligned(bias, 16)))
+  if (!g.a || !g.b || !g.a_sf || !g.b_sf || !g.alpha) return NVFP4_ERR_INVALID_ARGUMENT;
+  if (!aligned(g.a, 16) || !aligned(g.b, 16) || !aligned(g.a_sf, 16) || !aligned(g.b_sf, 16) || !aligned(g.alpha, 4))
     return NVFP4_ERR_INVALID_ARGUMENT;
-  if (kGrouped && (!mask || !aligned(mask, 4))) return NVFP4_ERR_INVALID_ARGUMENT;
-  if (kLowRank && (!d || !l1 || !aligned(d, 16) || !aligned(l1, 16))) return NVFP4_ERR_INVALID_ARGUMENT;
+  if (kSwiGLU) {
+    if (!g.b2 || !g.b2_sf || !g.alpha2 || !g.q || !g.sf || !g.gsf_h) return NVFP4_ERR_INVALID_ARGUMENT;
+    if (!aligned(g.b2, 16) || !aligned(g.b2_sf, 16) || !aligned(g.alpha2, 4) || !aligned(g.q, 16) ||
+        !aligned(g.sf, 16) || !aligned(g.gsf_h, 4))
+      return NVFP4_ERR_INVALID_ARGUMENT;
+  } else {
+    if (!g.out || !aligned(g.out, 16) || (g.bias && !aligned(g.bias, 16))) return NVFP4_ERR_INVALID_ARGUMENT;
+  }
+  if (kGrouped && (!g.mask || !aligned(g.mask, 4))) return NVFP4_ERR_INVALID_ARGUMENT;
+  if (kLowRank && (!g.d || !g.l1 || !aligned(g.d, 16) || !aligned(g.l1, 16))) return NVFP4_ERR_INVALID_ARGUMENT;
 
   DeviceInfo info;
   int st = current_device(&info);
@@ -609,33 +738,46 @@ int launch_gemm(const uint8_t* a, const uint8_t* b, const uint8_t* a_sf, const u
 
   Maps maps;
   memset(&maps, 0, sizeof(maps));
-  if ((st = make_operand_map(&maps.a, a, E, m, k, kGrouped)) != NVFP4_OK) return st;
-  if ((st = make_operand_map(&maps.b, b, E, n, k, kGrouped)) != NVFP4_OK) return st;
-  if ((st = make_scale_map(&maps.sfa, a_sf, E, m, k, kGrouped)) != NVFP4_OK) return st;
-  if ((st = make_scale_map(&maps.sfb, b_sf, E, n, k, kGrouped)) != NVFP4_OK) return st;
+  if ((st = make_operand_map(&maps.a, g.a, E, m, k, kGrouped)) != NVFP4_OK) return st;
+  if ((st = make_operand_map(&maps.b, g.b, E, n, k, kGrouped)) != NVFP4_OK) return st;
+  if ((st = make_scale_map(&maps.sfa, g.a_sf, E, m, k, kGrouped)) != NVFP4_OK) return st;
+  if ((st = make_scale_map(&maps.sfb, g.b_sf, E, n, k, kGrouped)) != NVFP4_OK) return st;
+  if (kSwiGLU) {
+    if ((st = make_operand_map(&maps.b2, g.b2, E, n, k, kGrouped)) != NVFP4_OK) return st;
+    if ((st = make_scale_map(&maps.sfb2, g.b2_sf, E, n, k, kGrouped)) != NVFP4_OK) return st;
+  }
   if (kLowRank) {
-    if ((st = make_lowrank_map(&maps.d, d, m, r)) != NVFP4_OK) return st;
-    if ((st = make_lowrank_map(&maps.l1, l1, n, r)) != NVFP4_OK) return st;
+    if ((st = make_lowrank_map(&maps.d, g.d, m, g.r)) != NVFP4_OK) return st;
+    if ((st = make_lowrank_map(&maps.l1, g.l1, n, g.r)) != NVFP4_OK) return st;
   }
 
   GemmParams p;
-  p.alpha = alpha;
-  p.bias = static_cast<const __nv_bfloat16*>(bias);
-  p.out = static_cast<__nv_bfloat16*>(out);
-  p.mask = mask;
+  memset(&p, 0, sizeof(p));
+  p.alpha = g.alpha;
+  p.bias = static_cast<const __nv_bfloat16*>(g.bias);
+  p.out = static_cast<__nv_bfloat16*>(g.out);
+  p.mask = g.mask;
   p.status = info.status;
   p.m = static_cast<int32_t>(m);
   p.n = static_cast<int32_t>(n);
   p.k = static_cast<int32_t>(k);
   p.experts = static_cast<int32_t>(E);
-  p.rank = static_cast<int32_t>(r);
-  p.n_tiles = static_cast<int32_t>((n + kBN - 1) / kBN);
+  p.rank = static_cast<int32_t>(g.r);
+  p.n_tiles = static_cast<int32_t>(kSwiGLU ? n / kBNHalf : (n + kBN - 1) / kBN);
   p.m_tiles = static_cast<int32_t>((m + kTileM - 1) / kTileM);
   p.k_stages = static_cast<int32_t>((k + kStageK - 1) / kStageK);
   p.k_steps = static_cast<int32_t>(k / 64);
   p.sf_groups = static_cast<int32_t>(k / 64);
+  if (kSwiGLU) {
+    p.alpha_up = g.alpha2;
+    p.gsf_h = g.gsf_h;
+    p.q = g.q;
+    p.sf = g.sf;
+    p.sf_item_stride = nvfp4_scale_bytes(m, n);
+    p.rows_pad = static_cast<int32_t>((m + 127) / 128 * 128);
+  }
 
-  auto kernel = nvfp4_gemm_kernel<kGrouped, kLowRank>;
+  auto kernel = nvfp4_gemm_kernel<kGrouped, kLowRank, kSwiGLU>;
   // One-time set-up per kernel instantiation: the dynamic shared memory opt-in and the
   // number of 2-CTA clusters that fit on the device at once (the persistent grid size).
   static int max_clusters = 0;
@@ -646,7 +788,7 @@ int launch_gemm(const uint8_t* a, const uint8_t* b, const uint8_t* a_sf, const u
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(info.sm_count / 2 * 2);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(kThreads<kSwiGLU>);
     cfg.dynamicSmemBytes = kSmemBytes;
     int clusters = 0;
     if (cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg) != cudaSuccess || clusters <= 0) {
@@ -660,7 +802,7 @@ int launch_gemm(const uint8_t* a, const uint8_t* b, const uint8_t* a_sf, const u
   if (tiles >= (int64_t(1) << 31)) return NVFP4_ERR_INVALID_ARGUMENT;
   const int64_t max_pairs = max_clusters;
   const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
-  kernel<<<2 * pairs, kThreads, kSmemBytes, stream>>>(maps, p);
+  kernel<<<2 * pairs, kThreads<kSwiGLU>, kSmemBytes, stream>>>(maps, p);
   return launch_status();
 }
 
@@ -673,23 +815,54 @@ extern "C" {
 
 int nvfp4_gemm(const uint8_t* a, const uint8_t* b, const uint8_t* a_sf, const uint8_t* b_sf, const float* alpha,
                const void* bias_bf16, void* out_bf16, int64_t m, int64_t n, int64_t k, nvfp4_stream_t stream) {
-  return launch_gemm<false, false>(a, b, a_sf, b_sf, alpha, nullptr, nullptr, 0, bias_bf16, nullptr, out_bf16, 1, m,
-                                   n, k, stream);
+  GemmArgs g;
+  g.a = a; g.b = b; g.a_sf = a_sf; g.b_sf = b_sf; g.alpha = alpha; g.bias = bias_bf16; g.out = out_bf16;
+  g.m = m; g.n = n; g.k = k;
+  return launch_gemm<false, false, false>(g, stream);
 }
 
 int nvfp4_grouped_gemm_masked(const uint8_t* a, const uint8_t* b, const uint8_t* a_sf, const uint8_t* b_sf,
                               const int32_t* mask, const float* alpha, void* out_bf16, int64_t E, int64_t mmax,
                               int64_t n, int64_t k, nvfp4_stream_t stream) {
-  return launch_gemm<true, false>(a, b, a_sf, b_sf, alpha, nullptr, nullptr, 0, nullptr, mask, out_bf16, E, mmax, n,
-                                  k, stream);
+  GemmArgs g;
+  g.a = a; g.b = b; g.a_sf = a_sf; g.b_sf = b_sf; g.alpha = alpha; g.mask = mask; g.out = out_bf16;
+  g.E = E; g.m = mmax; g.n = n; g.k = k;
+  return launch_gemm<true, false, false>(g, stream);
 }
 
 int nvfp4_gemm_lowrank_bias(const uint8_t* a, const uint8_t* b, const uint8_t* a_sf, const uint8_t* b_sf,
                             const float* alpha, const void* d_bf16, const void* l1_bf16, int64_t r,
                             const void* bias_bf16, void* out_bf16, int64_t m, int64_t n, int64_t k,
                             nvfp4_stream_t stream) {
-  return launch_gemm<false, true>(a, b, a_sf, b_sf, alpha, d_bf16, l1_bf16, r, bias_bf16, nullptr, out_bf16, 1, m, n,
-                                  k, stream);
+  GemmArgs g;
+  g.a = a; g.b = b; g.a_sf = a_sf; g.b_sf = b_sf; g.alpha = alpha; g.d = d_bf16; g.l1 = l1_bf16; g.r = r;
+  g.bias = bias_bf16; g.out = out_bf16;
+  g.m = m; g.n = n; g.k = k;
+  return launch_gemm<false, true, false>(g, stream);
+}
+
+int nvfp4_gemm_silu_mul_quantize(const uint8_t* a, const uint8_t* b_gate, const uint8_t* b_up, const uint8_t* a_sf,
+                                 const uint8_t* b_gate_sf, const uint8_t* b_up_sf, const float* alpha_gate,
+                                 const float* alpha_up, const float* gsf_h, uint8_t* q_out, uint8_t* sf_out,
+                                 int64_t m, int64_t n, int64_t k, nvfp4_stream_t stream) {
+  GemmArgs g;
+  g.a = a; g.b = b_gate; g.b2 = b_up; g.a_sf = a_sf; g.b_sf = b_gate_sf; g.b2_sf = b_up_sf;
+  g.alpha = alpha_gate; g.alpha2 = alpha_up; g.gsf_h = gsf_h; g.q = q_out; g.sf = sf_out;
+  g.m = m; g.n = n; g.k = k;
+  return launch_gemm<false, false, true>(g, stream);
+}
+
+int nvfp4_grouped_gemm_silu_mul_quantize_masked(const uint8_t* a, const uint8_t* b_gate, const uint8_t* b_up,
+                                                const uint8_t* a_sf, const uint8_t* b_gate_sf,
+                                                const uint8_t* b_up_sf, const int32_t* mask,
+                                                const float* alpha_gate, const float* alpha_up,
+                                                const float* gsf_h, uint8_t* q_out, uint8_t* sf_out, int64_t E,
+                                                int64_t mmax, int64_t n, int64_t k, nvfp4_stream_t stream) {
+  GemmArgs g;
+  g.a = a; g.b = b_gate; g.b2 = b_up; g.a_sf = a_sf; g.b_sf = b_gate_sf; g.b2_sf = b_up_sf; g.mask = mask;
+  g.alpha = alpha_gate; g.alpha2 = alpha_up; g.gsf_h = gsf_h; g.q = q_out; g.sf = sf_out;
+  g.E = E; g.m = mmax; g.n = n; g.k = k;
+  return launch_gemm<true, false, true>(g, stream);
 }
 
 }  // extern "C"

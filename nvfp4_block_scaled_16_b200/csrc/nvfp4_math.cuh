@@ -1,0 +1,195 @@
+// nvfp4_math.cuh -- device arithmetic of NVFP4 quantization shared by the quantizers and
+// the GEMM epilogue that quantizes SiLU(gate) * up: e4m3 / e2m1 conversions, the specified
+// fp32 exponential, h = bf16(silu(g) * u), and one 16-element block (scale + codes).
+//
+// Sources (page title, section): TensorRT-LLM NVFP4LinearMethod.create_weights (block size
+// 16, ue4m3 block scales, global scale 448*6/amax); flashinfer PR #1774 "Masked batch nvfp4
+// quantization" (silu_and_mul fused variant); flashinfer docs mm_nvfp4_svdquant,
+// Parameters a / a_sf (packed e2m1, 128x4-swizzled ue4m3 scales).
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+namespace nvfp4 {
+namespace {
+
+// ---- bf16 / fp8 / fp4 conversions ------------------------------------------------------
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// ue4m3 code of s >= 0: round to nearest even, saturate to 448.  Both halves of the
+// packed pair convert the same value, so the pair order does not matter.
+__device__ __forceinline__ uint32_t ue4m3_encode(float s) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %1;" : "=h"(r) : "f"(s));
+  return r & 0xffu;
+}
+
+// Exact value of an e4m3 code (through f16, which holds every e4m3 value).
+__device__ __forceinline__ float e4m3_decode(uint32_t code) {
+  const uint16_t pair = static_cast<uint16_t>(code | (code << 8));
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(pair));
+  return __half2float(__ushort_as_half(static_cast<uint16_t>(h2 & 0xffffu)));
+}
+
+// Eight e2m1 codes, round to nearest even, saturate to +-6; element 2i goes to the low
+// nibble of byte i (the cvt's second source is its low nibble).
+__device__ __forceinline__ uint32_t e2m1x8(const float* t) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(r)
+      : "f"(t[0]), "f"(t[1]), "f"(t[2]), "f"(t[3]), "f"(t[4]), "f"(t[5]), "f"(t[6]), "f"(t[7]));
+  return r;
+}
+
+// ---- the specified fp32 exponential used by SiLU -----------------------------------------
+// x = n*ln2 + r (Cody-Waite, ln2 split into a 16-significant-bit head and an fp32 tail),
+// e^r by the degree-7 Taylor polynomial in Horner form with fused multiply-adds, then an
+// exact multiplication by 2^n (two steps when 2^n is not a normal fp32).  Every step is a
+// single correctly rounded operation, so the result is reproducible bit for bit.
+
+__device__ __forceinline__ float pow2_int(int n) { return __uint_as_float(static_cast<uint32_t>(n + 127) << 23); }
+
+__device__ __forceinline__ float exp_specified(float x) {
+  if (x != x) return x;
+  if (x > 89.0f) return __uint_as_float(0x7f800000u);
+  if (x < -104.0f) return 0.0f;
+  const float n = rintf(__fmul_rn(x, 0x1.715476p+0f));
+  float r = __fmaf_rn(n, -0x1.62e4p-1f, x);
+  r = __fmaf_rn(n, -0x1.7f7d1cp-20f, r);
+  float p = 0x1.a01a02p-13f;
+  p = __fmaf_rn(p, r, 0x1.6c16c2p-10f);
+  p = __fmaf_rn(p, r, 0x1.111112p-7f);
+  p = __fmaf_rn(p, r, 0x1.555556p-5f);
+  p = __fmaf_rn(p, r, 0x1.555556p-3f);
+  p = __fmaf_rn(p, r, 0x1.0p-1f);
+  p = __fmaf_rn(p, r, 1.0f);
+  p = __fmaf_rn(p, r, 1.0f);
+  const int ni = static_cast<int>(n);
+  if (ni > 127) return __fmul_rn(__fmul_rn(p, pow2_int(127)), pow2_int(ni - 127));
+  if (ni < -126) return __fmul_rn(__fmul_rn(p, pow2_int(-126)), pow2_int(ni + 126));
+  return __fmul_rn(p, pow2_int(ni));
+}
+
+// h = bf16(silu(g) * u), returned as the fp32 value of that bf16.
+__device__ __forceinline__ float silu_mul_bf16(float g, float u) {
+  const float e = exp_specified(-g);
+  const float den = __fadd_rn(1.0f, e);
+  const float s = __fdiv_rn(g, den);
+  const float p = __fmul_rn(s, u);
+  return __bfloat162float(__float2bfloat16_rn(p));
+}
+
+// ---- the same arithmetic on pairs of values with packed f32x2 instructions -----------------
+// Each lane of fma/mul/add.rn.f32x2 is one correctly rounded fp32 operation, so the pair
+// functions return exactly what the scalar ones return.
+
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unpack2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t splat2(float v) { return pack2(v, v); }
+
+// exp_specified of a pair.  The input is clamped to [-104, 89], which leaves every result
+// unchanged (e^x overflows to +inf for x > 88.73 and rounds to 0 for x <= -104), and 2^n
+// is applied as two exact power-of-two multiplications 2^(n/2) * 2^(n - n/2): both halves
+// are normal numbers for n in [-150, 128], so only the last multiplication can round --
+// the same single rounding as the three-way scaling of exp_specified.  NaN stays NaN.
+__device__ __forceinline__ void exp_specified2(float x0, float x1, float& e0, float& e1) {
+  const float c0 = fmaxf(fminf(x0, 89.0f), -104.0f);
+  const float c1 = fmaxf(fminf(x1, 89.0f), -104.0f);
+  const uint64_t x = pack2(c0, c1);
+  float t0, t1;
+  unpack2(mul2(x, splat2(0x1.715476p+0f)), t0, t1);
+  const float n0 = rintf(t0), n1 = rintf(t1);
+  const uint64_t n = pack2(n0, n1);
+  uint64_t r = fma2(n, splat2(-0x1.62e4p-1f), x);
+  r = fma2(n, splat2(-0x1.7f7d1cp-20f), r);
+  uint64_t p = splat2(0x1.a01a02p-13f);
+  p = fma2(p, r, splat2(0x1.6c16c2p-10f));
+  p = fma2(p, r, splat2(0x1.111112p-7f));
+  p = fma2(p, r, splat2(0x1.555556p-5f));
+  p = fma2(p, r, splat2(0x1.555556p-3f));
+  p = fma2(p, r, splat2(0x1.0p-1f));
+  p = fma2(p, r, splat2(1.0f));
+  p = fma2(p, r, splat2(1.0f));
+  const int i0 = static_cast<int>(n0), i1 = static_cast<int>(n1);
+  const int h0 = i0 / 2, h1 = i1 / 2;
+  p = mul2(p, pack2(pow2_int(h0), pow2_int(h1)));
+  p = mul2(p, pack2(pow2_int(i0 - h0), pow2_int(i1 - h1)));
+  unpack2(p, e0, e1);
+  if (x0 != x0) e0 = x0;
+  if (x1 != x1) e1 = x1;
+}
+
+// silu_mul_bf16 of a pair: h = bf16((g / (1 + exp(-g))) * u), as fp32 values.
+__device__ __forceinline__ void silu_mul_bf16_2(float g0, float g1, float u0, float u1, float& h0, float& h1) {
+  float e0, e1;
+  exp_specified2(-g0, -g1, e0, e1);
+  const float s0 = __fdiv_rn(g0, __fadd_rn(1.0f, e0));
+  const float s1 = __fdiv_rn(g1, __fadd_rn(1.0f, e1));
+  float p0, p1;
+  unpack2(mul2(pack2(s0, s1), pack2(u0, u1)), p0, p1);
+  uint32_t b2;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(b2) : "f"(p1), "f"(p0));   // p0 -> low half
+  h0 = __uint_as_float(b2 << 16);
+  h1 = __uint_as_float(b2 & 0xffff0000u);
+}
+
+// ---- one 16-element block ------------------------------------------------------------------
+
+struct QBlock {
+  uint32_t lo, hi;  // 16 packed e2m1 codes
+  uint32_t s8;      // ue4m3 scale code
+};
+
+__device__ __forceinline__ QBlock quantize16(const float* v, float gsf) {
+  float vmax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) vmax = fmaxf(vmax, fabsf(v[i]));
+  const float s32 = __fmul_rn(__fdiv_rn(vmax, 6.0f), gsf);
+  QBlock b;
+  b.s8 = ue4m3_encode(s32);
+  const float sd = e4m3_decode(b.s8);
+  const float inv = sd == 0.0f ? 0.0f : __fdiv_rn(gsf, sd);
+  const uint64_t inv2 = pack2(inv, inv);
+  float t[16];
+#pragma unroll
+  for (int i = 0; i < 16; i += 2) unpack2(mul2(pack2(v[i], v[i + 1]), inv2), t[i], t[i + 1]);
+  b.lo = e2m1x8(t);
+  b.hi = e2m1x8(t + 8);
+  return b;
+}
+
+// Byte offset of the scale of (row r, block c) in the 128x4 swizzled layout;
+// groups = pad_up(k/16, 4) / 4.
+__device__ __forceinline__ int64_t sf_offset(uint32_t r, uint32_t c, uint32_t groups) {
+  const int64_t chunk = static_cast<int64_t>(r >> 7) * groups + (c >> 2);
+  return chunk * 512 + (r & 31u) * 16 + ((r >> 5) & 3u) * 4 + (c & 3u);
+}
+
+}  // namespace
+}  // namespace nvfp4

@@ -57,6 +57,14 @@ def lib():
                                             _u16p, _i64, _i64p, _i64p, _i64, _f64p]),
             "nvo_grouped_gemm_ref": (None, [_u8p, _u8p, _u8p, _u8p, _i32p, _f32p, _i64, _i64, _i64, _i64,
                                             _f64p]),
+            "nvo_f64_to_bf16": (ctypes.c_uint16, [ctypes.c_double]),
+            "nvo_gemm_silu_mul_quantize": (None, [_u8p] * 6 + [ctypes.c_float] * 3 + [_i64, _i64, _i64,
+                                                                                      _u8p, _u8p]),
+            "nvo_grouped_gemm_silu_mul_quantize": (None, [_u8p] * 6 + [_i32p, _f32p, _f32p, _f32p, _i64, _i64,
+                                                                       _i64, _i64, _u8p, _u8p]),
+            "nvo_gemm_gate_up_bf16": (None, [_u8p] * 6 + [ctypes.c_float] * 2 + [_i64, _i64, _i64p, _i64, _u16p]),
+            "nvo_gemm_silu_mul_quantize_rows": (None, [_u8p] * 6 + [ctypes.c_float] * 3 + [_i64, _i64, _i64p,
+                                                                                           _i64, _u8p, _u8p]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -246,3 +254,70 @@ def grouped_gemm_ref(a, b, a_sf, b_sf, mask, alphas, E, mmax, n, k):
     lib().nvo_grouped_gemm_ref(_p(a, _u8p), _p(b, _u8p), _p(a_sf, _u8p), _p(b_sf, _u8p), _p(mk, _i32p),
                                _p(al, _f32p), E, mmax, n, k, _p(out, _f64p))
     return out
+
+
+def f64_to_bf16(v: float) -> int:
+    """bf16 bits nearest to the double v (ties to even)."""
+    return int(lib().nvo_f64_to_bf16(float(v)))
+
+
+def _u8(*arrs):
+    return [np.ascontiguousarray(x, np.uint8) for x in arrs]
+
+
+def gemm_silu_mul_quantize(a, b_gate, b_up, a_sf, b_gate_sf, b_up_sf, alpha_gate, alpha_up, gsf_h, m, n, k,
+                           sf_fill=0):
+    """Gate/up projections, h = bf16(silu(g) * u), NVFP4 quantization of h with gsf_h.
+
+    Returns (q [m, n/2] uint8, sf [scale_bytes(m, n)] uint8)."""
+    a, b_gate, b_up, a_sf, b_gate_sf, b_up_sf = _u8(a, b_gate, b_up, a_sf, b_gate_sf, b_up_sf)
+    q = np.zeros((m, n // 2), np.uint8)
+    sf = np.full(scale_bytes(m, n), sf_fill, np.uint8)
+    lib().nvo_gemm_silu_mul_quantize(_p(a, _u8p), _p(b_gate, _u8p), _p(b_up, _u8p), _p(a_sf, _u8p),
+                                     _p(b_gate_sf, _u8p), _p(b_up_sf, _u8p), float(np.float32(alpha_gate)),
+                                     float(np.float32(alpha_up)), float(np.float32(gsf_h)), m, n, k,
+                                     _p(q, _u8p), _p(sf, _u8p))
+    return q, sf
+
+
+def grouped_gemm_silu_mul_quantize(a, b_gate, b_up, a_sf, b_gate_sf, b_up_sf, mask, alpha_gate, alpha_up, gsf_h,
+                                   E, mmax, n, k, q_fill=0, sf_fill=0):
+    """Masked grouped form; rows >= mask[e] keep q_fill / sf_fill.
+
+    Returns (q [E, mmax, n/2], sf [E, scale_bytes(mmax, n)])."""
+    a, b_gate, b_up, a_sf, b_gate_sf, b_up_sf = _u8(a, b_gate, b_up, a_sf, b_gate_sf, b_up_sf)
+    mk = np.ascontiguousarray(mask, np.int32)
+    ag, au, g = (np.ascontiguousarray(v, np.float32).reshape(E) for v in (alpha_gate, alpha_up, gsf_h))
+    q = np.full((E, mmax, n // 2), q_fill, np.uint8)
+    sf = np.full((E, scale_bytes(mmax, n)), sf_fill, np.uint8)
+    lib().nvo_grouped_gemm_silu_mul_quantize(_p(a, _u8p), _p(b_gate, _u8p), _p(b_up, _u8p), _p(a_sf, _u8p),
+                                             _p(b_gate_sf, _u8p), _p(b_up_sf, _u8p), _p(mk, _i32p),
+                                             _p(ag, _f32p), _p(au, _f32p), _p(g, _f32p), E, mmax, n, k,
+                                             _p(q, _u8p), _p(sf, _u8p))
+    return q, sf
+
+
+def gemm_silu_mul_quantize_rows(a, b_gate, b_up, a_sf, b_gate_sf, b_up_sf, alpha_gate, alpha_up, gsf_h, n, k,
+                                rows):
+    """The dense result at the listed rows only: (q_rows [len, n/2], scale codes [len, n/16] in
+    logical order)."""
+    a, b_gate, b_up, a_sf, b_gate_sf, b_up_sf = _u8(a, b_gate, b_up, a_sf, b_gate_sf, b_up_sf)
+    ii = np.ascontiguousarray(rows, np.int64)
+    q = np.zeros((len(ii), n // 2), np.uint8)
+    s = np.zeros((len(ii), n // 16), np.uint8)
+    lib().nvo_gemm_silu_mul_quantize_rows(_p(a, _u8p), _p(b_gate, _u8p), _p(b_up, _u8p), _p(a_sf, _u8p),
+                                          _p(b_gate_sf, _u8p), _p(b_up_sf, _u8p), float(np.float32(alpha_gate)),
+                                          float(np.float32(alpha_up)), float(np.float32(gsf_h)), n, k,
+                                          _p(ii, _i64p), len(ii), _p(q, _u8p), _p(s, _u8p))
+    return q, s
+
+
+def gemm_gate_up_bf16(a, b_gate, b_up, a_sf, b_gate_sf, b_up_sf, alpha_gate, alpha_up, n, k, rows):
+    """[g | u] = [bf16(alpha_gate A.Bg^T) | bf16(alpha_up A.Bu^T)] at the listed rows -> uint16 [len, 2n]."""
+    a, b_gate, b_up, a_sf, b_gate_sf, b_up_sf = _u8(a, b_gate, b_up, a_sf, b_gate_sf, b_up_sf)
+    ii = np.ascontiguousarray(rows, np.int64)
+    x = np.zeros((len(ii), 2 * n), np.uint16)
+    lib().nvo_gemm_gate_up_bf16(_p(a, _u8p), _p(b_gate, _u8p), _p(b_up, _u8p), _p(a_sf, _u8p),
+                                _p(b_gate_sf, _u8p), _p(b_up_sf, _u8p), float(np.float32(alpha_gate)),
+                                float(np.float32(alpha_up)), n, k, _p(ii, _i64p), len(ii), _p(x, _u16p))
+    return x

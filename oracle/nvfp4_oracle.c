@@ -37,6 +37,7 @@
 #include <float.h>
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #ifdef _OPENMP
@@ -480,4 +481,111 @@ NVO_API void nvo_grouped_gemm_ref(const uint8_t *a, const uint8_t *b, const uint
                 out[(e * mmax + i) * n + j] =
                     ref_element(ae, be, ase, bse, (double)alpha[e], NULL, NULL, 0, NULL, i, j, k);
     }
+}
+
+/* ------------------------------------------------------------------------------- */
+/* SwiGLU first half: gate/up projections, then SiLU-and-mul quantization           */
+/* [NVF] NVIDIA/Fuser PR #5737, module tree: NVFP4InferenceSwiGLU (gate_proj,       */
+/* up_proj, down_proj) and its grouped form for the routed experts; [FI3] the        */
+/* silu_and_mul quantizer that consumes [gate | up].                                 */
+/*   g = bf16(alpha_gate * A.Bg^T),  u = bf16(alpha_up * A.Bu^T)                     */
+/*   (q, sf) = nvo_silu_mul_quantize_batched([g | u], gsf_h)                         */
+/* The projections are the fp64 GEMM reference rounded once to bf16.                 */
+/* ------------------------------------------------------------------------------- */
+
+/* bf16 nearest to the double v, ties to even: 8 significant bits, fp32's exponent
+ * range (subnormal spacing 2^-133), overflow to infinity. */
+static uint16_t f64_to_bf16_rne(double v) {
+    if (isnan(v)) return 0x7FC0;
+    uint16_t sign = signbit(v) ? 0x8000 : 0;
+    double a = fabs(v);
+    if (a == 0.0) return sign;
+    int e;
+    frexp(a, &e);                           /* 2^(e-1) <= a < 2^e */
+    int q = e - 8;                          /* spacing of 8 significant bits */
+    if (q < -133) q = -133;
+    double r = ldexp(nearbyint(ldexp(a, -q)), q);   /* default mode: ties to even */
+    if (r > 0x1.FEp127) return sign | 0x7F80;
+    float f = (float)r;                     /* exact */
+    uint32_t bits;
+    memcpy(&bits, &f, 4);
+    return sign | (uint16_t)(bits >> 16);
+}
+
+NVO_API uint16_t nvo_f64_to_bf16(double v) { return f64_to_bf16_rne(v); }
+
+/* [g | u] rows (bf16 bits, [rows, 2n]) for rows ii[0..count) of A. */
+static void gate_up_rows(const uint8_t *a, const uint8_t *b_gate, const uint8_t *b_up, const uint8_t *a_sf,
+                         const uint8_t *b_gate_sf, const uint8_t *b_up_sf, float alpha_gate, float alpha_up,
+                         int64_t n, int64_t k, const int64_t *ii, int64_t count, uint16_t *x) {
+    #pragma omp parallel for schedule(dynamic, 1) num_threads(g_threads)
+    for (int64_t s = 0; s < count; ++s)
+        for (int64_t j = 0; j < n; ++j) {
+            double g = ref_element(a, b_gate, a_sf, b_gate_sf, (double)alpha_gate, NULL, NULL, 0, NULL, ii[s], j, k);
+            double u = ref_element(a, b_up, a_sf, b_up_sf, (double)alpha_up, NULL, NULL, 0, NULL, ii[s], j, k);
+            x[s * 2 * n + j] = f64_to_bf16_rne(g);
+            x[s * 2 * n + n + j] = f64_to_bf16_rne(u);
+        }
+}
+
+/* The bf16 [g | u] rows ii[0..count) -> x [count, 2n] (e.g. to calibrate gsf_h). */
+NVO_API void nvo_gemm_gate_up_bf16(const uint8_t *a, const uint8_t *b_gate, const uint8_t *b_up,
+                                   const uint8_t *a_sf, const uint8_t *b_gate_sf, const uint8_t *b_up_sf,
+                                   float alpha_gate, float alpha_up, int64_t n, int64_t k, const int64_t *ii,
+                                   int64_t count, uint16_t *x) {
+    gate_up_rows(a, b_gate, b_up, a_sf, b_gate_sf, b_up_sf, alpha_gate, alpha_up, n, k, ii, count, x);
+}
+
+/* Dense: a [m, k/2], b_gate / b_up [n, k/2] -> q [m, n/2], sf [scale_bytes(m, n)]. */
+NVO_API void nvo_gemm_silu_mul_quantize(const uint8_t *a, const uint8_t *b_gate, const uint8_t *b_up,
+                                        const uint8_t *a_sf, const uint8_t *b_gate_sf, const uint8_t *b_up_sf,
+                                        float alpha_gate, float alpha_up, float gsf_h, int64_t m, int64_t n,
+                                        int64_t k, uint8_t *q, uint8_t *sf) {
+    uint16_t *x = (uint16_t *)malloc((size_t)(m > 0 ? m : 1) * 2 * n * sizeof(uint16_t));
+    int64_t *ii = (int64_t *)malloc((size_t)(m > 0 ? m : 1) * sizeof(int64_t));
+    for (int64_t i = 0; i < m; ++i) ii[i] = i;
+    gate_up_rows(a, b_gate, b_up, a_sf, b_gate_sf, b_up_sf, alpha_gate, alpha_up, n, k, ii, m, x);
+    nvo_silu_mul_quantize_batched(x, 1, m, n, NULL, &gsf_h, q, sf);
+    free(ii);
+    free(x);
+}
+
+/* Masked grouped: per expert e, rows i < mask[e] only (other rows and their scale
+ * entries untouched), with alpha_gate[e], alpha_up[e], gsf_h[e]. */
+NVO_API void nvo_grouped_gemm_silu_mul_quantize(const uint8_t *a, const uint8_t *b_gate, const uint8_t *b_up,
+                                                const uint8_t *a_sf, const uint8_t *b_gate_sf,
+                                                const uint8_t *b_up_sf, const int32_t *mask,
+                                                const float *alpha_gate, const float *alpha_up,
+                                                const float *gsf_h, int64_t E, int64_t mmax, int64_t n,
+                                                int64_t k, uint8_t *q, uint8_t *sf) {
+    int64_t sba = nvo_scale_bytes(mmax, k), sbb = nvo_scale_bytes(n, k), sbh = nvo_scale_bytes(mmax, n);
+    uint16_t *x = (uint16_t *)calloc((size_t)(mmax > 0 ? mmax : 1) * 2 * n, sizeof(uint16_t));
+    int64_t *ii = (int64_t *)malloc((size_t)(mmax > 0 ? mmax : 1) * sizeof(int64_t));
+    for (int64_t i = 0; i < mmax; ++i) ii[i] = i;
+    for (int64_t e = 0; e < E; ++e) {
+        int64_t valid = mask[e] < 0 ? 0 : (mask[e] > mmax ? mmax : mask[e]);
+        gate_up_rows(a + e * mmax * (k / 2), b_gate + e * n * (k / 2), b_up + e * n * (k / 2), a_sf + e * sba,
+                     b_gate_sf + e * sbb, b_up_sf + e * sbb, alpha_gate[e], alpha_up[e], n, k, ii, valid, x);
+        nvo_silu_mul_quantize_batched(x, 1, mmax, n, mask + e, gsf_h + e, q + e * mmax * (n / 2), sf + e * sbh);
+    }
+    free(ii);
+    free(x);
+}
+
+/* Rows ii[0..count) of the dense result, each quantized on its own: q_rows [count, n/2]
+ * and the row's scale codes in logical order, s_rows [count, n/16]. */
+NVO_API void nvo_gemm_silu_mul_quantize_rows(const uint8_t *a, const uint8_t *b_gate, const uint8_t *b_up,
+                                             const uint8_t *a_sf, const uint8_t *b_gate_sf,
+                                             const uint8_t *b_up_sf, float alpha_gate, float alpha_up,
+                                             float gsf_h, int64_t n, int64_t k, const int64_t *ii,
+                                             int64_t count, uint8_t *q_rows, uint8_t *s_rows) {
+    uint16_t *x = (uint16_t *)malloc((size_t)(count > 0 ? count : 1) * 2 * n * sizeof(uint16_t));
+    uint8_t *sf1 = (uint8_t *)malloc((size_t)nvo_scale_bytes(1, n));
+    gate_up_rows(a, b_gate, b_up, a_sf, b_gate_sf, b_up_sf, alpha_gate, alpha_up, n, k, ii, count, x);
+    for (int64_t s = 0; s < count; ++s) {
+        nvo_silu_mul_quantize_batched(x + s * 2 * n, 1, 1, n, NULL, &gsf_h, q_rows + s * (n / 2), sf1);
+        for (int64_t c = 0; c < n / 16; ++c) s_rows[s * (n / 16) + c] = sf1[nvo_sf_offset(0, c, n)];
+    }
+    free(sf1);
+    free(x);
 }

@@ -114,3 +114,28 @@ def test_valid_call_without_gpu_fails_loudly(lib):
     # valid arguments reach the device query, which must report an error (no fallback)
     st = lib.nvfp4_quantize(A16, 4, 32, A16, A16, A16, None)
     assert st != 0
+
+
+@pytest.mark.parametrize("n", [0 + 64, 200, 136])
+def test_silu_mul_gemm_rejects_width_not_multiple_of_128(lib, n):
+    args = [A16] * 11
+    assert lib.nvfp4_gemm_silu_mul_quantize(*args, 256, n, 256, None) == INVALID
+
+
+def test_silu_mul_gemm_rejects_null_and_misaligned(lib):
+    for i in range(11):                     # every pointer argument is required
+        args = [A16] * 11
+        args[i] = None
+        assert lib.nvfp4_gemm_silu_mul_quantize(*args, 256, 256, 256, None) == INVALID, i
+    args = [A16] * 11
+    args[2] = A1                            # b_up misaligned
+    assert lib.nvfp4_gemm_silu_mul_quantize(*args, 256, 256, 256, None) == INVALID
+    assert lib.nvfp4_gemm_silu_mul_quantize(*([A16] * 11), 256, 256, 96, None) == INVALID    # k % 64
+
+
+def test_grouped_silu_mul_gemm_argument_checks(lib):
+    args = [A16] * 12
+    assert lib.nvfp4_grouped_gemm_silu_mul_quantize_masked(*args, 2000, 128, 256, 256, None) == INVALID
+    args[6] = None                          # mask required
+    assert lib.nvfp4_grouped_gemm_silu_mul_quantize_masked(*args, 2, 128, 256, 256, None) == INVALID
+    assert lib.nvfp4_grouped_gemm_silu_mul_quantize_masked(*([A16] * 12), 0, 128, 256, 256, None) == 0  # empty

@@ -471,3 +471,125 @@ def test_grouped_ref_equals_per_expert(oracle):
         if v:
             ref = oracle.gemm_ref(qa[e], qw[e], sfa[e], sfw[e], alphas[e], mmax, n, k)[:v]
             assert (out[e, :v] == ref).all()
+
+
+# --------------------------------------------------------------------------------------
+# SwiGLU first half: gate/up projections, SiLU-and-mul quantization of h
+# --------------------------------------------------------------------------------------
+
+def _bf16_value(bits):
+    """Exact value of one bf16 bit pattern (reinterpretation of the upper half of an fp32)."""
+    w = np.array([int(bits) << 16], np.uint32)
+    return float(w.view(np.float32)[0])
+
+
+def test_f64_to_bf16_is_nearest_ties_even(oracle):
+    # brute force on the definition: of the two bf16 neighbours (by bit pattern) of v, the
+    # nearer one; on a tie the one with the even bit pattern
+    g = np.random.default_rng(3)
+    vals = list(g.standard_normal(3000) * 10.0 ** g.integers(-30, 30, 3000))
+    # exact midpoints between neighbours, and points just beside them
+    for bits in g.integers(0x0080, 0x7F00, 400):
+        lo, hi = _bf16_value(bits), _bf16_value(bits + 1)
+        mid = (lo + hi) / 2
+        vals += [mid, np.nextafter(mid, 0.0), np.nextafter(mid, np.inf), -mid]
+    vals += [0.0, -0.0, 2.0 ** -133, 2.0 ** -134, 3 * 2.0 ** -135, 1e39,
+             float.fromhex("0x1.FEp127"), float.fromhex("0x1.FFp127")]
+    for v in vals:
+        got = oracle.f64_to_bf16(v)
+        a = abs(v)
+        sign = 0x8000 if math.copysign(1.0, v) < 0 else 0
+        if a >= float.fromhex("0x1.FFp127"):     # at or past the overflow midpoint: infinity
+            assert got == sign | 0x7F80, v
+            continue
+        t = int(np.array([a], np.float32).view(np.uint32)[0] >> 16)   # neighbour by truncation
+        cands = [c for c in (t - 1, t, t + 1) if 0 <= c <= 0x7F7F]
+        dist = [abs(_bf16_value(c) - a) for c in cands]
+        best = min(dist)
+        near = [c for c, d in zip(cands, dist) if d == best]
+        want = near[0] if len(near) == 1 else [c for c in near if c % 2 == 0][0]
+        assert got == sign | want, (v, hex(got), hex(sign | want))
+
+
+def _pack(codes):
+    codes = np.asarray(codes, np.uint8)
+    return (codes[..., 0::2] | (codes[..., 1::2] << 4)).astype(np.uint8)
+
+
+def test_gemm_silu_mul_closed_form(oracle):
+    # A = 1 everywhere, gate weight = 1, up weight = +-1 per output column (unit scales):
+    # acc_g = k, acc_u = +-k.  With alpha_gate = 1, alpha_up = 1/64 and k = 128: g = 128
+    # (silu(128) = 128 exactly in fp32), u = +-2, h = +-256, and gsf_h = 2688/256 makes
+    # every block scale 448 (0x7E) and every code +-6 (0x7 / 0xF).  Swapping gate and up,
+    # or their alphas, changes h.
+    m, n, k = 130, 256, 128
+    sign = np.random.default_rng(5).integers(0, 2, n).astype(np.uint8)   # 1: negative up row
+    a = _pack(np.full((m, k), 0x2, np.uint8))
+    bg = _pack(np.full((n, k), 0x2, np.uint8))
+    bu = _pack(np.where(sign[:, None] == 1, 0xA, 0x2).astype(np.uint8) * np.ones((1, k), np.uint8))
+    sa = np.full(oracle.scale_bytes(m, k), 0x38, np.uint8)
+    sb = np.full(oracle.scale_bytes(n, k), 0x38, np.uint8)
+    q, sf = oracle.gemm_silu_mul_quantize(a, bg, bu, sa, sb, sb, 1.0, 1.0 / 64, 2688.0 / 256, m, n, k)
+    want_codes = np.where(sign == 1, 0xF, 0x7).astype(np.uint8)
+    assert (unpack_codes(q) == want_codes[None, :]).all()
+    for r in range(-(-m // 128) * 128):
+        for c in range(n // 16):
+            want = 0x7E if r < m else 0x00          # padding rows of the dense output are 0
+            assert sf[oracle.sf_offset(r, c, n)] == want
+    # swapped roles give something else
+    q2, _ = oracle.gemm_silu_mul_quantize(a, bu, bg, sa, sb, sb, 1.0, 1.0 / 64, 2688.0 / 256, m, n, k)
+    assert (q2 != q).any()
+    _, sf3 = oracle.gemm_silu_mul_quantize(a, bg, bu, sa, sb, sb, 1.0 / 64, 1.0, 2688.0 / 256, m, n, k)
+    assert (sf3 != sf).any()          # h = silu(2) * 128: the codes saturate alike, the scales differ
+
+
+def test_gemm_silu_mul_zero_up_weight_gives_zero(oracle):
+    m, n, k = 40, 128, 64
+    xa = S.normal_bf16((m, k), 1.0, seed=11)
+    xg = S.normal_bf16((n, k), 0.02, seed=11, tensor_id=2)
+    _, ga = oracle.global_scale(xa)
+    _, gg = oracle.global_scale(xg)
+    qa, sa = oracle.quantize(xa, ga)
+    qg, sg = oracle.quantize(xg, gg)
+    qu = np.zeros_like(qg)
+    su = np.zeros_like(sg)
+    q, sf = oracle.gemm_silu_mul_quantize(qa, qg, qu, sa, sg, su, 0.5, 0.5, 100.0, m, n, k)
+    assert ((q & 0x77) == 0).all() and (sf == 0).all()
+
+
+def test_gemm_silu_mul_rows_and_grouped_agree_with_dense(oracle):
+    # invariants: a row of the result depends only on that row of A; a masked expert equals
+    # the dense result on its valid rows and leaves the other rows untouched
+    E, mmax, n, k = 3, 150, 128, 128
+    xa = S.normal_bf16((E, mmax, k), 1.0, seed=12)
+    xg = S.normal_bf16((E, n, k), 0.02, seed=12, tensor_id=2)
+    xu = S.normal_bf16((E, n, k), 0.02, seed=12, tensor_id=3)
+    mask = np.array([150, 0, 77], np.int32)
+    _, ga = oracle.global_scale_batched(xa, None)
+    _, gg = oracle.global_scale_batched(xg, None)
+    _, gu = oracle.global_scale_batched(xu, None)
+    qa, sa = oracle.quantize_masked_batched(xa, ga)
+    qg, sg = oracle.quantize_masked_batched(xg, gg)
+    qu, su = oracle.quantize_masked_batched(xu, gu)
+    al_g = np.array([0.7, 0.9, 1.1], np.float32)
+    al_u = np.array([1.3, 0.6, 0.8], np.float32)
+    gsf = np.array([40.0, 50.0, 60.0], np.float32)
+    qG, sG = oracle.grouped_gemm_silu_mul_quantize(qa, qg, qu, sa, sg, su, mask, al_g, al_u, gsf, E, mmax, n, k,
+                                                   q_fill=0xAB, sf_fill=0xCD)
+    for e in range(E):
+        v = int(mask[e])
+        qd, sd = oracle.gemm_silu_mul_quantize(qa[e], qg[e], qu[e], sa[e], sg[e], su[e], al_g[e], al_u[e], gsf[e],
+                                               mmax, n, k)
+        assert (qG[e, :v] == qd[:v]).all() and (qG[e, v:] == 0xAB).all()
+        for r in range(-(-mmax // 128) * 128):
+            offs = [oracle.sf_offset(r, c, n) for c in range(n // 16)]
+            if r < v:
+                assert (sG[e, offs] == sd[offs]).all()
+            else:
+                assert (sG[e, offs] == 0xCD).all()
+        rows = np.array([0, 3, mmax - 1])
+        qr, sr = oracle.gemm_silu_mul_quantize_rows(qa[e], qg[e], qu[e], sa[e], sg[e], su[e], al_g[e], al_u[e],
+                                                    gsf[e], n, k, rows)
+        assert (qr == qd[rows]).all()
+        for i, r in enumerate(rows):
+            assert (sr[i] == sd[[oracle.sf_offset(r, c, n) for c in range(n // 16)]]).all()
