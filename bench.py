@@ -211,13 +211,17 @@ class Workload:
 
 
 class SwigluBlock(Workload):
+    """Dense SwiGLU block.  fused=True: amax(x), quantize(x), the gate/up GEMM whose
+    epilogue emits SiLU(g)*u as NVFP4, the down GEMM.  fused=False: the same with the
+    gate/up GEMM writing bf16 [g | u] and the SiLU-and-mul quantizer as its own kernel."""
     name = "swiglu_block"
     unit = "TFLOP/s"
-    dominant = "gemm_gate_up"
 
-    def __init__(self, nv, seed=0):
+    def __init__(self, nv, seed=0, fused=True):
         import torch
         self.nv = nv
+        self.fused = fused
+        self.dominant = "gemm_gate_up_silu_quantize" if fused else "gemm_gate_up"
         self.M, self.H, self.I = 8192, 5120, 8192
         d = S.swiglu_block(self.M, self.H, self.I, seed)
         self.x_host = d["x"]
@@ -234,16 +238,39 @@ class SwigluBlock(Workload):
         self.hq = torch.empty((1, self.M, self.I // 2), dtype=torch.uint8, device=dev)
         self.hsf = torch.empty((1, nv.nvfp4_scale_bytes(self.M, self.I)), dtype=torch.uint8, device=dev)
         self.y = torch.empty((self.M, self.H), dtype=torch.bfloat16, device=dev)
-        # calibration pass: static scale of h = silu(gate) * up and the down-projection alpha
-        for _, fn in self.launches()[:3]:
-            fn()
+        # the gate and up weights are the two row halves of the one quantized [2I, H] tensor
+        half = nv.nvfp4_scale_bytes(self.I, self.H)
+        self.wg_q, self.wu_q = self.wgu_q[:self.I], self.wgu_q[self.I:]
+        self.wg_sf, self.wu_sf = self.wgu_sf[:half], self.wgu_sf[half:]
+        # calibration pass (offline, unfused): static scale of h = silu(gate) * up and the
+        # down-projection alpha
+        self._unfused_launches()[0][1]()
+        self._unfused_launches()[1][1]()
+        self._unfused_launches()[2][1]()
         amax_h, self.gsf_h = nv.nvfp4_global_scale_batched(self.gu.view(1, self.M, 2 * self.I), None, silu_mul=True)
+        if fused:
+            del self.gu
         a_h = np.float32(amax_h.item())
         a_w = np.float32(self.amax_wd.item())
         self.alpha2 = torch.tensor([np.float32(a_h * a_w) / np.float32(7225344.0)], dtype=torch.float32, device=dev)
         torch.cuda.synchronize()
 
     def launches(self):
+        if not self.fused:
+            return self._unfused_launches()
+        nv = self
+        lib = self.nv
+        return [
+            ("global_scale_x", lambda: lib.nvfp4_global_scale(nv.x, nv.amax_x, nv.gsf_x, nv.amax_wgu, nv.alpha1)),
+            ("quantize_x", lambda: lib.nvfp4_quantize(nv.x, nv.gsf_x, nv.xq, nv.xsf)),
+            ("gemm_gate_up_silu_quantize", lambda: lib.nvfp4_gemm_silu_mul_quantize(
+                nv.xq, nv.wg_q, nv.wu_q, nv.xsf, nv.wg_sf, nv.wu_sf, nv.alpha1, nv.alpha1, nv.gsf_h,
+                nv.hq.view(nv.M, nv.I // 2), nv.hsf.view(-1))),
+            ("gemm_down", lambda: lib.nvfp4_gemm(nv.hq.view(nv.M, nv.I // 2), nv.wd_q, nv.hsf.view(-1), nv.wd_sf,
+                                                 nv.alpha2, None, nv.y)),
+        ]
+
+    def _unfused_launches(self):
         nv = self
         lib = self.nv
         return [
@@ -261,13 +288,15 @@ class SwigluBlock(Workload):
 
     def kernel_work(self):
         M, H, I = self.M, self.H, self.I
-        return {
+        names = {name for name, _ in self.launches()}
+        return {k: v for k, v in {
             "global_scale_x": (2.0 * M * H, "GB/s"),
             "quantize_x": (2.5625 * M * H, "GB/s"),
             "gemm_gate_up": (2.0 * M * H * 2 * I, "TFLOP/s"),
+            "gemm_gate_up_silu_quantize": (2.0 * M * H * 2 * I, "TFLOP/s"),
             "silu_mul_quantize": (4.5625 * M * I, "GB/s"),
             "gemm_down": (2.0 * M * I * H, "TFLOP/s"),
-        }
+        }.items() if k in names}
 
     def e2e_io(self):
         """(host input, device input, device output) of the end-to-end measurement."""
@@ -278,6 +307,8 @@ class SwigluBlock(Workload):
                             "intermediate 8192; gate/up [8192x5120]@[16384x5120]^T, silu*mul requantize, "
                             "down [8192x8192]@[5120x8192]^T; x~N(0,1), W~N(0,0.02)",
                 "tokens": self.M, "hidden": self.H, "intermediate": self.I,
+                "path": ("gate/up GEMM with the SiLU*mul NVFP4 quantizer in its epilogue" if self.fused else
+                         "gate/up GEMM to bf16, then the SiLU*mul quantizer kernel"),
                 "l2": "flushed between steps (512 MB write, outside the timed events)"}
 
 
@@ -402,6 +433,90 @@ class GroupedMoE(Workload):
                 "l2": "flushed between steps"}
 
 
+class GroupedSwiglu(Workload):
+    """Routed-expert SwiGLU: masked quantize of every expert's tokens, the grouped gate/up
+    GEMM whose epilogue emits SiLU(g)*u as NVFP4, the grouped down GEMM.  Activation scales
+    (x and h, per expert) are static, calibrated once, as the masked quantizer's global
+    scale input is."""
+    name = "grouped_swiglu"
+    unit = "TFLOP/s"
+    dominant = "grouped_gemm_gate_up_silu_quantize"
+
+    def __init__(self, nv, seed=0):
+        import torch
+        self.nv = nv
+        self.E, self.mmax, self.H, self.I = 16, 2048, 5120, 8192
+        d = S.grouped_swiglu(self.E, self.mmax, self.H, self.I, 512, seed)
+        E, mmax, H, I = self.E, self.mmax, self.H, self.I
+        self.mask_host = d["mask"]
+        self.mask = torch.from_numpy(d["mask"]).cuda()
+        self.x_host = d["x"]
+        self.x = to_dev_bf16(d["x"])
+        amax_x, self.gsf_x = nv.nvfp4_global_scale_batched(self.x, self.mask)      # calibration
+        amaxes = {}
+        for name in ("w_gate", "w_up", "w_down"):
+            w = to_dev_bf16(d[name])
+            amax, g = nv.nvfp4_global_scale_batched(w, None)
+            q, sf = nv.nvfp4_quantize_masked_batched(w, g, None)
+            setattr(self, name + "_q", q)
+            setattr(self, name + "_sf", sf)
+            amaxes[name] = amax.cpu().numpy().astype(np.float32)
+            del w
+        ax = amax_x.cpu().numpy().astype(np.float32)
+
+        def alpha(a, b):
+            return torch.from_numpy(((a * b) / np.float32(7225344.0)).astype(np.float32)).cuda()
+
+        self.alpha_g = alpha(ax, amaxes["w_gate"])
+        self.alpha_u = alpha(ax, amaxes["w_up"])
+        self.xq = torch.empty((E, mmax, H // 2), dtype=torch.uint8, device="cuda")
+        self.xsf = torch.empty((E, nv.nvfp4_scale_bytes(mmax, H)), dtype=torch.uint8, device="cuda")
+        self.hq = torch.empty((E, mmax, I // 2), dtype=torch.uint8, device="cuda")
+        self.hsf = torch.empty((E, nv.nvfp4_scale_bytes(mmax, I)), dtype=torch.uint8, device="cuda")
+        self.y = torch.empty((E, mmax, H), dtype=torch.bfloat16, device="cuda")
+        # calibration of the static h scales (offline, unfused): [g | u] in bf16, amax of silu(g)*u
+        nv.nvfp4_quantize_masked_batched(self.x, self.gsf_x, self.mask, self.xq, self.xsf)
+        g = nv.nvfp4_grouped_gemm_masked(self.xq, self.w_gate_q, self.xsf, self.w_gate_sf, self.mask, self.alpha_g)
+        u = nv.nvfp4_grouped_gemm_masked(self.xq, self.w_up_q, self.xsf, self.w_up_sf, self.mask, self.alpha_u)
+        gu = torch.cat([g, u], dim=-1)
+        del g, u
+        amax_h, self.gsf_h = nv.nvfp4_global_scale_batched(gu, self.mask, silu_mul=True)
+        del gu
+        self.alpha_d = alpha(amax_h.cpu().numpy().astype(np.float32), amaxes["w_down"])
+        torch.cuda.synchronize()
+
+    def launches(self):
+        lib, s = self.nv, self
+        return [
+            ("quantize_x_masked", lambda: lib.nvfp4_quantize_masked_batched(s.x, s.gsf_x, s.mask, s.xq, s.xsf)),
+            ("grouped_gemm_gate_up_silu_quantize", lambda: lib.nvfp4_grouped_gemm_silu_mul_quantize_masked(
+                s.xq, s.w_gate_q, s.w_up_q, s.xsf, s.w_gate_sf, s.w_up_sf, s.mask, s.alpha_g, s.alpha_u, s.gsf_h,
+                s.hq, s.hsf)),
+            ("grouped_gemm_down", lambda: lib.nvfp4_grouped_gemm_masked(s.hq, s.w_down_q, s.hsf, s.w_down_sf, s.mask,
+                                                                        s.alpha_d, s.y)),
+        ]
+
+    def work(self):
+        return 6.0 * int(self.mask_host.sum()) * self.H * self.I
+
+    def kernel_work(self):
+        rows = int(self.mask_host.sum())
+        return {"quantize_x_masked": (2.5625 * rows * self.H, "GB/s"),
+                "grouped_gemm_gate_up_silu_quantize": (4.0 * rows * self.H * self.I, "TFLOP/s"),
+                "grouped_gemm_down": (2.0 * rows * self.I * self.H, "TFLOP/s")}
+
+    def e2e_io(self):
+        return self.x_host, self.x, self.y
+
+    def config(self):
+        return {"workload": f"routed-expert NVFP4 SwiGLU, E=16 experts, Mmax=2048 tokens each, valid rows "
+                            f"min(Poisson(512),2048) (sum {int(self.mask_host.sum())}), hidden 5120, "
+                            f"intermediate 8192; masked quantize, grouped gate/up GEMM with the SiLU*mul NVFP4 "
+                            f"epilogue, grouped down GEMM; static per-expert activation scales",
+                "experts": self.E, "mmax": self.mmax, "hidden": self.H, "intermediate": self.I,
+                "l2": "flushed between steps (512 MB write, outside the timed events)"}
+
+
 class LowRank(Workload):
     name = "lowrank"
     unit = "TFLOP/s"
@@ -481,9 +596,9 @@ class PR1Linear(Workload):
         return {"workload": "single NVFP4 linear x[128,256] W[256,256] (latency-bound)", "l2": "flushed between steps"}
 
 
-def make_workload(name, nv, rank_lr):
+def make_workload(name, nv, rank_lr, swiglu_path="fused"):
     if name == "swiglu_block":
-        return SwigluBlock(nv)
+        return SwigluBlock(nv, fused=swiglu_path == "fused")
     if name == "quant_dense":
         return QuantDense(nv)
     if name == "quant_masked":
@@ -492,6 +607,8 @@ def make_workload(name, nv, rank_lr):
         return QuantMasked(nv, True)
     if name == "grouped_moe":
         return GroupedMoE(nv)
+    if name == "grouped_swiglu":
+        return GroupedSwiglu(nv)
     if name == "lowrank":
         return LowRank(nv, rank_lr)
     if name == "pr1_linear":
@@ -527,6 +644,14 @@ class OracleSample:
             self.H, self.I = 5120, 8192
             self.sample = f"{self.rows} of 8192 token rows through the whole block (amax, quantize, gate/up GEMM, " \
                           f"SiLU-mul quantize, down GEMM)"
+        elif w == "grouped_swiglu":
+            self.rows = rows or 2
+            d = S.grouped_swiglu(16, 2048, 5120, 8192, 512, 0, experts=1)
+            self.x = d["x"][0, :self.rows].copy()
+            self.wg, self.wu, self.wd = d["w_gate"][0], d["w_up"][0], d["w_down"][0]
+            self.H, self.I = 5120, 8192
+            self.sample = f"{self.rows} token rows of expert 0 through the routed-expert block (quantize, gate/up " \
+                          f"GEMMs, SiLU-mul quantize, down GEMM)"
         elif w == "pr1_linear":
             self.rows = 128
             d = S.pr1_linear(0)
@@ -557,6 +682,14 @@ class OracleSample:
             self.qw, self.sfw = O.quantize(self.wgu, gw)
             self.ad, gd = O.global_scale(self.wd)
             self.qd, self.sfd = O.quantize(self.wd, gd)
+        elif self.workload == "grouped_swiglu":
+            self.ag, gg = O.global_scale(self.wg)
+            self.qg, self.sfg = O.quantize(self.wg, gg)
+            self.au, gu = O.global_scale(self.wu)
+            self.qu, self.sfu = O.quantize(self.wu, gu)
+            self.ad, gd = O.global_scale(self.wd)
+            self.qd, self.sfd = O.quantize(self.wd, gd)
+            self.ax, self.gx = O.global_scale(self.x)          # static activation scale (calibration)
         elif self.workload in ("pr1_linear", "grouped_moe", "lowrank"):
             self.aw, gw = O.global_scale(self.w)
             self.qw, self.sfw = O.quantize(self.w, gw)
@@ -569,12 +702,24 @@ class OracleSample:
             rows, H, I = self.rows, self.H, self.I
             ax, gx = O.global_scale(self.x)
             qx, sfx = O.quantize(self.x, gx)
-            gu = O.gemm_ref(qx, self.qw, sfx, self.sfw, O.alpha(float(ax), float(self.aw)), rows, 2 * I, H)
-            gu_bits = S.f32_to_bf16_bits(gu.astype(np.float32)).reshape(1, rows, 2 * I)
+            al = O.alpha(float(ax), float(self.aw))
+            half = O.scale_bytes(I, H)
+            gu_bits = O.gemm_gate_up_bf16(qx, self.qw[:I], self.qw[I:], sfx, self.sfw[:half], self.sfw[half:],
+                                          al, al, I, H, np.arange(rows)).reshape(1, rows, 2 * I)
             ah, gh = O.global_scale_batched(gu_bits, None, silu_mul=True)
             hq, hsf = O.silu_mul_quantize_batched(gu_bits, gh)
             O.gemm_ref(hq[0], self.qd, hsf[0], self.sfd, O.alpha(float(ah[0]), float(self.ad)), rows, H, I)
             work = 2.0 * rows * H * 2 * I + 2.0 * rows * I * H
+        elif w == "grouped_swiglu":
+            rows, H, I = self.rows, self.H, self.I
+            qx, sfx = O.quantize(self.x, self.gx)
+            ax = float(self.ax)
+            gu_bits = O.gemm_gate_up_bf16(qx, self.qg, self.qu, sfx, self.sfg, self.sfu, O.alpha(ax, float(self.ag)),
+                                          O.alpha(ax, float(self.au)), I, H, np.arange(rows)).reshape(1, rows, 2 * I)
+            ah, gh = O.global_scale_batched(gu_bits, None, silu_mul=True)
+            hq, hsf = O.silu_mul_quantize_batched(gu_bits, gh)
+            O.gemm_ref(hq[0], self.qd, hsf[0], self.sfd, O.alpha(float(ah[0]), float(self.ad)), rows, H, I)
+            work = 6.0 * rows * H * I
         elif w == "pr1_linear":
             ax, gx = O.global_scale(self.x)
             qx, sfx = O.quantize(self.x, gx)
@@ -613,7 +758,7 @@ def run_reference(args, world, rank):
     if rank != 0:
         return       # the oracle runs on rank 0 only; the other ranks exit without work
     wl = args.workload
-    rows = 1 if wl == "swiglu_block" else None
+    rows = 1 if wl in ("swiglu_block", "grouped_swiglu") else None
     o = OracleSample(wl, rows)
     o.measure(min(args.warmup, 1))
     t0 = time.perf_counter()
@@ -636,9 +781,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="nvfp4", choices=["nvfp4", "reference"])
     ap.add_argument("--workload", default="swiglu_block",
-                    choices=["swiglu_block", "quant_dense", "quant_masked", "quant_silu", "grouped_moe", "lowrank",
-                             "pr1_linear"])
+                    choices=["swiglu_block", "quant_dense", "quant_masked", "quant_silu", "grouped_moe",
+                             "grouped_swiglu", "lowrank", "pr1_linear"])
     ap.add_argument("--rank-lr", type=int, default=64)
+    ap.add_argument("--swiglu-path", default="fused", choices=["fused", "unfused"],
+                    help="swiglu_block: SiLU*mul quantization in the gate/up GEMM epilogue, or as its own kernel")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
@@ -654,7 +801,7 @@ def main():
     import nvfp4_block_scaled_16_b200 as nv
     world, rank, local = dist_setup(args.gpus)
     nv.load_library()
-    wl = make_workload(args.workload, nv, args.rank_lr)
+    wl = make_workload(args.workload, nv, args.rank_lr, args.swiglu_path)
     launches = wl.launches()
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
     stream = torch.cuda.Stream()

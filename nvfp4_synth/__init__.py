@@ -28,7 +28,7 @@ import numpy as np
 # Tensor ids: one independent stream per tensor of a workload.
 TID = {
     "x": 1, "w": 2, "w_gate_up": 3, "w_down": 4, "mask": 5, "d": 6, "l1": 7, "bias": 8,
-    "outlier": 9, "sample": 10,
+    "outlier": 9, "sample": 10, "w_gate": 11, "w_up": 12,
 }
 
 
@@ -60,8 +60,12 @@ def bf16_bits_to_f32(u) -> np.ndarray:
 CHUNK = 1 << 24
 
 
-def _chunked(shape, fill):
-    """Fill a flat uint16 array chunk by chunk; chunk c gets its own generator."""
+def _chunked(shape, fill, items=None):
+    """Fill a flat uint16 array chunk by chunk; chunk c gets its own generator.  With
+    `items`, only the leading `items` entries of dimension 0 are produced (the same values
+    as in the whole tensor)."""
+    if items is not None:
+        shape = (int(items),) + tuple(shape[1:])
     n = int(np.prod(shape))
     out = np.empty(n, np.uint16)
     starts = list(range(0, n, CHUNK))
@@ -76,14 +80,15 @@ def _chunked(shape, fill):
     return out.reshape(shape)
 
 
-def normal_bf16(shape, std=1.0, seed=0, tensor_id=TID["x"]) -> np.ndarray:
-    """N(0, std^2) drawn in fp32 and rounded to bf16."""
+def normal_bf16(shape, std=1.0, seed=0, tensor_id=TID["x"], items=None) -> np.ndarray:
+    """N(0, std^2) drawn in fp32 and rounded to bf16 (optionally only the leading `items`
+    entries of dimension 0)."""
     def fill(c, dst):
         v = np.random.default_rng([int(seed), int(tensor_id), c]).standard_normal(dst.size, dtype=np.float32)
         if std != 1.0:
             v *= np.float32(std)
         dst[:] = f32_to_bf16_bits(v)
-    return _chunked(shape, fill)
+    return _chunked(shape, fill, items)
 
 
 def normal_with_outliers_bf16(shape, p=0.001, factor=50.0, seed=0, tensor_id=TID["x"]) -> np.ndarray:
@@ -137,6 +142,16 @@ def swiglu_block(m=8192, hidden=5120, inter=8192, seed=0):
 def grouped_moe(E=16, mmax=2048, k=5120, n=8192, mean=512, seed=0):
     return {"a": normal_bf16((E, mmax, k), 1.0, seed, TID["x"]),
             "w": normal_bf16((E, n, k), 0.02, seed, TID["w"]),
+            "mask": masks_poisson(E, mean, mmax, seed)}
+
+
+def grouped_swiglu(E=16, mmax=2048, hidden=5120, inter=8192, mean=512, seed=0, experts=None):
+    """Routed experts: tokens per expert min(Poisson(mean), mmax); per-expert gate, up and
+    down weights.  With `experts`, only the leading experts' tensors are produced."""
+    return {"x": normal_bf16((E, mmax, hidden), 1.0, seed, TID["x"], experts),
+            "w_gate": normal_bf16((E, inter, hidden), 0.02, seed, TID["w_gate"], experts),
+            "w_up": normal_bf16((E, inter, hidden), 0.02, seed, TID["w_up"], experts),
+            "w_down": normal_bf16((E, hidden, inter), 0.02, seed, TID["w_down"], experts),
             "mask": masks_poisson(E, mean, mmax, seed)}
 
 

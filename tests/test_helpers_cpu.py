@@ -48,3 +48,14 @@ def test_nvfp4_close_accepts_identical_and_rejects_planted_mistakes(oracle):
         q2, s2, _ = _silu_case(oracle, 1, **kw)
         with pytest.raises(AssertionError):
             assert_nvfp4_close(q2, s2, q, s, gsf)
+
+
+def test_synth_leading_items_match_whole_tensor(monkeypatch):
+    # small chunks so the test stays small: items of 1200 values, item 1 straddles the
+    # 2048-value chunk boundary
+    monkeypatch.setattr(S, "CHUNK", 1 << 11)
+    whole = S.normal_bf16((3, 40, 30), 0.02, 4, 11)
+    for items in (1, 2):
+        part = S.normal_bf16((3, 40, 30), 0.02, 4, 11, items=items)
+        assert part.shape == (items, 40, 30)
+        assert (part == whole[:items]).all()
