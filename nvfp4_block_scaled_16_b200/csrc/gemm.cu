@@ -188,6 +188,11 @@ __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile 
   }
 }
 
+// mbar_wait with the common case (the phase already completed) inlined into the caller.
+__device__ __forceinline__ bool mbar_wait_fast(uint64_t* bar, uint32_t parity, volatile int32_t* abort, int* status) {
+  return mbar_try_wait(bar, parity) || mbar_wait(bar, parity, abort, status);
+}
+
 // Tiled TMA loads into this CTA's shared memory, completing on the barrier at the
 // shared::cluster address `bar` (the leader's; the .cta_group::2 form allows either CTA
 // of the pair).
@@ -431,7 +436,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kSwiGLU>, 1
     }
     __syncwarp();
     const int lr_stages = kLowRank ? (p.rank + 63) / 64 : 0;
-    uint32_t it = 0;
+    uint32_t s = 0, phase = 0;
+    bool wrapped = false;      // the ring has been filled once: every later stage waits for its slot
     bool ok = true;
     TileCoord t;
     for (int tile = pair; ok && tile_coord<kGrouped>(p, ctl, tile, t); tile += pairs) {
@@ -447,9 +453,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kSwiGLU>, 1
       const int sfa_row0 = ((2 * t.m_tile + static_cast<int>(rank)) * p.sf_groups) * 4;
       const int sfb_row0 = (b_tile0 * p.sf_groups) * 4;
       const int sfb_row1 = (b_tile1 * p.sf_groups) * 4;
-      for (int ks = 0; ks < p.k_stages + lr_stages; ++ks, ++it) {
-        const uint32_t s = it % kStages, round = it / kStages;
-        if (round > 0 && !(ok = mbar_wait(&ctl.empty[s], (round - 1) & 1, abort, p.status))) break;
+      for (int ks = 0; ks < p.k_stages + lr_stages; ++ks) {
+        if (wrapped && !(ok = mbar_wait_fast(&ctl.empty[s], phase, abort, p.status))) break;
         uint8_t* st = smem + s * kStageBytes;
         const uint32_t full_bar = map_to_rank(&ctl.full[s], 0);
         if (elect_one()) {
@@ -477,48 +482,75 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kSwiGLU>, 1
           }
         }
         __syncwarp();
+        if (++s == kStages) {
+          s = 0;
+          if (wrapped) phase ^= 1u;
+          wrapped = true;
+        }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer (leader)
-    // The whole warp runs the loop; one elected lane issues each batch of tcgen05 ops.
+    // The whole warp runs the loop; one elected lane issues each stage's tcgen05 ops.  The
+    // loop is kept lean (stage slot and phase tracked incrementally, descriptors built
+    // once per stage and advanced by 32 bytes per K-step): the tensor pipe finishes one
+    // M256 N256 K64 MMA every ~128 cycles, so issue overhead shows directly in the rate.
     if (leader) {
       const int lr_stages = kLowRank ? (p.rank + 63) / 64 : 0;
-      uint32_t it = 0, tcount = 0;
+      const uint32_t smem0 = smem_u32(smem);
+      const uint64_t a_desc0 = operand_desc(smem0);
+      const uint64_t b_desc0 = operand_desc(smem0 + kABytes);
+      const uint64_t sfa_desc0 = sf_desc(smem0 + kABytes + kBBytes);
+      const uint64_t sfb_desc0 = sf_desc(smem0 + kABytes + kBBytes + kSfaBytes);
+      uint32_t s = 0, phase = 0, tcount = 0;
       bool ok = true;
       TileCoord t;
       for (int tile = pair; ok && tile_coord<kGrouped>(p, ctl, tile, t); tile += pairs, ++tcount) {
         const uint32_t acc = tmem + ((tcount & 1) ? kAccOverlapCol : 0u);
         if (tcount > 0) {
-          if (!(ok = mbar_wait(&ctl.acc_empty, (tcount - 1) & 1, abort, p.status))) break;
+          if (!(ok = mbar_wait_fast(&ctl.acc_empty, (tcount - 1) & 1, abort, p.status))) break;
           tc_fence_after();
         }
-        for (int ks = 0; ks < p.k_stages + lr_stages; ++ks, ++it) {
-          const uint32_t s = it % kStages;
-          if (!(ok = mbar_wait(&ctl.full[s], (it / kStages) & 1, abort, p.status))) break;
+        for (int ks = 0; ks < p.k_stages + lr_stages; ++ks) {
+          if (!(ok = mbar_wait_fast(&ctl.full[s], phase, abort, p.status))) break;
           tc_fence_after();
-          const uint32_t st = smem_u32(smem + s * kStageBytes);
+          const uint64_t off = (s * kStageBytes) >> 4;     // descriptor address units (16 bytes)
+          const uint64_t da = a_desc0 + off, db = b_desc0 + off;
           if (elect_one()) {
             if (ks < p.k_stages) {
-              const int nks = min(4, p.k_steps - 4 * ks);
-              const uint32_t sfa_s = st + kABytes + kBBytes;
-              const uint32_t sfb_s = sfa_s + kSfaBytes;
-              for (int j = 0; j < nks; ++j) {
-                tc_copy_sf(tmem + kSfaCol + 4 * j, sf_desc(sfa_s + 512 * j));
-                tc_copy_sf(tmem + kSfbCol + 8 * j, sf_desc(sfb_s + 512 * j));
-                tc_copy_sf(tmem + kSfbCol + 8 * j + 4, sf_desc(sfb_s + kSfaBytes + 512 * j));
-                mma_fp4(acc, operand_desc(st + 32 * j), operand_desc(st + kABytes + 32 * j), tmem + kSfaCol + 4 * j,
-                        tmem + kSfbCol + 8 * j, (ks > 0 || j > 0) ? 1u : 0u);
+              const uint64_t dsa = sfa_desc0 + off, dsb = sfb_desc0 + off;
+              const uint32_t acc_first = ks > 0 ? 1u : 0u;
+              const int nks = p.k_steps - 4 * ks;
+              if (nks >= 4) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  tc_copy_sf(tmem + kSfaCol + 4 * j, dsa + 32 * j);
+                  tc_copy_sf(tmem + kSfbCol + 8 * j, dsb + 32 * j);
+                  tc_copy_sf(tmem + kSfbCol + 8 * j + 4, dsb + (kSfaBytes >> 4) + 32 * j);
+                  mma_fp4(acc, da + 2 * j, db + 2 * j, tmem + kSfaCol + 4 * j, tmem + kSfbCol + 8 * j,
+                          j > 0 ? 1u : acc_first);
+                }
+              } else {
+                for (int j = 0; j < nks; ++j) {
+                  tc_copy_sf(tmem + kSfaCol + 4 * j, dsa + 32 * j);
+                  tc_copy_sf(tmem + kSfbCol + 8 * j, dsb + 32 * j);
+                  tc_copy_sf(tmem + kSfbCol + 8 * j + 4, dsb + (kSfaBytes >> 4) + 32 * j);
+                  mma_fp4(acc, da + 2 * j, db + 2 * j, tmem + kSfaCol + 4 * j, tmem + kSfbCol + 8 * j,
+                          j > 0 ? 1u : acc_first);
+                }
               }
             } else if constexpr (kLowRank) {
               const int c = ks - p.k_stages;
               const int steps = min(4, (p.rank - 64 * c) / 16);
-              for (int j = 0; j < steps; ++j)
-                mma_bf16(acc, operand_desc(st + 32 * j), operand_desc(st + kABytes + 32 * j), 1u);
+              for (int j = 0; j < steps; ++j) mma_bf16(acc, da + 2 * j, db + 2 * j, 1u);
             }
             mma_commit_both(&ctl.empty[s]);
           }
           __syncwarp();
+          if (++s == kStages) {
+            s = 0;
+            phase ^= 1u;
+          }
         }
         if (!ok) break;
         if (elect_one()) mma_commit_both(&ctl.acc_full);
