@@ -34,7 +34,8 @@
 //               into its own tensor memory, then the MMA; the low-rank term follows as kind::f16 (bf16) MMAs into the same
 //               accumulator.  Commits are multicast to both CTAs.
 //   warps 2-5   epilogue (both CTAs): tcgen05.ld of the CTA's 128 x 256 fp32 accumulator
-//               (each warp owns its 32-lane TMEM quarter), alpha * acc + bias, bf16 stores.
+//               (each warp owns its 32-lane TMEM quarter), alpha * acc + bias, bf16 staged
+//               in shared memory and written by TMA stores (one 32 x 64 tile at a time).
 //               The SiLU * up epilogue uses warps 2-9: two per lane quarter, one per half
 //               of the tile's 128 h columns.
 // Two accumulators of 256 columns share TMEM columns [192, 256): the epilogue drains that
@@ -95,7 +96,13 @@ struct __align__(8) Control {
   int32_t abort;
   int32_t prefix[kMaxExperts + 1];   // grouped: prefix sums of pair tiles per expert
 };
-constexpr int kSmemBytes = kStages * kStageBytes + sizeof(Control) + 1024;
+// bf16 epilogue: one 32-row x 64-column bf16 staging tile (4 KB, 128-byte swizzle) per
+// epilogue warp, written to global memory by a TMA store.
+constexpr int kStoreTileBytes = 32 * 128;
+template <bool kSwiGLU>
+constexpr int kStagingBytes = kSwiGLU ? 0 : kEpiWarps<false> * kStoreTileBytes;
+template <bool kSwiGLU>
+constexpr int kSmemBytes = kStages * kStageBytes + kStagingBytes<kSwiGLU> + sizeof(Control) + 1024;
 
 // Instruction descriptors (tcgen05 "instruction descriptor" bit fields).
 //   kind::mxf4nvf4: A/B format E2M1 (1) at bits 7..9 / 10..12, both K-major, N>>3 at
@@ -209,6 +216,28 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       "[%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
+}
+
+// TMA stores of a staged shared-memory tile (bulk-group completion, issued and waited on
+// by the same thread).  Elements outside the tensor are not written.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int c0, int c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(src)), "r"(c0), "r"(c1)
+               : "memory");
+}
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
 }
 
 __device__ __forceinline__ void prefetch_map(const CUtensorMap* map) {
@@ -366,6 +395,7 @@ __device__ __forceinline__ bool tile_coord(const GemmParams& p, const Control& c
 struct Maps {
   CUtensorMap a, b, sfa, sfb, d, l1;
   CUtensorMap b2, sfb2;       // SiLU * up: the up weight and its scales
+  CUtensorMap out;            // bf16 output [E, mmax, n], boxes of 32 rows x 64 columns
 };
 
 // ---- the kernel ---------------------------------------------------------------------------------
@@ -375,7 +405,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kSwiGLU>, 1
     nvfp4_gemm_kernel(const __grid_constant__ Maps maps, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Control& ctl = *reinterpret_cast<Control*>(smem + kStages * kStageBytes);
+  uint8_t* staging = smem + kStages * kStageBytes;     // 1024-byte aligned (the ring is 190 KB)
+  Control& ctl = *reinterpret_cast<Control*>(staging + kStagingBytes<kSwiGLU>);
   volatile int32_t* abort = &ctl.abort;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -621,6 +652,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kSwiGLU>, 1
           }
         }
       } else {
+        // This warp's 32-row slab of the tile goes out through its staging tile and a TMA
+        // store (rows >= m and columns >= n are clipped by the tensor bounds).  A grouped
+        // slab that crosses the expert's mask is stored row by row instead, so rows beyond
+        // the mask stay untouched.
+        const int slab_row = t.m_tile * kTileM + static_cast<int>(rank) * kBM + quarter * 32;
+        const bool use_tma = kGrouped ? slab_row + 32 <= t.valid_rows : slab_row < p.m;
+        uint8_t* stage_tile = staging + (warp - 2) * kStoreTileBytes;
+        const uint32_t stage_row = smem_u32(stage_tile) + lane * 128;
         __nv_bfloat16* out_row = p.out + (static_cast<int64_t>(t.expert) * p.m + row) * p.n;
         for (int i = 0; i < 4; ++i) {
           // accumulator 0 drains its last 64 columns first, accumulator 1 its first 64
@@ -634,37 +673,58 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kSwiGLU>, 1
             if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
           }
           const int col_base = t.n_tile * kBN + sub * 64;
-          if (row_ok) {
+          if (col_base >= p.n || !(use_tma || row_ok)) continue;
+          uint4 o[8];
 #pragma unroll
-            for (int g = 0; g < 8; ++g) {
-              const int col = col_base + 8 * g;
-              if (col < p.n) {
-                float f[8];
+          for (int g = 0; g < 8; ++g) {
+            const int col = col_base + 8 * g;
+            float f[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * g + e]);
-                if (p.bias) {
-                  const uint4 bw = __ldg(reinterpret_cast<const uint4*>(p.bias + col));
-                  const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w};
+            for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * g + e]);
+            if (p.bias && col < p.n) {
+              const uint4 bw = __ldg(reinterpret_cast<const uint4*>(p.bias + col));
+              const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w};
 #pragma unroll
-                  for (int e = 0; e < 4; ++e) {
-                    f[2 * e] = __fmaf_rn(alpha, f[2 * e], __uint_as_float(bb[e] << 16));
-                    f[2 * e + 1] = __fmaf_rn(alpha, f[2 * e + 1], __uint_as_float(bb[e] & 0xffff0000u));
-                  }
-                } else {
-#pragma unroll
-                  for (int e = 0; e < 8; ++e) f[e] = __fmul_rn(alpha, f[e]);
-                }
-                uint4 o;
-                o.x = pack_bf16x2(f[0], f[1]);
-                o.y = pack_bf16x2(f[2], f[3]);
-                o.z = pack_bf16x2(f[4], f[5]);
-                o.w = pack_bf16x2(f[6], f[7]);
-                *reinterpret_cast<uint4*>(out_row + col) = o;
+              for (int e = 0; e < 4; ++e) {
+                f[2 * e] = __fmaf_rn(alpha, f[2 * e], __uint_as_float(bb[e] << 16));
+                f[2 * e + 1] = __fmaf_rn(alpha, f[2 * e + 1], __uint_as_float(bb[e] & 0xffff0000u));
               }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) f[e] = __fmul_rn(alpha, f[e]);
             }
+            o[g].x = pack_bf16x2(f[0], f[1]);
+            o[g].y = pack_bf16x2(f[2], f[3]);
+            o[g].z = pack_bf16x2(f[4], f[5]);
+            o[g].w = pack_bf16x2(f[6], f[7]);
+          }
+          if (use_tma) {
+            if (lane == 0) bulk_wait_read();      // the previous store has read the staging tile
+            __syncwarp();
+            // 128-byte swizzle: 16-byte chunk g of row r sits at chunk position g ^ (r % 8)
+#pragma unroll
+            for (int g = 0; g < 8; ++g) st_shared_v4(stage_row + ((g ^ (lane & 7)) << 4), o[g]);
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              if constexpr (kGrouped) {
+                tma_store_3d(&maps.out, stage_tile, col_base, slab_row, t.expert);
+              } else {
+                tma_store_2d(&maps.out, stage_tile, col_base, slab_row);
+              }
+              bulk_commit();
+            }
+          } else {
+#pragma unroll
+            for (int g = 0; g < 8; ++g)
+              if (col_base + 8 * g < p.n) *reinterpret_cast<uint4*>(out_row + col_base + 8 * g) = o[g];
           }
         }
       }
+    }
+    if constexpr (!kSwiGLU) {
+      if (lane == 0) bulk_wait_all();         // this warp's TMA stores are complete
+      __syncwarp();
     }
   }
 
@@ -717,6 +777,16 @@ int make_scale_map(CUtensorMap* map, const uint8_t* base, int64_t experts, int64
   const uint32_t box[3] = {128, 16, 1};
   return make_map(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, grouped ? 3 : 2, base, dims, strides, box,
                   CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+// bf16 output [experts, rows, n] with boxes of 64 columns (128 bytes) by 32 rows, 128-byte
+// swizzle (the epilogue's staging layout).
+int make_output_map(CUtensorMap* map, const void* base, int64_t experts, int64_t rows, int64_t n, bool grouped) {
+  const uint64_t dims[3] = {static_cast<uint64_t>(n), static_cast<uint64_t>(rows), static_cast<uint64_t>(experts)};
+  const uint64_t strides[2] = {static_cast<uint64_t>(n * 2), static_cast<uint64_t>(rows * n * 2)};
+  const uint32_t box[3] = {64, 32, 1};
+  return make_map(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, grouped ? 3 : 2, base, dims, strides, box,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // bf16 low-rank operand [rows, r] with boxes of 64 values (128 bytes) by 128 rows.
@@ -777,6 +847,8 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream) {
   if (kSwiGLU) {
     if ((st = make_operand_map(&maps.b2, g.b2, E, n, k, kGrouped)) != NVFP4_OK) return st;
     if ((st = make_scale_map(&maps.sfb2, g.b2_sf, E, n, k, kGrouped)) != NVFP4_OK) return st;
+  } else {
+    if ((st = make_output_map(&maps.out, g.out, E, m, n, kGrouped)) != NVFP4_OK) return st;
   }
   if (kLowRank) {
     if ((st = make_lowrank_map(&maps.d, g.d, m, g.r)) != NVFP4_OK) return st;
@@ -814,14 +886,15 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream) {
   // number of 2-CTA clusters that fit on the device at once (the persistent grid size).
   static int max_clusters = 0;
   if (max_clusters == 0) {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes<kSwiGLU>) !=
+        cudaSuccess) {
       cudaGetLastError();
       return NVFP4_ERR_CUDA;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(info.sm_count / 2 * 2);
     cfg.blockDim = dim3(kThreads<kSwiGLU>);
-    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.dynamicSmemBytes = kSmemBytes<kSwiGLU>;
     int clusters = 0;
     if (cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg) != cudaSuccess || clusters <= 0) {
       cudaGetLastError();
@@ -834,7 +907,7 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream) {
   if (tiles >= (int64_t(1) << 31)) return NVFP4_ERR_INVALID_ARGUMENT;
   const int64_t max_pairs = max_clusters;
   const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
-  kernel<<<2 * pairs, kThreads<kSwiGLU>, kSmemBytes, stream>>>(maps, p);
+  kernel<<<2 * pairs, kThreads<kSwiGLU>, kSmemBytes<kSwiGLU>, stream>>>(maps, p);
   return launch_status();
 }
 
