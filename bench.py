@@ -1,25 +1,32 @@
 """Benchmark of the NVFP4 linear-layer hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl nvfp4|reference]
-                    [--workload swiglu_block|quant_dense|quant_masked|quant_silu|grouped_moe|lowrank|pr1_linear]
-                    [--rank-lr R]
+                    [--workload swiglu_block|quant_dense|quant_masked|quant_silu|grouped_moe|grouped_swiglu|
+                                lowrank|pr1_linear]
+                    [--rank-lr R] [--swiglu-path fused|unfused] [--no-pdl]
 
 Default workload: the dense NVFP4 SwiGLU shared-expert block, M = 8192 tokens, hidden
 5120, intermediate 8192.  One step is the whole hot path over one batch:
     global amax of x (dynamic activation scale; also yields the gate/up alpha)
     -> quantize x [8192, 5120]
-    -> gate/up GEMM [8192 x 5120] @ [16384 x 5120]^T  (bf16 out, [gate | up])
-    -> SiLU-and-mul fused quantize [8192, 16384] -> [8192, 8192] (calibrated static scale)
+    -> gate/up GEMM [8192 x 5120] @ [16384 x 5120]^T whose epilogue forms
+       h = bf16(silu(gate) * up) and quantizes it with the calibrated static scale of h
+       (--swiglu-path unfused: the GEMM writes bf16 [gate | up] and the SiLU-and-mul
+       quantizer runs as its own kernel)
     -> down GEMM [8192 x 8192] @ [5120 x 8192]^T  (bf16 out)
 Weights are quantized once before timing (offline weight quantization), and the static
 activation scale of h is calibrated once, as a deployed layer would.
 
-Timing: the step is captured once into a CUDA graph with a CUDA event node before and
-after every kernel; W warm-up replays, then K timed replays bracketed by a barrier and a
-device synchronize.  L2 is flushed (a 512 MB write) before every replay, outside the
-events; the step time is the device time between the first and the last event.  The value is whole-job throughput (sum over
-ranks of the work / the max over ranks of the device time).  With N > 1 every rank runs
-its own independent batch (data parallel, no collective on the data path): weak scaling.
+Timing: the step is captured into a CUDA graph with event nodes only at its start and
+end (its kernels chained by programmatic dependent launch unless --no-pdl), and into a
+second graph with an event node around every kernel.  W warm-up replays, then K timed
+replays of each graph bracketed by a barrier and a device synchronize.  Before every
+replay L2 is flushed outside the events (a 512 MB write, then a 256 MB read that leaves
+no dirty line of the flush to be written back inside the timing).  ms_per_step and the
+value come from the step graph; per-kernel times (parts, roofline) from the kernel
+graph.  The value is whole-job throughput (sum over ranks of the work / the max over
+ranks of the device time).  With N > 1 every rank runs its own independent batch (data
+parallel, no collective on the data path): weak scaling.
 
 ``--impl reference`` times the CPU oracle (the plain C reference implementation) on a
 bounded sample of the same workload on this machine's host cores.
@@ -43,7 +50,10 @@ import nvfp4_synth as S  # noqa: E402
 METRIC = "NVFP4 GEMM TFLOPS (% of FP4 peak); quantize HBM GB/s (% of HBM peak)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP4_OVER_BF16 = 4.0          # nominal dense ratio 9 PFLOP/s / 2.25 PFLOP/s
-L2_FLUSH_BYTES = 512 << 20
+L2_FLUSH_BYTES = 512 << 20      # written before every step (L2 is 126 MB) ...
+L2_CLEAN_BYTES = 256 << 20      # ... then read, so the flush's dirty lines are written back outside the timing
+L2_NOTE = ("flushed before every step outside the timed events: 512 MB written, then 256 MB read so that "
+           "no dirty line of the flush is written back inside the timing")
 
 
 def load_peaks():
@@ -309,7 +319,7 @@ class SwigluBlock(Workload):
                 "tokens": self.M, "hidden": self.H, "intermediate": self.I,
                 "path": ("gate/up GEMM with the SiLU*mul NVFP4 quantizer in its epilogue" if self.fused else
                          "gate/up GEMM to bf16, then the SiLU*mul quantizer kernel"),
-                "l2": "flushed between steps (512 MB write, outside the timed events)"}
+                "l2": L2_NOTE}
 
 
 class QuantDense(Workload):
@@ -344,7 +354,7 @@ class QuantDense(Workload):
 
     def config(self):
         return {"workload": "quantize bf16 [8192,8192] ~N(0,1) with 0.1% outliers x50 (amax + quantize)",
-                "l2": "flushed between steps"}
+                "l2": L2_NOTE}
 
 
 class QuantMasked(Workload):
@@ -385,7 +395,7 @@ class QuantMasked(Workload):
     def config(self):
         w = "[8,4096,2*7168] silu(gate)*up fused" if self.silu else "[8,4096,7168]"
         return {"workload": f"masked batched quantize {w}, valid rows per item U[0,4096] (sum {int(self.mask_host.sum())})",
-                "l2": "flushed between steps"}
+                "l2": L2_NOTE}
 
 
 class GroupedMoE(Workload):
@@ -430,7 +440,7 @@ class GroupedMoE(Workload):
     def config(self):
         return {"workload": f"masked grouped NVFP4 GEMM E=16 Mmax=2048 K=5120 N=8192, valid rows "
                             f"min(Poisson(512),2048) (sum {int(self.mask_host.sum())})",
-                "l2": "flushed between steps"}
+                "l2": L2_NOTE}
 
 
 class GroupedSwiglu(Workload):
@@ -514,7 +524,7 @@ class GroupedSwiglu(Workload):
                             f"intermediate 8192; masked quantize, grouped gate/up GEMM with the SiLU*mul NVFP4 "
                             f"epilogue, grouped down GEMM; static per-expert activation scales",
                 "experts": self.E, "mmax": self.mmax, "hidden": self.H, "intermediate": self.I,
-                "l2": "flushed between steps (512 MB write, outside the timed events)"}
+                "l2": L2_NOTE}
 
 
 class LowRank(Workload):
@@ -555,7 +565,7 @@ class LowRank(Workload):
 
     def config(self):
         return {"workload": f"low-rank-corrected NVFP4 GEMM M=4096 K=3072 N=3072 r={self.r} + bias",
-                "l2": "flushed between steps"}
+                "l2": L2_NOTE}
 
 
 class PR1Linear(Workload):
@@ -593,7 +603,7 @@ class PR1Linear(Workload):
         return self.x_host, self.x, self.out
 
     def config(self):
-        return {"workload": "single NVFP4 linear x[128,256] W[256,256] (latency-bound)", "l2": "flushed between steps"}
+        return {"workload": "single NVFP4 linear x[128,256] W[256,256] (latency-bound)", "l2": L2_NOTE}
 
 
 def make_workload(name, nv, rank_lr, swiglu_path="fused"):
@@ -788,6 +798,8 @@ def main():
                     help="swiglu_block: SiLU*mul quantization in the gate/up GEMM epilogue, or as its own kernel")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-pdl", action="store_true",
+                    help="launch without programmatic dependent launch (the library default is on)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -803,8 +815,15 @@ def main():
     nv.load_library()
     wl = make_workload(args.workload, nv, args.rank_lr, args.swiglu_path)
     launches = wl.launches()
+    if args.no_pdl:
+        nv.nvfp4_set_pdl(False)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    clean = torch.ones(L2_CLEAN_BYTES // 4, dtype=torch.float32, device="cuda")
     stream = torch.cuda.Stream()
+
+    def flush_l2():
+        flush.zero_()
+        clean.max()
 
     def step(evs=None):
         for i, (_, fn) in enumerate(launches):
@@ -815,10 +834,13 @@ def main():
             evs[len(launches)].record()
 
     # One eager pass on the launch stream (allocates the library's per-stream scratch),
-    # then the step is captured once into a CUDA graph with an external event node
-    # around every kernel, so host launch overhead never appears inside the timed
-    # kernels.  Should the driver refuse timing on graph event nodes, every kernel is
-    # captured into its own graph and timed by events recorded around its replay.
+    # then two CUDA graphs of the step.  The step graph has an external event node only at
+    # its start and end, so consecutive kernels keep their programmatic-dependent-launch
+    # edges: it gives the step time (value).  The kernel graph has an event node around
+    # every kernel (consecutive kernels then cannot overlap): it gives each kernel's own
+    # duration (parts, roofline).  Both run inside the timed region, one pass each.  Should
+    # the driver refuse timing on graph event nodes, every kernel is captured into its own
+    # graph and timed by events recorded around its replay (no overlap either way).
     with torch.cuda.stream(stream):
         step()
     torch.cuda.synchronize()
@@ -827,23 +849,35 @@ def main():
         for g in graphs:
             g.replay()
 
-    events = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(launches) + 1)]
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        step(events)
+    step_events = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+    kernel_events = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(launches) + 1)]
+    graph_s, graph_k = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_s, stream=stream):
+        step_events[0].record()
+        step()
+        step_events[1].record()
+    with torch.cuda.graph(graph_k, stream=stream):
+        step(kernel_events)
     torch.cuda.synchronize()
-    timing_mode = "event nodes inside one CUDA graph per step"
+    timing_mode = ("step: one CUDA graph per step, event nodes at its start and end (kernels chained by "
+                   "programmatic dependent launch: %s); kernels: a second pass with an event node around every "
+                   "kernel" % ("on" if nv.nvfp4_get_pdl() else "off"))
 
     def run_step_graph():
-        graph.replay()
+        graph_s.replay()
         stream.synchronize()
-        return [events[i].elapsed_time(events[i + 1]) for i in range(len(launches))] + \
-               [events[0].elapsed_time(events[-1])]
+        return step_events[0].elapsed_time(step_events[1])
 
-    run_step = run_step_graph
+    def run_kernels_graph():
+        graph_k.replay()
+        stream.synchronize()
+        return [kernel_events[i].elapsed_time(kernel_events[i + 1]) for i in range(len(launches))]
+
+    run_step, run_kernels = run_step_graph, run_kernels_graph
     try:
         with torch.cuda.stream(stream):
             run_step()
+            run_kernels()
     except Exception:                                      # noqa: BLE001
         torch.cuda.synchronize()
         graphs = []
@@ -853,43 +887,49 @@ def main():
                 fn()
             graphs.append(g)
         outer = [torch.cuda.Event(enable_timing=True) for _ in range(len(launches) + 1)]
-        timing_mode = "one CUDA graph per kernel, events around each replay"
+        timing_mode = "one CUDA graph per kernel, events around each replay (step time = first to last event)"
 
-        def run_step_split():
+        def run_kernels_split():
             for i, g in enumerate(graphs):
                 outer[i].record()
                 g.replay()
             outer[-1].record()
             stream.synchronize()
-            return [outer[i].elapsed_time(outer[i + 1]) for i in range(len(launches))] + \
-                   [outer[0].elapsed_time(outer[-1])]
+            return [outer[i].elapsed_time(outer[i + 1]) for i in range(len(launches))]
 
-        run_step = run_step_split
-        graph = None
+        def run_step_split():
+            run_kernels_split()
+            return outer[0].elapsed_time(outer[-1])
+
+        run_step, run_kernels = run_step_split, run_kernels_split
+        graph_s = None
 
         def replay_step():
             replay_all(graphs)
     else:
         def replay_step():
-            graph.replay()
+            graph_s.replay()
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
-            flush.zero_()
+            flush_l2()
             replay_step()
     torch.cuda.synchronize()
     if nv.nvfp4_device_status(clear=True) != 0:
         raise SystemExit("device-side timeout during warm-up")
 
-    samples = []
+    step_ms, samples = [], []
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
         t_wall = time.perf_counter()
         with torch.cuda.stream(stream):
             for s in range(args.steps):
-                flush.zero_()
-                samples.append(run_step())
+                flush_l2()
+                step_ms.append(run_step())
+            for s in range(args.steps):
+                flush_l2()
+                samples.append(run_kernels())
         torch.cuda.synchronize()
         t_wall = time.perf_counter() - t_wall
     barrier(world)
@@ -898,7 +938,6 @@ def main():
         raise SystemExit(f"device-side timeout in the timed region (status {status})")
 
     per_kernel = {name: [smp[i] for smp in samples] for i, (name, _) in enumerate(launches)}
-    step_ms = [smp[-1] for smp in samples]
     total_ms = sum(step_ms)
     total_ms_max = max_over_ranks(world, total_ms)
     work_all = sum_over_ranks(world, wl.work() * args.steps)
@@ -938,7 +977,7 @@ def main():
         e_end = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
         with torch.cuda.stream(stream):
             for s in range(args.steps + args.warmup):
-                flush.zero_()
+                flush_l2()
                 i = s - args.warmup
                 if i >= 0:
                     e_start[i].record()

@@ -258,6 +258,21 @@ NVFP4_API int nvfp4_grouped_gemm_silu_mul_quantize_masked(
     int64_t n, int64_t k, nvfp4_stream_t stream);
 
 /*
+ * Programmatic dependent launch [FI5 mm_nvfp4_svdquant, Parameters: enable_pdl, which
+ * defaults to the device default].  When enabled (the default: compute capability 10.0
+ * supports it), every kernel of the library is launched with programmatic stream
+ * serialization: it may start while the preceding kernel of its stream is finishing, runs
+ * its set-up (barriers, tensor memory, descriptor prefetch), and waits for that kernel to
+ * complete before its first global memory access; it lets the next kernel start in the
+ * same way.  Results are identical either way; only launch latency overlaps.  The setting
+ * is process-wide and applies to launches made after the call, including launches
+ * captured into CUDA graphs.  nvfp4_set_pdl returns NVFP4_OK; nvfp4_get_pdl returns the
+ * current setting (0 or 1).
+ */
+NVFP4_API int nvfp4_set_pdl(int enable);
+NVFP4_API int nvfp4_get_pdl(void);
+
+/*
  * Device-side status word of the current device.  GEMM kernels bound every wait; a
  * wait that runs out records NVFP4_ERR_DEVICE_TIMEOUT here and the kernel returns
  * without hanging the GPU.  Synchronizes the device, then stores the word in

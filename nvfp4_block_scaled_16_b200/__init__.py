@@ -26,5 +26,7 @@ from .binding import (  # noqa: F401
     nvfp4_gemm_lowrank_bias,
     nvfp4_gemm_silu_mul_quantize,
     nvfp4_grouped_gemm_silu_mul_quantize_masked,
+    nvfp4_set_pdl,
+    nvfp4_get_pdl,
     nvfp4_device_status,
 )

@@ -27,6 +27,8 @@ EXPORTED_SYMBOLS = (
     "nvfp4_gemm_lowrank_bias",
     "nvfp4_gemm_silu_mul_quantize",
     "nvfp4_grouped_gemm_silu_mul_quantize_masked",
+    "nvfp4_set_pdl",
+    "nvfp4_get_pdl",
     "nvfp4_device_status",
 )
 
@@ -48,6 +50,8 @@ _SIGNATURES = {
     "nvfp4_gemm_lowrank_bias": (_INT, [_P, _P, _P, _P, _P, _P, _P, _I64, _P, _P, _I64, _I64, _I64, _P]),
     "nvfp4_gemm_silu_mul_quantize": (_INT, [_P] * 11 + [_I64, _I64, _I64, _P]),
     "nvfp4_grouped_gemm_silu_mul_quantize_masked": (_INT, [_P] * 12 + [_I64, _I64, _I64, _I64, _P]),
+    "nvfp4_set_pdl": (_INT, [_INT]),
+    "nvfp4_get_pdl": (_INT, []),
     "nvfp4_device_status": (_INT, [ctypes.POINTER(_INT), _INT]),
 }
 
@@ -273,6 +277,15 @@ def nvfp4_grouped_gemm_silu_mul_quantize_masked(a, b_gate, b_up, a_sf, b_gate_sf
             _stream(stream))
     _check("nvfp4_grouped_gemm_silu_mul_quantize_masked", st)
     return q_out, sf_out
+
+
+def nvfp4_set_pdl(enable: bool) -> None:
+    """Launch subsequent kernels with (True) or without programmatic dependent launch."""
+    _check("nvfp4_set_pdl", load_library().nvfp4_set_pdl(1 if enable else 0))
+
+
+def nvfp4_get_pdl() -> bool:
+    return bool(load_library().nvfp4_get_pdl())
 
 
 def nvfp4_device_status(clear: bool = True) -> int:

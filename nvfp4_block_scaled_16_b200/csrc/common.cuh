@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstdint>
+#include <utility>
 
 #include "nvfp4.h"
 
@@ -29,6 +30,44 @@ int stream_workspace(cudaStream_t stream, uint32_t** out);
 
 // Maps the last CUDA error (launch configuration, ...) to a status code.
 int launch_status();
+
+// Whether kernels are launched with programmatic dependent launch (nvfp4_set_pdl).
+bool pdl_enabled();
+
+// Launches `kernel` on `stream`, with the programmatic-stream-serialization attribute when
+// PDL is enabled: the kernel may then start while its predecessor in the stream finishes,
+// and every kernel of this library waits (griddepcontrol.wait) before its first global
+// memory access, so the predecessor's results are complete when it reads or overwrites
+// them.  Returns NVFP4_OK or NVFP4_ERR_CUDA.
+template <typename... KernelArgs, typename... Args>
+int launch_kernel(void (*kernel)(KernelArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                  Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  if (cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) != cudaSuccess) {
+    cudaGetLastError();
+    return NVFP4_ERR_CUDA;
+  }
+  return NVFP4_OK;
+}
+
+// ---- device side --------------------------------------------------------------------
+
+// Lets the next kernel of the stream (launched with PDL) start its launch and prologue.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Waits until the preceding kernel of the stream has completed and its memory operations
+// are visible (returns at once when the kernel was not launched with PDL).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 

@@ -1,4 +1,5 @@
 // context.cu -- per-device state, per-stream reduction scratch, status codes.
+#include <atomic>
 #include <map>
 #include <mutex>
 #include <utility>
@@ -9,6 +10,7 @@ namespace nvfp4 {
 namespace {
 
 std::mutex g_mu;
+std::atomic<int> g_pdl{1};      // programmatic dependent launch, on by default (sm_100 supports it)
 DeviceInfo g_dev[64];
 std::map<std::pair<int, cudaStream_t>, uint32_t*> g_ws;
 
@@ -76,6 +78,8 @@ int stream_workspace(cudaStream_t stream, uint32_t** out) {
   return NVFP4_OK;
 }
 
+bool pdl_enabled() { return g_pdl.load(std::memory_order_relaxed) != 0; }
+
 int launch_status() {
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
@@ -117,6 +121,13 @@ int64_t nvfp4_scale_bytes(int64_t rows, int64_t k) {
   const int64_t cp = (k / 16 + 3) / 4 * 4;
   return rp * cp;
 }
+
+int nvfp4_set_pdl(int enable) {
+  nvfp4::g_pdl.store(enable ? 1 : 0, std::memory_order_relaxed);
+  return NVFP4_OK;
+}
+
+int nvfp4_get_pdl(void) { return nvfp4::g_pdl.load(std::memory_order_relaxed); }
 
 int nvfp4_device_status(int* status_out, int clear) {
   if (!status_out) return NVFP4_ERR_INVALID_ARGUMENT;

@@ -51,6 +51,7 @@
 // Every mbarrier wait is bounded (about one second of global time); a wait that runs out
 // records NVFP4_ERR_DEVICE_TIMEOUT in the device status word and the CTA unwinds without
 // hanging the GPU.
+#include <cstddef>
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -96,13 +97,26 @@ struct __align__(8) Control {
   int32_t abort;
   int32_t prefix[kMaxExperts + 1];   // grouped: prefix sums of pair tiles per expert
 };
-// bf16 epilogue: one 32-row x 64-column bf16 staging tile (4 KB, 128-byte swizzle) per
-// epilogue warp, written to global memory by a TMA store.
+// bf16 epilogue: 32-row x 64-column bf16 staging tiles (4 KB, 128-byte swizzle) per
+// epilogue warp, written to global memory by TMA stores; two per warp (one store in flight
+// while the next tile is written) where shared memory allows, one in the grouped kernels
+// (whose expert prefix table takes the room).
 constexpr int kStoreTileBytes = 32 * 128;
-template <bool kSwiGLU>
-constexpr int kStagingBytes = kSwiGLU ? 0 : kEpiWarps<false> * kStoreTileBytes;
-template <bool kSwiGLU>
-constexpr int kSmemBytes = kStages * kStageBytes + kStagingBytes<kSwiGLU> + sizeof(Control) + 1024;
+template <bool kGrouped, bool kSwiGLU>
+constexpr int kStagingBuffers = kSwiGLU ? 0 : (kGrouped ? 1 : 2);
+template <bool kGrouped, bool kSwiGLU>
+constexpr int kStagingBytes = kStagingBuffers<kGrouped, kSwiGLU> * kEpiWarps<false> * kStoreTileBytes;
+// The expert prefix table (the last member of Control) is only allocated for grouped kernels.
+template <bool kGrouped>
+constexpr int kControlBytes = kGrouped ? static_cast<int>(sizeof(Control))
+                                       : static_cast<int>(offsetof(Control, prefix)) + 8;
+template <bool kGrouped, bool kSwiGLU>
+constexpr int kSmemBytes =
+    kStages * kStageBytes + kStagingBytes<kGrouped, kSwiGLU> + kControlBytes<kGrouped> + 1024;
+constexpr int kMaxDynamicSmem = 227 * 1024;      // sm_100 opt-in limit per block
+static_assert(kSmemBytes<false, false> <= kMaxDynamicSmem && kSmemBytes<true, false> <= kMaxDynamicSmem &&
+                  kSmemBytes<false, true> <= kMaxDynamicSmem && kSmemBytes<true, true> <= kMaxDynamicSmem,
+              "shared memory layout exceeds the per-block limit");
 
 // Instruction descriptors (tcgen05 "instruction descriptor" bit fields).
 //   kind::mxf4nvf4: A/B format E2M1 (1) at bits 7..9 / 10..12, both K-major, N>>3 at
@@ -231,7 +245,9 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void*
                : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Waits until at most N of this thread's committed bulk groups have not yet read their source.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
@@ -406,7 +422,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kSwiGLU>, 1
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* staging = smem + kStages * kStageBytes;     // 1024-byte aligned (the ring is 190 KB)
-  Control& ctl = *reinterpret_cast<Control*>(staging + kStagingBytes<kSwiGLU>);
+  Control& ctl = *reinterpret_cast<Control*>(staging + kStagingBytes<kGrouped, kSwiGLU>);
   volatile int32_t* abort = &ctl.abort;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -425,17 +441,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kSwiGLU>, 1
     ctl.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if constexpr (kGrouped) {
-    if (threadIdx.x == 32) {
-      int acc = 0;
-      ctl.prefix[0] = 0;
-      for (int e = 0; e < p.experts; ++e) {
-        const int valid = min(max(p.mask[e], 0), p.m);
-        acc += (valid + kTileM - 1) / kTileM * p.n_tiles;
-        ctl.prefix[e + 1] = acc;
-      }
-    }
-  }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&ctl.tmem_base)),
                  "r"(kTmemCols)
@@ -447,6 +452,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kSwiGLU>, 1
   cluster_sync();      // the leader's barriers are initialized before the peer signals them
   tc_fence_after();
   const uint32_t tmem = ctl.tmem_base;
+
+  // Programmatic dependent launch: the set-up above touched only this CTA's own resources;
+  // global memory is accessed only after the preceding kernel of the stream has finished.
+  pdl_launch_dependents();
+  pdl_wait();
+  if constexpr (kGrouped) {
+    if (threadIdx.x == 32) {
+      int acc = 0;
+      ctl.prefix[0] = 0;
+      for (int e = 0; e < p.experts; ++e) {
+        const int valid = min(max(p.mask[e], 0), p.m);
+        acc += (valid + kTileM - 1) / kTileM * p.n_tiles;
+        ctl.prefix[e + 1] = acc;
+      }
+    }
+    __syncthreads();
+  }
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -597,19 +619,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kSwiGLU>, 1
     const uint32_t acc_empty_leader = map_to_rank(&ctl.acc_empty, 0);
     uint32_t tcount = 0;
     TileCoord t;
+    uint32_t nstore = 0;                       // TMA stores issued by this warp (bf16 epilogue)
     for (int tile = pair; tile_coord<kGrouped>(p, ctl, tile, t); tile += pairs, ++tcount) {
+      // per-tile scalars, loaded before the wait so their latency hides behind the mainloop
+      const float alpha = __ldg(p.alpha + t.expert);
+      float gsf = 0.0f, alpha_u = 0.0f;
+      if constexpr (kSwiGLU) {
+        gsf = __ldg(p.gsf_h + t.expert);
+        alpha_u = __ldg(p.alpha_up + t.expert);
+      }
       if (!mbar_wait(&ctl.acc_full, tcount & 1, abort, p.status)) break;
       tc_fence_after();
       const uint32_t buf = tcount & 1;
       const uint32_t col0 = buf ? kAccOverlapCol : 0u;
-      const float alpha = __ldg(p.alpha + t.expert);
       const int row = t.m_tile * kTileM + static_cast<int>(rank) * kBM + row_in_tile;
       const bool row_ok = row < t.valid_rows;
       if constexpr (kSwiGLU) {
         // h columns [128 n_tile, 128 n_tile + 128): g in accumulator columns [0, 128), u in
         // [128, 256); this warp's half of them is loaded whole, then the accumulator released.
-        const float gsf = __ldg(p.gsf_h + t.expert);
-        const float alpha_u = __ldg(p.alpha_up + t.expert);
         const bool pad_row = !kGrouped && row >= p.m && row < p.rows_pad;   // zero scales
         uint8_t* q_row = p.q + (static_cast<int64_t>(t.expert) * p.m + row) * (p.n / 2) + t.n_tile * 64;
         uint8_t* sf_e = p.sf + static_cast<int64_t>(t.expert) * p.sf_item_stride;
@@ -658,12 +685,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kSwiGLU>, 1
         // the mask stay untouched.
         const int slab_row = t.m_tile * kTileM + static_cast<int>(rank) * kBM + quarter * 32;
         const bool use_tma = kGrouped ? slab_row + 32 <= t.valid_rows : slab_row < p.m;
-        uint8_t* stage_tile = staging + (warp - 2) * kStoreTileBytes;
-        const uint32_t stage_row = smem_u32(stage_tile) + lane * 128;
+        constexpr int kBufs = kStagingBuffers<kGrouped, kSwiGLU>;
+        uint8_t* stage_warp = staging + (warp - 2) * kBufs * kStoreTileBytes;
         __nv_bfloat16* out_row = p.out + (static_cast<int64_t>(t.expert) * p.m + row) * p.n;
         for (int i = 0; i < 4; ++i) {
           // accumulator 0 drains its last 64 columns first, accumulator 1 its first 64
           const int sub = buf ? i : 3 - i;
+          const int col_base = t.n_tile * kBN + sub * 64;
+          uint4 bias8[8];                      // issued before the TMEM load to hide its latency
+#pragma unroll
+          for (int g = 0; g < 8; ++g)
+            bias8[g] = (p.bias && col_base + 8 * g < p.n)
+                           ? __ldg(reinterpret_cast<const uint4*>(p.bias + col_base + 8 * g))
+                           : make_uint4(0u, 0u, 0u, 0u);
           uint32_t v[64];
           tmem_load_64(tmem + col0 + sub * 64 + lane_base, v);
           tmem_wait_ld<64>(v);
@@ -672,7 +706,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kSwiGLU>, 1
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
           }
-          const int col_base = t.n_tile * kBN + sub * 64;
           if (col_base >= p.n || !(use_tma || row_ok)) continue;
           uint4 o[8];
 #pragma unroll
@@ -682,8 +715,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kSwiGLU>, 1
 #pragma unroll
             for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * g + e]);
             if (p.bias && col < p.n) {
-              const uint4 bw = __ldg(reinterpret_cast<const uint4*>(p.bias + col));
-              const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w};
+              const uint32_t bb[4] = {bias8[g].x, bias8[g].y, bias8[g].z, bias8[g].w};
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
                 f[2 * e] = __fmaf_rn(alpha, f[2 * e], __uint_as_float(bb[e] << 16));
@@ -699,7 +731,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kSwiGLU>, 1
             o[g].w = pack_bf16x2(f[6], f[7]);
           }
           if (use_tma) {
-            if (lane == 0) bulk_wait_read();      // the previous store has read the staging tile
+            uint8_t* stage_tile = stage_warp + (nstore % kBufs) * kStoreTileBytes;
+            const uint32_t stage_row = smem_u32(stage_tile) + lane * 128;
+            if (lane == 0) bulk_wait_read<kBufs - 1>();   // the store that last used this tile has read it
             __syncwarp();
             // 128-byte swizzle: 16-byte chunk g of row r sits at chunk position g ^ (r % 8)
 #pragma unroll
@@ -714,6 +748,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kSwiGLU>, 1
               }
               bulk_commit();
             }
+            ++nstore;
           } else {
 #pragma unroll
             for (int g = 0; g < 8; ++g)
@@ -886,7 +921,7 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream) {
   // number of 2-CTA clusters that fit on the device at once (the persistent grid size).
   static int max_clusters = 0;
   if (max_clusters == 0) {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes<kSwiGLU>) !=
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes<kGrouped, kSwiGLU>) !=
         cudaSuccess) {
       cudaGetLastError();
       return NVFP4_ERR_CUDA;
@@ -894,7 +929,7 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(info.sm_count / 2 * 2);
     cfg.blockDim = dim3(kThreads<kSwiGLU>);
-    cfg.dynamicSmemBytes = kSmemBytes<kSwiGLU>;
+    cfg.dynamicSmemBytes = kSmemBytes<kGrouped, kSwiGLU>;
     int clusters = 0;
     if (cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg) != cudaSuccess || clusters <= 0) {
       cudaGetLastError();
@@ -907,8 +942,8 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream) {
   if (tiles >= (int64_t(1) << 31)) return NVFP4_ERR_INVALID_ARGUMENT;
   const int64_t max_pairs = max_clusters;
   const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
-  kernel<<<2 * pairs, kThreads<kSwiGLU>, kSmemBytes<kSwiGLU>, stream>>>(maps, p);
-  return launch_status();
+  return launch_kernel(kernel, dim3(2 * pairs), dim3(kThreads<kSwiGLU>), kSmemBytes<kGrouped, kSwiGLU>, stream, maps,
+                       p);
 }
 
 }  // namespace

@@ -65,6 +65,8 @@ struct QuantParams {
 
 template <bool kSilu, int kUnroll>
 __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantParams p) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int item = blockIdx.y;
   int valid = p.m;
   if (p.mask) valid = min(max(__ldg(p.mask + item), 0), p.m);
@@ -185,6 +187,8 @@ __device__ void reduce_and_finalize(float local, uint32_t* ws, int item, int ite
 __global__ void __launch_bounds__(kThreads) amax_dense_kernel(const uint16_t* x, int64_t numel, uint32_t* ws,
                                                               float* amax_out, float* gsf_out,
                                                               const float* other_amax, float* alpha_out) {
+  pdl_launch_dependents();
+  pdl_wait();
   float m = 0.0f;
   const int64_t nvec = numel / 8;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
@@ -210,6 +214,8 @@ template <bool kSilu>
 __global__ void __launch_bounds__(kThreads) amax_batched_kernel(const uint16_t* x, int32_t m, int32_t k,
                                                                 const int32_t* mask, uint32_t* ws,
                                                                 float* amax_out, float* gsf_out) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int item = blockIdx.y;
   const int valid = mask ? min(max(__ldg(mask + item), 0), m) : m;
   const int64_t width = kSilu ? 2 * static_cast<int64_t>(k) : k;
@@ -271,13 +277,11 @@ int launch_quantize(const void* x, int64_t b, int64_t m, int64_t k, bool silu, c
   if (silu) {
     constexpr int U = 2;
     dim3 grid(static_cast<unsigned>((p.blocks + kThreads * U - 1) / (kThreads * U)), static_cast<unsigned>(b));
-    quantize_kernel<true, U><<<grid, kThreads, 0, stream>>>(p);
-  } else {
-    constexpr int U = 4;
-    dim3 grid(static_cast<unsigned>((p.blocks + kThreads * U - 1) / (kThreads * U)), static_cast<unsigned>(b));
-    quantize_kernel<false, U><<<grid, kThreads, 0, stream>>>(p);
+    return launch_kernel(quantize_kernel<true, U>, grid, dim3(kThreads), 0, stream, p);
   }
-  return launch_status();
+  constexpr int U = 4;
+  dim3 grid(static_cast<unsigned>((p.blocks + kThreads * U - 1) / (kThreads * U)), static_cast<unsigned>(b));
+  return launch_kernel(quantize_kernel<false, U>, grid, dim3(kThreads), 0, stream, p);
 }
 
 }  // namespace
@@ -303,9 +307,8 @@ int nvfp4_global_scale(const void* x_bf16, int64_t numel, float* amax_out, float
   const int64_t nvec = numel / 8;
   int64_t blocks = (nvec + kThreads * 4 - 1) / (kThreads * 4);
   blocks = blocks < 1 ? 1 : (blocks > info.sm_count * 8 ? info.sm_count * 8 : blocks);
-  amax_dense_kernel<<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
-      static_cast<const uint16_t*>(x_bf16), numel, ws, amax_out, gsf_out, other_amax, alpha_out);
-  return launch_status();
+  return launch_kernel(amax_dense_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), 0, stream,
+                       static_cast<const uint16_t*>(x_bf16), numel, ws, amax_out, gsf_out, other_amax, alpha_out);
 }
 
 int nvfp4_global_scale_batched(const void* x_bf16, int64_t b, int64_t m, int64_t k, const int32_t* mask,
@@ -329,13 +332,8 @@ int nvfp4_global_scale_batched(const void* x_bf16, int64_t b, int64_t m, int64_t
   gx = gx < 1 ? 1 : (gx > cap ? cap : gx);
   dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(b));
   const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
-  if (silu_mul)
-    amax_batched_kernel<true><<<grid, kThreads, 0, stream>>>(x, static_cast<int32_t>(m), static_cast<int32_t>(k),
-                                                             mask, ws, amax_out, gsf_out);
-  else
-    amax_batched_kernel<false><<<grid, kThreads, 0, stream>>>(x, static_cast<int32_t>(m), static_cast<int32_t>(k),
-                                                              mask, ws, amax_out, gsf_out);
-  return launch_status();
+  return launch_kernel(silu_mul ? amax_batched_kernel<true> : amax_batched_kernel<false>, grid, dim3(kThreads), 0,
+                       stream, x, static_cast<int32_t>(m), static_cast<int32_t>(k), mask, ws, amax_out, gsf_out);
 }
 
 int nvfp4_quantize(const void* x_bf16, int64_t m, int64_t k, const float* gsf, uint8_t* q_out, uint8_t* sf_out,
@@ -438,11 +436,6 @@ extern "C" int nvfp4_global_scale_batched_noalloc(const void* x_bf16, int64_t b,
   gx = gx < 1 ? 1 : (gx > cap ? cap : gx);
   dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(b));
   const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
-  if (silu_mul)
-    amax_batched_kernel<true><<<grid, kThreads, 0, stream>>>(x, static_cast<int32_t>(m), static_cast<int32_t>(k), mask,
-                                                             scratch, amax_out, gsf_out);
-  else
-    amax_batched_kernel<false><<<grid, kThreads, 0, stream>>>(x, static_cast<int32_t>(m), static_cast<int32_t>(k), mask,
-                                                              scratch, amax_out, gsf_out);
-  return launch_status();
+  return launch_kernel(silu_mul ? amax_batched_kernel<true> : amax_batched_kernel<false>, grid, dim3(kThreads), 0,
+                       stream, x, static_cast<int32_t>(m), static_cast<int32_t>(k), mask, scratch, amax_out, gsf_out);
 }

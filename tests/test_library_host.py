@@ -139,3 +139,12 @@ def test_grouped_silu_mul_gemm_argument_checks(lib):
     args[6] = None                          # mask required
     assert lib.nvfp4_grouped_gemm_silu_mul_quantize_masked(*args, 2, 128, 256, 256, None) == INVALID
     assert lib.nvfp4_grouped_gemm_silu_mul_quantize_masked(*([A16] * 12), 0, 128, 256, 256, None) == 0  # empty
+
+
+def test_pdl_switch(lib):
+    import nvfp4_block_scaled_16_b200 as nv
+    assert nv.nvfp4_get_pdl() is True              # on by default
+    nv.nvfp4_set_pdl(False)
+    assert nv.nvfp4_get_pdl() is False
+    nv.nvfp4_set_pdl(True)
+    assert nv.nvfp4_get_pdl() is True
