@@ -568,6 +568,65 @@ class LowRank(Workload):
                 "l2": L2_NOTE}
 
 
+class SvdquantLinear(Workload):
+    """The whole SVDQuant NVFP4 linear layer at the low-rank GEMM's sizes: smooth quantize of x
+    and the LoRA-down product in one pass (nvfp4_quantize_smooth_lora_down), then the residual
+    FP4 GEMM with the rank-r correction and bias.  The activation scale of x_hat is static
+    (calibrated once)."""
+    name = "svdquant_linear"
+    unit = "TFLOP/s"
+    dominant = "gemm_lowrank"
+
+    def __init__(self, nv, r=64, seed=0):
+        import torch
+        self.nv, self.r = nv, r
+        self.m, self.k, self.n = 4096, 3072, 3072
+        d = S.svdquant_linear(self.m, self.k, self.n, r, seed)
+        self.x_host = d["x"]
+        self.x = to_dev_bf16(d["x"])
+        self.pqs = to_dev_bf16(d["pqs"])
+        self.w_down = to_dev_bf16(d["w_down"])
+        # calibration (offline): amax of x_hat = bf16(x * pre_quant_scale)
+        xh = S.f32_to_bf16_bits(S.bf16_bits_to_f32(d["x"]) * S.bf16_bits_to_f32(d["pqs"])[None, :])
+        amax_x = np.float32(np.abs(S.bf16_bits_to_f32(xh)).max())
+        self.gsf = torch.tensor([np.float32(2688.0) / amax_x], dtype=torch.float32, device="cuda")
+        self.wq, self.wsf, amax_w = quantize_weight(nv, to_dev_bf16(d["w"]))
+        alpha = np.float32(amax_x * np.float32(amax_w.item())) / np.float32(7225344.0)
+        self.alpha = torch.tensor([alpha], dtype=torch.float32, device="cuda")
+        self.l1 = to_dev_bf16(S.f32_to_bf16_bits(d["l1_f32"] / alpha))
+        self.bias = to_dev_bf16(d["bias"])
+        self.xq = torch.empty((self.m, self.k // 2), dtype=torch.uint8, device="cuda")
+        self.xsf = torch.empty((nv.nvfp4_scale_bytes(self.m, self.k),), dtype=torch.uint8, device="cuda")
+        self.dd = torch.empty((self.m, r), dtype=torch.bfloat16, device="cuda")
+        self.out = torch.empty((self.m, self.n), dtype=torch.bfloat16, device="cuda")
+        torch.cuda.synchronize()
+
+    def launches(self):
+        lib, s = self.nv, self
+        return [("quantize_smooth_lora_down", lambda: lib.nvfp4_quantize_smooth_lora_down(
+                    s.x, s.pqs, s.gsf, s.w_down, s.xq, s.xsf, s.dd)),
+                ("gemm_lowrank", lambda: lib.nvfp4_gemm_lowrank_bias(s.xq, s.wq, s.xsf, s.wsf, s.alpha, s.dd, s.l1,
+                                                                      s.bias, s.out))]
+
+    def work(self):
+        return 2.0 * self.m * self.n * self.k + 2.0 * self.m * self.n * self.r + 2.0 * self.m * self.k * self.r
+
+    def kernel_work(self):
+        m, n, k, r = self.m, self.n, self.k, self.r
+        # input stage: HBM-bound (x read; codes, scales and d written)
+        return {"quantize_smooth_lora_down": (2.0 * m * k + 0.5625 * m * k + 2.0 * m * r, "GB/s"),
+                "gemm_lowrank": (2.0 * m * n * k + 2.0 * m * n * r, "TFLOP/s")}
+
+    def e2e_io(self):
+        return self.x_host, self.x, self.out
+
+    def config(self):
+        return {"workload": f"SVDQuant NVFP4 linear layer M=4096 K=3072 N=3072 r={self.r} + bias: smooth quantize "
+                            f"and LoRA-down in one pass over x, then the residual FP4 GEMM with the rank-r "
+                            f"correction; x~N(0,1), pre_quant_scale~U[0.25,4], static x_hat scale",
+                "l2": L2_NOTE}
+
+
 class PR1Linear(Workload):
     name = "pr1_linear"
     unit = "TFLOP/s"
@@ -621,6 +680,8 @@ def make_workload(name, nv, rank_lr, swiglu_path="fused"):
         return GroupedSwiglu(nv)
     if name == "lowrank":
         return LowRank(nv, rank_lr)
+    if name == "svdquant_linear":
+        return SvdquantLinear(nv, rank_lr)
     if name == "pr1_linear":
         return PR1Linear(nv)
     raise SystemExit(f"unknown workload {name}")
@@ -675,6 +736,15 @@ class OracleSample:
                 k = 7168
                 self.x = S.normal_bf16((1, self.rows, 2 * k if w == "quant_silu" else k), 1.0, 0, S.TID["x"])
             self.sample = f"{self.rows} valid rows"
+        elif w == "svdquant_linear":
+            self.rows = rows or 2
+            d = S.svdquant_linear(4096, 3072, 3072, 64, 0)
+            self.x = d["x"][:self.rows].copy()
+            self.pqs, self.wd, self.w = d["pqs"], d["w_down"], d["w"]
+            self.l1_f32, self.bias = d["l1_f32"], d["bias"]
+            self.m, self.k, self.n = self.rows, 3072, 3072
+            self.sample = f"{self.rows} token rows through the SVDQuant layer (smooth quantize, LoRA-down, residual " \
+                          f"GEMM with the rank-64 correction and bias)"
         elif w in ("grouped_moe", "lowrank"):
             self.rows = rows or 2
             self.m, self.k, self.n = (self.rows, 5120, 8192) if w == "grouped_moe" else (self.rows, 3072, 3072)
@@ -700,7 +770,7 @@ class OracleSample:
             self.ad, gd = O.global_scale(self.wd)
             self.qd, self.sfd = O.quantize(self.wd, gd)
             self.ax, self.gx = O.global_scale(self.x)          # static activation scale (calibration)
-        elif self.workload in ("pr1_linear", "grouped_moe", "lowrank"):
+        elif self.workload in ("pr1_linear", "grouped_moe", "lowrank", "svdquant_linear"):
             self.aw, gw = O.global_scale(self.w)
             self.qw, self.sfw = O.quantize(self.w, gw)
 
@@ -730,6 +800,17 @@ class OracleSample:
             hq, hsf = O.silu_mul_quantize_batched(gu_bits, gh)
             O.gemm_ref(hq[0], self.qd, hsf[0], self.sfd, O.alpha(float(ah[0]), float(self.ad)), rows, H, I)
             work = 6.0 * rows * H * I
+        elif w == "svdquant_linear":
+            m, k, n = self.m, self.k, self.n
+            xh = S.f32_to_bf16_bits(S.bf16_bits_to_f32(self.x) * S.bf16_bits_to_f32(self.pqs)[None, :])
+            ax, gx = O.global_scale(xh)
+            qx, sfx = O.quantize_smooth(self.x, self.pqs, gx)
+            dd = O.lora_down(self.x, self.wd)
+            d_bf16 = np.vectorize(O.f64_to_bf16, otypes=[np.uint16])(dd)
+            al = O.alpha(float(ax), float(self.aw))
+            l1 = S.f32_to_bf16_bits(self.l1_f32 / np.float32(al))
+            O.gemm_ref(qx, self.qw, sfx, self.sfw, al, m, n, k, d=d_bf16, l1=l1, bias=self.bias)
+            work = 2.0 * m * n * k + 2.0 * m * n * 64 + 2.0 * m * k * 64
         elif w == "pr1_linear":
             ax, gx = O.global_scale(self.x)
             qx, sfx = O.quantize(self.x, gx)
@@ -792,7 +873,7 @@ def main():
     ap.add_argument("--impl", default="nvfp4", choices=["nvfp4", "reference"])
     ap.add_argument("--workload", default="swiglu_block",
                     choices=["swiglu_block", "quant_dense", "quant_masked", "quant_silu", "grouped_moe",
-                             "grouped_swiglu", "lowrank", "pr1_linear"])
+                             "grouped_swiglu", "lowrank", "svdquant_linear", "pr1_linear"])
     ap.add_argument("--rank-lr", type=int, default=64)
     ap.add_argument("--swiglu-path", default="fused", choices=["fused", "unfused"],
                     help="swiglu_block: SiLU*mul quantization in the gate/up GEMM epilogue, or as its own kernel")

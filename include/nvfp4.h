@@ -258,6 +258,42 @@ NVFP4_API int nvfp4_grouped_gemm_silu_mul_quantize_masked(
     int64_t n, int64_t k, nvfp4_stream_t stream);
 
 /*
+ * Smooth quantize: the SVDQuant activation quantizer [FI5 mm_nvfp4_svdquant, Parameters a:
+ * produced by nvfp4_quantize_smooth, which folds the pre-quantization scale in; TRT
+ * pre_quant_scale].  x_hat[r, c] = bf16(x[r, c] * pre_quant_scale[c]) (one fp32
+ * multiplication rounded to bf16), then quantized exactly as nvfp4_quantize.
+ *   x_bf16 [m, k] bf16; pre_quant_scale_bf16 [k] bf16 (16-byte aligned); k % 16 == 0.
+ *   gsf    fp32 [1] device: the global scale of x_hat (448*6 / amax(x_hat)).
+ *   q_out, sf_out as nvfp4_quantize.
+ */
+NVFP4_API int nvfp4_quantize_smooth(const void *x_bf16, int64_t m, int64_t k, const void *pre_quant_scale_bf16,
+                                    const float *gsf, uint8_t *q_out, uint8_t *sf_out, nvfp4_stream_t stream);
+
+/*
+ * LoRA-down product of an SVDQuant layer [FI5 mm_nvfp4_svdquant, Parameters d: the rank-r
+ * operand is x times the pre-quantization-scaled down projection, in bf16]:
+ *   d = bf16(x @ w^T), accumulated in fp32 on the tensor cores.
+ *   x_bf16 [m, k] bf16 (the unsmoothed activation), k % 64 == 0.
+ *   w_bf16 [r, k] bf16: row j is (pre_quant_scale * L2[j, :]), prepared once per layer.
+ *   r      rank: a multiple of 32 in [32, 256].
+ *   d_bf16 [m, r] bf16 output, 16-byte aligned.
+ */
+NVFP4_API int nvfp4_lora_down(const void *x_bf16, int64_t m, int64_t k, const void *w_bf16, int64_t r,
+                              void *d_bf16, nvfp4_stream_t stream);
+
+/*
+ * Both of the above in one pass over x (the pages run them as two ops): the NVFP4 operand
+ * of nvfp4_quantize_smooth and the d of nvfp4_lora_down, bit-identical to the separate
+ * calls' q_out / sf_out and to nvfp4_lora_down's d.  Arguments as in the two calls;
+ * k % 64 == 0.  Each 128-row tile of x is read once by a cluster of 4 CTAs that split its
+ * K range; their partial d are summed through distributed shared memory.
+ */
+NVFP4_API int nvfp4_quantize_smooth_lora_down(const void *x_bf16, int64_t m, int64_t k,
+                                              const void *pre_quant_scale_bf16, const float *gsf,
+                                              const void *w_bf16, int64_t r, uint8_t *q_out,
+                                              uint8_t *sf_out, void *d_bf16, nvfp4_stream_t stream);
+
+/*
  * Programmatic dependent launch [FI5 mm_nvfp4_svdquant, Parameters: enable_pdl, which
  * defaults to the device default].  When enabled (the default: compute capability 10.0
  * supports it), every kernel of the library is launched with programmatic stream

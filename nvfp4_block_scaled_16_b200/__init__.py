@@ -26,6 +26,9 @@ from .binding import (  # noqa: F401
     nvfp4_gemm_lowrank_bias,
     nvfp4_gemm_silu_mul_quantize,
     nvfp4_grouped_gemm_silu_mul_quantize_masked,
+    nvfp4_quantize_smooth,
+    nvfp4_lora_down,
+    nvfp4_quantize_smooth_lora_down,
     nvfp4_set_pdl,
     nvfp4_get_pdl,
     nvfp4_device_status,

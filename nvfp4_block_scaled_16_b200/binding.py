@@ -27,6 +27,9 @@ EXPORTED_SYMBOLS = (
     "nvfp4_gemm_lowrank_bias",
     "nvfp4_gemm_silu_mul_quantize",
     "nvfp4_grouped_gemm_silu_mul_quantize_masked",
+    "nvfp4_quantize_smooth",
+    "nvfp4_lora_down",
+    "nvfp4_quantize_smooth_lora_down",
     "nvfp4_set_pdl",
     "nvfp4_get_pdl",
     "nvfp4_device_status",
@@ -50,6 +53,9 @@ _SIGNATURES = {
     "nvfp4_gemm_lowrank_bias": (_INT, [_P, _P, _P, _P, _P, _P, _P, _I64, _P, _P, _I64, _I64, _I64, _P]),
     "nvfp4_gemm_silu_mul_quantize": (_INT, [_P] * 11 + [_I64, _I64, _I64, _P]),
     "nvfp4_grouped_gemm_silu_mul_quantize_masked": (_INT, [_P] * 12 + [_I64, _I64, _I64, _I64, _P]),
+    "nvfp4_quantize_smooth": (_INT, [_P, _I64, _I64, _P, _P, _P, _P, _P]),
+    "nvfp4_lora_down": (_INT, [_P, _I64, _I64, _P, _I64, _P, _P]),
+    "nvfp4_quantize_smooth_lora_down": (_INT, [_P, _I64, _I64, _P, _P, _P, _I64, _P, _P, _P, _P]),
     "nvfp4_set_pdl": (_INT, [_INT]),
     "nvfp4_get_pdl": (_INT, []),
     "nvfp4_device_status": (_INT, [ctypes.POINTER(_INT), _INT]),
@@ -277,6 +283,50 @@ def nvfp4_grouped_gemm_silu_mul_quantize_masked(a, b_gate, b_up, a_sf, b_gate_sf
             _stream(stream))
     _check("nvfp4_grouped_gemm_silu_mul_quantize_masked", st)
     return q_out, sf_out
+
+
+def nvfp4_quantize_smooth(x, pre_quant_scale, gsf, q_out=None, sf_out=None, stream=None):
+    """x [m, k] bf16, pre_quant_scale [k] bf16 -> NVFP4 of bf16(x * pre_quant_scale): (q [m, k/2], sf)."""
+    m, k = x.shape
+    if q_out is None:
+        q_out = torch.empty((m, k // 2), dtype=torch.uint8, device=x.device)
+    if sf_out is None:
+        sf_out = torch.empty((nvfp4_scale_bytes(m, k),), dtype=torch.uint8, device=x.device)
+    with torch.cuda.device(x.device):
+        st = load_library().nvfp4_quantize_smooth(_ptr(x), m, k, _ptr(pre_quant_scale), _ptr(gsf), _ptr(q_out),
+                                                  _ptr(sf_out), _stream(stream))
+    _check("nvfp4_quantize_smooth", st)
+    return q_out, sf_out
+
+
+def nvfp4_lora_down(x, w, d_out=None, stream=None):
+    """d [m, r] bf16 = x [m, k] @ w [r, k]^T (w: the pre-quantization-scaled LoRA-down weight)."""
+    m, k = x.shape
+    r = w.shape[0]
+    if d_out is None:
+        d_out = torch.empty((m, r), dtype=torch.bfloat16, device=x.device)
+    with torch.cuda.device(x.device):
+        st = load_library().nvfp4_lora_down(_ptr(x), m, k, _ptr(w), r, _ptr(d_out), _stream(stream))
+    _check("nvfp4_lora_down", st)
+    return d_out
+
+
+def nvfp4_quantize_smooth_lora_down(x, pre_quant_scale, gsf, w, q_out=None, sf_out=None, d_out=None, stream=None):
+    """Both in one pass over x: (q [m, k/2], sf, d [m, r])."""
+    m, k = x.shape
+    r = w.shape[0]
+    if q_out is None:
+        q_out = torch.empty((m, k // 2), dtype=torch.uint8, device=x.device)
+    if sf_out is None:
+        sf_out = torch.empty((nvfp4_scale_bytes(m, k),), dtype=torch.uint8, device=x.device)
+    if d_out is None:
+        d_out = torch.empty((m, r), dtype=torch.bfloat16, device=x.device)
+    with torch.cuda.device(x.device):
+        st = load_library().nvfp4_quantize_smooth_lora_down(_ptr(x), m, k, _ptr(pre_quant_scale), _ptr(gsf),
+                                                            _ptr(w), r, _ptr(q_out), _ptr(sf_out), _ptr(d_out),
+                                                            _stream(stream))
+    _check("nvfp4_quantize_smooth_lora_down", st)
+    return q_out, sf_out, d_out
 
 
 def nvfp4_set_pdl(enable: bool) -> None:

@@ -55,6 +55,7 @@ struct QuantParams {
   int64_t sf_item_stride;  // bytes
   const int32_t* mask;     // nullable
   const float* gsf;        // [items]
+  const uint16_t* pqs;     // smoothing: bf16 [k] pre-quantization scale (x_hat = bf16(x * pqs))
   int32_t m;               // rows per item
   int32_t k;               // output width (elements)
   uint32_t nb;             // k / 16
@@ -63,7 +64,7 @@ struct QuantParams {
   uint32_t blocks;         // rows_pad * cpad (per item)
 };
 
-template <bool kSilu, int kUnroll>
+template <bool kSilu, bool kSmooth, int kUnroll>
 __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantParams p) {
   pdl_launch_dependents();
   pdl_wait();
@@ -119,6 +120,22 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantParams p)
         unpack_bf16x8(raw[u][3], up + 8);
 #pragma unroll
         for (int i = 0; i < 16; i += 2) silu_mul_bf16_2(v[i], v[i + 1], up[i], up[i + 1], v[i], v[i + 1]);
+      }
+      if constexpr (kSmooth) {
+        // x_hat = bf16(x * pre_quant_scale) for the block's 16 columns (the scale vector is
+        // the same for every row: these loads hit in L1 / L2)
+        float sc[16];
+        unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(p.pqs + c * 16)), sc);
+        unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(p.pqs + c * 16 + 8)), sc + 8);
+#pragma unroll
+        for (int i = 0; i < 16; i += 2) {
+          float a, b;
+          unpack2(mul2(pack2(v[i], v[i + 1]), pack2(sc[i], sc[i + 1])), a, b);
+          uint32_t w;
+          asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w) : "f"(b), "f"(a));   // a -> low half
+          v[i] = bf16_lo(w);
+          v[i + 1] = bf16_hi(w);
+        }
       }
       const QBlock b = quantize16(v, gsf);
       *reinterpret_cast<uint2*>(q + static_cast<int64_t>(r) * (p.k / 2) + c * 8) = make_uint2(b.lo, b.hi);
@@ -245,11 +262,12 @@ __global__ void __launch_bounds__(kThreads) amax_batched_kernel(const uint16_t* 
 // ---- host helpers -------------------------------------------------------------------------
 
 int launch_quantize(const void* x, int64_t b, int64_t m, int64_t k, bool silu, const int32_t* mask,
-                    const float* gsf, uint8_t* q, uint8_t* sf, cudaStream_t stream) {
+                    const float* gsf, uint8_t* q, uint8_t* sf, cudaStream_t stream, const void* pqs = nullptr) {
   if (b < 0 || m < 0 || k < 0 || k % 16 != 0) return NVFP4_ERR_INVALID_ARGUMENT;
   if (b == 0 || m == 0 || k == 0) return NVFP4_OK;
   if (!x || !gsf || !q || !sf) return NVFP4_ERR_INVALID_ARGUMENT;
-  if (!aligned(x, 16) || !aligned(q, 8) || !aligned(gsf, 4) || (mask && !aligned(mask, 4)))
+  if (!aligned(x, 16) || !aligned(q, 8) || !aligned(gsf, 4) || (mask && !aligned(mask, 4)) ||
+      (pqs && !aligned(pqs, 16)))
     return NVFP4_ERR_INVALID_ARGUMENT;
   if (b > 65535 || m > (1 << 30) || k > (1 << 30)) return NVFP4_ERR_INVALID_ARGUMENT;
   const int64_t nb = k / 16, cpad = (nb + 3) / 4 * 4, rows_pad = (m + 127) / 128 * 128;
@@ -268,6 +286,7 @@ int launch_quantize(const void* x, int64_t b, int64_t m, int64_t k, bool silu, c
   p.sf_item_stride = rows_pad * cpad;
   p.mask = mask;
   p.gsf = gsf;
+  p.pqs = static_cast<const uint16_t*>(pqs);
   p.m = static_cast<int32_t>(m);
   p.k = static_cast<int32_t>(k);
   p.nb = static_cast<uint32_t>(nb);
@@ -277,11 +296,12 @@ int launch_quantize(const void* x, int64_t b, int64_t m, int64_t k, bool silu, c
   if (silu) {
     constexpr int U = 2;
     dim3 grid(static_cast<unsigned>((p.blocks + kThreads * U - 1) / (kThreads * U)), static_cast<unsigned>(b));
-    return launch_kernel(quantize_kernel<true, U>, grid, dim3(kThreads), 0, stream, p);
+    return launch_kernel(quantize_kernel<true, false, U>, grid, dim3(kThreads), 0, stream, p);
   }
   constexpr int U = 4;
   dim3 grid(static_cast<unsigned>((p.blocks + kThreads * U - 1) / (kThreads * U)), static_cast<unsigned>(b));
-  return launch_kernel(quantize_kernel<false, U>, grid, dim3(kThreads), 0, stream, p);
+  if (pqs) return launch_kernel(quantize_kernel<false, true, U>, grid, dim3(kThreads), 0, stream, p);
+  return launch_kernel(quantize_kernel<false, false, U>, grid, dim3(kThreads), 0, stream, p);
 }
 
 }  // namespace
@@ -339,6 +359,12 @@ int nvfp4_global_scale_batched(const void* x_bf16, int64_t b, int64_t m, int64_t
 int nvfp4_quantize(const void* x_bf16, int64_t m, int64_t k, const float* gsf, uint8_t* q_out, uint8_t* sf_out,
                    nvfp4_stream_t stream) {
   return launch_quantize(x_bf16, 1, m, k, false, nullptr, gsf, q_out, sf_out, stream);
+}
+
+int nvfp4_quantize_smooth(const void* x_bf16, int64_t m, int64_t k, const void* pre_quant_scale_bf16,
+                          const float* gsf, uint8_t* q_out, uint8_t* sf_out, nvfp4_stream_t stream) {
+  if (!pre_quant_scale_bf16 && m > 0 && k > 0) return NVFP4_ERR_INVALID_ARGUMENT;
+  return launch_quantize(x_bf16, 1, m, k, false, nullptr, gsf, q_out, sf_out, stream, pre_quant_scale_bf16);
 }
 
 int nvfp4_quantize_masked_batched(const void* x_bf16, int64_t b, int64_t m, int64_t k, const int32_t* mask,

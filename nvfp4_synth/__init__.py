@@ -28,7 +28,7 @@ import numpy as np
 # Tensor ids: one independent stream per tensor of a workload.
 TID = {
     "x": 1, "w": 2, "w_gate_up": 3, "w_down": 4, "mask": 5, "d": 6, "l1": 7, "bias": 8,
-    "outlier": 9, "sample": 10, "w_gate": 11, "w_up": 12,
+    "outlier": 9, "sample": 10, "w_gate": 11, "w_up": 12, "pqs": 13, "lora_down": 14,
 }
 
 
@@ -153,6 +153,18 @@ def grouped_swiglu(E=16, mmax=2048, hidden=5120, inter=8192, mean=512, seed=0, e
             "w_up": normal_bf16((E, inter, hidden), 0.02, seed, TID["w_up"], experts),
             "w_down": normal_bf16((E, hidden, inter), 0.02, seed, TID["w_down"], experts),
             "mask": masks_poisson(E, mean, mmax, seed)}
+
+
+def svdquant_linear(m=4096, k=3072, n=3072, r=64, seed=0):
+    """SVDQuant layer: activations, pre-quantization scale U[0.25, 4] (per input channel),
+    the pre-scaled LoRA-down weight [r, k] ~ N(0, 0.05), residual weight ~ N(0, 0.02), LoRA-up
+    draws N(0, 0.01) (fp32; the caller divides by alpha and rounds), bias ~ N(0, 0.1)."""
+    return {"x": normal_bf16((m, k), 1.0, seed, TID["x"]),
+            "pqs": f32_to_bf16_bits(rng(seed, TID["pqs"]).uniform(0.25, 4.0, k).astype(np.float32)),
+            "w_down": normal_bf16((r, k), 0.05, seed, TID["lora_down"]),
+            "w": normal_bf16((n, k), 0.02, seed, TID["w"]),
+            "l1_f32": rng(seed, TID["l1"]).standard_normal((n, r), dtype=np.float32) * np.float32(0.01),
+            "bias": normal_bf16((n,), 0.1, seed, TID["bias"])}
 
 
 def lowrank(m=4096, k=3072, n=3072, r=64, seed=0):

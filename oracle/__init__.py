@@ -58,6 +58,8 @@ def lib():
             "nvo_grouped_gemm_ref": (None, [_u8p, _u8p, _u8p, _u8p, _i32p, _f32p, _i64, _i64, _i64, _i64,
                                             _f64p]),
             "nvo_f64_to_bf16": (ctypes.c_uint16, [ctypes.c_double]),
+            "nvo_quantize_smooth": (None, [_u16p, _i64, _i64, _u16p, ctypes.c_float, _u8p, _u8p]),
+            "nvo_lora_down": (None, [_u16p, _i64, _i64, _u16p, _i64, _f64p]),
             "nvo_gemm_silu_mul_quantize": (None, [_u8p] * 6 + [ctypes.c_float] * 3 + [_i64, _i64, _i64,
                                                                                       _u8p, _u8p]),
             "nvo_grouped_gemm_silu_mul_quantize": (None, [_u8p] * 6 + [_i32p, _f32p, _f32p, _f32p, _i64, _i64,
@@ -321,3 +323,25 @@ def gemm_gate_up_bf16(a, b_gate, b_up, a_sf, b_gate_sf, b_up_sf, alpha_gate, alp
                                 _p(b_gate_sf, _u8p), _p(b_up_sf, _u8p), float(np.float32(alpha_gate)),
                                 float(np.float32(alpha_up)), n, k, _p(ii, _i64p), len(ii), _p(x, _u16p))
     return x
+
+
+def quantize_smooth(x, pqs, gsf, sf_fill=0):
+    """Smooth quantize: NVFP4 quantization of x_hat = bf16(x * pqs) -> (q [m, k/2], sf)."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    pq = np.ascontiguousarray(pqs, dtype=np.uint16)
+    m, k = x.shape
+    q = np.zeros((m, k // 2), np.uint8)
+    sf = np.full(scale_bytes(m, k), sf_fill, np.uint8)
+    lib().nvo_quantize_smooth(_p(x, _u16p), m, k, _p(pq, _u16p), float(np.float32(gsf)), _p(q, _u8p), _p(sf, _u8p))
+    return q, sf
+
+
+def lora_down(x, w):
+    """d = x @ w^T in fp64 for bf16 bits x [m, k], w [r, k] -> [m, r]."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    w = np.ascontiguousarray(w, dtype=np.uint16)
+    m, k = x.shape
+    r = w.shape[0]
+    out = np.zeros((m, r), np.float64)
+    lib().nvo_lora_down(_p(x, _u16p), m, k, _p(w, _u16p), r, _p(out, _f64p))
+    return out

@@ -589,3 +589,39 @@ NVO_API void nvo_gemm_silu_mul_quantize_rows(const uint8_t *a, const uint8_t *b_
     free(sf1);
     free(x);
 }
+
+/* ------------------------------------------------------------------------------- */
+/* SVDQuant input stage [FI5] Parameters a and d: the activation operand is x        */
+/* quantized with the pre-quantization scale folded in, and d is the LoRA-down       */
+/* product of x with the pre-quantization-scaled down projection.                    */
+/* ------------------------------------------------------------------------------- */
+
+/* Smooth quantize (reading R20): x_hat[r, c] = bf16(float(x[r, c]) * float(pqs[c])),
+ * one fp32 multiplication rounded to bf16, then the dense quantizer with gsf. */
+NVO_API void nvo_quantize_smooth(const uint16_t *x, int64_t m, int64_t k, const uint16_t *pqs, float gsf,
+                                 uint8_t *q, uint8_t *sf) {
+    #pragma omp parallel for schedule(static) num_threads(g_threads)
+    for (int64_t r = 0; r < m; ++r) {
+        float xr[k > 0 ? k : 1];
+        for (int64_t i = 0; i < k; ++i) {
+            float prod = bf16_to_f32(x[r * k + i]) * bf16_to_f32(pqs[i]);
+            xr[i] = bf16_to_f32(f32_to_bf16_rne(prod));
+        }
+        quantize_row(xr, k, gsf, q + r * (k / 2), sf, r, k);
+        zero_row_padding_cols(sf, r, k);
+    }
+    zero_padding_rows(sf, m, k);
+}
+
+/* LoRA-down: d[i, j] = sum_c x[i, c] * w[j, c] in fp64 (w = [r, k], the down projection
+ * already scaled by the pre-quantization scale); out is [m, r]. */
+NVO_API void nvo_lora_down(const uint16_t *x, int64_t m, int64_t k, const uint16_t *w, int64_t r, double *out) {
+    #pragma omp parallel for schedule(static) num_threads(g_threads)
+    for (int64_t i = 0; i < m; ++i)
+        for (int64_t j = 0; j < r; ++j) {
+            double acc = 0.0;
+            for (int64_t c = 0; c < k; ++c)
+                acc += (double)bf16_to_f32(x[i * k + c]) * (double)bf16_to_f32(w[j * k + c]);
+            out[i * r + j] = acc;
+        }
+}

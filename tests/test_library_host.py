@@ -148,3 +148,19 @@ def test_pdl_switch(lib):
     assert nv.nvfp4_get_pdl() is False
     nv.nvfp4_set_pdl(True)
     assert nv.nvfp4_get_pdl() is True
+
+
+def test_svdquant_input_argument_checks(lib):
+    # k % 64, rank in [32, 256] and a multiple of 32, required pointers
+    assert lib.nvfp4_lora_down(A16, 128, 96, A16, 64, A16, None) == INVALID
+    for r in (0, 16, 48, 288):
+        assert lib.nvfp4_lora_down(A16, 128, 128, A16, r, A16, None) == INVALID
+    assert lib.nvfp4_lora_down(A16, 128, 128, None, 64, A16, None) == INVALID
+    assert lib.nvfp4_lora_down(A16, 0, 128, A16, 64, A16, None) == 0                      # empty
+    args = [A16, 128, 128, A16, A16, A16, 64, A16, A16, A16, None]
+    for i in (3, 4, 7, 8):                                                                 # pqs, gsf, q, sf
+        bad = list(args)
+        bad[i] = None
+        assert lib.nvfp4_quantize_smooth_lora_down(*bad) == INVALID, i
+    assert lib.nvfp4_quantize_smooth(A16, 4, 32, None, A16, A16, A16, None) == INVALID       # pqs required
+    assert lib.nvfp4_quantize_smooth(A16, 4, 32, A1, A16, A16, A16, None) == INVALID         # misaligned pqs

@@ -593,3 +593,58 @@ def test_gemm_silu_mul_rows_and_grouped_agree_with_dense(oracle):
         assert (qr == qd[rows]).all()
         for i, r in enumerate(rows):
             assert (sr[i] == sd[[oracle.sf_offset(r, c, n) for c in range(n // 16)]]).all()
+
+
+# --------------------------------------------------------------------------------------
+# SVDQuant input stage: smooth quantize and LoRA-down
+# --------------------------------------------------------------------------------------
+
+BF16_ONE = 0x3F80
+
+
+def test_quantize_smooth_unit_scale_is_quantize(oracle):
+    x = S.normal_bf16((70, 96), 1.0, seed=21)
+    _, gsf = oracle.global_scale(x)
+    q1, s1 = oracle.quantize_smooth(x, np.full(96, BF16_ONE, np.uint16), gsf)
+    q2, s2 = oracle.quantize(x, gsf)
+    assert (q1 == q2).all() and (s1 == s2).all()
+
+
+def test_quantize_smooth_power_of_two_scales_are_exact(oracle):
+    # pqs[c] = 2^e[c]: x * pqs is exact in bf16 (no overflow / underflow at these sizes), so
+    # the smoothed tensor is x with e[c] added to every exponent of column c
+    m, k = 40, 64
+    x = S.normal_bf16((m, k), 1.0, seed=22)
+    e = np.random.default_rng(3).integers(-3, 4, k)
+    pqs = ((127 + e).astype(np.uint16) << 7).astype(np.uint16)             # bf16 2^e
+    xs = x.astype(np.int32)
+    expo = (xs >> 7) & 0xFF
+    nz = expo != 0
+    xs = np.where(nz, (xs & ~(0xFF << 7)) | ((expo + e[None, :]) << 7), xs).astype(np.uint16)
+    _, gsf = oracle.global_scale(xs)
+    q1, s1 = oracle.quantize_smooth(x, pqs, gsf)
+    q2, s2 = oracle.quantize(xs, gsf)
+    assert (q1 == q2).all() and (s1 == s2).all()
+
+
+def test_quantize_smooth_matches_numpy_rounding(oracle):
+    m, k = 33, 128
+    x = S.normal_bf16((m, k), 1.0, seed=23)
+    pqs = S.f32_to_bf16_bits(np.random.default_rng(4).uniform(0.25, 4.0, k).astype(np.float32))
+    xh = S.f32_to_bf16_bits(S.bf16_bits_to_f32(x) * S.bf16_bits_to_f32(pqs)[None, :])
+    _, gsf = oracle.global_scale(xh)
+    q1, s1 = oracle.quantize_smooth(x, pqs, gsf)
+    q2, s2 = oracle.quantize(xh, gsf)
+    assert (q1 == q2).all() and (s1 == s2).all()
+
+
+def test_lora_down_matches_numpy_and_identity(oracle):
+    m, k, r = 50, 96, 32
+    x = S.normal_bf16((m, k), 1.0, seed=24)
+    w = S.normal_bf16((r, k), 0.05, seed=24, tensor_id=2)
+    d = oracle.lora_down(x, w)
+    ref = S.bf16_bits_to_f32(x).astype(np.float64) @ S.bf16_bits_to_f32(w).astype(np.float64).T
+    assert np.allclose(d, ref, rtol=1e-12, atol=1e-12)
+    eye = np.zeros((r, k), np.uint16)
+    eye[np.arange(r), np.arange(r)] = BF16_ONE
+    assert (oracle.lora_down(x, eye) == S.bf16_bits_to_f32(x[:, :r]).astype(np.float64)).all()
