@@ -18,13 +18,14 @@
 //   warp 1      TMEM allocator and MMA issuer: per stage four tcgen05.mma.cta_group::1
 //               kind::f16 (bf16 x bf16 -> fp32, M = 128, N = r, K = 16) into a 128 x r fp32
 //               accumulator in tensor memory.
-//   warps 2-5   quantizer (fused op only): thread t owns row t of the tile; per stage it reads
-//               its 64 values from the swizzled tile, forms x_hat, and writes 4 blocks: 32
-//               code bytes and one 4-byte word of scales (the stage is exactly one 4-block
-//               group of the 128x4 scale layout).  Afterwards the same warps drain the
-//               accumulator into shared memory (column-major fp32) and, after a cluster
-//               barrier, CTA c sums rows [32c, 32c + 32) over the 4 CTAs' partials through
-//               distributed shared memory and writes them as bf16.
+//   warps 2-9   quantizer (fused op only): a thread owns one row of the tile and half of the
+//               stage's 4 blocks (two warps per 32 rows); per stage it reads its 32 values
+//               from the swizzled tile, forms x_hat, and writes 2 blocks: 16 code bytes and
+//               two scale bytes (a stage is exactly one 4-block group of the 128x4 scale
+//               layout).  Afterwards warps 2-5 drain the accumulator into shared memory
+//               (column-major fp32) and, after a cluster barrier, CTA c sums rows
+//               [32c, 32c + 32) over the 4 CTAs' partials through distributed shared memory
+//               and writes them as bf16.
 // Every mbarrier wait is bounded; the two cluster barriers are executed on every path.
 #include <cuda_bf16.h>
 
@@ -41,7 +42,12 @@ constexpr int kSvdStages = 4;
 constexpr int kSvdSplit = 4;             // CTAs per cluster, splitting K
 constexpr int kSvdXBytes = kSvdRows * 128;   // 16 KB per stage
 constexpr int kSvdMaxRank = 256;
-constexpr int kSvdThreads = 192;
+// Quantizer warps: 16 / kSvdQuantWarps of a row's 4 blocks per stage per thread; the first
+// four of them also drain and reduce the accumulator.
+constexpr int kSvdQuantWarps = 8;
+constexpr int kSvdBlocksPerThread = 16 / kSvdQuantWarps;
+constexpr int kSvdThreads = 64 + 32 * kSvdQuantWarps;
+static_assert(kSvdQuantWarps == 4 || kSvdQuantWarps == 8 || kSvdQuantWarps == 16, "1, 2 or 4 blocks per thread");
 
 struct __align__(8) SvdControl {
   uint64_t full[kSvdStages];
@@ -139,7 +145,7 @@ __global__ void __cluster_dims__(kSvdSplit, 1, 1) __launch_bounds__(kSvdThreads,
   if (threadIdx.x == 0) {
     for (int s = 0; s < kSvdStages; ++s) {
       mbar_init(&ctl.full[s], 1);
-      mbar_init(&ctl.empty[s], kQuant ? 5 : 1);   // the MMA commit (+ the 4 quantizer warps)
+      mbar_init(&ctl.empty[s], kQuant ? 1 + kSvdQuantWarps : 1);   // the MMA commit (+ the quantizer warps)
     }
     mbar_init(&ctl.acc_full, 1);
     ctl.abort = 0;
@@ -200,7 +206,9 @@ __global__ void __cluster_dims__(kSvdSplit, 1, 1) __launch_bounds__(kSvdThreads,
     __syncwarp();
   } else {
     // ------------------------------------------------------------------ quantizer + epilogue
-    const int row = (warp - 2) * 32 + lane;         // row of the tile; also its TMEM lane
+    const int qw = warp - 2;
+    const int row = (qw & 3) * 32 + lane;           // row of the tile; also its TMEM lane
+    const int part = qw >> 2;                       // which blocks of the stage this thread takes
     const int grow = row0 + row;
     bool ok = true;
     if constexpr (kQuant) {
@@ -209,23 +217,28 @@ __global__ void __cluster_dims__(kSvdSplit, 1, 1) __launch_bounds__(kSvdThreads,
       for (int i = 0; i < nch; ++i) {
         const int s = i % kSvdStages;
         const int kc = (c_begin + i) * kSvdChunk;
-        uint4 sc_raw[8];                      // the stage's 64 pre-quantization scales
+        const int b0 = part * kSvdBlocksPerThread;   // first block (of 4) of this thread
+        uint4 sc_raw[2 * kSvdBlocksPerThread];      // its pre-quantization scales
 #pragma unroll
-        for (int c = 0; c < 8; ++c) sc_raw[c] = __ldg(reinterpret_cast<const uint4*>(p.pqs + kc + 8 * c));
+        for (int c = 0; c < 2 * kSvdBlocksPerThread; ++c)
+          sc_raw[c] = __ldg(reinterpret_cast<const uint4*>(p.pqs + kc + 16 * b0 + 8 * c));
         if (!(ok = mbar_wait_fast(&ctl.full[s], (i / kSvdStages) & 1, abort, p.status))) break;
         const uint32_t tile = smem_u32(smem + s * stage_bytes);
+        const uint32_t sf_word = static_cast<uint32_t>(
+            sf_offset(static_cast<uint32_t>(grow), static_cast<uint32_t>(kc / 16 + b0), groups));
         if (grow < p.m) {
-          uint32_t codes[8];
+          uint32_t codes[2 * kSvdBlocksPerThread];
           uint32_t scales = 0;
 #pragma unroll
-          for (int blk = 0; blk < 4; ++blk) {
+          for (int blk = 0; blk < kSvdBlocksPerThread; ++blk) {
             float v[16];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-              const int c = 2 * blk + h;
+              const int c = 2 * (b0 + blk) + h;       // 16-byte chunk of the 128-byte row
               const uint4 xr = ld_swizzled_chunk(tile, row, c);
+              const uint4 sr = sc_raw[2 * blk + h];
               const uint32_t xw[4] = {xr.x, xr.y, xr.z, xr.w};
-              const uint32_t sw[4] = {sc_raw[c].x, sc_raw[c].y, sc_raw[c].z, sc_raw[c].w};
+              const uint32_t sw[4] = {sr.x, sr.y, sr.z, sr.w};
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
                 float a, b;
@@ -241,14 +254,26 @@ __global__ void __cluster_dims__(kSvdSplit, 1, 1) __launch_bounds__(kSvdThreads,
             codes[2 * blk + 1] = qb.hi;
             scales |= qb.s8 << (8 * blk);
           }
-          uint4* dst = reinterpret_cast<uint4*>(p.q + static_cast<int64_t>(grow) * (p.k / 2) + kc / 2);
-          dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
-          dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
-          *reinterpret_cast<uint32_t*>(p.sf + sf_offset(static_cast<uint32_t>(grow), static_cast<uint32_t>(kc / 16),
-                                                        groups)) = scales;
+          uint8_t* qdst = p.q + static_cast<int64_t>(grow) * (p.k / 2) + kc / 2 + 8 * b0;
+          if constexpr (kSvdBlocksPerThread == 4) {
+            reinterpret_cast<uint4*>(qdst)[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+            reinterpret_cast<uint4*>(qdst)[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+            *reinterpret_cast<uint32_t*>(p.sf + sf_word) = scales;
+          } else if constexpr (kSvdBlocksPerThread == 2) {
+            *reinterpret_cast<uint4*>(qdst) = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+            *reinterpret_cast<uint16_t*>(p.sf + sf_word) = static_cast<uint16_t>(scales);
+          } else {
+            *reinterpret_cast<uint2*>(qdst) = make_uint2(codes[0], codes[1]);
+            p.sf[sf_word] = static_cast<uint8_t>(scales);
+          }
         } else if (grow < p.rows_pad) {
-          *reinterpret_cast<uint32_t*>(p.sf + sf_offset(static_cast<uint32_t>(grow), static_cast<uint32_t>(kc / 16),
-                                                        groups)) = 0u;
+          if constexpr (kSvdBlocksPerThread == 4) {
+            *reinterpret_cast<uint32_t*>(p.sf + sf_word) = 0u;
+          } else if constexpr (kSvdBlocksPerThread == 2) {
+            *reinterpret_cast<uint16_t*>(p.sf + sf_word) = 0;
+          } else {
+            p.sf[sf_word] = 0;
+          }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive_local(&ctl.empty[s]);
@@ -256,24 +281,26 @@ __global__ void __cluster_dims__(kSvdSplit, 1, 1) __launch_bounds__(kSvdThreads,
     }
     // The partials overwrite the stage ring: every quantizer warp must be done reading it
     // (a warp whose rows all lie beyond m has no quantizing work and would get here first).
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    // drain this CTA's partial accumulator into shared memory, column-major: part[col][row]
-    float* part = reinterpret_cast<float*>(smem);
-    if (ok && nch > 0 && mbar_wait(&ctl.acc_full, 0, abort, p.status)) {
-      tc_fence_after();
-      const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-      for (int c0 = 0; c0 < p.r; c0 += 64) {
-        uint32_t v[64];
-        tmem_load_64(tmem + c0 + lane_base, v);
-        tmem_wait_ld<64>(v);
-        const int tmem_row = (warp & 3) * 32 + lane;   // TMEM lane quarter of this warp
+    asm volatile("bar.sync 1, %0;" ::"n"(32 * kSvdQuantWarps) : "memory");
+    // warps 2-5 drain this CTA's partial accumulator into shared memory, column-major:
+    // part[col][row]
+    if (qw < 4) {
+      float* partial = reinterpret_cast<float*>(smem);
+      const int tmem_row = (warp & 3) * 32 + lane;   // TMEM lane quarter of this warp
+      if (ok && nch > 0 && mbar_wait(&ctl.acc_full, 0, abort, p.status)) {
+        tc_fence_after();
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        for (int c0 = 0; c0 < p.r; c0 += 64) {
+          uint32_t v[64];
+          tmem_load_64(tmem + c0 + lane_base, v);
+          tmem_wait_ld<64>(v);
 #pragma unroll
-        for (int j = 0; j < 64; ++j)
-          if (c0 + j < p.r) part[(c0 + j) * kSvdRows + tmem_row] = __uint_as_float(v[j]);
+          for (int j = 0; j < 64; ++j)
+            if (c0 + j < p.r) partial[(c0 + j) * kSvdRows + tmem_row] = __uint_as_float(v[j]);
+        }
+      } else {
+        for (int j = 0; j < p.r; ++j) partial[j * kSvdRows + tmem_row] = 0.0f;
       }
-    } else {
-      const int tmem_row = (warp & 3) * 32 + lane;
-      for (int j = 0; j < p.r; ++j) part[j * kSvdRows + tmem_row] = 0.0f;
     }
   }
 
@@ -282,7 +309,7 @@ __global__ void __cluster_dims__(kSvdSplit, 1, 1) __launch_bounds__(kSvdThreads,
   __syncwarp();
   __syncthreads();
   cluster_sync();          // every CTA's partials are in its shared memory
-  if (warp >= 2 && !*abort) {
+  if (warp >= 2 && warp < 6 && !*abort) {
     const int row = static_cast<int>(rank) * 32 + lane;   // this CTA's quarter of the tile rows
     const int grow = row0 + row;
     const int cols = p.r / 4;                             // columns per epilogue warp
