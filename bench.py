@@ -112,24 +112,30 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(world, v):
+def _reduce(world, v, op, device):
     if world == 1:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=op)
     return t.item()
 
 
-def sum_over_ranks(world, v):
-    if world == 1:
-        return v
-    import torch
+def max_over_ranks(world, v, device="cuda"):
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return t.item()
+    return _reduce(world, v, dist.ReduceOp.MAX if world > 1 else None, device)
+
+
+def sum_over_ranks(world, v, device="cuda"):
+    import torch.distributed as dist
+    return _reduce(world, v, dist.ReduceOp.SUM if world > 1 else None, device)
+
+
+def aggregate(world, work_local, ms_local, device="cuda"):
+    """Whole-job throughput of a data-parallel run: (sum over ranks of the work) / (max over
+    ranks of the device time).  Returns (work of all ranks, max time in ms)."""
+    return sum_over_ranks(world, work_local, device), max_over_ranks(world, ms_local, device)
 
 
 # ---------------------------------------------------------------------------------------
@@ -1020,8 +1026,7 @@ def main():
 
     per_kernel = {name: [smp[i] for smp in samples] for i, (name, _) in enumerate(launches)}
     total_ms = sum(step_ms)
-    total_ms_max = max_over_ranks(world, total_ms)
-    work_all = sum_over_ranks(world, wl.work() * args.steps)
+    work_all, total_ms_max = aggregate(world, wl.work() * args.steps, total_ms)
     value = scale(work_all / (total_ms_max * 1e-3), wl.unit)
     ms_per_step = total_ms_max / args.steps
 
@@ -1069,8 +1074,8 @@ def main():
                     e_end[i].record()
         torch.cuda.synchronize()
         e2e_ms = sum(a.elapsed_time(b) for a, b in zip(e_start, e_end))
-        e2e_ms = max_over_ranks(world, e2e_ms)
-        e2e_val = scale(sum_over_ranks(world, wl.work() * args.steps) / (e2e_ms * 1e-3), wl.unit)
+        e2e_work, e2e_ms = aggregate(world, wl.work() * args.steps, e2e_ms)
+        e2e_val = scale(e2e_work / (e2e_ms * 1e-3), wl.unit)
         e2e = {"value": round(e2e_val, 3), "unit": wl.unit, "h2d_bytes_per_step": int(x_pinned.numel() * x_pinned.element_size()),
                "d2h_bytes_per_step": int(y_pinned.numel() * y_pinned.element_size()), "ms_per_step": round(e2e_ms / args.steps, 4)}
 

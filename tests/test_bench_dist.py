@@ -1,0 +1,73 @@
+"""The multi-rank plumbing of bench.py on the CPU: two processes over gloo (world size 2)
+check the barrier, the max / sum reductions, the whole-job aggregation of a
+data-parallel run (sum of work over ranks / max of device time), and that under torchrun
+only rank 0 of the reference arm runs and prints."""
+import io
+import os
+import socket
+import sys
+from contextlib import redirect_stdout
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, results):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    sys.path.insert(0, ROOT)
+    import datetime
+    import torch.distributed as dist
+    import bench
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        bench.barrier(world)
+        mx = bench.max_over_ranks(world, float(rank + 1) * 10.0, device="cpu")
+        sm = bench.sum_over_ranks(world, float(rank + 1), device="cpu")
+        # rank r did (r + 1) * 1e12 FLOP in (r + 1) * 100 ms
+        work, ms = bench.aggregate(world, (rank + 1) * 1e12, (rank + 1) * 100.0, device="cpu")
+        # reference arm: rank 1 must return without work or output
+        out = io.StringIO()
+        if rank == 1:
+            class Args:
+                workload, steps, warmup, gpus = "quant_dense", 1, 1, world
+            with redirect_stdout(out):
+                bench.run_reference(Args, world, rank)
+        results[rank] = (mx, sm, work, ms, out.getvalue())
+        bench.barrier(world)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_reductions_and_aggregation():
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
+        results = mgr.dict()
+        port = _free_port()
+        procs = [ctx.Process(target=_worker, args=(r, 2, port, results)) for r in range(2)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(timeout=120)
+        assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+        res = dict(results)
+    for rank in range(2):
+        mx, sm, work, ms, out = res[rank]
+        assert mx == 20.0 and sm == 3.0
+        assert work == 3e12 and ms == 200.0          # value = 3e12 FLOP / 0.2 s = 15 TFLOP/s
+    assert res[1][4] == ""                            # the reference arm ran on rank 0 only
+
+
+def test_single_rank_helpers_are_identity():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(1, 5.0) == 5.0
+    assert bench.sum_over_ranks(1, 5.0) == 5.0
+    assert bench.aggregate(1, 7.0, 3.0) == (7.0, 3.0)
