@@ -36,14 +36,14 @@
 //   warps 2-5   epilogue (both CTAs): tcgen05.ld of the CTA's 128 x 256 fp32 accumulator
 //               (each warp owns its 32-lane TMEM quarter), alpha * acc + bias, bf16 staged
 //               in shared memory and written by TMA stores (one 32 x 64 tile at a time).
-//               The SiLU * up epilogue uses warps 2-9: two per lane quarter, one per half
+//               The SiLU * up epilogue uses warps 2-9: two per lane quarter, each with 64
 //               of the tile's 128 h columns.
 // Two accumulators of 256 columns share TMEM columns [192, 256): the epilogue drains that
 // overlap first and releases the accumulator, so the next tile's MMAs overlap the rest of
 // the epilogue.  Scale factors use columns [448, 496).
 // SiLU * up epilogue: the B half of CTA 0 is 128 rows of the gate weight and the B half of
 // CTA 1 the same 128 rows of the up weight, so accumulator columns [0, 128) hold g and
-// [128, 256) hold u for 128 columns of h.  Each thread owns one row: it rounds g and u to
+// [128, 256) hold u for 128 columns of h.  Each thread owns 64 columns of one row: it rounds g and u to
 // bf16 exactly as the bf16 epilogue would, forms h, and quantizes each 16-value block with
 // the caller's global scale (64 code bytes and 8 scale bytes per row and tile).  Every
 // epilogue warp loads all its accumulator columns before any arithmetic and releases the
@@ -76,8 +76,9 @@ constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;  // 38 KB
 constexpr uint32_t kFp4TxBytes = 2u * kStageBytes;              // both CTAs
 constexpr uint32_t kLrTxBytes = 2u * (kABytes + kBBytes);
 constexpr int kMaxExperts = 1024;
-// Warps: 0 TMA producer, 1 MMA issuer, then the epilogue warps (two per TMEM lane quarter
-// for the SiLU * up epilogue, whose arithmetic needs more warps to hide its latency).
+// Warps: 0 TMA producer, 1 MMA issuer, then the epilogue warps: one per TMEM lane quarter
+// for the bf16 epilogue, two per quarter for the SiLU * up epilogue, whose arithmetic would
+// otherwise outlast the tile's mainloop (four per quarter measured the same).
 template <bool kSwiGLU>
 constexpr int kEpiWarps = kSwiGLU ? 8 : 4;
 template <bool kSwiGLU>
@@ -482,21 +483,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kSwiGLU>, 1
         uint8_t* sf_e = p.sf + static_cast<int64_t>(t.expert) * p.sf_item_stride;
         const uint32_t groups = static_cast<uint32_t>(p.n / 64);
         {
-          const int half = (warp - 2) >> 2;        // warps 2-5: columns [0, 64), warps 6-9: [64, 128)
-          uint32_t g[64], u[64];
-          tmem_load_64(tmem + col0 + half * 64 + lane_base, g);
-          tmem_load_64(tmem + col0 + 128 + half * 64 + lane_base, u);
-          tmem_wait_ld<64>(g);
-          tmem_wait_ld<64>(u);
+          constexpr int kQuarterWarps = kEpiWarps<true> / 4;   // epilogue warps per lane quarter
+          constexpr int kCols = 128 / kQuarterWarps;            // h columns of this warp
+          constexpr int kBlocks = kCols / 16;                   // 16-value blocks per thread
+          const int part = (warp - 2) >> 2;                     // which kCols-wide slice
+          uint32_t g[kCols], u[kCols];
+          if constexpr (kCols == 64) {
+            tmem_load_64(tmem + col0 + part * kCols + lane_base, g);
+            tmem_load_64(tmem + col0 + 128 + part * kCols + lane_base, u);
+          } else {
+            tmem_load_32(tmem + col0 + part * kCols + lane_base, g);
+            tmem_load_32(tmem + col0 + 128 + part * kCols + lane_base, u);
+          }
+          tmem_wait_ld<kCols>(g);
+          tmem_wait_ld<kCols>(u);
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
-          const uint32_t c0 = static_cast<uint32_t>(t.n_tile * 8 + half * 4);   // first block column
+          const uint32_t c0 = static_cast<uint32_t>(t.n_tile * 8 + part * kBlocks);   // first block column
           if (row_ok) {
-            uint32_t codes[8];
+            uint32_t codes[2 * kBlocks];
             uint32_t scales = 0;
 #pragma unroll
-            for (int blk = 0; blk < 4; ++blk) {
+            for (int blk = 0; blk < kBlocks; ++blk) {
               float h[16];
 #pragma unroll
               for (int e = 0; e < 16; e += 2) {
@@ -510,12 +519,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kSwiGLU>, 1
               codes[2 * blk + 1] = qb.hi;
               scales |= qb.s8 << (8 * blk);
             }
-            uint4* dst = reinterpret_cast<uint4*>(q_row + half * 32);
-            dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
-            dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
-            *reinterpret_cast<uint32_t*>(sf_e + sf_offset(static_cast<uint32_t>(row), c0, groups)) = scales;
+            uint4* dst = reinterpret_cast<uint4*>(q_row + part * (kCols / 2));
+            uint8_t* sdst = sf_e + sf_offset(static_cast<uint32_t>(row), c0, groups);
+            if constexpr (kBlocks == 4) {
+              dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+              dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+              *reinterpret_cast<uint32_t*>(sdst) = scales;
+            } else {
+              dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+              *reinterpret_cast<uint16_t*>(sdst) = static_cast<uint16_t>(scales);
+            }
           } else if (pad_row) {
-            *reinterpret_cast<uint32_t*>(sf_e + sf_offset(static_cast<uint32_t>(row), c0, groups)) = 0u;
+            uint8_t* sdst = sf_e + sf_offset(static_cast<uint32_t>(row), c0, groups);
+            if constexpr (kBlocks == 4) {
+              *reinterpret_cast<uint32_t*>(sdst) = 0u;
+            } else {
+              *reinterpret_cast<uint16_t*>(sdst) = 0;
+            }
           }
         }
       } else {
