@@ -316,6 +316,26 @@ NVFP4_API int nvfp4_get_pdl(void);
  */
 NVFP4_API int nvfp4_device_status(int *status_out, int clear);
 
+/*
+ * Self-tests of the failure detection (the pages have no counterpart; they exist so that
+ * the bounded waits can be exercised on a GPU without faulting or hanging it).
+ *
+ * nvfp4_selftest_bounded_wait launches one thread that waits, through the same bounded
+ * wait the GEMM kernels use, for an mbarrier phase that nothing ever completes; after about
+ * one second the wait gives up and NVFP4_ERR_DEVICE_TIMEOUT is recorded in the device
+ * status word (read it with nvfp4_device_status).
+ *
+ * nvfp4_selftest_gemm_stall runs nvfp4_gemm on the given operands (same arguments and
+ * constraints) with the loads of the first K stage of each pair's first tile withheld: the
+ * MMA issuer's wait for that stage runs out, records NVFP4_ERR_DEVICE_TIMEOUT, and every
+ * role of both CTAs of each pair unwinds (bounded drain, cluster barrier, tensor memory
+ * freed) within a few seconds.  out_bf16 is left unspecified.  The device stays usable.
+ */
+NVFP4_API int nvfp4_selftest_bounded_wait(nvfp4_stream_t stream);
+NVFP4_API int nvfp4_selftest_gemm_stall(const uint8_t *a, const uint8_t *b, const uint8_t *a_sf,
+                                        const uint8_t *b_sf, const float *alpha, void *out_bf16, int64_t m,
+                                        int64_t n, int64_t k, nvfp4_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -31,5 +31,7 @@ from .binding import (  # noqa: F401
     nvfp4_quantize_smooth_lora_down,
     nvfp4_set_pdl,
     nvfp4_get_pdl,
+    nvfp4_selftest_bounded_wait,
+    nvfp4_selftest_gemm_stall,
     nvfp4_device_status,
 )

@@ -32,6 +32,8 @@ EXPORTED_SYMBOLS = (
     "nvfp4_quantize_smooth_lora_down",
     "nvfp4_set_pdl",
     "nvfp4_get_pdl",
+    "nvfp4_selftest_bounded_wait",
+    "nvfp4_selftest_gemm_stall",
     "nvfp4_device_status",
 )
 
@@ -58,6 +60,8 @@ _SIGNATURES = {
     "nvfp4_quantize_smooth_lora_down": (_INT, [_P, _I64, _I64, _P, _P, _P, _I64, _P, _P, _P, _P]),
     "nvfp4_set_pdl": (_INT, [_INT]),
     "nvfp4_get_pdl": (_INT, []),
+    "nvfp4_selftest_bounded_wait": (_INT, [_P]),
+    "nvfp4_selftest_gemm_stall": (_INT, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "nvfp4_device_status": (_INT, [ctypes.POINTER(_INT), _INT]),
 }
 
@@ -336,6 +340,24 @@ def nvfp4_set_pdl(enable: bool) -> None:
 
 def nvfp4_get_pdl() -> bool:
     return bool(load_library().nvfp4_get_pdl())
+
+
+def nvfp4_selftest_bounded_wait(stream=None):
+    """Launch a wait that nothing completes; its bounded wait records NVFP4_ERR_DEVICE_TIMEOUT."""
+    with torch.cuda.device(torch.cuda.current_device()):
+        _check("nvfp4_selftest_bounded_wait", load_library().nvfp4_selftest_bounded_wait(_stream(stream)))
+
+
+def nvfp4_selftest_gemm_stall(a, b, a_sf, b_sf, alpha, out=None, stream=None):
+    """nvfp4_gemm with the first K stage's loads withheld: the MMA wait runs out and the kernel unwinds."""
+    m, kh = a.shape
+    n = b.shape[0]
+    out = torch.empty((m, n), dtype=torch.bfloat16, device=a.device) if out is None else out
+    with torch.cuda.device(a.device):
+        st = load_library().nvfp4_selftest_gemm_stall(_ptr(a), _ptr(b), _ptr(a_sf), _ptr(b_sf), _ptr(alpha),
+                                                      _ptr(out), m, n, 2 * kh, _stream(stream))
+    _check("nvfp4_selftest_gemm_stall", st)
+    return out
 
 
 def nvfp4_device_status(clear: bool = True) -> int:

@@ -220,6 +220,8 @@ struct GemmParams {
   uint8_t* sf;                // [E][nvfp4_scale_bytes(mmax, n)] swizzled scales of h
   int64_t sf_item_stride;     // nvfp4_scale_bytes(mmax, n)
   int32_t rows_pad;           // pad_up(mmax, 128)
+  int32_t stall_stage;        // self-test only: K stage of each pair's first tile whose loads
+                              // are withheld, so a bounded wait runs out (-1: none)
 };
 
 struct TileCoord {
@@ -351,7 +353,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kSwiGLU>, 1
         if (wrapped && !(ok = mbar_wait_fast(&ctl.empty[s], phase, abort, p.status))) break;
         uint8_t* st = smem + s * kStageBytes;
         const uint32_t full_bar = map_to_rank(&ctl.full[s], 0);
-        if (elect_one()) {
+        const bool withheld = ks == p.stall_stage && tile == pair;   // self-test: nothing completes it
+        if (!withheld && elect_one()) {
           if (ks < p.k_stages) {
             if (leader) mbar_arrive_expect_tx(&ctl.full[s], kFp4TxBytes);
             if constexpr (kGrouped) {
@@ -705,6 +708,7 @@ struct GemmArgs {
   const float *alpha2 = nullptr, *gsf_h = nullptr;
   uint8_t *q = nullptr, *sf = nullptr;
   int64_t E = 1, m = 0, n = 0, k = 0;      // n: output width (the width of h for SiLU * up)
+  int32_t stall_stage = -1;                // self-test only
 };
 
 template <bool kGrouped, bool kLowRank, bool kSwiGLU>
@@ -767,6 +771,7 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream) {
   p.k_stages = static_cast<int32_t>((k + kStageK - 1) / kStageK);
   p.k_steps = static_cast<int32_t>(k / 64);
   p.sf_groups = static_cast<int32_t>(k / 64);
+  p.stall_stage = g.stall_stage;
   if (kSwiGLU) {
     p.alpha_up = g.alpha2;
     p.gsf_h = g.gsf_h;
@@ -804,6 +809,19 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream) {
   const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
   return launch_kernel(kernel, dim3(2 * pairs), dim3(kThreads<kSwiGLU>), kSmemBytes<kGrouped, kSwiGLU>, stream, maps,
                        p);
+}
+
+// Self-test of the bounded wait: one thread waits for an mbarrier phase that nothing ever
+// completes; the wait gives up after its limit and records NVFP4_ERR_DEVICE_TIMEOUT.
+__global__ void bounded_wait_selftest_kernel(int* status) {
+  __shared__ uint64_t bar;
+  __shared__ int32_t abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, status);
 }
 
 }  // namespace
@@ -863,6 +881,23 @@ int nvfp4_grouped_gemm_silu_mul_quantize_masked(const uint8_t* a, const uint8_t*
   g.alpha = alpha_gate; g.alpha2 = alpha_up; g.gsf_h = gsf_h; g.q = q_out; g.sf = sf_out;
   g.E = E; g.m = mmax; g.n = n; g.k = k;
   return launch_gemm<true, false, true>(g, stream);
+}
+
+int nvfp4_selftest_bounded_wait(nvfp4_stream_t stream) {
+  DeviceInfo info;
+  int st = current_device(&info);
+  if (st != NVFP4_OK) return st;
+  return launch_kernel(bounded_wait_selftest_kernel, dim3(1), dim3(32), 0, stream, info.status);
+}
+
+int nvfp4_selftest_gemm_stall(const uint8_t* a, const uint8_t* b, const uint8_t* a_sf, const uint8_t* b_sf,
+                              const float* alpha, void* out_bf16, int64_t m, int64_t n, int64_t k,
+                              nvfp4_stream_t stream) {
+  GemmArgs g;
+  g.a = a; g.b = b; g.a_sf = a_sf; g.b_sf = b_sf; g.alpha = alpha; g.out = out_bf16;
+  g.m = m; g.n = n; g.k = k;
+  g.stall_stage = 0;
+  return launch_gemm<false, false, false>(g, stream);
 }
 
 }  // extern "C"
