@@ -258,6 +258,15 @@ NVFP4_API int nvfp4_grouped_gemm_silu_mul_quantize_masked(
     int64_t n, int64_t k, nvfp4_stream_t stream);
 
 /*
+ * SiLU-and-mul without quantization [FI3 silu_and_mul, the unfused reference of the
+ * fused quantizer]: h[r, c] = bf16(silu(x[r, c]) * x[r, k + c]) with silu(g) = g / (1 + exp(-g))
+ * and the library's specified fp32 exponential -- the same arithmetic, bit for bit, as
+ * nvfp4_silu_mul_quantize_batched and the SiLU * up GEMM epilogue.
+ *   x_bf16 [rows, 2k] bf16 (gate | up), h_bf16 [rows, k] bf16; k % 8 == 0; 16-byte aligned.
+ */
+NVFP4_API int nvfp4_silu_and_mul(const void *x_bf16, int64_t rows, int64_t k, void *h_bf16, nvfp4_stream_t stream);
+
+/*
  * Smooth quantize: the SVDQuant activation quantizer [FI5 mm_nvfp4_svdquant, Parameters a:
  * produced by nvfp4_quantize_smooth, which folds the pre-quantization scale in; TRT
  * pre_quant_scale].  x_hat[r, c] = bf16(x[r, c] * pre_quant_scale[c]) (one fp32

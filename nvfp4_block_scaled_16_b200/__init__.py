@@ -26,6 +26,7 @@ from .binding import (  # noqa: F401
     nvfp4_gemm_lowrank_bias,
     nvfp4_gemm_silu_mul_quantize,
     nvfp4_grouped_gemm_silu_mul_quantize_masked,
+    nvfp4_silu_and_mul,
     nvfp4_quantize_smooth,
     nvfp4_lora_down,
     nvfp4_quantize_smooth_lora_down,

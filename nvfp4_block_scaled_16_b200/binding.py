@@ -27,6 +27,7 @@ EXPORTED_SYMBOLS = (
     "nvfp4_gemm_lowrank_bias",
     "nvfp4_gemm_silu_mul_quantize",
     "nvfp4_grouped_gemm_silu_mul_quantize_masked",
+    "nvfp4_silu_and_mul",
     "nvfp4_quantize_smooth",
     "nvfp4_lora_down",
     "nvfp4_quantize_smooth_lora_down",
@@ -55,6 +56,7 @@ _SIGNATURES = {
     "nvfp4_gemm_lowrank_bias": (_INT, [_P, _P, _P, _P, _P, _P, _P, _I64, _P, _P, _I64, _I64, _I64, _P]),
     "nvfp4_gemm_silu_mul_quantize": (_INT, [_P] * 11 + [_I64, _I64, _I64, _P]),
     "nvfp4_grouped_gemm_silu_mul_quantize_masked": (_INT, [_P] * 12 + [_I64, _I64, _I64, _I64, _P]),
+    "nvfp4_silu_and_mul": (_INT, [_P, _I64, _I64, _P, _P]),
     "nvfp4_quantize_smooth": (_INT, [_P, _I64, _I64, _P, _P, _P, _P, _P]),
     "nvfp4_lora_down": (_INT, [_P, _I64, _I64, _P, _I64, _P, _P]),
     "nvfp4_quantize_smooth_lora_down": (_INT, [_P, _I64, _I64, _P, _P, _P, _I64, _P, _P, _P, _P]),
@@ -287,6 +289,18 @@ def nvfp4_grouped_gemm_silu_mul_quantize_masked(a, b_gate, b_up, a_sf, b_gate_sf
             _stream(stream))
     _check("nvfp4_grouped_gemm_silu_mul_quantize_masked", st)
     return q_out, sf_out
+
+
+def nvfp4_silu_and_mul(x, h_out=None, stream=None):
+    """x [rows, 2k] bf16 (gate | up) -> h [rows, k] bf16 = bf16(silu(gate) * up)."""
+    rows, w = x.shape
+    k = w // 2
+    if h_out is None:
+        h_out = torch.empty((rows, k), dtype=torch.bfloat16, device=x.device)
+    with torch.cuda.device(x.device):
+        st = load_library().nvfp4_silu_and_mul(_ptr(x), rows, k, _ptr(h_out), _stream(stream))
+    _check("nvfp4_silu_and_mul", st)
+    return h_out
 
 
 def nvfp4_quantize_smooth(x, pre_quant_scale, gsf, q_out=None, sf_out=None, stream=None):

@@ -114,18 +114,40 @@ __device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
 __device__ __forceinline__ uint64_t splat2(float v) { return pack2(v, v); }
 
 // exp_specified of a pair.  The input is clamped to [-104, 89], which leaves every result
-// unchanged (e^x overflows to +inf for x > 88.73 and rounds to 0 for x <= -104), and 2^n
-// is applied as two exact power-of-two multiplications 2^(n/2) * 2^(n - n/2): both halves
-// are normal numbers for n in [-150, 128], so only the last multiplication can round --
-// the same single rounding as the three-way scaling of exp_specified.  NaN stays NaN.
+// unchanged (e^x overflows to +inf for x > 88.73 and rounds to 0 for x <= -104).  The
+// polynomial value p lies in [0.7, 1.42], so p * 2^n is an exact normal number for
+// -125 <= n <= 127 (an exponent-field addition); otherwise 2^n is applied as two exact
+// power-of-two multiplications 2^(n/2) * 2^(n - n/2), both normal for n in [-150, 128], so
+// only the last can round -- the same single rounding as the scaling of exp_specified.
+// NaN stays NaN.
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// x * 2^n for an integer n given a normal p in [0.5, 2): the exponent field of p plus n when
+// the result is a normal number (-125 <= n <= 127), otherwise the two-step exact scaling.
+// Both give the correctly rounded p * 2^n (the first exactly, as the product is exact).
+__device__ __forceinline__ float scale_pow2(float p, int n) {
+  if (n >= -125 && n <= 127) return __int_as_float(__float_as_int(p) + (n << 23));
+  const int h = n / 2;
+  return __fmul_rn(__fmul_rn(p, pow2_int(h)), pow2_int(n - h));
+}
+
 __device__ __forceinline__ void exp_specified2(float x0, float x1, float& e0, float& e1) {
   const float c0 = fmaxf(fminf(x0, 89.0f), -104.0f);
   const float c1 = fmaxf(fminf(x1, 89.0f), -104.0f);
   const uint64_t x = pack2(c0, c1);
-  float t0, t1;
-  unpack2(mul2(x, splat2(0x1.715476p+0f)), t0, t1);
-  const float n0 = rintf(t0), n1 = rintf(t1);
-  const uint64_t n = pack2(n0, n1);
+  // n = rint(x * log2(e)): adding 1.5 * 2^23 rounds |t| < 2^22 to an integer (nearest,
+  // ties to even, as rint does); subtracting it back is exact, and the integer is the
+  // difference of the bit patterns.
+  const uint64_t t = mul2(x, splat2(0x1.715476p+0f));
+  const uint64_t tm = add2(t, splat2(0x1.8p+23f));
+  const uint64_t n = add2(tm, splat2(-0x1.8p+23f));
+  float tm0, tm1;
+  unpack2(tm, tm0, tm1);
+  const int i0 = __float_as_int(tm0) - 0x4B400000, i1 = __float_as_int(tm1) - 0x4B400000;
   uint64_t r = fma2(n, splat2(-0x1.62e4p-1f), x);
   r = fma2(n, splat2(-0x1.7f7d1cp-20f), r);
   uint64_t p = splat2(0x1.a01a02p-13f);
@@ -136,11 +158,10 @@ __device__ __forceinline__ void exp_specified2(float x0, float x1, float& e0, fl
   p = fma2(p, r, splat2(0x1.0p-1f));
   p = fma2(p, r, splat2(1.0f));
   p = fma2(p, r, splat2(1.0f));
-  const int i0 = static_cast<int>(n0), i1 = static_cast<int>(n1);
-  const int h0 = i0 / 2, h1 = i1 / 2;
-  p = mul2(p, pack2(pow2_int(h0), pow2_int(h1)));
-  p = mul2(p, pack2(pow2_int(i0 - h0), pow2_int(i1 - h1)));
-  unpack2(p, e0, e1);
+  float p0, p1;
+  unpack2(p, p0, p1);
+  e0 = scale_pow2(p0, i0);
+  e1 = scale_pow2(p1, i1);
   if (x0 != x0) e0 = x0;
   if (x1 != x1) e1 = x1;
 }

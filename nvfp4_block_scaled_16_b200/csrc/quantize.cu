@@ -150,6 +150,33 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantParams p)
   }
 }
 
+// ---- SiLU-and-mul without quantization ---------------------------------------------------
+
+// h[r, c] = bf16(silu(x[r, c]) * x[r, k + c]) for rows of width 2k; 8 outputs per thread.
+__global__ void __launch_bounds__(kThreads) silu_and_mul_kernel(const uint16_t* x, int64_t rows, int32_t k,
+                                                                uint16_t* h) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int64_t per_row = k / 8;
+  const int64_t total = rows * per_row;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * kThreads) {
+    const int64_t r = i / per_row;
+    const int64_t c = (i - r * per_row) * 8;
+    float g[8], u[8], o[8];
+    unpack_bf16x8(load_stream(x + r * 2 * k + c), g);
+    unpack_bf16x8(load_stream(x + r * 2 * k + k + c), u);
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) silu_mul_bf16_2(g[e], g[e + 1], u[e], u[e + 1], o[e], o[e + 1]);
+    uint4 w;
+    w.x = (__float_as_uint(o[0]) >> 16) | (__float_as_uint(o[1]) & 0xffff0000u);
+    w.y = (__float_as_uint(o[2]) >> 16) | (__float_as_uint(o[3]) & 0xffff0000u);
+    w.z = (__float_as_uint(o[4]) >> 16) | (__float_as_uint(o[5]) & 0xffff0000u);
+    w.w = (__float_as_uint(o[6]) >> 16) | (__float_as_uint(o[7]) & 0xffff0000u);
+    *reinterpret_cast<uint4*>(h + r * k + c) = w;
+  }
+}
+
 // ---- global scale reductions -------------------------------------------------------------
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -359,6 +386,21 @@ int nvfp4_global_scale_batched(const void* x_bf16, int64_t b, int64_t m, int64_t
 int nvfp4_quantize(const void* x_bf16, int64_t m, int64_t k, const float* gsf, uint8_t* q_out, uint8_t* sf_out,
                    nvfp4_stream_t stream) {
   return launch_quantize(x_bf16, 1, m, k, false, nullptr, gsf, q_out, sf_out, stream);
+}
+
+int nvfp4_silu_and_mul(const void* x_bf16, int64_t rows, int64_t k, void* h_bf16, nvfp4_stream_t stream) {
+  if (rows < 0 || k < 0 || k % 8 != 0 || k > (1 << 30)) return NVFP4_ERR_INVALID_ARGUMENT;
+  if (rows == 0 || k == 0) return NVFP4_OK;
+  if (!x_bf16 || !h_bf16 || !aligned(x_bf16, 16) || !aligned(h_bf16, 16)) return NVFP4_ERR_INVALID_ARGUMENT;
+  DeviceInfo info;
+  int st = current_device(&info);
+  if (st != NVFP4_OK) return st;
+  const int64_t total = rows * (k / 8);
+  int64_t blocks = (total + kThreads - 1) / kThreads;
+  blocks = blocks > info.sm_count * 16 ? info.sm_count * 16 : blocks;
+  return launch_kernel(silu_and_mul_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), 0, stream,
+                       static_cast<const uint16_t*>(x_bf16), rows, static_cast<int32_t>(k),
+                       static_cast<uint16_t*>(h_bf16));
 }
 
 int nvfp4_quantize_smooth(const void* x_bf16, int64_t m, int64_t k, const void* pre_quant_scale_bf16,

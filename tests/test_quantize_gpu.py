@@ -183,3 +183,25 @@ def test_silu_zero_up_and_zero_gate(oracle):
     check_masked(oracle, x, None, True)
     x = np.concatenate([np.zeros_like(g), g], axis=-1)      # silu(0) = 0
     check_masked(oracle, x, None, True)
+
+
+@pytest.mark.parametrize("u_kind", ["one", "negative", "random"])
+def test_silu_and_mul_every_bf16_gate_bit_exact(oracle, u_kind):
+    # every finite bf16 value as the gate (both signs, subnormals, |g| up to 3.4e38: the
+    # exponential's clamps at -104 / 89 and its 2^n scaling outside [-125, 127] are reached)
+    pats = np.arange(65536, dtype=np.uint32)
+    finite = ((pats >> 7) & 0xFF) != 0xFF
+    g = pats[finite].astype(np.uint16)
+    k = 256
+    g = np.concatenate([g, np.zeros((-len(g)) % k, np.uint16)]).reshape(-1, k)
+    if u_kind == "one":
+        u = np.full_like(g, 0x3F80)
+    elif u_kind == "negative":
+        u = np.full_like(g, S.f32_to_bf16_bits(np.float32([-3.5]))[0])
+    else:
+        u = S.normal_bf16(g.shape, 1.0, 5, S.TID["x"])
+    x = np.concatenate([g, u], axis=1)
+    h = nv.nvfp4_silu_and_mul(dev_bf16(x))
+    want = oracle.silu_mul(x)
+    got = host(h)
+    assert (got == want).all(), np.argwhere(got != want)[:5]
