@@ -648,3 +648,30 @@ def test_lora_down_matches_numpy_and_identity(oracle):
     eye = np.zeros((r, k), np.uint16)
     eye[np.arange(r), np.arange(r)] = BF16_ONE
     assert (oracle.lora_down(x, eye) == S.bf16_bits_to_f32(x[:, :r]).astype(np.float64)).all()
+
+
+def test_gemm_gate_up_bf16_rows(oracle):
+    # the [g | u] rows are the gate and up references rounded once to bf16; in the closed
+    # form of test_gemm_silu_mul_closed_form they are exactly 128 and +-2
+    m, n, k = 20, 64, 128
+    xa = S.normal_bf16((m, k), 1.0, seed=25)
+    xg = S.normal_bf16((n, k), 0.05, seed=25, tensor_id=2)
+    xu = S.normal_bf16((n, k), 0.05, seed=25, tensor_id=3)
+    ops = []
+    for x in (xa, xg, xu):
+        _, g = oracle.global_scale(x)
+        ops.append(oracle.quantize(x, g))
+    (qa, sa), (qg, sg), (qu, su) = ops
+    rows = np.array([0, 7, 19])
+    x = oracle.gemm_gate_up_bf16(qa, qg, qu, sa, sg, su, 0.75, 1.25, n, k, rows)
+    rg = oracle.gemm_ref(qa, qg, sa, sg, 0.75, m, n, k)[rows]
+    ru = oracle.gemm_ref(qa, qu, sa, su, 1.25, m, n, k)[rows]
+    to_bf16 = np.vectorize(oracle.f64_to_bf16, otypes=[np.uint16])
+    assert (x[:, :n] == to_bf16(rg)).all() and (x[:, n:] == to_bf16(ru)).all()
+    a = _pack(np.full((4, k), 0x2, np.uint8))
+    bg = _pack(np.full((n, k), 0x2, np.uint8))
+    bu = _pack(np.full((n, k), 0xA, np.uint8))
+    sa1 = np.full(oracle.scale_bytes(4, k), 0x38, np.uint8)
+    sb1 = np.full(oracle.scale_bytes(n, k), 0x38, np.uint8)
+    x = oracle.gemm_gate_up_bf16(a, bg, bu, sa1, sb1, sb1, 1.0, 1.0 / 64, n, k, np.arange(4))
+    assert (x[:, :n] == 0x4300).all() and (x[:, n:] == 0xC000).all()      # bf16 128 and -2
