@@ -16,10 +16,12 @@ struct DeviceInfo {
   int device = -1;
   int sm_count = 0;
   int* status = nullptr;  // device-side status word (NVFP4_OK or NVFP4_ERR_DEVICE_TIMEOUT)
+  const float* silu_table = nullptr;  // SiLU of every bf16 value the closed forms do not cover
 };
 
 // Checks that the current device is compute capability 10.0 and returns its info; the
-// first call on a device allocates the status word.
+// first call on a device allocates the status word and computes the SiLU table (one kernel
+// on the legacy default stream, waited for before returning).
 int current_device(DeviceInfo* out);
 
 // Library-owned scratch of the global-scale reductions, one per (device, stream): word 0

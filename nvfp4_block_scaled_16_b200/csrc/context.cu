@@ -5,9 +5,15 @@
 #include <utility>
 
 #include "common.cuh"
+#include "nvfp4_math.cuh"
 
 namespace nvfp4 {
 namespace {
+
+__global__ void silu_table_kernel(float* tab) {
+  const uint32_t i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < kSiluEntries) tab[i] = silu_table_entry(i);
+}
 
 std::mutex g_mu;
 std::atomic<int> g_pdl{1};      // programmatic dependent launch, on by default (sm_100 supports it)
@@ -43,7 +49,21 @@ int current_device(DeviceInfo* out) {
       cudaFree(status);
       return NVFP4_ERR_CUDA;
     }
+    float* tab = nullptr;
+    if (cudaMalloc(&tab, kSiluTableBytes) != cudaSuccess) {
+      cudaGetLastError();
+      cudaFree(status);
+      return NVFP4_ERR_OUT_OF_MEMORY;
+    }
+    silu_table_kernel<<<(kSiluEntries + 255) / 256, 256>>>(tab);
+    if (cudaGetLastError() != cudaSuccess || cudaStreamSynchronize(0) != cudaSuccess) {
+      cudaGetLastError();
+      cudaFree(tab);
+      cudaFree(status);
+      return NVFP4_ERR_CUDA;
+    }
     d.status = status;
+    d.silu_table = tab;
     d.sm_count = sms;
     d.device = dev;
   }

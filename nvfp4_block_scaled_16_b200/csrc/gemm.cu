@@ -107,13 +107,16 @@ template <bool kGrouped, bool kSwiGLU>
 constexpr int kStagingBuffers = kSwiGLU ? 0 : (kGrouped ? 1 : 2);
 template <bool kGrouped, bool kSwiGLU>
 constexpr int kStagingBytes = kStagingBuffers<kGrouped, kSwiGLU> * kEpiWarps<false> * kStoreTileBytes;
+// SiLU * up epilogue: the SiLU table (31 KB) after the ring.
+template <bool kSwiGLU>
+constexpr int kTableBytes = kSwiGLU ? static_cast<int>(kSiluTableBytes) : 0;
 // The expert prefix table (the last member of Control) is only allocated for grouped kernels.
 template <bool kGrouped>
 constexpr int kControlBytes = kGrouped ? static_cast<int>(sizeof(Control))
                                        : static_cast<int>(offsetof(Control, prefix)) + 8;
 template <bool kGrouped, bool kSwiGLU>
 constexpr int kSmemBytes =
-    kStages * kStageBytes + kStagingBytes<kGrouped, kSwiGLU> + kControlBytes<kGrouped> + 1024;
+    kStages * kStageBytes + kStagingBytes<kGrouped, kSwiGLU> + kTableBytes<kSwiGLU> + kControlBytes<kGrouped> + 1024;
 constexpr int kMaxDynamicSmem = 227 * 1024;      // sm_100 opt-in limit per block
 static_assert(kSmemBytes<false, false> <= kMaxDynamicSmem && kSmemBytes<true, false> <= kMaxDynamicSmem &&
                   kSmemBytes<false, true> <= kMaxDynamicSmem && kSmemBytes<true, true> <= kMaxDynamicSmem,
@@ -222,6 +225,7 @@ struct GemmParams {
   int32_t rows_pad;           // pad_up(mmax, 128)
   int32_t stall_stage;        // self-test only: K stage of each pair's first tile whose loads
                               // are withheld, so a bounded wait runs out (-1: none)
+  const float* silu_tab;      // SiLU * up epilogue: the SiLU table in global memory
 };
 
 struct TileCoord {
@@ -265,7 +269,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kSwiGLU>, 1
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* staging = smem + kStages * kStageBytes;     // 1024-byte aligned (the ring is 190 KB)
-  Control& ctl = *reinterpret_cast<Control*>(staging + kStagingBytes<kGrouped, kSwiGLU>);
+  float* silu_tab = reinterpret_cast<float*>(staging + kStagingBytes<kGrouped, kSwiGLU>);
+  Control& ctl = *reinterpret_cast<Control*>(staging + kStagingBytes<kGrouped, kSwiGLU> + kTableBytes<kSwiGLU>);
   volatile int32_t* abort = &ctl.abort;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -461,6 +466,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kSwiGLU>, 1
     const int row_in_tile = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t acc_empty_leader = map_to_rank(&ctl.acc_empty, 0);
+    if constexpr (kSwiGLU) {
+      // the epilogue warps load the SiLU table while the first tile's mainloop runs
+      silu_table_load(silu_tab, p.silu_tab, threadIdx.x - 64, 32 * kEpiWarps<true>);
+      asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpiWarps<true>) : "memory");
+    }
     uint32_t tcount = 0;
     TileCoord t;
     uint32_t nstore = 0;                       // TMA stores issued by this warp (bf16 epilogue)
@@ -515,7 +525,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kSwiGLU>, 1
                 float g0, g1, u0, u1;
                 scale_round_bf16_2(alpha, g[16 * blk + e], g[16 * blk + e + 1], g0, g1);
                 scale_round_bf16_2(alpha_u, u[16 * blk + e], u[16 * blk + e + 1], u0, u1);
-                silu_mul_bf16_2(g0, g1, u0, u1, h[e], h[e + 1]);
+                silu_mul_bf16_tab2(silu_tab, g0, g1, u0, u1, h[e], h[e + 1]);
               }
               const QBlock qb = quantize16(h, gsf);
               codes[2 * blk] = qb.lo;
@@ -761,6 +771,7 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream) {
   p.out = static_cast<__nv_bfloat16*>(g.out);
   p.mask = g.mask;
   p.status = info.status;
+  p.silu_tab = info.silu_table;
   p.m = static_cast<int32_t>(m);
   p.n = static_cast<int32_t>(n);
   p.k = static_cast<int32_t>(k);

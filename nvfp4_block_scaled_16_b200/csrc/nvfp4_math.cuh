@@ -113,71 +113,62 @@ __device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
 }
 __device__ __forceinline__ uint64_t splat2(float v) { return pack2(v, v); }
 
-// exp_specified of a pair.  The input is clamped to [-104, 89], which leaves every result
-// unchanged (e^x overflows to +inf for x > 88.73 and rounds to 0 for x <= -104).  The
-// polynomial value p lies in [0.7, 1.42], so p * 2^n is an exact normal number for
-// -125 <= n <= 127 (an exponent-field addition); otherwise 2^n is applied as two exact
-// power-of-two multiplications 2^(n/2) * 2^(n - n/2), both normal for n in [-150, 128], so
-// only the last can round -- the same single rounding as the scaling of exp_specified.
-// NaN stays NaN.
-__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
+// ---- SiLU of a bf16 value: closed forms and a per-device table ---------------------------
+// s(g) = g / (1 + exp_specified(-g)) (one correctly rounded addition and division) depends
+// only on the 16 bits of a bf16 g, so the kernels read it from a table that is computed once
+// per device with exactly that arithmetic.  Outside the magnitude ranges the table covers,
+// s has closed forms that follow from the definition of exp_specified:
+//   |g| < 2^-25: n = 0 and both Horner steps that add 1 round to 1, so e = 1, 1 + e = 2 and
+//     s = g / 2, exact for every bf16 g (subnormal ones included);
+//   g >= 24: e = exp_specified(-g) < 2^-34 is below half an ulp of 1, so 1 + e = 1 and s = g;
+//   g <= -96: the argument of exp_specified exceeds 89, e = +inf and s = g / inf = -0,
+//     written g * 0 so that -inf and NaN give NaN as the division does.
+// Table entry i < kSiluPos holds s(+g) and entry kSiluPos + i holds s(-g) for the bf16 g of
+// magnitude pattern kSiluMagLo + i.
+constexpr uint32_t kSiluMagLo = 0x3300;                 // 2^-25
+constexpr uint32_t kSiluPos = 0x41c0 - kSiluMagLo;      // up to 24: 3776 entries
+constexpr uint32_t kSiluNeg = 0x42c0 - kSiluMagLo;      // up to 96: 4032 entries
+constexpr uint32_t kSiluEntries = kSiluPos + kSiluNeg;
+constexpr uint32_t kSiluTableBytes = kSiluEntries * 4;  // 31 232 bytes, a multiple of 16
+
+// Table entry i, computed with the scalar definition.
+__device__ __forceinline__ float silu_table_entry(uint32_t i) {
+  const bool neg = i >= kSiluPos;
+  const uint32_t mag = kSiluMagLo + (neg ? i - kSiluPos : i);
+  const float g = __uint_as_float(((neg ? 0x8000u : 0u) | mag) << 16);
+  return __fdiv_rn(g, __fadd_rn(1.0f, exp_specified(-g)));
 }
 
-// x * 2^n for an integer n given a normal p in [0.5, 2): the exponent field of p plus n when
-// the result is a normal number (-125 <= n <= 127), otherwise the two-step exact scaling.
-// Both give the correctly rounded p * 2^n (the first exactly, as the product is exact).
-__device__ __forceinline__ float scale_pow2(float p, int n) {
-  if (n >= -125 && n <= 127) return __int_as_float(__float_as_int(p) + (n << 23));
-  const int h = n / 2;
-  return __fmul_rn(__fmul_rn(p, pow2_int(h)), pow2_int(n - h));
+// s(g) for a bf16-valued g (the low 16 bits of its fp32 pattern are zero), from the table
+// `tab` (shared memory) or the closed forms.
+__device__ __forceinline__ float silu_lookup(const float* tab, float g) {
+  const uint32_t bits = __float_as_uint(g);
+  const uint32_t neg = bits >> 31;
+  const uint32_t off = ((bits >> 16) & 0x7fffu) - kSiluMagLo;   // wraps below 2^-25
+  if (off < (neg ? kSiluNeg : kSiluPos)) return tab[off + (neg ? kSiluPos : 0u)];
+  const float f = (off & 0x80000000u) ? 0.5f : (neg ? 0.0f : 1.0f);
+  return __fmul_rn(g, f);
 }
 
-__device__ __forceinline__ void exp_specified2(float x0, float x1, float& e0, float& e1) {
-  const float c0 = fmaxf(fminf(x0, 89.0f), -104.0f);
-  const float c1 = fmaxf(fminf(x1, 89.0f), -104.0f);
-  const uint64_t x = pack2(c0, c1);
-  // n = rint(x * log2(e)): adding 1.5 * 2^23 rounds |t| < 2^22 to an integer (nearest,
-  // ties to even, as rint does); subtracting it back is exact, and the integer is the
-  // difference of the bit patterns.
-  const uint64_t t = mul2(x, splat2(0x1.715476p+0f));
-  const uint64_t tm = add2(t, splat2(0x1.8p+23f));
-  const uint64_t n = add2(tm, splat2(-0x1.8p+23f));
-  float tm0, tm1;
-  unpack2(tm, tm0, tm1);
-  const int i0 = __float_as_int(tm0) - 0x4B400000, i1 = __float_as_int(tm1) - 0x4B400000;
-  uint64_t r = fma2(n, splat2(-0x1.62e4p-1f), x);
-  r = fma2(n, splat2(-0x1.7f7d1cp-20f), r);
-  uint64_t p = splat2(0x1.a01a02p-13f);
-  p = fma2(p, r, splat2(0x1.6c16c2p-10f));
-  p = fma2(p, r, splat2(0x1.111112p-7f));
-  p = fma2(p, r, splat2(0x1.555556p-5f));
-  p = fma2(p, r, splat2(0x1.555556p-3f));
-  p = fma2(p, r, splat2(0x1.0p-1f));
-  p = fma2(p, r, splat2(1.0f));
-  p = fma2(p, r, splat2(1.0f));
-  float p0, p1;
-  unpack2(p, p0, p1);
-  e0 = scale_pow2(p0, i0);
-  e1 = scale_pow2(p1, i1);
-  if (x0 != x0) e0 = x0;
-  if (x1 != x1) e1 = x1;
-}
-
-// silu_mul_bf16 of a pair: h = bf16((g / (1 + exp(-g))) * u), as fp32 values.
-__device__ __forceinline__ void silu_mul_bf16_2(float g0, float g1, float u0, float u1, float& h0, float& h1) {
-  float e0, e1;
-  exp_specified2(-g0, -g1, e0, e1);
-  const float s0 = __fdiv_rn(g0, __fadd_rn(1.0f, e0));
-  const float s1 = __fdiv_rn(g1, __fadd_rn(1.0f, e1));
+// h = bf16(s(g) * u) for a pair of bf16-valued g, as fp32 values; equal to silu_mul_bf16.
+__device__ __forceinline__ void silu_mul_bf16_tab2(const float* tab, float g0, float g1, float u0, float u1,
+                                                   float& h0, float& h1) {
+  const float s0 = silu_lookup(tab, g0);
+  const float s1 = silu_lookup(tab, g1);
   float p0, p1;
   unpack2(mul2(pack2(s0, s1), pack2(u0, u1)), p0, p1);
   uint32_t b2;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(b2) : "f"(p1), "f"(p0));   // p0 -> low half
   h0 = __uint_as_float(b2 << 16);
   h1 = __uint_as_float(b2 & 0xffff0000u);
+}
+
+// Copies the table from global memory into shared memory with `threads` threads starting at
+// thread index `t`; the caller synchronizes before the first lookup.
+__device__ __forceinline__ void silu_table_load(float* dst, const float* src, int t, int threads) {
+  const uint4* s = reinterpret_cast<const uint4*>(src);
+  uint4* d = reinterpret_cast<uint4*>(dst);
+  for (int i = t; i < static_cast<int>(kSiluTableBytes / 16); i += threads) d[i] = __ldg(s + i);
 }
 
 // ---- one 16-element block ------------------------------------------------------------------
@@ -187,11 +178,22 @@ struct QBlock {
   uint32_t s8;      // ue4m3 scale code
 };
 
+// vmax / 6, correctly rounded, for a bf16-valued vmax >= 0: the product with fp32(1/6)
+// followed by one Markstein correction step (the remainder vmax - 6q is exact as an fma,
+// and q + rem/6 is rounded once).  It equals the IEEE division for every non-negative
+// finite bf16 value (checked exhaustively); +inf passes through as the division would.
+__device__ __forceinline__ float div6_bf16(float vmax) {
+  const float q = __fmul_rn(vmax, 0x1.555556p-3f);
+  const float rem = __fmaf_rn(-q, 6.0f, vmax);
+  return vmax == __uint_as_float(0x7f800000u) ? vmax : __fmaf_rn(rem, 0x1.555556p-3f, q);
+}
+
+// One 16-element block of bf16-valued inputs.
 __device__ __forceinline__ QBlock quantize16(const float* v, float gsf) {
   float vmax = 0.0f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) vmax = fmaxf(vmax, fabsf(v[i]));
-  const float s32 = __fmul_rn(__fdiv_rn(vmax, 6.0f), gsf);
+  const float s32 = __fmul_rn(div6_bf16(vmax), gsf);
   QBlock b;
   b.s8 = ue4m3_encode(s32);
   const float sd = e4m3_decode(b.s8);

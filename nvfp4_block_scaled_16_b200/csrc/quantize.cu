@@ -62,19 +62,21 @@ struct QuantParams {
   uint32_t cpad;           // pad_up(nb, 4)
   uint32_t rows_pad;       // pad_up(m, 128)
   uint32_t blocks;         // rows_pad * cpad (per item)
+  const float* silu_tab;   // SiLU table in global memory (SiLU variant)
+  uint32_t chunks_per_item;
+  uint32_t items;
 };
 
+// One chunk of kThreads * kUnroll consecutive 16-element blocks of item `item`, starting at
+// block `base` (row-major over rows_pad x cpad).  With kSilu, `tab` is the SiLU table in
+// shared memory.
 template <bool kSilu, bool kSmooth, int kUnroll>
-__global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantParams p) {
-  pdl_launch_dependents();
-  pdl_wait();
-  const int item = blockIdx.y;
+__device__ __forceinline__ void quantize_chunk(const QuantParams& p, int item, uint32_t base, const float* tab) {
   int valid = p.m;
   if (p.mask) valid = min(max(__ldg(p.mask + item), 0), p.m);
   // Rows at or beyond `limit` are never touched: with a mask, rows >= mask; without one,
   // only the padding rows beyond rows_pad (which do not exist).
   const uint32_t limit = p.mask ? static_cast<uint32_t>(valid) : p.rows_pad;
-  const uint32_t base = blockIdx.x * (kThreads * kUnroll);
   if (base / p.cpad >= limit) return;
 
   const float gsf = __ldg(p.gsf + item);
@@ -119,7 +121,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantParams p)
         unpack_bf16x8(raw[u][2], up);
         unpack_bf16x8(raw[u][3], up + 8);
 #pragma unroll
-        for (int i = 0; i < 16; i += 2) silu_mul_bf16_2(v[i], v[i + 1], up[i], up[i + 1], v[i], v[i + 1]);
+        for (int i = 0; i < 16; i += 2) silu_mul_bf16_tab2(tab, v[i], v[i + 1], up[i], up[i + 1], v[i], v[i + 1]);
       }
       if constexpr (kSmooth) {
         // x_hat = bf16(x * pre_quant_scale) for the block's 16 columns (the scale vector is
@@ -150,13 +152,47 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantParams p)
   }
 }
 
+// One chunk per CTA: grid (chunks per item, items).
+template <bool kSmooth, int kUnroll>
+__global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantParams p) {
+  pdl_launch_dependents();
+  pdl_wait();
+  quantize_chunk<false, kSmooth, kUnroll>(p, blockIdx.y, blockIdx.x * (kThreads * kUnroll), nullptr);
+}
+
+// SiLU * up: persistent CTAs that load the SiLU table into shared memory once and walk the
+// chunks of all items (item-major) with a grid stride, so the live chunks of every item are
+// spread over all CTAs whatever the masks are.
+constexpr int kSiluUnroll = 2;
+constexpr int kSiluCtasPerSm = 4;
+// The table fits the default 48 KB of dynamic shared memory (no opt-in attribute needed).
+static_assert(kSiluTableBytes <= 48 * 1024, "SiLU table exceeds the default dynamic shared memory");
+__global__ void __launch_bounds__(kThreads, kSiluCtasPerSm) silu_quantize_kernel(const QuantParams p) {
+  extern __shared__ float4 silu_smem[];
+  float* tab = reinterpret_cast<float*>(silu_smem);
+  pdl_launch_dependents();
+  pdl_wait();
+  silu_table_load(tab, p.silu_tab, threadIdx.x, kThreads);
+  __syncthreads();
+  const uint64_t total = static_cast<uint64_t>(p.chunks_per_item) * p.items;
+  for (uint64_t chunk = blockIdx.x; chunk < total; chunk += gridDim.x) {
+    const uint32_t item = static_cast<uint32_t>(chunk / p.chunks_per_item);
+    const uint32_t local = static_cast<uint32_t>(chunk - static_cast<uint64_t>(item) * p.chunks_per_item);
+    quantize_chunk<true, false, kSiluUnroll>(p, static_cast<int>(item), local * (kThreads * kSiluUnroll), tab);
+  }
+}
+
 // ---- SiLU-and-mul without quantization ---------------------------------------------------
 
 // h[r, c] = bf16(silu(x[r, c]) * x[r, k + c]) for rows of width 2k; 8 outputs per thread.
 __global__ void __launch_bounds__(kThreads) silu_and_mul_kernel(const uint16_t* x, int64_t rows, int32_t k,
-                                                                uint16_t* h) {
+                                                                uint16_t* h, const float* silu_tab) {
+  extern __shared__ float4 silu_smem[];
+  float* tab = reinterpret_cast<float*>(silu_smem);
   pdl_launch_dependents();
   pdl_wait();
+  silu_table_load(tab, silu_tab, threadIdx.x, kThreads);
+  __syncthreads();
   const int64_t per_row = k / 8;
   const int64_t total = rows * per_row;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; i < total;
@@ -167,7 +203,7 @@ __global__ void __launch_bounds__(kThreads) silu_and_mul_kernel(const uint16_t* 
     unpack_bf16x8(load_stream(x + r * 2 * k + c), g);
     unpack_bf16x8(load_stream(x + r * 2 * k + k + c), u);
 #pragma unroll
-    for (int e = 0; e < 8; e += 2) silu_mul_bf16_2(g[e], g[e + 1], u[e], u[e + 1], o[e], o[e + 1]);
+    for (int e = 0; e < 8; e += 2) silu_mul_bf16_tab2(tab, g[e], g[e + 1], u[e], u[e + 1], o[e], o[e + 1]);
     uint4 w;
     w.x = (__float_as_uint(o[0]) >> 16) | (__float_as_uint(o[1]) & 0xffff0000u);
     w.y = (__float_as_uint(o[2]) >> 16) | (__float_as_uint(o[3]) & 0xffff0000u);
@@ -320,15 +356,21 @@ int launch_quantize(const void* x, int64_t b, int64_t m, int64_t k, bool silu, c
   p.cpad = static_cast<uint32_t>(cpad);
   p.rows_pad = static_cast<uint32_t>(rows_pad);
   p.blocks = static_cast<uint32_t>(rows_pad * cpad);
+  p.silu_tab = info.silu_table;
+  p.items = static_cast<uint32_t>(b);
   if (silu) {
-    constexpr int U = 2;
-    dim3 grid(static_cast<unsigned>((p.blocks + kThreads * U - 1) / (kThreads * U)), static_cast<unsigned>(b));
-    return launch_kernel(quantize_kernel<true, false, U>, grid, dim3(kThreads), 0, stream, p);
+    constexpr int U = kSiluUnroll;
+    p.chunks_per_item = (p.blocks + kThreads * U - 1) / (kThreads * U);
+    const int64_t chunks = static_cast<int64_t>(p.chunks_per_item) * b;
+    const int64_t cap = static_cast<int64_t>(info.sm_count) * kSiluCtasPerSm;
+    return launch_kernel(silu_quantize_kernel, dim3(static_cast<unsigned>(chunks < cap ? chunks : cap)),
+                         dim3(kThreads), kSiluTableBytes, stream, p);
   }
   constexpr int U = 4;
-  dim3 grid(static_cast<unsigned>((p.blocks + kThreads * U - 1) / (kThreads * U)), static_cast<unsigned>(b));
-  if (pqs) return launch_kernel(quantize_kernel<false, true, U>, grid, dim3(kThreads), 0, stream, p);
-  return launch_kernel(quantize_kernel<false, false, U>, grid, dim3(kThreads), 0, stream, p);
+  p.chunks_per_item = (p.blocks + kThreads * U - 1) / (kThreads * U);
+  dim3 grid(p.chunks_per_item, static_cast<unsigned>(b));
+  if (pqs) return launch_kernel(quantize_kernel<true, U>, grid, dim3(kThreads), 0, stream, p);
+  return launch_kernel(quantize_kernel<false, U>, grid, dim3(kThreads), 0, stream, p);
 }
 
 }  // namespace
@@ -397,10 +439,10 @@ int nvfp4_silu_and_mul(const void* x_bf16, int64_t rows, int64_t k, void* h_bf16
   if (st != NVFP4_OK) return st;
   const int64_t total = rows * (k / 8);
   int64_t blocks = (total + kThreads - 1) / kThreads;
-  blocks = blocks > info.sm_count * 16 ? info.sm_count * 16 : blocks;
-  return launch_kernel(silu_and_mul_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), 0, stream,
-                       static_cast<const uint16_t*>(x_bf16), rows, static_cast<int32_t>(k),
-                       static_cast<uint16_t*>(h_bf16));
+  blocks = blocks > info.sm_count * 4 ? info.sm_count * 4 : blocks;
+  return launch_kernel(silu_and_mul_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), kSiluTableBytes,
+                       stream, static_cast<const uint16_t*>(x_bf16), rows, static_cast<int32_t>(k),
+                       static_cast<uint16_t*>(h_bf16), info.silu_table);
 }
 
 int nvfp4_quantize_smooth(const void* x_bf16, int64_t m, int64_t k, const void* pre_quant_scale_bf16,
