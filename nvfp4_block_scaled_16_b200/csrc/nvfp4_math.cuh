@@ -89,9 +89,8 @@ __device__ __forceinline__ float silu_mul_bf16(float g, float u) {
   return __bfloat162float(__float2bfloat16_rn(p));
 }
 
-// ---- the same arithmetic on pairs of values with packed f32x2 instructions -----------------
-// Each lane of fma/mul/add.rn.f32x2 is one correctly rounded fp32 operation, so the pair
-// functions return exactly what the scalar ones return.
+// ---- pairs of values in packed f32x2 registers ----------------------------------------------
+// Each lane of mul.rn.f32x2 is one correctly rounded fp32 multiplication.
 
 __device__ __forceinline__ uint64_t pack2(float lo, float hi) {
   uint64_t r;
@@ -100,11 +99,6 @@ __device__ __forceinline__ uint64_t pack2(float lo, float hi) {
 }
 __device__ __forceinline__ void unpack2(uint64_t v, float& lo, float& hi) {
   asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
 }
 __device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
   uint64_t d;
