@@ -76,13 +76,14 @@ constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;  // 38 KB
 constexpr uint32_t kFp4TxBytes = 2u * kStageBytes;              // both CTAs
 constexpr uint32_t kLrTxBytes = 2u * (kABytes + kBBytes);
 constexpr int kMaxExperts = 1024;
-// Warps: 0 TMA producer, 1 MMA issuer, then the epilogue warps: one per TMEM lane quarter
-// for the bf16 epilogue, two per quarter for the SiLU * up epilogue, whose arithmetic would
-// otherwise outlast the tile's mainloop (four per quarter measured the same).
-template <bool kSwiGLU>
-constexpr int kEpiWarps = kSwiGLU ? 8 : 4;
-template <bool kSwiGLU>
-constexpr int kThreads = 64 + 32 * kEpiWarps<kSwiGLU>;
+// Warps: 0 TMA producer, 1 MMA issuer, then the epilogue warps: two per TMEM lane quarter
+// (each drains half of the tile's columns, so a tile's epilogue takes about half the time of
+// one warp per quarter), except in the grouped bf16 kernel, whose expert prefix table leaves
+// shared memory for the staging tiles of one warp per quarter only.
+template <bool kGrouped, bool kSwiGLU>
+constexpr int kEpiWarps = (kGrouped && !kSwiGLU) ? 4 : 8;
+template <bool kGrouped, bool kSwiGLU>
+constexpr int kThreads = 64 + 32 * kEpiWarps<kGrouped, kSwiGLU>;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccOverlapCol = 192;          // accumulator 1 starts here
 constexpr uint32_t kSfaCol = 448;                 // SFA: 448 + 4j, SFB: 464 + 8j (+4 upper half)
@@ -98,16 +99,14 @@ struct __align__(8) Control {
   int32_t abort;
   int32_t prefix[kMaxExperts + 1];   // grouped: prefix sums of pair tiles per expert
 };
-// bf16 epilogue: 32-row x 64-column bf16 staging tiles (4 KB, 128-byte swizzle) per
-// epilogue warp, written to global memory by TMA stores; two per warp (one store in flight
-// while the next tile is written) where shared memory allows, one in the grouped kernels
-// (whose expert prefix table takes the room).
+// bf16 epilogue: one 32-row x 64-column bf16 staging tile (4 KB, 128-byte swizzle) per
+// epilogue warp, written to global memory by TMA stores.
 constexpr int kStoreTileBytes = 32 * 128;
 template <bool kGrouped, bool kSwiGLU>
-constexpr int kStagingBuffers = kSwiGLU ? 0 : (kGrouped ? 1 : 2);
+constexpr int kStagingBuffers = kSwiGLU ? 0 : 1;
 template <bool kGrouped, bool kSwiGLU>
-constexpr int kStagingBytes = kStagingBuffers<kGrouped, kSwiGLU> * kEpiWarps<false> * kStoreTileBytes;
-// SiLU * up epilogue: the SiLU table (31 KB) after the ring.
+constexpr int kStagingBytes = kStagingBuffers<kGrouped, kSwiGLU> * kEpiWarps<kGrouped, kSwiGLU> * kStoreTileBytes;
+// SiLU * up epilogue: the SiLU table (32 KB) after the ring.
 template <bool kSwiGLU>
 constexpr int kTableBytes = kSwiGLU ? static_cast<int>(kSiluTableBytes) : 0;
 // The expert prefix table (the last member of Control) is only allocated for grouped kernels.
@@ -188,14 +187,14 @@ __device__ __forceinline__ void mma_commit_both(uint64_t* bar) {
       : "memory");
 }
 
-// bf16(alpha * a), bf16(alpha * b) as fp32 values: the rounding of the bf16 epilogue.
-__device__ __forceinline__ void scale_round_bf16_2(float alpha, uint32_t a, uint32_t b, float& ra, float& rb) {
+// bf16(alpha * a), bf16(alpha * b) packed (a in the low half): the rounding of the bf16
+// epilogue, applied to two fp32 accumulator values given as bits.
+__device__ __forceinline__ uint32_t scale_round_bf16x2(float alpha, uint32_t a, uint32_t b) {
   float pa, pb;
   unpack2(mul2(pack2(__uint_as_float(a), __uint_as_float(b)), splat2(alpha)), pa, pb);
   uint32_t w;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w) : "f"(pb), "f"(pa));   // pa -> low half
-  ra = __uint_as_float(w << 16);
-  rb = __uint_as_float(w & 0xffff0000u);
+  return w;
 }
 
 // ---- problem description ----------------------------------------------------------------------
@@ -264,7 +263,7 @@ struct Maps {
 // ---- the kernel ---------------------------------------------------------------------------------
 
 template <bool kGrouped, bool kLowRank, bool kSwiGLU>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kSwiGLU>, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kGrouped, kSwiGLU>, 1)
     nvfp4_gemm_kernel(const __grid_constant__ Maps maps, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -285,7 +284,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kSwiGLU>, 1
       mbar_init(&ctl.empty[s], 1);
     }
     mbar_init(&ctl.acc_full, 1);
-    mbar_init(&ctl.acc_empty, 2 * kEpiWarps<kSwiGLU>);   // every epilogue warp of both CTAs
+    mbar_init(&ctl.acc_empty, 2 * kEpiWarps<kGrouped, kSwiGLU>);   // every epilogue warp of both CTAs
     ctl.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -468,8 +467,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kSwiGLU>, 1
     const uint32_t acc_empty_leader = map_to_rank(&ctl.acc_empty, 0);
     if constexpr (kSwiGLU) {
       // the epilogue warps load the SiLU table while the first tile's mainloop runs
-      silu_table_load(silu_tab, p.silu_tab, threadIdx.x - 64, 32 * kEpiWarps<true>);
-      asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpiWarps<true>) : "memory");
+      silu_table_load(silu_tab, p.silu_tab, threadIdx.x - 64, 32 * kEpiWarps<kGrouped, true>);
+      asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpiWarps<kGrouped, true>) : "memory");
     }
     uint32_t tcount = 0;
     TileCoord t;
@@ -496,7 +495,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kSwiGLU>, 1
         uint8_t* sf_e = p.sf + static_cast<int64_t>(t.expert) * p.sf_item_stride;
         const uint32_t groups = static_cast<uint32_t>(p.n / 64);
         {
-          constexpr int kQuarterWarps = kEpiWarps<true> / 4;   // epilogue warps per lane quarter
+          constexpr int kQuarterWarps = kEpiWarps<kGrouped, true> / 4;   // epilogue warps per lane quarter
           constexpr int kCols = 128 / kQuarterWarps;            // h columns of this warp
           constexpr int kBlocks = kCols / 16;                   // 16-value blocks per thread
           const int part = (warp - 2) >> 2;                     // which kCols-wide slice
@@ -522,10 +521,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kSwiGLU>, 1
               float h[16];
 #pragma unroll
               for (int e = 0; e < 16; e += 2) {
-                float g0, g1, u0, u1;
-                scale_round_bf16_2(alpha, g[16 * blk + e], g[16 * blk + e + 1], g0, g1);
-                scale_round_bf16_2(alpha_u, u[16 * blk + e], u[16 * blk + e + 1], u0, u1);
-                silu_mul_bf16_tab2(silu_tab, g0, g1, u0, u1, h[e], h[e + 1]);
+                const uint32_t g2 = scale_round_bf16x2(alpha, g[16 * blk + e], g[16 * blk + e + 1]);
+                const uint32_t u2 = scale_round_bf16x2(alpha_u, u[16 * blk + e], u[16 * blk + e + 1]);
+                silu_mul_bf16_tab2(silu_tab, g2, bf16_lo(u2), bf16_hi(u2), h[e], h[e + 1]);
               }
               const QBlock qb = quantize16(h, gsf);
               codes[2 * blk] = qb.lo;
@@ -558,11 +556,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kSwiGLU>, 1
         // the mask stay untouched.
         const int slab_row = t.m_tile * kTileM + static_cast<int>(rank) * kBM + quarter * 32;
         const bool use_tma = kGrouped ? slab_row + 32 <= t.valid_rows : slab_row < p.m;
-        constexpr int kBufs = kStagingBuffers<kGrouped, kSwiGLU>;
-        uint8_t* stage_warp = staging + (warp - 2) * kBufs * kStoreTileBytes;
+        uint8_t* stage_tile = staging + (warp - 2) * kStoreTileBytes;
         __nv_bfloat16* out_row = p.out + (static_cast<int64_t>(t.expert) * p.m + row) * p.n;
-        for (int i = 0; i < 4; ++i) {
-          // accumulator 0 drains its last 64 columns first, accumulator 1 its first 64
+        // The quarter's warps split the four 64-column subtiles in drain order: accumulator 0
+        // drains its last 64 columns first, accumulator 1 its first 64 (the columns the next
+        // tile's accumulator overlaps), and each warp releases the accumulator after its
+        // first subtile.  A warp that never reads the overlap may release it at once; the
+        // tile after next reuses this accumulator only after every warp has released the
+        // next tile's, which it does after finishing this one.
+        constexpr int kSubs = 16 / kEpiWarps<kGrouped, kSwiGLU>;   // subtiles per warp
+        const int part = (warp - 2) >> 2;
+        for (int j = 0; j < kSubs; ++j) {
+          const int i = part * kSubs + j;
           const int sub = buf ? i : 3 - i;
           const int col_base = t.n_tile * kBN + sub * 64;
           uint4 bias8[8];                      // issued before the TMEM load to hide its latency
@@ -574,7 +579,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kSwiGLU>, 1
           uint32_t v[64];
           tmem_load_64(tmem + col0 + sub * 64 + lane_base, v);
           tmem_wait_ld<64>(v);
-          if (i == 0) {
+          if (j == 0) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
@@ -604,9 +609,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kSwiGLU>, 1
             o[g].w = pack_bf16x2(f[6], f[7]);
           }
           if (use_tma) {
-            uint8_t* stage_tile = stage_warp + (nstore % kBufs) * kStoreTileBytes;
             const uint32_t stage_row = smem_u32(stage_tile) + lane * 128;
-            if (lane == 0) bulk_wait_read<kBufs - 1>();   // the store that last used this tile has read it
+            if (nstore > 0 && lane == 0) bulk_wait_read<0>();   // the previous store has read the tile
             __syncwarp();
             // 128-byte swizzle: 16-byte chunk g of row r sits at chunk position g ^ (r % 8)
 #pragma unroll
@@ -804,7 +808,7 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream) {
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(info.sm_count / 2 * 2);
-    cfg.blockDim = dim3(kThreads<kSwiGLU>);
+    cfg.blockDim = dim3(kThreads<kGrouped, kSwiGLU>);
     cfg.dynamicSmemBytes = kSmemBytes<kGrouped, kSwiGLU>;
     int clusters = 0;
     if (cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg) != cudaSuccess || clusters <= 0) {
@@ -818,8 +822,8 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream) {
   if (tiles >= (int64_t(1) << 31)) return NVFP4_ERR_INVALID_ARGUMENT;
   const int64_t max_pairs = max_clusters;
   const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
-  return launch_kernel(kernel, dim3(2 * pairs), dim3(kThreads<kSwiGLU>), kSmemBytes<kGrouped, kSwiGLU>, stream, maps,
-                       p);
+  return launch_kernel(kernel, dim3(2 * pairs), dim3(kThreads<kGrouped, kSwiGLU>), kSmemBytes<kGrouped, kSwiGLU>,
+                       stream, maps, p);
 }
 
 // Self-test of the bounded wait: one thread waits for an mbarrier phase that nothing ever

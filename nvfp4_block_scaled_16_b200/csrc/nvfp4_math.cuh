@@ -107,48 +107,61 @@ __device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
 }
 __device__ __forceinline__ uint64_t splat2(float v) { return pack2(v, v); }
 
-// ---- SiLU of a bf16 value: closed forms and a per-device table ---------------------------
+// ---- SiLU of a bf16 value: a per-device table and closed forms ----------------------------
 // s(g) = g / (1 + exp_specified(-g)) (one correctly rounded addition and division) depends
-// only on the 16 bits of a bf16 g, so the kernels read it from a table that is computed once
-// per device with exactly that arithmetic.  Outside the magnitude ranges the table covers,
-// s has closed forms that follow from the definition of exp_specified:
+// only on the 16 bits of a bf16 g, so the kernels read it from a table computed once per
+// device with exactly that arithmetic, for both signs of every magnitude in [2^-25, 96):
+// entry 2 * (mag - kSiluMagLo) + sign.  Outside that range s has closed forms that follow
+// from the definition of exp_specified:
 //   |g| < 2^-25: n = 0 and both Horner steps that add 1 round to 1, so e = 1, 1 + e = 2 and
 //     s = g / 2, exact for every bf16 g (subnormal ones included);
-//   g >= 24: e = exp_specified(-g) < 2^-34 is below half an ulp of 1, so 1 + e = 1 and s = g;
+//   g >= 96: e = exp_specified(-g) < 2^-138 is below half an ulp of 1, so 1 + e = 1, s = g;
 //   g <= -96: the argument of exp_specified exceeds 89, e = +inf and s = g / inf = -0,
 //     written g * 0 so that -inf and NaN give NaN as the division does.
-// Table entry i < kSiluPos holds s(+g) and entry kSiluPos + i holds s(-g) for the bf16 g of
-// magnitude pattern kSiluMagLo + i.
-constexpr uint32_t kSiluMagLo = 0x3300;                 // 2^-25
-constexpr uint32_t kSiluPos = 0x41c0 - kSiluMagLo;      // up to 24: 3776 entries
-constexpr uint32_t kSiluNeg = 0x42c0 - kSiluMagLo;      // up to 96: 4032 entries
-constexpr uint32_t kSiluEntries = kSiluPos + kSiluNeg;
-constexpr uint32_t kSiluTableBytes = kSiluEntries * 4;  // 31 232 bytes, a multiple of 16
+constexpr uint32_t kSiluMagLo = 0x3300;                                 // 2^-25
+constexpr uint32_t kSiluMagHi = 0x42c0;                                 // 96
+constexpr uint32_t kSiluEntries = 2 * (kSiluMagHi - kSiluMagLo);        // 8064
+constexpr uint32_t kSiluTableBytes = kSiluEntries * 4;                  // 32 256, a multiple of 16
 
 // Table entry i, computed with the scalar definition.
 __device__ __forceinline__ float silu_table_entry(uint32_t i) {
-  const bool neg = i >= kSiluPos;
-  const uint32_t mag = kSiluMagLo + (neg ? i - kSiluPos : i);
-  const float g = __uint_as_float(((neg ? 0x8000u : 0u) | mag) << 16);
+  const uint32_t mag = kSiluMagLo + (i >> 1);
+  const float g = __uint_as_float((((i & 1u) << 15) | mag) << 16);
   return __fdiv_rn(g, __fadd_rn(1.0f, exp_specified(-g)));
 }
 
-// s(g) for a bf16-valued g (the low 16 bits of its fp32 pattern are zero), from the table
-// `tab` (shared memory) or the closed forms.
-__device__ __forceinline__ float silu_lookup(const float* tab, float g) {
-  const uint32_t bits = __float_as_uint(g);
-  const uint32_t neg = bits >> 31;
-  const uint32_t off = ((bits >> 16) & 0x7fffu) - kSiluMagLo;   // wraps below 2^-25
-  if (off < (neg ? kSiluNeg : kSiluPos)) return tab[off + (neg ? kSiluPos : 0u)];
-  const float f = (off & 0x80000000u) ? 0.5f : (neg ? 0.0f : 1.0f);
+// Table index of the bf16 pattern b (16 bits): 2 * magnitude + sign, less the start of the
+// table; magnitudes outside [kSiluMagLo, kSiluMagHi) give kSiluEntries or more (unsigned).
+__device__ __forceinline__ uint32_t silu_index(uint32_t b) {
+  return (((b << 1) & 0xfffeu) | (b >> 15)) - 2 * kSiluMagLo;
+}
+
+// s(g) for a bf16-valued g outside the table's magnitude range.
+__device__ __forceinline__ float silu_closed(float g) {
+  const uint32_t b = __float_as_uint(g) >> 16;
+  const float f = (b & 0x7fffu) < kSiluMagLo ? 0.5f : ((b & 0x8000u) ? 0.0f : 1.0f);
   return __fmul_rn(g, f);
 }
 
-// h = bf16(s(g) * u) for a pair of bf16-valued g, as fp32 values; equal to silu_mul_bf16.
-__device__ __forceinline__ void silu_mul_bf16_tab2(const float* tab, float g0, float g1, float u0, float u1,
-                                                   float& h0, float& h1) {
-  const float s0 = silu_lookup(tab, g0);
-  const float s1 = silu_lookup(tab, g1);
+// s of the two bf16 values packed in w (element 0 in the low half), from the table `tab`
+// (shared memory); both loads are clamped into the table, and the rare element outside its
+// range is replaced by its closed form.
+__device__ __forceinline__ void silu_pair(const float* tab, uint32_t w, float& s0, float& s1) {
+  const uint32_t i0 = silu_index(w & 0xffffu), i1 = silu_index(w >> 16);
+  s0 = tab[min(i0, kSiluEntries - 1)];
+  s1 = tab[min(i1, kSiluEntries - 1)];
+  if (max(i0, i1) >= kSiluEntries) {
+    if (i0 >= kSiluEntries) s0 = silu_closed(bf16_lo(w));
+    if (i1 >= kSiluEntries) s1 = silu_closed(bf16_hi(w));
+  }
+}
+
+// h = bf16(s(g) * u) for the pair of bf16 gate values packed in g2 and up values u0, u1, as
+// fp32 values; equal to silu_mul_bf16.
+__device__ __forceinline__ void silu_mul_bf16_tab2(const float* tab, uint32_t g2, float u0, float u1, float& h0,
+                                                   float& h1) {
+  float s0, s1;
+  silu_pair(tab, g2, s0, s1);
   float p0, p1;
   unpack2(mul2(pack2(s0, s1), pack2(u0, u1)), p0, p1);
   uint32_t b2;

@@ -67,61 +67,78 @@ struct QuantParams {
   uint32_t items;
 };
 
-// One chunk of kThreads * kUnroll consecutive 16-element blocks of item `item`, starting at
-// block `base` (row-major over rows_pad x cpad).  With kSilu, `tab` is the SiLU table in
-// shared memory.
-template <bool kSilu, bool kSmooth, int kUnroll>
-__device__ __forceinline__ void quantize_chunk(const QuantParams& p, int item, uint32_t base, const float* tab) {
+// One chunk: kThreads * kUnroll consecutive 16-element blocks of one item, row-major over
+// rows_pad x cpad; thread t owns blocks base + u * kThreads + t.  chunk_load issues the
+// chunk's loads, chunk_store computes and writes it, so a caller can overlap the loads of the
+// next chunk with the arithmetic of this one.
+template <bool kSilu, int kUnroll>
+struct Chunk {
+  static constexpr int kVec = kSilu ? 4 : 2;   // 16-byte loads per block
+  uint4 raw[kUnroll][kVec];
+  uint32_t r[kUnroll], c[kUnroll];
+  bool live[kUnroll];     // a block of a valid row and column: quantized
+  bool active;            // false: the chunk lies beyond the item's row limit, nothing is touched
+  int item, valid;
+  uint32_t base;
+};
+
+template <bool kSilu, int kUnroll>
+__device__ __forceinline__ void chunk_load(const QuantParams& p, int item, uint32_t base, Chunk<kSilu, kUnroll>& ch) {
   int valid = p.m;
   if (p.mask) valid = min(max(__ldg(p.mask + item), 0), p.m);
   // Rows at or beyond `limit` are never touched: with a mask, rows >= mask; without one,
   // only the padding rows beyond rows_pad (which do not exist).
   const uint32_t limit = p.mask ? static_cast<uint32_t>(valid) : p.rows_pad;
-  if (base / p.cpad >= limit) return;
-
-  const float gsf = __ldg(p.gsf + item);
+  ch.item = item;
+  ch.valid = valid;
+  ch.base = base;
+  ch.active = base / p.cpad < limit;
+  if (!ch.active) return;
   const uint16_t* x = p.x + item * p.x_item_stride;
-  uint8_t* q = p.q + item * p.q_item_stride;
-  uint8_t* sf = p.sf + item * p.sf_item_stride;
-  const uint32_t groups = p.cpad >> 2;
-
-  constexpr int kVec = kSilu ? 4 : 2;
-  uint4 raw[kUnroll][kVec];
-  uint32_t rr[kUnroll], cc[kUnroll];
-  bool live[kUnroll];
-
 #pragma unroll
   for (int u = 0; u < kUnroll; ++u) {
     const uint32_t f = base + u * kThreads + threadIdx.x;
     const uint32_t r = f / p.cpad;
     const uint32_t c = f - r * p.cpad;
-    rr[u] = r;
-    cc[u] = c;
-    live[u] = f < p.blocks && r < static_cast<uint32_t>(valid) && c < p.nb;
-    if (live[u]) {
+    ch.r[u] = r;
+    ch.c[u] = c;
+    ch.live[u] = f < p.blocks && r < static_cast<uint32_t>(valid) && c < p.nb;
+    if (ch.live[u]) {
       const uint16_t* src = x + static_cast<int64_t>(r) * p.x_row_stride + c * 16;
-      raw[u][0] = load_stream(src);
-      raw[u][1] = load_stream(src + 8);
+      ch.raw[u][0] = load_stream(src);
+      ch.raw[u][1] = load_stream(src + 8);
       if constexpr (kSilu) {
-        raw[u][2] = load_stream(src + p.k);
-        raw[u][3] = load_stream(src + p.k + 8);
+        ch.raw[u][2] = load_stream(src + p.k);
+        ch.raw[u][3] = load_stream(src + p.k + 8);
       }
     }
   }
+}
 
+// With kSilu, `tab` is the SiLU table in shared memory.
+template <bool kSilu, bool kSmooth, int kUnroll>
+__device__ __forceinline__ void chunk_store(const QuantParams& p, const Chunk<kSilu, kUnroll>& ch, const float* tab) {
+  if (!ch.active) return;
+  const float gsf = __ldg(p.gsf + ch.item);
+  uint8_t* q = p.q + ch.item * p.q_item_stride;
+  uint8_t* sf = p.sf + ch.item * p.sf_item_stride;
+  const uint32_t groups = p.cpad >> 2;
 #pragma unroll
   for (int u = 0; u < kUnroll; ++u) {
-    const uint32_t r = rr[u], c = cc[u];
-    if (live[u]) {
+    const uint32_t r = ch.r[u], c = ch.c[u];
+    if (ch.live[u]) {
       float v[16];
-      unpack_bf16x8(raw[u][0], v);
-      unpack_bf16x8(raw[u][1], v + 8);
       if constexpr (kSilu) {
         float up[16];
-        unpack_bf16x8(raw[u][2], up);
-        unpack_bf16x8(raw[u][3], up + 8);
+        unpack_bf16x8(ch.raw[u][2], up);
+        unpack_bf16x8(ch.raw[u][3], up + 8);
+        const uint32_t gw[8] = {ch.raw[u][0].x, ch.raw[u][0].y, ch.raw[u][0].z, ch.raw[u][0].w,
+                                ch.raw[u][1].x, ch.raw[u][1].y, ch.raw[u][1].z, ch.raw[u][1].w};
 #pragma unroll
-        for (int i = 0; i < 16; i += 2) silu_mul_bf16_tab2(tab, v[i], v[i + 1], up[i], up[i + 1], v[i], v[i + 1]);
+        for (int i = 0; i < 8; ++i) silu_mul_bf16_tab2(tab, gw[i], up[2 * i], up[2 * i + 1], v[2 * i], v[2 * i + 1]);
+      } else {
+        unpack_bf16x8(ch.raw[u][0], v);
+        unpack_bf16x8(ch.raw[u][1], v + 8);
       }
       if constexpr (kSmooth) {
         // x_hat = bf16(x * pre_quant_scale) for the block's 16 columns (the scale vector is
@@ -142,10 +159,10 @@ __device__ __forceinline__ void quantize_chunk(const QuantParams& p, int item, u
       const QBlock b = quantize16(v, gsf);
       *reinterpret_cast<uint2*>(q + static_cast<int64_t>(r) * (p.k / 2) + c * 8) = make_uint2(b.lo, b.hi);
       sf[sf_offset(r, c, groups)] = static_cast<uint8_t>(b.s8);
-    } else if (base + u * kThreads + threadIdx.x < p.blocks) {
+    } else if (ch.base + u * kThreads + threadIdx.x < p.blocks) {
       // Padding scale entries: a column beyond the last block of a valid row, or (no mask)
       // a padding row below m.
-      const bool pad_col = r < static_cast<uint32_t>(valid) && c >= p.nb;
+      const bool pad_col = r < static_cast<uint32_t>(ch.valid) && c >= p.nb;
       const bool pad_row = p.mask == nullptr && r >= static_cast<uint32_t>(p.m);
       if (pad_col || pad_row) sf[sf_offset(r, c, groups)] = 0;
     }
@@ -157,12 +174,16 @@ template <bool kSmooth, int kUnroll>
 __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantParams p) {
   pdl_launch_dependents();
   pdl_wait();
-  quantize_chunk<false, kSmooth, kUnroll>(p, blockIdx.y, blockIdx.x * (kThreads * kUnroll), nullptr);
+  Chunk<false, kUnroll> ch;
+  chunk_load(p, blockIdx.y, blockIdx.x * (kThreads * kUnroll), ch);
+  chunk_store<false, kSmooth>(p, ch, nullptr);
 }
 
 // SiLU * up: persistent CTAs that load the SiLU table into shared memory once and walk the
 // chunks of all items (item-major) with a grid stride, so the live chunks of every item are
-// spread over all CTAs whatever the masks are.
+// spread over all CTAs whatever the masks are.  (Issuing the next chunk's loads before the
+// current chunk's arithmetic, with one or two blocks per thread and 2-6 CTAs per SM, measured
+// 2-15% slower than this plain loop with two blocks per thread and four CTAs per SM.)
 constexpr int kSiluUnroll = 2;
 constexpr int kSiluCtasPerSm = 4;
 // The table fits the default 48 KB of dynamic shared memory (no opt-in attribute needed).
@@ -175,10 +196,12 @@ __global__ void __launch_bounds__(kThreads, kSiluCtasPerSm) silu_quantize_kernel
   silu_table_load(tab, p.silu_tab, threadIdx.x, kThreads);
   __syncthreads();
   const uint64_t total = static_cast<uint64_t>(p.chunks_per_item) * p.items;
+  Chunk<true, kSiluUnroll> ch;
   for (uint64_t chunk = blockIdx.x; chunk < total; chunk += gridDim.x) {
     const uint32_t item = static_cast<uint32_t>(chunk / p.chunks_per_item);
     const uint32_t local = static_cast<uint32_t>(chunk - static_cast<uint64_t>(item) * p.chunks_per_item);
-    quantize_chunk<true, false, kSiluUnroll>(p, static_cast<int>(item), local * (kThreads * kSiluUnroll), tab);
+    chunk_load(p, static_cast<int>(item), local * (kThreads * kSiluUnroll), ch);
+    chunk_store<true, false>(p, ch, tab);
   }
 }
 
@@ -199,11 +222,12 @@ __global__ void __launch_bounds__(kThreads) silu_and_mul_kernel(const uint16_t* 
        i += static_cast<int64_t>(gridDim.x) * kThreads) {
     const int64_t r = i / per_row;
     const int64_t c = (i - r * per_row) * 8;
-    float g[8], u[8], o[8];
-    unpack_bf16x8(load_stream(x + r * 2 * k + c), g);
+    float u[8], o[8];
+    const uint4 g = load_stream(x + r * 2 * k + c);
     unpack_bf16x8(load_stream(x + r * 2 * k + k + c), u);
+    const uint32_t gw[4] = {g.x, g.y, g.z, g.w};
 #pragma unroll
-    for (int e = 0; e < 8; e += 2) silu_mul_bf16_tab2(tab, g[e], g[e + 1], u[e], u[e + 1], o[e], o[e + 1]);
+    for (int e = 0; e < 4; ++e) silu_mul_bf16_tab2(tab, gw[e], u[2 * e], u[2 * e + 1], o[2 * e], o[2 * e + 1]);
     uint4 w;
     w.x = (__float_as_uint(o[0]) >> 16) | (__float_as_uint(o[1]) & 0xffff0000u);
     w.y = (__float_as_uint(o[2]) >> 16) | (__float_as_uint(o[3]) & 0xffff0000u);

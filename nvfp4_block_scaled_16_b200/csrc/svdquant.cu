@@ -11,8 +11,8 @@
 // ([r, k], prepared offline), computed in bf16.  TensorRT-LLM NVFP4LinearMethod.create_weights
 // carries the same pre_quant_scale for o_proj / down_proj style layers.
 //
-// Kernel structure.  A cluster of 4 CTAs shares one 128-row tile of x and splits its K range
-// in four; every CTA streams its 128 x (k/4) slice of x (and the matching columns of w)
+// Kernel structure.  A cluster of kSvdSplit CTAs shares one 128-row tile of x and splits its
+// K range; every CTA streams its 128 x (k/kSvdSplit) slice of x (and the matching columns of w)
 // through a 4-stage ring of 64-column TMA tiles (128-byte swizzle).
 //   warp 0      TMA producer (one elected lane).
 //   warp 1      TMEM allocator and MMA issuer: per stage four tcgen05.mma.cta_group::1
@@ -23,9 +23,9 @@
 //               from the swizzled tile, forms x_hat, and writes 2 blocks: 16 code bytes and
 //               two scale bytes (a stage is exactly one 4-block group of the 128x4 scale
 //               layout).  Afterwards warps 2-5 drain the accumulator into shared memory
-//               (column-major fp32) and, after a cluster barrier, CTA c sums rows
-//               [32c, 32c + 32) over the 4 CTAs' partials through distributed shared memory
-//               and writes them as bf16.
+//               (column-major fp32) and, after a cluster barrier, CTA c sums its share of
+//               the tile's rows over the cluster's partials through distributed shared
+//               memory and writes them as bf16.
 // Every mbarrier wait is bounded; the two cluster barriers are executed on every path.
 #include <cuda_bf16.h>
 
@@ -40,6 +40,7 @@ constexpr int kSvdRows = 128;            // rows of x per cluster (MMA M)
 constexpr int kSvdChunk = 64;            // bf16 values of K per stage (128-byte rows)
 constexpr int kSvdStages = 4;
 constexpr int kSvdSplit = 4;             // CTAs per cluster, splitting K
+static_assert(kSvdSplit == 4 || kSvdSplit == 8, "the reduction splits 128 threads over 128 / kSvdSplit rows");
 constexpr int kSvdXBytes = kSvdRows * 128;   // 16 KB per stage
 constexpr int kSvdMaxRank = 256;
 // Quantizer warps: 16 / kSvdQuantWarps of a row's 4 blocks per stage per thread; the first
@@ -310,32 +311,32 @@ __global__ void __cluster_dims__(kSvdSplit, 1, 1) __launch_bounds__(kSvdThreads,
   __syncthreads();
   cluster_sync();          // every CTA's partials are in its shared memory
   if (warp >= 2 && warp < 6 && !*abort) {
-    const int row = static_cast<int>(rank) * 32 + lane;   // this CTA's quarter of the tile rows
+    // CTA c reduces rows [c * kRows, (c + 1) * kRows) of the tile; the 128 threads of warps
+    // 2-5 take one row and one of kGroups column ranges each
+    constexpr int kRows = kSvdRows / kSvdSplit;
+    constexpr int kGroups = 128 / kRows;
+    const int t = threadIdx.x - 64;
+    const int row = static_cast<int>(rank) * kRows + t % kRows;
     const int grow = row0 + row;
-    const int cols = p.r / 4;                             // columns per epilogue warp
-    const int col0 = (warp - 2) * cols;
+    const int cols = p.r / kGroups;                       // a multiple of 4 (r is a multiple of 32)
+    const int col0 = (t / kRows) * cols;
     const float* part = reinterpret_cast<const float*>(smem);
     uint32_t peer[kSvdSplit];
 #pragma unroll
     for (int q = 0; q < kSvdSplit; ++q) peer[q] = map_to_rank(part, static_cast<uint32_t>(q));
     if (grow < p.m) {
       __nv_bfloat16* drow = p.d + static_cast<int64_t>(grow) * p.r + col0;
-      for (int j = 0; j < cols; j += 8) {
-        float acc[8];
+      for (int j = 0; j < cols; j += 4) {
+        float acc[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
+        for (int e = 0; e < 4; ++e) {
           const uint32_t off = static_cast<uint32_t>(((col0 + j + e) * kSvdRows + row) * 4);
           float sum = 0.0f;
 #pragma unroll
           for (int q = 0; q < kSvdSplit; ++q) sum = __fadd_rn(sum, ld_shared_cluster_f32(peer[q] + off));
           acc[e] = sum;
         }
-        uint4 o;
-        o.x = pack_bf16x2(acc[0], acc[1]);
-        o.y = pack_bf16x2(acc[2], acc[3]);
-        o.z = pack_bf16x2(acc[4], acc[5]);
-        o.w = pack_bf16x2(acc[6], acc[7]);
-        *reinterpret_cast<uint4*>(drow + j) = o;
+        *reinterpret_cast<uint2*>(drow + j) = make_uint2(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]));
       }
     }
   }
