@@ -1,18 +1,18 @@
 """Benchmark of the NVFP4 linear-layer hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl nvfp4|reference]
-                    [--workload swiglu_block|quant_dense|quant_masked|quant_silu|grouped_moe|grouped_swiglu|
-                                lowrank|pr1_linear]
+                    [--workload swiglu_block|quant_dense|quant_dense_fused|quant_masked|quant_silu|grouped_moe|
+                                grouped_swiglu|lowrank|svdquant_linear|pr1_linear]
                     [--rank-lr R] [--swiglu-path fused|unfused] [--no-pdl]
 
 Default workload: the dense NVFP4 SwiGLU shared-expert block, M = 8192 tokens, hidden
 5120, intermediate 8192.  One step is the whole hot path over one batch:
-    global amax of x (dynamic activation scale; also yields the gate/up alpha)
-    -> quantize x [8192, 5120]
+    global amax of x (dynamic activation scale; also yields the gate/up alpha) and the
+    quantization of x [8192, 5120] in one launch
     -> gate/up GEMM [8192 x 5120] @ [16384 x 5120]^T whose epilogue forms
        h = bf16(silu(gate) * up) and quantizes it with the calibrated static scale of h
-       (--swiglu-path unfused: the GEMM writes bf16 [gate | up] and the SiLU-and-mul
-       quantizer runs as its own kernel)
+       (--swiglu-path unfused: the pages' sequence of separate kernels -- amax, quantize,
+       the GEMM writing bf16 [gate | up], the SiLU-and-mul quantizer)
     -> down GEMM [8192 x 8192] @ [5120 x 8192]^T  (bf16 out)
 Weights are quantized once before timing (offline weight quantization), and the static
 activation scale of h is calibrated once, as a deployed layer would.
@@ -227,9 +227,10 @@ class Workload:
 
 
 class SwigluBlock(Workload):
-    """Dense SwiGLU block.  fused=True: amax(x), quantize(x), the gate/up GEMM whose
-    epilogue emits SiLU(g)*u as NVFP4, the down GEMM.  fused=False: the same with the
-    gate/up GEMM writing bf16 [g | u] and the SiLU-and-mul quantizer as its own kernel."""
+    """Dense SwiGLU block.  fused=True: amax(x) and quantize(x) in one launch, the gate/up
+    GEMM whose epilogue emits SiLU(g)*u as NVFP4, the down GEMM.  fused=False: the pages'
+    sequence of separate kernels -- amax(x), quantize(x), the gate/up GEMM writing bf16
+    [g | u], the SiLU-and-mul quantizer, the down GEMM."""
     name = "swiglu_block"
     unit = "TFLOP/s"
 
@@ -277,8 +278,8 @@ class SwigluBlock(Workload):
         nv = self
         lib = self.nv
         return [
-            ("global_scale_x", lambda: lib.nvfp4_global_scale(nv.x, nv.amax_x, nv.gsf_x, nv.amax_wgu, nv.alpha1)),
-            ("quantize_x", lambda: lib.nvfp4_quantize(nv.x, nv.gsf_x, nv.xq, nv.xsf)),
+            ("global_scale_quantize_x", lambda: lib.nvfp4_global_scale_quantize(
+                nv.x, nv.amax_wgu, nv.amax_x, nv.gsf_x, nv.alpha1, nv.xq, nv.xsf)),
             ("gemm_gate_up_silu_quantize", lambda: lib.nvfp4_gemm_silu_mul_quantize(
                 nv.xq, nv.wg_q, nv.wu_q, nv.xsf, nv.wg_sf, nv.wu_sf, nv.alpha1, nv.alpha1, nv.gsf_h,
                 nv.hq.view(nv.M, nv.I // 2), nv.hsf.view(-1))),
@@ -308,6 +309,7 @@ class SwigluBlock(Workload):
         return {k: v for k, v in {
             "global_scale_x": (2.0 * M * H, "GB/s"),
             "quantize_x": (2.5625 * M * H, "GB/s"),
+            "global_scale_quantize_x": (2.5625 * M * H, "GB/s"),
             "gemm_gate_up": (2.0 * M * H * 2 * I, "TFLOP/s"),
             "gemm_gate_up_silu_quantize": (2.0 * M * H * 2 * I, "TFLOP/s"),
             "silu_mul_quantize": (4.5625 * M * I, "GB/s"),
@@ -361,6 +363,25 @@ class QuantDense(Workload):
     def config(self):
         return {"workload": "quantize bf16 [8192,8192] ~N(0,1) with 0.1% outliers x50 (amax + quantize)",
                 "l2": L2_NOTE}
+
+
+class QuantDenseFused(QuantDense):
+    """The quant_dense workload through nvfp4_global_scale_quantize: amax and quantize in
+    one launch."""
+    name = "quant_dense_fused"
+    dominant = "global_scale_quantize"
+
+    def launches(self):
+        lib, s = self.nv, self
+        return [("global_scale_quantize", lambda: lib.nvfp4_global_scale_quantize(s.x, None, s.amax, s.gsf, None,
+                                                                                   s.q, s.sf))]
+
+    def kernel_work(self):
+        return {"global_scale_quantize": (2.5625 * self.m * self.k, "GB/s")}
+
+    def config(self):
+        return {"workload": "quantize bf16 [8192,8192] ~N(0,1) with 0.1% outliers x50 (amax and quantize in one "
+                            "launch)", "l2": L2_NOTE}
 
 
 class QuantMasked(Workload):
@@ -676,6 +697,8 @@ def make_workload(name, nv, rank_lr, swiglu_path="fused"):
         return SwigluBlock(nv, fused=swiglu_path == "fused")
     if name == "quant_dense":
         return QuantDense(nv)
+    if name == "quant_dense_fused":
+        return QuantDenseFused(nv)
     if name == "quant_masked":
         return QuantMasked(nv, False)
     if name == "quant_silu":
@@ -734,9 +757,9 @@ class OracleSample:
             d = S.pr1_linear(0)
             self.x, self.w = d["x"], d["w"]
             self.sample = "the whole 128x256x256 linear (amax, quantize, GEMM)"
-        elif w in ("quant_dense", "quant_masked", "quant_silu"):
+        elif w in ("quant_dense", "quant_dense_fused", "quant_masked", "quant_silu"):
             self.rows = rows or 256
-            if w == "quant_dense":
+            if w in ("quant_dense", "quant_dense_fused"):
                 self.x = S.quant_dense(8192, 8192, 0)["x"][:self.rows].copy()
             else:
                 k = 7168
@@ -822,7 +845,7 @@ class OracleSample:
             qx, sfx = O.quantize(self.x, gx)
             O.gemm_ref(qx, self.qw, sfx, self.sfw, O.alpha(float(ax), float(self.aw)), 128, 256, 256)
             work = 2.0 * 128 * 256 * 256
-        elif w == "quant_dense":
+        elif w in ("quant_dense", "quant_dense_fused"):
             a, g = O.global_scale(self.x)
             O.quantize(self.x, g)
             work = 2.5625 * self.x.size
@@ -878,7 +901,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="nvfp4", choices=["nvfp4", "reference"])
     ap.add_argument("--workload", default="swiglu_block",
-                    choices=["swiglu_block", "quant_dense", "quant_masked", "quant_silu", "grouped_moe",
+                    choices=["swiglu_block", "quant_dense", "quant_dense_fused", "quant_masked", "quant_silu", "grouped_moe",
                              "grouped_swiglu", "lowrank", "svdquant_linear", "pr1_linear"])
     ap.add_argument("--rank-lr", type=int, default=64)
     ap.add_argument("--swiglu-path", default="fused", choices=["fused", "unfused"],

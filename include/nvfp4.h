@@ -134,6 +134,29 @@ NVFP4_API int nvfp4_quantize(const void *x_bf16, int64_t m, int64_t k, const flo
                    uint8_t *q_out, uint8_t *sf_out, nvfp4_stream_t stream);
 
 /*
+ * Global scale and dense quantize in one launch: the results of nvfp4_global_scale
+ * followed by nvfp4_quantize with its gsf, bit for bit [FV _global_sf; TRT input_scale;
+ * FI3 fp4_quantize].  The pages compute the two in sequence; fusing them is this
+ * library's: one persistent grid reduces max|x| (keeping x in L2), meets at a grid-wide
+ * barrier, and quantizes, reading most of x a second time from L2 instead of HBM.
+ *   x_bf16     [m, k] bf16, 16-byte aligned; k % 16 == 0, k > 0, m >= 0 (m = 0 writes
+ *              only the scalars: amax = 1e-12).
+ *   amax_out   nullable fp32 [1]; gsf_out required fp32 [1]; other_amax / alpha_out as in
+ *              nvfp4_global_scale (both or neither).
+ *   q_out      uint8 [m, k/2] (8-byte aligned); sf_out uint8 [nvfp4_scale_bytes(m, k)] (both may
+ *              be NULL when m = 0).
+ * Uses the stream's reduction workspace (allocated on the stream's first use, like
+ * nvfp4_global_scale).  The grid is a cooperative launch (all CTAs resident) of at most
+ * three CTAs per SM; it is not chained to its predecessor by programmatic dependent
+ * launch.  The barrier wait is bounded (1 s): if it runs out, nothing is written,
+ * NVFP4_ERR_DEVICE_TIMEOUT is recorded in the device status word, and clearing that word
+ * with nvfp4_device_status also re-zeroes the device's reduction workspaces.
+ */
+NVFP4_API int nvfp4_global_scale_quantize(const void *x_bf16, int64_t m, int64_t k, float *amax_out,
+                                          float *gsf_out, const float *other_amax, float *alpha_out,
+                                          uint8_t *q_out, uint8_t *sf_out, nvfp4_stream_t stream);
+
+/*
  * Masked batched quantize [FI3 nvfp4_batched_quantize(..., mask)].
  *   x_bf16 [b, m, k] bf16; mask nullable int32 [b] (NULL: all rows); gsf fp32 [b].
  *   q_out  uint8 [b, m, k/2]; sf_out uint8 [b][nvfp4_scale_bytes(m, k)].
@@ -339,11 +362,19 @@ NVFP4_API int nvfp4_device_status(int *status_out, int clear);
  * MMA issuer's wait for that stage runs out, records NVFP4_ERR_DEVICE_TIMEOUT, and every
  * role of both CTAs of each pair unwinds (bounded drain, cluster barrier, tensor memory
  * freed) within a few seconds.  out_bf16 is left unspecified.  The device stays usable.
+ *
+ * nvfp4_selftest_grid_barrier runs nvfp4_global_scale_quantize (same constraints) with one
+ * more barrier arrival expected than the grid has CTAs: every CTA's barrier wait runs out
+ * after about one second, NVFP4_ERR_DEVICE_TIMEOUT is recorded, and nothing is written.
+ * The stream's reduction workspace is left set until the status word is cleared with
+ * nvfp4_device_status (which re-zeroes it); the next call then computes correctly.
  */
 NVFP4_API int nvfp4_selftest_bounded_wait(nvfp4_stream_t stream);
 NVFP4_API int nvfp4_selftest_gemm_stall(const uint8_t *a, const uint8_t *b, const uint8_t *a_sf,
                                         const uint8_t *b_sf, const float *alpha, void *out_bf16, int64_t m,
                                         int64_t n, int64_t k, nvfp4_stream_t stream);
+NVFP4_API int nvfp4_selftest_grid_barrier(const void *x_bf16, int64_t m, int64_t k, float *gsf_out,
+                                          uint8_t *q_out, uint8_t *sf_out, nvfp4_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -19,6 +19,7 @@ from .binding import (  # noqa: F401
     nvfp4_global_scale_batched,
     nvfp4_global_scale_batched_noalloc,
     nvfp4_quantize,
+    nvfp4_global_scale_quantize,
     nvfp4_quantize_masked_batched,
     nvfp4_silu_mul_quantize_batched,
     nvfp4_gemm,
@@ -34,5 +35,6 @@ from .binding import (  # noqa: F401
     nvfp4_get_pdl,
     nvfp4_selftest_bounded_wait,
     nvfp4_selftest_gemm_stall,
+    nvfp4_selftest_grid_barrier,
     nvfp4_device_status,
 )

@@ -20,6 +20,7 @@ EXPORTED_SYMBOLS = (
     "nvfp4_global_scale_batched",
     "nvfp4_global_scale_batched_noalloc",
     "nvfp4_quantize",
+    "nvfp4_global_scale_quantize",
     "nvfp4_quantize_masked_batched",
     "nvfp4_silu_mul_quantize_batched",
     "nvfp4_gemm",
@@ -35,6 +36,7 @@ EXPORTED_SYMBOLS = (
     "nvfp4_get_pdl",
     "nvfp4_selftest_bounded_wait",
     "nvfp4_selftest_gemm_stall",
+    "nvfp4_selftest_grid_barrier",
     "nvfp4_device_status",
 )
 
@@ -49,6 +51,7 @@ _SIGNATURES = {
     "nvfp4_global_scale_batched": (_INT, [_P, _I64, _I64, _I64, _P, _INT, _P, _P, _P]),
     "nvfp4_global_scale_batched_noalloc": (_INT, [_P, _I64, _I64, _I64, _P, _INT, _P, _P, _P]),
     "nvfp4_quantize": (_INT, [_P, _I64, _I64, _P, _P, _P, _P]),
+    "nvfp4_global_scale_quantize": (_INT, [_P, _I64, _I64, _P, _P, _P, _P, _P, _P, _P]),
     "nvfp4_quantize_masked_batched": (_INT, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P]),
     "nvfp4_silu_mul_quantize_batched": (_INT, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P]),
     "nvfp4_gemm": (_INT, [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
@@ -64,6 +67,7 @@ _SIGNATURES = {
     "nvfp4_get_pdl": (_INT, []),
     "nvfp4_selftest_bounded_wait": (_INT, [_P]),
     "nvfp4_selftest_gemm_stall": (_INT, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
+    "nvfp4_selftest_grid_barrier": (_INT, [_P, _I64, _I64, _P, _P, _P, _P]),
     "nvfp4_device_status": (_INT, [ctypes.POINTER(_INT), _INT]),
 }
 
@@ -180,6 +184,27 @@ def nvfp4_quantize(x, gsf, q_out=None, sf_out=None, stream=None):
         st = load_library().nvfp4_quantize(_ptr(x), m, k, _ptr(gsf), _ptr(q_out), _ptr(sf_out), _stream(stream))
     _check("nvfp4_quantize", st)
     return q_out, sf_out
+
+
+def nvfp4_global_scale_quantize(x, other_amax=None, amax_out=None, gsf_out=None, alpha_out=None, q_out=None,
+                                sf_out=None, stream=None):
+    """x [m, k] bf16 -> (amax [1], gsf [1], alpha [1] or None, q [m, k/2] uint8, sf [scale_bytes(m, k)] uint8):
+    nvfp4_global_scale and nvfp4_quantize in one launch."""
+    m, k = x.shape
+    dev = x.device
+    amax_out = torch.empty(1, dtype=torch.float32, device=dev) if amax_out is None else amax_out
+    gsf_out = torch.empty(1, dtype=torch.float32, device=dev) if gsf_out is None else gsf_out
+    if other_amax is not None and alpha_out is None:
+        alpha_out = torch.empty(1, dtype=torch.float32, device=dev)
+    q_out = torch.empty((m, k // 2), dtype=torch.uint8, device=dev) if q_out is None else q_out
+    if sf_out is None:
+        sf_out = torch.empty(max(nvfp4_scale_bytes(m, k), 0), dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        st = load_library().nvfp4_global_scale_quantize(_ptr(x), m, k, _ptr(amax_out), _ptr(gsf_out),
+                                                        _ptr(other_amax), _ptr(alpha_out), _ptr(q_out),
+                                                        _ptr(sf_out), _stream(stream))
+    _check("nvfp4_global_scale_quantize", st)
+    return amax_out, gsf_out, alpha_out, q_out, sf_out
 
 
 def _batched_outputs(x, b, m, k, q_out, sf_out):
@@ -372,6 +397,19 @@ def nvfp4_selftest_gemm_stall(a, b, a_sf, b_sf, alpha, out=None, stream=None):
                                                       _ptr(out), m, n, 2 * kh, _stream(stream))
     _check("nvfp4_selftest_gemm_stall", st)
     return out
+
+
+def nvfp4_selftest_grid_barrier(x, stream=None):
+    """nvfp4_global_scale_quantize whose grid barrier waits for one arrival too many: every
+    CTA's wait runs out, NVFP4_ERR_DEVICE_TIMEOUT is recorded and nothing is written."""
+    m, k = x.shape
+    gsf = torch.full((1,), -1.0, dtype=torch.float32, device=x.device)
+    q = torch.zeros((m, k // 2), dtype=torch.uint8, device=x.device)
+    sf = torch.zeros(max(nvfp4_scale_bytes(m, k), 0), dtype=torch.uint8, device=x.device)
+    with torch.cuda.device(x.device):
+        st = load_library().nvfp4_selftest_grid_barrier(_ptr(x), m, k, _ptr(gsf), _ptr(q), _ptr(sf), _stream(stream))
+    _check("nvfp4_selftest_grid_barrier", st)
+    return gsf, q, sf
 
 
 def nvfp4_device_status(clear: bool = True) -> int:

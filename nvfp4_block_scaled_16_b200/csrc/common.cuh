@@ -61,6 +61,30 @@ int launch_kernel(void (*kernel)(KernelArgs...), dim3 grid, dim3 block, size_t s
   return NVFP4_OK;
 }
 
+// Launches `kernel` as a cooperative grid (every CTA resident at once; the launch fails
+// if the grid cannot be) for kernels whose CTAs wait on one another.  It is not given the
+// programmatic-serialization attribute, so it starts after its predecessor in the stream
+// completes.
+template <typename... KernelArgs, typename... Args>
+int launch_kernel_cooperative(void (*kernel)(KernelArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) != cudaSuccess) {
+    cudaGetLastError();
+    return NVFP4_ERR_CUDA;
+  }
+  return NVFP4_OK;
+}
+
 // ---- device side --------------------------------------------------------------------
 
 // Lets the next kernel of the stream (launched with PDL) start its launch and prologue.

@@ -167,6 +167,18 @@ int nvfp4_device_status(int* status_out, int clear) {
     cudaGetLastError();
     return NVFP4_ERR_CUDA;
   }
+  if (clear && v != NVFP4_OK) {
+    // a kernel that gave up a wait may have left its reduction words set: zero this
+    // device's per-stream workspaces (the device is idle after the synchronize above)
+    std::lock_guard<std::mutex> lock(nvfp4::g_mu);
+    for (auto& kv : nvfp4::g_ws) {
+      if (kv.first.first == info.device &&
+          cudaMemset(kv.second, 0, sizeof(uint32_t) * (1 + nvfp4::kMaxItems)) != cudaSuccess) {
+        cudaGetLastError();
+        return NVFP4_ERR_CUDA;
+      }
+    }
+  }
   *status_out = v;
   return NVFP4_OK;
 }

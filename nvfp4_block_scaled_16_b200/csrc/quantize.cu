@@ -24,6 +24,7 @@
 
 #include "common.cuh"
 #include "nvfp4_math.cuh"
+#include "tc_common.cuh"
 
 namespace nvfp4 {
 namespace {
@@ -80,10 +81,14 @@ struct Chunk {
   bool active;            // false: the chunk lies beyond the item's row limit, nothing is touched
   int item, valid;
   uint32_t base;
+  uint32_t end;           // blocks at or beyond end belong to someone else
 };
 
-template <bool kSilu, int kUnroll>
-__device__ __forceinline__ void chunk_load(const QuantParams& p, int item, uint32_t base, Chunk<kSilu, kUnroll>& ch) {
+// Blocks f = base + u * kThreads + threadIdx.x with f < end (and f < p.blocks) are this
+// chunk's.  kKeep: the loads keep x in the caches (a second pass will read it again).
+template <bool kSilu, int kUnroll, bool kKeep = false>
+__device__ __forceinline__ void chunk_load(const QuantParams& p, int item, uint32_t base, Chunk<kSilu, kUnroll>& ch,
+                                           uint32_t end = 0xffffffffu) {
   int valid = p.m;
   if (p.mask) valid = min(max(__ldg(p.mask + item), 0), p.m);
   // Rows at or beyond `limit` are never touched: with a mask, rows >= mask; without one,
@@ -92,6 +97,7 @@ __device__ __forceinline__ void chunk_load(const QuantParams& p, int item, uint3
   ch.item = item;
   ch.valid = valid;
   ch.base = base;
+  ch.end = end;
   ch.active = base / p.cpad < limit;
   if (!ch.active) return;
   const uint16_t* x = p.x + item * p.x_item_stride;
@@ -102,11 +108,16 @@ __device__ __forceinline__ void chunk_load(const QuantParams& p, int item, uint3
     const uint32_t c = f - r * p.cpad;
     ch.r[u] = r;
     ch.c[u] = c;
-    ch.live[u] = f < p.blocks && r < static_cast<uint32_t>(valid) && c < p.nb;
+    ch.live[u] = f < p.blocks && f < end && r < static_cast<uint32_t>(valid) && c < p.nb;
     if (ch.live[u]) {
       const uint16_t* src = x + static_cast<int64_t>(r) * p.x_row_stride + c * 16;
-      ch.raw[u][0] = load_stream(src);
-      ch.raw[u][1] = load_stream(src + 8);
+      if constexpr (kKeep) {
+        ch.raw[u][0] = __ldg(reinterpret_cast<const uint4*>(src));
+        ch.raw[u][1] = __ldg(reinterpret_cast<const uint4*>(src + 8));
+      } else {
+        ch.raw[u][0] = load_stream(src);
+        ch.raw[u][1] = load_stream(src + 8);
+      }
       if constexpr (kSilu) {
         ch.raw[u][2] = load_stream(src + p.k);
         ch.raw[u][3] = load_stream(src + p.k + 8);
@@ -116,10 +127,12 @@ __device__ __forceinline__ void chunk_load(const QuantParams& p, int item, uint3
 }
 
 // With kSilu, `tab` is the SiLU table in shared memory.
+// gsf_given >= 0 replaces the item's global scale from p.gsf.
 template <bool kSilu, bool kSmooth, int kUnroll>
-__device__ __forceinline__ void chunk_store(const QuantParams& p, const Chunk<kSilu, kUnroll>& ch, const float* tab) {
+__device__ __forceinline__ void chunk_store(const QuantParams& p, const Chunk<kSilu, kUnroll>& ch, const float* tab,
+                                            float gsf_given = -1.0f) {
   if (!ch.active) return;
-  const float gsf = __ldg(p.gsf + ch.item);
+  const float gsf = gsf_given >= 0.0f ? gsf_given : __ldg(p.gsf + ch.item);
   uint8_t* q = p.q + ch.item * p.q_item_stride;
   uint8_t* sf = p.sf + ch.item * p.sf_item_stride;
   const uint32_t groups = p.cpad >> 2;
@@ -159,7 +172,7 @@ __device__ __forceinline__ void chunk_store(const QuantParams& p, const Chunk<kS
       const QBlock b = quantize16(v, gsf);
       *reinterpret_cast<uint2*>(q + static_cast<int64_t>(r) * (p.k / 2) + c * 8) = make_uint2(b.lo, b.hi);
       sf[sf_offset(r, c, groups)] = static_cast<uint8_t>(b.s8);
-    } else if (ch.base + u * kThreads + threadIdx.x < p.blocks) {
+    } else if (ch.base + u * kThreads + threadIdx.x < min(p.blocks, ch.end)) {
       // Padding scale entries: a column beyond the last block of a valid row, or (no mask)
       // a padding row below m.
       const bool pad_col = r < static_cast<uint32_t>(ch.valid) && c >= p.nb;
@@ -346,6 +359,99 @@ __global__ void __launch_bounds__(kThreads) amax_batched_kernel(const uint16_t* 
   reduce_and_finalize(mx, ws, item, gridDim.y, gridDim.x * gridDim.y, amax_out, gsf_out, nullptr, nullptr);
 }
 
+// ---- global scale and quantize in one launch -----------------------------------------------
+//
+// The global scale needs the amax of the whole tensor before any block can be quantized.
+// One persistent grid, every CTA resident at once (a cooperative launch), does both: CTA j
+// takes the contiguous range of 16-element blocks [j B / G, (j + 1) B / G); it reduces the
+// max |x| of its range (loads that keep x in L2), folds it into the workspace with an atomic
+// max, and arrives on a grid barrier; once every CTA has arrived, each computes gsf from the
+// same maximum and quantizes its range, last chunk first, so that the lines it read most
+// recently (the ones most likely still in L2) are read again first.  Workspace words:
+// 0 = barrier arrivals, 1 = amax bits, 2 = CTAs done reading the maximum; the last of
+// those resets all three for the next call on the stream.
+constexpr int kGsqUnroll = 4;
+constexpr int kGsqCtasPerSm = 3;
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__global__ void __launch_bounds__(kThreads, kGsqCtasPerSm)
+    global_scale_quantize_kernel(const QuantParams p, uint32_t* ws, float* amax_out, float* gsf_out,
+                                 const float* other_amax, float* alpha_out, int* status, uint32_t withheld) {
+  __shared__ float red[kThreads / 32];
+  __shared__ float s_amax;
+  pdl_wait();
+  const uint32_t grid = gridDim.x;
+  const uint32_t expected = grid + withheld;   // self-test: arrivals that never come
+  const uint32_t lo = static_cast<uint32_t>(static_cast<uint64_t>(p.blocks) * blockIdx.x / grid);
+  const uint32_t hi = static_cast<uint32_t>(static_cast<uint64_t>(p.blocks) * (blockIdx.x + 1) / grid);
+  constexpr uint32_t kChunk = kThreads * kGsqUnroll;
+
+  // phase 1: max |x| over this CTA's blocks
+  float mx = 0.0f;
+  for (uint32_t base = lo; base < hi; base += kChunk) {
+    Chunk<false, kGsqUnroll> ch;
+    chunk_load<false, kGsqUnroll, true>(p, 0, base, ch, hi);
+#pragma unroll
+    for (int u = 0; u < kGsqUnroll; ++u)
+      if (ch.live[u]) mx = absmax8(ch.raw[u][1], absmax8(ch.raw[u][0], mx));   // fmaxf drops NaN
+  }
+  mx = warp_max(mx);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float v = red[0];
+#pragma unroll
+    for (int w = 1; w < kThreads / 32; ++w) v = fmaxf(v, red[w]);
+    atomicMax(ws + 1, __float_as_uint(v));
+    __threadfence();
+    atomicAdd(ws, 1u);
+    // grid barrier, bounded: every CTA is resident, so only a fault elsewhere can stall it
+    const uint64_t t0 = global_ns();
+    bool ok = true;
+    while (ld_acquire_gpu(ws) < expected) {
+      if (global_ns() - t0 > kWaitLimitNs) {
+        ok = false;
+        atomicExch(status, NVFP4_ERR_DEVICE_TIMEOUT);
+        break;
+      }
+      __nanosleep(100);
+    }
+    float a = -1.0f;                                   // -1: give up, write nothing
+    if (ok) {
+      a = fmaxf(fminf(__uint_as_float(ld_acquire_gpu(ws + 1)), FLT_MAX), 1e-12f);
+      if (atomicAdd(ws + 2, 1u) == grid - 1) {         // every CTA has read the maximum
+        atomicExch(ws + 1, 0u);
+        atomicExch(ws + 2, 0u);
+        atomicExch(ws, 0u);
+      }
+    }
+    s_amax = a;
+  }
+  __syncthreads();
+  const float amax = s_amax;
+  if (amax < 0.0f) return;
+  pdl_launch_dependents();            // every CTA of this grid is past the barrier
+  const float gsf = __fdiv_rn(2688.0f, amax);
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    if (amax_out) *amax_out = amax;
+    *gsf_out = gsf;
+    if (other_amax) *alpha_out = __fdiv_rn(__fmul_rn(amax, *other_amax), 7225344.0f);
+  }
+
+  // phase 2: quantize this CTA's blocks, last chunk first
+  const uint32_t chunks = (hi - lo + kChunk - 1) / kChunk;
+  for (uint32_t j = chunks; j-- > 0;) {
+    Chunk<false, kGsqUnroll> ch;
+    chunk_load<false, kGsqUnroll, false>(p, 0, lo + j * kChunk, ch, hi);
+    chunk_store<false, false>(p, ch, nullptr, gsf);
+  }
+}
+
 // ---- host helpers -------------------------------------------------------------------------
 
 int launch_quantize(const void* x, int64_t b, int64_t m, int64_t k, bool silu, const int32_t* mask,
@@ -395,6 +501,54 @@ int launch_quantize(const void* x, int64_t b, int64_t m, int64_t k, bool silu, c
   dim3 grid(p.chunks_per_item, static_cast<unsigned>(b));
   if (pqs) return launch_kernel(quantize_kernel<true, U>, grid, dim3(kThreads), 0, stream, p);
   return launch_kernel(quantize_kernel<false, U>, grid, dim3(kThreads), 0, stream, p);
+}
+
+// nvfp4_global_scale_quantize; `withheld` > 0 (self-test only) makes the grid barrier wait
+// for arrivals that never come.
+int launch_global_scale_quantize(const void* x_bf16, int64_t m, int64_t k, float* amax_out, float* gsf_out,
+                                 const float* other_amax, float* alpha_out, uint8_t* q_out, uint8_t* sf_out,
+                                 cudaStream_t stream, uint32_t withheld) {
+  if (m < 0 || k <= 0 || k % 16 != 0 || m > (1 << 30) || k > (1 << 30)) return NVFP4_ERR_INVALID_ARGUMENT;
+  if ((other_amax == nullptr) != (alpha_out == nullptr)) return NVFP4_ERR_INVALID_ARGUMENT;
+  if (!gsf_out || (m > 0 && (!x_bf16 || !q_out || !sf_out))) return NVFP4_ERR_INVALID_ARGUMENT;
+  if ((x_bf16 && !aligned(x_bf16, 16)) || !aligned(q_out, 8) || !aligned(gsf_out, 4) ||
+      (amax_out && !aligned(amax_out, 4)) || (other_amax && (!aligned(other_amax, 4) || !aligned(alpha_out, 4))))
+    return NVFP4_ERR_INVALID_ARGUMENT;
+  const int64_t nb = k / 16, cpad = (nb + 3) / 4 * 4, rows_pad = (m + 127) / 128 * 128;
+  if (rows_pad * cpad >= (int64_t(1) << 31)) return NVFP4_ERR_INVALID_ARGUMENT;
+  DeviceInfo info;
+  int st = current_device(&info);
+  if (st != NVFP4_OK) return st;
+  uint32_t* ws = nullptr;
+  st = stream_workspace(stream, &ws);
+  if (st != NVFP4_OK) return st;
+  static int per_sm = 0;          // co-resident CTAs per SM, found once
+  if (per_sm == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, global_scale_quantize_kernel, kThreads, 0) != cudaSuccess ||
+        n <= 0) {
+      cudaGetLastError();
+      return NVFP4_ERR_CUDA;
+    }
+    per_sm = n < kGsqCtasPerSm ? n : kGsqCtasPerSm;
+  }
+  QuantParams p = {};
+  p.x = static_cast<const uint16_t*>(x_bf16);
+  p.x_row_stride = k;
+  p.q = q_out;
+  p.sf = sf_out;
+  p.m = static_cast<int32_t>(m);
+  p.k = static_cast<int32_t>(k);
+  p.nb = static_cast<uint32_t>(nb);
+  p.cpad = static_cast<uint32_t>(cpad);
+  p.rows_pad = static_cast<uint32_t>(rows_pad);
+  p.blocks = static_cast<uint32_t>(rows_pad * cpad);
+  p.items = 1;
+  const int64_t chunks = (p.blocks + kThreads * kGsqUnroll - 1) / (kThreads * kGsqUnroll);
+  const int64_t cap = static_cast<int64_t>(info.sm_count) * per_sm;
+  const unsigned grid = static_cast<unsigned>(chunks < 1 ? 1 : (chunks < cap ? chunks : cap));
+  return launch_kernel_cooperative(global_scale_quantize_kernel, dim3(grid), dim3(kThreads), 0, stream, p, ws, amax_out,
+                                   gsf_out, other_amax, alpha_out, info.status, withheld);
 }
 
 }  // namespace
@@ -473,6 +627,17 @@ int nvfp4_quantize_smooth(const void* x_bf16, int64_t m, int64_t k, const void* 
                           const float* gsf, uint8_t* q_out, uint8_t* sf_out, nvfp4_stream_t stream) {
   if (!pre_quant_scale_bf16 && m > 0 && k > 0) return NVFP4_ERR_INVALID_ARGUMENT;
   return launch_quantize(x_bf16, 1, m, k, false, nullptr, gsf, q_out, sf_out, stream, pre_quant_scale_bf16);
+}
+
+int nvfp4_global_scale_quantize(const void* x_bf16, int64_t m, int64_t k, float* amax_out, float* gsf_out,
+                                const float* other_amax, float* alpha_out, uint8_t* q_out, uint8_t* sf_out,
+                                nvfp4_stream_t stream) {
+  return launch_global_scale_quantize(x_bf16, m, k, amax_out, gsf_out, other_amax, alpha_out, q_out, sf_out, stream, 0);
+}
+
+int nvfp4_selftest_grid_barrier(const void* x_bf16, int64_t m, int64_t k, float* gsf_out, uint8_t* q_out,
+                                uint8_t* sf_out, nvfp4_stream_t stream) {
+  return launch_global_scale_quantize(x_bf16, m, k, nullptr, gsf_out, nullptr, nullptr, q_out, sf_out, stream, 1);
 }
 
 int nvfp4_quantize_masked_batched(const void* x_bf16, int64_t b, int64_t m, int64_t k, const int32_t* mask,

@@ -1,13 +1,15 @@
 """Failure detection on the GPU without a fault: a bounded wait that nothing completes must
 give up (about one second), record NVFP4_ERR_DEVICE_TIMEOUT in the device status word,
 and leave the context usable; a GEMM whose first K stage is withheld must unwind the same
-way, after which the same GEMM runs correctly."""
+way, after which the same GEMM runs correctly; a global-scale quantize whose grid barrier
+waits for an arrival that never comes must give up, write nothing, and — once the status
+is cleared — leave its stream's workspace clean for the next call."""
 import numpy as np
 import pytest
 
 import nvfp4_block_scaled_16_b200 as nv
 import nvfp4_synth as S
-from tests.helpers import assert_gemm_close, bf16_to_f64, dev_f32, dev_u8
+from tests.helpers import assert_gemm_close, bf16_to_f64, dev_bf16, dev_f32, dev_u8, host
 
 pytestmark = pytest.mark.gpu
 
@@ -48,3 +50,18 @@ def test_gemm_stall_unwinds_and_the_device_stays_usable(oracle):
     assert nv.nvfp4_device_status(clear=True) == 0
     ref = oracle.gemm_ref(qa, qb, sfa, sfb, alpha, m, n, k)
     assert_gemm_close(bf16_to_f64(out), ref, "gemm after a stalled launch")
+
+
+def test_grid_barrier_timeout_writes_nothing_and_recovers(oracle):
+    x = S.normal_bf16((512, 1024), 4.0, 9, S.TID["x"])
+    xd = dev_bf16(x)
+    assert nv.nvfp4_device_status(clear=True) == 0
+    gsf, q, sf = nv.nvfp4_selftest_grid_barrier(xd)
+    assert nv.nvfp4_device_status(clear=True) == NVFP4_ERR_DEVICE_TIMEOUT    # clearing re-zeroes the workspace
+    assert host(gsf)[0] == -1.0 and not host(q).any() and not host(sf).any()
+    _, gsf_o = oracle.global_scale(x)
+    q_o, sf_o = oracle.quantize(x, gsf_o)
+    _, g2, _, q2, s2 = nv.nvfp4_global_scale_quantize(xd)
+    assert nv.nvfp4_device_status(clear=True) == 0
+    assert host(g2)[0] == gsf_o
+    assert (host(q2) == q_o).all() and (host(s2) == sf_o).all()

@@ -111,6 +111,59 @@ def test_quantize_full_size_with_outliers(oracle):
     check_dense(oracle, x)
 
 
+# ---- global scale and quantize in one launch ------------------------------------------------
+
+def check_global_scale_quantize(oracle, x, other=np.float32(0.75)):
+    """amax, gsf, alpha, codes and scales bit-exact against the oracle's global scale and
+    quantizer (the fused launch must equal the two-call definition)."""
+    m, k = x.shape
+    amax_o, gsf_o = oracle.global_scale(x)
+    q = torch.full((m, k // 2), 0xA5, dtype=torch.uint8, device="cuda")
+    sf = torch.full((nv.nvfp4_scale_bytes(m, k),), 0x5A, dtype=torch.uint8, device="cuda")
+    amax, gsf, alpha, _, _ = nv.nvfp4_global_scale_quantize(dev_bf16(x), other_amax=dev_f32(other), q_out=q,
+                                                             sf_out=sf)
+    torch.cuda.synchronize()
+    assert host(amax)[0] == amax_o and host(gsf)[0] == gsf_o
+    assert host(alpha)[0] == np.float32(oracle.alpha(float(amax_o), float(other)))
+    if m:
+        q_o, sf_o = oracle.quantize(x, gsf_o)
+        assert first_diff(host(q), q_o) is None, first_diff(host(q), q_o)
+        assert first_diff(host(sf), sf_o) is None, first_diff(host(sf), sf_o)
+
+
+@pytest.mark.parametrize("m,k", [(1, 16), (3, 48), (130, 80), (300, 272), (257, 512), (64, 4096), (2048, 5120)])
+def test_global_scale_quantize_matches_oracle(oracle, m, k):
+    check_global_scale_quantize(oracle, S.normal_with_outliers_bf16((m, k), 0.01, 50.0, seed=m * 11 + k))
+
+
+def test_global_scale_quantize_full_size(oracle):
+    # the activation of the SwiGLU block: x [8192, 5120] ~ N(0, 1)
+    check_global_scale_quantize(oracle, S.normal_bf16((8192, 5120), 1.0, 0, S.TID["x"]))
+
+
+def test_global_scale_quantize_empty_rows_and_zeros(oracle):
+    check_global_scale_quantize(oracle, np.zeros((0, 64), np.uint16))          # scalars only: amax = 1e-12
+    check_global_scale_quantize(oracle, np.zeros((5, 32), np.uint16))
+
+
+def test_global_scale_quantize_equals_two_calls_and_reuses_its_workspace():
+    # repeated calls on one stream with different maxima (a workspace left set would leak
+    # the previous maximum), NaN and inf included: the fused launch equals
+    # nvfp4_global_scale followed by nvfp4_quantize
+    for seed, scale in ((0, 8.0), (1, 0.5), (2, 3.0)):
+        x = S.normal_bf16((700, 1024), scale, seed=seed)
+        if seed == 2:
+            x[3, 5] = 0x7FC0                      # NaN (counted as 0 by the amax)
+            x[9, 100] = 0xFF80                    # -inf
+        xd = dev_bf16(x)
+        a1, g1, _ = nv.nvfp4_global_scale(xd)
+        q1, s1 = nv.nvfp4_quantize(xd, g1)
+        a2, g2, _, q2, s2 = nv.nvfp4_global_scale_quantize(xd)
+        torch.cuda.synchronize()
+        assert torch.equal(a1, a2) and torch.equal(g1, g2)
+        assert torch.equal(q1, q2) and torch.equal(s1, s2)
+
+
 def test_quantize_empty_and_invalid():
     x = torch.zeros((0, 32), dtype=torch.bfloat16, device="cuda")
     q, sf = nv.nvfp4_quantize(x, torch.ones(1, device="cuda"))
