@@ -195,23 +195,43 @@ __device__ __forceinline__ float div6_bf16(float vmax) {
   return vmax == __uint_as_float(0x7f800000u) ? vmax : __fmaf_rn(rem, 0x1.555556p-3f, q);
 }
 
-// One 16-element block of bf16-valued inputs.
-__device__ __forceinline__ QBlock quantize16(const float* v, float gsf) {
-  float vmax = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) vmax = fmaxf(vmax, fabsf(v[i]));
-  const float s32 = __fmul_rn(div6_bf16(vmax), gsf);
-  QBlock b;
-  b.s8 = ue4m3_encode(s32);
-  const float sd = e4m3_decode(b.s8);
-  const float inv = sd == 0.0f ? 0.0f : __fdiv_rn(gsf, sd);
+// The codes and scale of one 16-element block given its scale code s8 and the factor
+// inv = gsf / e4m3(s8) (0 when the scale decodes to 0).
+__device__ __forceinline__ QBlock quantize16_codes(const float* v, uint32_t s8, float inv) {
   const uint64_t inv2 = pack2(inv, inv);
   float t[16];
 #pragma unroll
   for (int i = 0; i < 16; i += 2) unpack2(mul2(pack2(v[i], v[i + 1]), inv2), t[i], t[i + 1]);
+  QBlock b;
+  b.s8 = s8;
   b.lo = e2m1x8(t);
   b.hi = e2m1x8(t + 8);
   return b;
+}
+
+__device__ __forceinline__ uint32_t block_scale_code(const float* v, float gsf) {
+  float vmax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) vmax = fmaxf(vmax, fabsf(v[i]));
+  return ue4m3_encode(__fmul_rn(div6_bf16(vmax), gsf));
+}
+
+__device__ __forceinline__ float inv_scale(uint32_t s8, float gsf) {
+  const float sd = e4m3_decode(s8);
+  return sd == 0.0f ? 0.0f : __fdiv_rn(gsf, sd);
+}
+
+// One 16-element block of bf16-valued inputs.
+__device__ __forceinline__ QBlock quantize16(const float* v, float gsf) {
+  const uint32_t s8 = block_scale_code(v, gsf);
+  return quantize16_codes(v, s8, inv_scale(s8, gsf));
+}
+
+// The same block with inv read from inv_tab[code] = inv_scale(code, gsf) for the 128 scale
+// codes a block can get (one division per code instead of one per block).
+__device__ __forceinline__ QBlock quantize16(const float* v, float gsf, const float* inv_tab) {
+  const uint32_t s8 = block_scale_code(v, gsf);
+  return quantize16_codes(v, s8, inv_tab[s8]);
 }
 
 // Byte offset of the scale of (row r, block c) in the 128x4 swizzled layout;

@@ -63,10 +63,31 @@ struct QuantParams {
   uint32_t cpad;           // pad_up(nb, 4)
   uint32_t rows_pad;       // pad_up(m, 128)
   uint32_t blocks;         // rows_pad * cpad (per item)
+  uint32_t cpad_magic;     // f / cpad = umulhi(f, cpad_magic) >> cpad_shift for f < 2^31
+  uint32_t cpad_shift;
   const float* silu_tab;   // SiLU table in global memory (SiLU variant)
   uint32_t chunks_per_item;
   uint32_t items;
 };
+
+// Division by cpad (a multiple of 4) with the Granlund-Montgomery multiplier of 31-bit
+// dividends: with l = ceil(log2 cpad) and m = ceil(2^(31+l) / cpad), floor(f / cpad) =
+// floor(f m / 2^(31+l)) for every f < 2^31.
+__device__ __forceinline__ uint32_t div_cpad(const QuantParams& p, uint32_t f) {
+  return __umulhi(f, p.cpad_magic) >> p.cpad_shift;
+}
+
+void set_cpad_divisor(QuantParams& p) {
+  uint32_t l = 0;
+  while ((uint64_t(1) << l) < p.cpad) ++l;
+  p.cpad_magic = static_cast<uint32_t>(((uint64_t(1) << (31 + l)) + p.cpad - 1) / p.cpad);
+  p.cpad_shift = l - 1;
+}
+
+// inv_tab[code] = inv_scale(code, gsf) for the 128 block-scale codes, by threads [0, 128).
+__device__ __forceinline__ void inv_table_build(float* inv_tab, float gsf) {
+  if (threadIdx.x < 128) inv_tab[threadIdx.x] = inv_scale(threadIdx.x, gsf);
+}
 
 // One chunk: kThreads * kUnroll consecutive 16-element blocks of one item, row-major over
 // rows_pad x cpad; thread t owns blocks base + u * kThreads + t.  chunk_load issues the
@@ -98,13 +119,13 @@ __device__ __forceinline__ void chunk_load(const QuantParams& p, int item, uint3
   ch.valid = valid;
   ch.base = base;
   ch.end = end;
-  ch.active = base / p.cpad < limit;
+  ch.active = div_cpad(p, base) < limit;
   if (!ch.active) return;
   const uint16_t* x = p.x + item * p.x_item_stride;
 #pragma unroll
   for (int u = 0; u < kUnroll; ++u) {
     const uint32_t f = base + u * kThreads + threadIdx.x;
-    const uint32_t r = f / p.cpad;
+    const uint32_t r = div_cpad(p, f);
     const uint32_t c = f - r * p.cpad;
     ch.r[u] = r;
     ch.c[u] = c;
@@ -127,12 +148,11 @@ __device__ __forceinline__ void chunk_load(const QuantParams& p, int item, uint3
 }
 
 // With kSilu, `tab` is the SiLU table in shared memory.
-// gsf_given >= 0 replaces the item's global scale from p.gsf.
+// inv_tab: the inverse block scales of the chunk's item (inv_table_build with its gsf).
 template <bool kSilu, bool kSmooth, int kUnroll>
 __device__ __forceinline__ void chunk_store(const QuantParams& p, const Chunk<kSilu, kUnroll>& ch, const float* tab,
-                                            float gsf_given = -1.0f) {
+                                            float gsf, const float* inv_tab) {
   if (!ch.active) return;
-  const float gsf = gsf_given >= 0.0f ? gsf_given : __ldg(p.gsf + ch.item);
   uint8_t* q = p.q + ch.item * p.q_item_stride;
   uint8_t* sf = p.sf + ch.item * p.sf_item_stride;
   const uint32_t groups = p.cpad >> 2;
@@ -169,7 +189,7 @@ __device__ __forceinline__ void chunk_store(const QuantParams& p, const Chunk<kS
           v[i + 1] = bf16_hi(w);
         }
       }
-      const QBlock b = quantize16(v, gsf);
+      const QBlock b = quantize16(v, gsf, inv_tab);
       *reinterpret_cast<uint2*>(q + static_cast<int64_t>(r) * (p.k / 2) + c * 8) = make_uint2(b.lo, b.hi);
       sf[sf_offset(r, c, groups)] = static_cast<uint8_t>(b.s8);
     } else if (ch.base + u * kThreads + threadIdx.x < min(p.blocks, ch.end)) {
@@ -185,11 +205,15 @@ __device__ __forceinline__ void chunk_store(const QuantParams& p, const Chunk<kS
 // One chunk per CTA: grid (chunks per item, items).
 template <bool kSmooth, int kUnroll>
 __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantParams p) {
+  __shared__ float inv_tab[128];
   pdl_launch_dependents();
   pdl_wait();
   Chunk<false, kUnroll> ch;
   chunk_load(p, blockIdx.y, blockIdx.x * (kThreads * kUnroll), ch);
-  chunk_store<false, kSmooth>(p, ch, nullptr);
+  const float gsf = __ldg(p.gsf + blockIdx.y);
+  inv_table_build(inv_tab, gsf);
+  __syncthreads();
+  chunk_store<false, kSmooth>(p, ch, nullptr, gsf, inv_tab);
 }
 
 // SiLU * up: persistent CTAs that load the SiLU table into shared memory once and walk the
@@ -203,18 +227,27 @@ constexpr int kSiluCtasPerSm = 4;
 static_assert(kSiluTableBytes <= 48 * 1024, "SiLU table exceeds the default dynamic shared memory");
 __global__ void __launch_bounds__(kThreads, kSiluCtasPerSm) silu_quantize_kernel(const QuantParams p) {
   extern __shared__ float4 silu_smem[];
+  __shared__ float inv_tab[128];
   float* tab = reinterpret_cast<float*>(silu_smem);
   pdl_launch_dependents();
   pdl_wait();
   silu_table_load(tab, p.silu_tab, threadIdx.x, kThreads);
-  __syncthreads();
   const uint64_t total = static_cast<uint64_t>(p.chunks_per_item) * p.items;
   Chunk<true, kSiluUnroll> ch;
+  uint32_t table_item = 0xffffffffu;           // the item whose inverse scales inv_tab holds
+  float gsf = 0.0f;
   for (uint64_t chunk = blockIdx.x; chunk < total; chunk += gridDim.x) {
     const uint32_t item = static_cast<uint32_t>(chunk / p.chunks_per_item);
     const uint32_t local = static_cast<uint32_t>(chunk - static_cast<uint64_t>(item) * p.chunks_per_item);
     chunk_load(p, static_cast<int>(item), local * (kThreads * kSiluUnroll), ch);
-    chunk_store<true, false>(p, ch, tab);
+    if (item != table_item) {                   // uniform over the CTA
+      __syncthreads();                          // the previous item's table is no longer read
+      gsf = __ldg(p.gsf + item);
+      inv_table_build(inv_tab, gsf);
+      table_item = item;
+      __syncthreads();                          // (also orders the SiLU table's first load)
+    }
+    chunk_store<true, false>(p, ch, tab, gsf, inv_tab);
   }
 }
 
@@ -384,6 +417,7 @@ __global__ void __launch_bounds__(kThreads, kGsqCtasPerSm)
                                  const float* other_amax, float* alpha_out, int* status, uint32_t withheld) {
   __shared__ float red[kThreads / 32];
   __shared__ float s_amax;
+  __shared__ float inv_tab[128];
   pdl_wait();
   const uint32_t grid = gridDim.x;
   const uint32_t expected = grid + withheld;   // self-test: arrivals that never come
@@ -444,11 +478,13 @@ __global__ void __launch_bounds__(kThreads, kGsqCtasPerSm)
   }
 
   // phase 2: quantize this CTA's blocks, last chunk first
+  inv_table_build(inv_tab, gsf);
+  __syncthreads();
   const uint32_t chunks = (hi - lo + kChunk - 1) / kChunk;
   for (uint32_t j = chunks; j-- > 0;) {
     Chunk<false, kGsqUnroll> ch;
     chunk_load<false, kGsqUnroll, false>(p, 0, lo + j * kChunk, ch, hi);
-    chunk_store<false, false>(p, ch, nullptr, gsf);
+    chunk_store<false, false>(p, ch, nullptr, gsf, inv_tab);
   }
 }
 
@@ -464,7 +500,7 @@ int launch_quantize(const void* x, int64_t b, int64_t m, int64_t k, bool silu, c
     return NVFP4_ERR_INVALID_ARGUMENT;
   if (b > 65535 || m > (1 << 30) || k > (1 << 30)) return NVFP4_ERR_INVALID_ARGUMENT;
   const int64_t nb = k / 16, cpad = (nb + 3) / 4 * 4, rows_pad = (m + 127) / 128 * 128;
-  if (rows_pad * cpad >= (int64_t(1) << 31)) return NVFP4_ERR_INVALID_ARGUMENT;
+  if (rows_pad * cpad >= (int64_t(1) << 31) - 4096) return NVFP4_ERR_INVALID_ARGUMENT;   // f < 2^31
   DeviceInfo info;
   int st = current_device(&info);
   if (st != NVFP4_OK) return st;
@@ -486,6 +522,7 @@ int launch_quantize(const void* x, int64_t b, int64_t m, int64_t k, bool silu, c
   p.cpad = static_cast<uint32_t>(cpad);
   p.rows_pad = static_cast<uint32_t>(rows_pad);
   p.blocks = static_cast<uint32_t>(rows_pad * cpad);
+  set_cpad_divisor(p);
   p.silu_tab = info.silu_table;
   p.items = static_cast<uint32_t>(b);
   if (silu) {
@@ -515,7 +552,7 @@ int launch_global_scale_quantize(const void* x_bf16, int64_t m, int64_t k, float
       (amax_out && !aligned(amax_out, 4)) || (other_amax && (!aligned(other_amax, 4) || !aligned(alpha_out, 4))))
     return NVFP4_ERR_INVALID_ARGUMENT;
   const int64_t nb = k / 16, cpad = (nb + 3) / 4 * 4, rows_pad = (m + 127) / 128 * 128;
-  if (rows_pad * cpad >= (int64_t(1) << 31)) return NVFP4_ERR_INVALID_ARGUMENT;
+  if (rows_pad * cpad >= (int64_t(1) << 31) - 4096) return NVFP4_ERR_INVALID_ARGUMENT;   // f < 2^31
   DeviceInfo info;
   int st = current_device(&info);
   if (st != NVFP4_OK) return st;
@@ -543,6 +580,7 @@ int launch_global_scale_quantize(const void* x_bf16, int64_t m, int64_t k, float
   p.cpad = static_cast<uint32_t>(cpad);
   p.rows_pad = static_cast<uint32_t>(rows_pad);
   p.blocks = static_cast<uint32_t>(rows_pad * cpad);
+  set_cpad_divisor(p);
   p.items = 1;
   const int64_t chunks = (p.blocks + kThreads * kGsqUnroll - 1) / (kThreads * kGsqUnroll);
   const int64_t cap = static_cast<int64_t>(info.sm_count) * per_sm;

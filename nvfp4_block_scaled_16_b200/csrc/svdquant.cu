@@ -214,6 +214,10 @@ __global__ void __cluster_dims__(kSvdSplit, 1, 1) __launch_bounds__(kSvdThreads,
     bool ok = true;
     if constexpr (kQuant) {
       const float gsf = __ldg(p.gsf);
+      // inverse block scales of the 128 scale codes, one division each
+      __shared__ float inv_tab[128];
+      if (threadIdx.x - 64 < 128) inv_tab[threadIdx.x - 64] = inv_scale(threadIdx.x - 64, gsf);
+      asm volatile("bar.sync 2, %0;" ::"n"(32 * kSvdQuantWarps) : "memory");
       const uint32_t groups = static_cast<uint32_t>(p.chunks);     // k / 64 scale groups per row
       for (int i = 0; i < nch; ++i) {
         const int s = i % kSvdStages;
@@ -250,7 +254,7 @@ __global__ void __cluster_dims__(kSvdSplit, 1, 1) __launch_bounds__(kSvdThreads,
                 v[8 * h + 2 * e + 1] = bf16_hi(w);
               }
             }
-            const QBlock qb = quantize16(v, gsf);
+            const QBlock qb = quantize16(v, gsf, inv_tab);
             codes[2 * blk] = qb.lo;
             codes[2 * blk + 1] = qb.hi;
             scales |= qb.s8 << (8 * blk);
