@@ -325,8 +325,9 @@ class SwigluBlock(Workload):
                             "intermediate 8192; gate/up [8192x5120]@[16384x5120]^T, silu*mul requantize, "
                             "down [8192x8192]@[5120x8192]^T; x~N(0,1), W~N(0,0.02)",
                 "tokens": self.M, "hidden": self.H, "intermediate": self.I,
-                "path": ("gate/up GEMM with the SiLU*mul NVFP4 quantizer in its epilogue" if self.fused else
-                         "gate/up GEMM to bf16, then the SiLU*mul quantizer kernel"),
+                "path": ("amax and quantize of x in one launch, gate/up GEMM with the SiLU*mul NVFP4 quantizer "
+                         "in its epilogue, down GEMM" if self.fused else
+                         "amax, quantize, gate/up GEMM to bf16, SiLU*mul quantizer, down GEMM (separate kernels)"),
                 "l2": L2_NOTE}
 
 
@@ -692,6 +693,26 @@ class PR1Linear(Workload):
         return {"workload": "single NVFP4 linear x[128,256] W[256,256] (latency-bound)", "l2": L2_NOTE}
 
 
+def workload_config(name, rank_lr, swiglu_path="fused"):
+    """The `config` of a workload without a GPU: its sizes and its seeded masks only (the
+    reference arm prints the same config as the CUDA arm)."""
+    cls = {"swiglu_block": SwigluBlock, "quant_dense": QuantDense, "quant_dense_fused": QuantDenseFused,
+           "quant_masked": QuantMasked, "quant_silu": QuantMasked, "grouped_moe": GroupedMoE,
+           "grouped_swiglu": GroupedSwiglu, "lowrank": LowRank, "svdquant_linear": SvdquantLinear,
+           "pr1_linear": PR1Linear}[name]
+    w = cls.__new__(cls)
+    w.fused = swiglu_path == "fused"
+    w.M, w.H, w.I = 8192, 5120, 8192
+    w.silu = name == "quant_silu"
+    w.r = rank_lr
+    w.E, w.mmax = 16, 2048
+    if name in ("quant_masked", "quant_silu"):
+        w.mask_host = S.masks_uniform(8, 4096, 0)
+    elif name in ("grouped_moe", "grouped_swiglu"):
+        w.mask_host = S.masks_poisson(16, 512, 2048, 0)
+    return w.config()
+
+
 def make_workload(name, nv, rank_lr, swiglu_path="fused"):
     if name == "swiglu_block":
         return SwigluBlock(nv, fused=swiglu_path == "fused")
@@ -886,7 +907,7 @@ def run_reference(args, world, rank):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": o.unit, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / max(args.steps, 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (plain C oracle)",
-            "data": "synthetic", "config": {"workload": wl},
+            "data": "synthetic", "config": workload_config(wl, args.rank_lr, args.swiglu_path),
             "cpu_baseline": {"value": value, "unit": o.unit, "cores": o.threads, "kind": "oracle",
                              "sample": o.sample + " per step"},
             "e2e": {"value": value, "unit": o.unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

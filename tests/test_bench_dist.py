@@ -71,3 +71,16 @@ def test_single_rank_helpers_are_identity():
     assert bench.max_over_ranks(1, 5.0) == 5.0
     assert bench.sum_over_ranks(1, 5.0) == 5.0
     assert bench.aggregate(1, 7.0, 3.0) == (7.0, 3.0)
+
+
+def test_reference_arm_config_is_computed_without_a_gpu():
+    # the reference arm prints the CUDA arm's config; it must build on a machine without a GPU
+    sys.path.insert(0, ROOT)
+    import bench
+    for name in ("swiglu_block", "quant_dense", "quant_dense_fused", "quant_masked", "quant_silu", "grouped_moe",
+                 "grouped_swiglu", "lowrank", "svdquant_linear", "pr1_linear"):
+        cfg = bench.workload_config(name, 64)
+        assert isinstance(cfg["workload"], str) and cfg["workload"]
+        assert "l2" in cfg
+    assert "sum 8088" in bench.workload_config("grouped_swiglu", 64)["workload"]
+    assert "r=32" in bench.workload_config("lowrank", 32)["workload"]
