@@ -20,7 +20,8 @@ activation scale of h is calibrated once, as a deployed layer would.
 Timing: the step is captured into a CUDA graph with event nodes only at its start and
 end (its kernels chained by programmatic dependent launch unless --no-pdl), and into a
 second graph with an event node around every kernel.  W warm-up replays, then K timed
-replays of each graph bracketed by a barrier and a device synchronize.  Before every
+replays of each graph, alternating (step graph, kernel graph) so both see the same clocks,
+bracketed by a barrier and a device synchronize.  Before every
 replay L2 is flushed outside the events (a 512 MB write, then a 256 MB read that leaves
 no dirty line of the flush to be written back inside the timing).  ms_per_step and the
 value come from the step graph; per-kernel times (parts, roofline) from the kernel
@@ -68,6 +69,16 @@ def load_peaks():
 def file_sha(path):
     with open(path, "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+# The CUDA kernel behind each launch name that can be a workload's dominant launch (the key of
+# its DRAM traffic in profiles/traffic.json).
+KERNEL_OF_LAUNCH = {
+    "quantize": "quantize_kernel", "quantize_masked": "quantize_kernel",
+    "silu_mul_quantize": "silu_quantize_kernel", "global_scale_quantize": "global_scale_quantize_kernel",
+    "global_scale_quantize_x": "global_scale_quantize_kernel",
+    "quantize_smooth_lora_down": "svdquant_input_kernel",
+}
 
 
 def recorded_traffic(kernel, workload):
@@ -676,8 +687,8 @@ class PR1Linear(Workload):
 
     def launches(self):
         lib, s = self.nv, self
-        return [("global_scale", lambda: lib.nvfp4_global_scale(s.x, s.amax, s.gsf, s.amax_w, s.alpha)),
-                ("quantize", lambda: lib.nvfp4_quantize(s.x, s.gsf, s.xq, s.xsf)),
+        return [("global_scale_quantize", lambda: lib.nvfp4_global_scale_quantize(s.x, s.amax_w, s.amax, s.gsf, s.alpha,
+                                                                                   s.xq, s.xsf)),
                 ("gemm", lambda: lib.nvfp4_gemm(s.xq, s.wq, s.xsf, s.wsf, s.alpha, None, s.out))]
 
     def work(self):
@@ -690,7 +701,8 @@ class PR1Linear(Workload):
         return self.x_host, self.x, self.out
 
     def config(self):
-        return {"workload": "single NVFP4 linear x[128,256] W[256,256] (latency-bound)", "l2": L2_NOTE}
+        return {"workload": "single NVFP4 linear x[128,256] W[256,256] (latency-bound): amax and quantize of x in "
+                            "one launch, then the GEMM", "l2": L2_NOTE}
 
 
 def workload_config(name, rank_lr, swiglu_path="fused"):
@@ -969,7 +981,7 @@ def main():
     # its start and end, so consecutive kernels keep their programmatic-dependent-launch
     # edges: it gives the step time (value).  The kernel graph has an event node around
     # every kernel (consecutive kernels then cannot overlap): it gives each kernel's own
-    # duration (parts, roofline).  Both run inside the timed region, one pass each.  Should
+    # duration (parts, roofline).  Both run inside the timed region, alternating step by step.  Should
     # the driver refuse timing on graph event nodes, every kernel is captured into its own
     # graph and timed by events recorded around its replay (no overlap either way).
     with torch.cuda.stream(stream):
@@ -1054,11 +1066,12 @@ def main():
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
         t_wall = time.perf_counter()
+        # the two passes alternate step by step, so that both see the same clocks and power
+        # state (a long run can reach the power cap)
         with torch.cuda.stream(stream):
             for s in range(args.steps):
                 flush_l2()
                 step_ms.append(run_step())
-            for s in range(args.steps):
                 flush_l2()
                 samples.append(run_kernels())
         torch.cuda.synchronize()
@@ -1090,7 +1103,7 @@ def main():
     dom_ms = statistics.mean(per_kernel[dom])
     achieved = scale(w / (dom_ms * 1e-3), unit)
     peak = fp4_peak if unit == "TFLOP/s" else hbm_peak
-    kernel_name = "nvfp4_gemm_kernel" if unit == "TFLOP/s" else "quantize_kernel"
+    kernel_name = KERNEL_OF_LAUNCH.get(dom, "nvfp4_gemm_kernel" if unit == "TFLOP/s" else "quantize_kernel")
     traffic = recorded_traffic(kernel_name, f"{wl.name}:{dom}")
     roofline = {"bound": "tensor" if unit == "TFLOP/s" else "hbm", "achieved": round(achieved, 2),
                 "peak": round(peak, 1), "unit": unit, "frac": round(achieved / peak, 4), "traffic": traffic,
