@@ -930,8 +930,8 @@ def run_reference(args, world, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="nvfp4", choices=["nvfp4", "reference"])
     ap.add_argument("--workload", default="swiglu_block",
                     choices=["swiglu_block", "quant_dense", "quant_dense_fused", "quant_masked", "quant_silu", "grouped_moe",

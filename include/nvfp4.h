@@ -177,7 +177,10 @@ NVFP4_API int nvfp4_quantize_masked_batched(const void *x_bf16, int64_t b, int64
  *   nvfp4_quantize_masked_batched.
  * h = bf16(silu(gate) * up) with silu(g) = g / (1 + exp(-g)), where exp is the
  * library's specified fp32 exponential (Cody-Waite reduction, degree-7 Taylor
- * polynomial, exact 2^n scaling); h is then quantized as above.
+ * polynomial, exact 2^n scaling); h is then quantized as above.  silu(g) of a bf16 g is
+ * read from a table the library computes once per device with exactly that arithmetic
+ * (32 KB of device memory, allocated with the status word on the first call on the
+ * device), so the kernel's h equals the definition for every bf16 input.
  */
 NVFP4_API int nvfp4_silu_mul_quantize_batched(const void *x_bf16, int64_t b, int64_t m, int64_t k,
                                     const int32_t *mask, const float *gsf, uint8_t *q_out,
