@@ -38,7 +38,9 @@ namespace {
 
 constexpr int kSvdRows = 128;            // rows of x per cluster (MMA M)
 constexpr int kSvdChunk = 64;            // bf16 values of K per stage (128-byte rows)
-constexpr int kSvdStages = 4;
+constexpr int kSvdMinStages = 4;
+constexpr int kSvdMaxStages = 8;         // the ring takes as many stages as fit (r = 64: 8)
+constexpr bool kSvdInterleave = true;    // CTA c of a cluster takes K chunks c, c + split, ...
 constexpr int kSvdSplit = 4;             // CTAs per cluster, splitting K
 static_assert(kSvdSplit == 4 || kSvdSplit == 8, "the reduction splits 128 threads over 128 / kSvdSplit rows");
 constexpr int kSvdXBytes = kSvdRows * 128;   // 16 KB per stage
@@ -51,21 +53,34 @@ constexpr int kSvdThreads = 64 + 32 * kSvdQuantWarps;
 static_assert(kSvdQuantWarps == 4 || kSvdQuantWarps == 8 || kSvdQuantWarps == 16, "1, 2 or 4 blocks per thread");
 
 struct __align__(8) SvdControl {
-  uint64_t full[kSvdStages];
-  uint64_t empty[kSvdStages];
+  uint64_t full[kSvdMaxStages];
+  uint64_t empty[kSvdMaxStages];
   uint64_t acc_full;
   uint32_t tmem_base;
   int32_t abort;
 };
 
 __host__ __device__ constexpr int svd_stage_bytes(int r) { return kSvdXBytes + r * 128; }
-__host__ __device__ constexpr int svd_smem_bytes(int r) {
-  return kSvdStages * svd_stage_bytes(r) + static_cast<int>(sizeof(SvdControl)) + 1024;
+// The stage's 64 pre-quantization scales (128 bytes) travel with it in a small ring of their
+// own after the main one (the main ring's tiles stay 1024-byte aligned).
+constexpr int kSvdPqsBytes = kSvdChunk * 2;
+// dynamic shared memory available to the ring (227 KB less the static inverse-scale table,
+// the pre-quantization-scale ring, the control block and the alignment slack)
+constexpr int kSvdRingBudget =
+    227 * 1024 - 512 - kSvdMaxStages * kSvdPqsBytes - static_cast<int>(sizeof(SvdControl)) - 1024;
+__host__ __device__ constexpr int svd_stages(int r) {
+  return kSvdRingBudget / svd_stage_bytes(r) < kSvdMaxStages ? kSvdRingBudget / svd_stage_bytes(r) : kSvdMaxStages;
 }
-static_assert(svd_smem_bytes(kSvdMaxRank) <= 227 * 1024, "shared memory layout exceeds the per-block limit");
+__host__ __device__ constexpr int svd_smem_bytes(int r) {
+  return svd_stages(r) * svd_stage_bytes(r) + kSvdMaxStages * kSvdPqsBytes + static_cast<int>(sizeof(SvdControl)) +
+         1024;
+}
+static_assert(svd_stages(kSvdMaxRank) >= kSvdMinStages, "the ring needs at least four stages");
+static_assert(svd_smem_bytes(32) <= 227 * 1024 - 512 && svd_smem_bytes(kSvdMaxRank) <= 227 * 1024 - 512,
+              "shared memory layout exceeds the per-block limit");
 // the fp32 partial accumulator (128 x r) reuses the stage ring after the K loop
-static_assert(kSvdRows * kSvdMaxRank * 4 <= kSvdStages * svd_stage_bytes(kSvdMaxRank), "partials do not fit");
-static_assert(kSvdRows * 32 * 4 <= kSvdStages * svd_stage_bytes(32), "partials do not fit");
+static_assert(kSvdRows * kSvdMaxRank * 4 <= svd_stages(kSvdMaxRank) * svd_stage_bytes(kSvdMaxRank), "partials do not fit");
+static_assert(kSvdRows * 32 * 4 <= svd_stages(32) * svd_stage_bytes(32), "partials do not fit");
 
 struct SvdParams {
   const uint16_t* pqs;      // [k] bf16 pre-quantization scale (fused op)
@@ -82,6 +97,15 @@ struct SvdParams {
 struct SvdMaps {
   CUtensorMap x, w;
 };
+
+// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from global memory
+// into this CTA's shared memory, completing on `bar`.
+__device__ __forceinline__ void bulk_load_cta(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
 
 // Tiled TMA load into this CTA's shared memory (plain, single-CTA form).
 __device__ __forceinline__ void tma_load_2d_cta(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1) {
@@ -130,21 +154,27 @@ __global__ void __cluster_dims__(kSvdSplit, 1, 1) __launch_bounds__(kSvdThreads,
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int stage_bytes = svd_stage_bytes(p.r);
-  SvdControl& ctl = *reinterpret_cast<SvdControl*>(smem + kSvdStages * stage_bytes);
+  const int stages = svd_stages(p.r);
+  uint8_t* pqs_ring = smem + stages * stage_bytes;
+  SvdControl& ctl = *reinterpret_cast<SvdControl*>(pqs_ring + kSvdMaxStages * kSvdPqsBytes);
   volatile int32_t* abort = &ctl.abort;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
   const int row0 = blockIdx.y * kSvdRows;
   // this CTA's share of the K chunks
+  // this CTA's K chunks: interleaved (c, c + split, ...), so that the cluster's CTAs read
+  // adjacent 128-byte pieces of the same rows at the same time; or one contiguous range
   const int per = (p.chunks + kSvdSplit - 1) / kSvdSplit;
-  const int c_begin = min(static_cast<int>(rank) * per, p.chunks);
-  const int nch = min(c_begin + per, p.chunks) - c_begin;
+  const int c_begin = kSvdInterleave ? static_cast<int>(rank) : min(static_cast<int>(rank) * per, p.chunks);
+  const int c_step = kSvdInterleave ? kSvdSplit : 1;
+  const int nch = kSvdInterleave ? (p.chunks - static_cast<int>(rank) + kSvdSplit - 1) / kSvdSplit
+                                 : min(c_begin + per, p.chunks) - c_begin;
   // the accumulator is drained 64 columns at a time, so at least 64 columns are allocated
   const uint32_t tmem_cols = p.r <= 64 ? 64u : (p.r <= 128 ? 128u : 256u);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kSvdStages; ++s) {
+    for (int s = 0; s < stages; ++s) {
       mbar_init(&ctl.full[s], 1);
       mbar_init(&ctl.empty[s], kQuant ? 1 + kSvdQuantWarps : 1);   // the MMA commit (+ the quantizer warps)
     }
@@ -172,15 +202,18 @@ __global__ void __cluster_dims__(kSvdSplit, 1, 1) __launch_bounds__(kSvdThreads,
       prefetch_map(&maps.w);
     }
     __syncwarp();
-    const uint32_t tx = static_cast<uint32_t>(stage_bytes);
+    const uint32_t tx = static_cast<uint32_t>(stage_bytes + (kQuant ? kSvdPqsBytes : 0));
     for (int i = 0; i < nch; ++i) {
-      const int s = i % kSvdStages;
-      if (i >= kSvdStages && !mbar_wait_fast(&ctl.empty[s], ((i / kSvdStages) - 1) & 1, abort, p.status)) break;
+      const int s = i % stages;
+      if (i >= stages && !mbar_wait_fast(&ctl.empty[s], ((i / stages) - 1) & 1, abort, p.status)) break;
       uint8_t* st = smem + s * stage_bytes;
       if (elect_one()) {
         mbar_arrive_expect_tx(&ctl.full[s], tx);
-        tma_load_2d_cta(st, &maps.x, &ctl.full[s], (c_begin + i) * kSvdChunk, row0);
-        tma_load_2d_cta(st + kSvdXBytes, &maps.w, &ctl.full[s], (c_begin + i) * kSvdChunk, 0);
+        tma_load_2d_cta(st, &maps.x, &ctl.full[s], (c_begin + i * c_step) * kSvdChunk, row0);
+        tma_load_2d_cta(st + kSvdXBytes, &maps.w, &ctl.full[s], (c_begin + i * c_step) * kSvdChunk, 0);
+        if constexpr (kQuant)
+          bulk_load_cta(pqs_ring + s * kSvdPqsBytes, p.pqs + (c_begin + i * c_step) * kSvdChunk, kSvdPqsBytes,
+                        &ctl.full[s]);
       }
       __syncwarp();
     }
@@ -192,8 +225,8 @@ __global__ void __cluster_dims__(kSvdSplit, 1, 1) __launch_bounds__(kSvdThreads,
     const uint64_t b0 = operand_desc(smem_u32(smem + kSvdXBytes));
     bool ok = true;
     for (int i = 0; i < nch; ++i) {
-      const int s = i % kSvdStages;
-      if (!(ok = mbar_wait_fast(&ctl.full[s], (i / kSvdStages) & 1, abort, p.status))) break;
+      const int s = i % stages;
+      if (!(ok = mbar_wait_fast(&ctl.full[s], (i / stages) & 1, abort, p.status))) break;
       tc_fence_after();
       const uint64_t off = static_cast<uint64_t>(s * stage_bytes) >> 4;
       if (elect_one()) {
@@ -220,14 +253,14 @@ __global__ void __cluster_dims__(kSvdSplit, 1, 1) __launch_bounds__(kSvdThreads,
       asm volatile("bar.sync 2, %0;" ::"n"(32 * kSvdQuantWarps) : "memory");
       const uint32_t groups = static_cast<uint32_t>(p.chunks);     // k / 64 scale groups per row
       for (int i = 0; i < nch; ++i) {
-        const int s = i % kSvdStages;
-        const int kc = (c_begin + i) * kSvdChunk;
+        const int s = i % stages;
+        const int kc = (c_begin + i * c_step) * kSvdChunk;
         const int b0 = part * kSvdBlocksPerThread;   // first block (of 4) of this thread
-        uint4 sc_raw[2 * kSvdBlocksPerThread];      // its pre-quantization scales
+        if (!(ok = mbar_wait_fast(&ctl.full[s], (i / stages) & 1, abort, p.status))) break;
+        uint4 sc_raw[2 * kSvdBlocksPerThread];      // its pre-quantization scales (arrived with the stage)
 #pragma unroll
         for (int c = 0; c < 2 * kSvdBlocksPerThread; ++c)
-          sc_raw[c] = __ldg(reinterpret_cast<const uint4*>(p.pqs + kc + 16 * b0 + 8 * c));
-        if (!(ok = mbar_wait_fast(&ctl.full[s], (i / kSvdStages) & 1, abort, p.status))) break;
+          sc_raw[c] = reinterpret_cast<const uint4*>(pqs_ring + s * kSvdPqsBytes)[2 * b0 + c];
         const uint32_t tile = smem_u32(smem + s * stage_bytes);
         const uint32_t sf_word = static_cast<uint32_t>(
             sf_offset(static_cast<uint32_t>(grow), static_cast<uint32_t>(kc / 16 + b0), groups));
@@ -402,15 +435,17 @@ int launch_svdquant(const void* x, int64_t m, int64_t k, const void* pqs, const 
   p.chunks = static_cast<int32_t>(k / kSvdChunk);
   auto kernel = svdquant_input_kernel<kQuant>;
   const int smem = svd_smem_bytes(static_cast<int>(r));
-  static int configured = 0;          // the largest dynamic smem size opted in so far
-  if (smem > configured) {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, svd_smem_bytes(kSvdMaxRank)) !=
-        cudaSuccess) {
+  constexpr int kOptIn = 227 * 1024 - 512;   // every ring size fits below this (static table: 512 B)
+  static_assert(svd_smem_bytes(96) <= kOptIn && svd_smem_bytes(128) <= kOptIn, "ring larger than the opt-in");
+  static bool configured = false;
+  if (!configured) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kOptIn) != cudaSuccess) {
       cudaGetLastError();
       return NVFP4_ERR_CUDA;
     }
-    configured = svd_smem_bytes(kSvdMaxRank);
+    configured = true;
   }
+  if (smem > kOptIn) return NVFP4_ERR_INVALID_ARGUMENT;
   dim3 grid(kSvdSplit, static_cast<unsigned>((m + kSvdRows - 1) / kSvdRows));
   return launch_kernel(kernel, grid, dim3(kSvdThreads), static_cast<size_t>(smem), stream, maps, p);
 }
