@@ -3,7 +3,7 @@
  * scales) quantization and block-scaled FP4 GEMMs for NVIDIA B200 (sm_100a).
  *
  * Sources, cited by page title and section:
- *   [TRT] TensorRT-LLM NVFP4LinearMethod.create_weights (linear.py:871-915)
+ *   [TRT] TensorRT-LLM NVFP4LinearMethod.create_weights
  *   [FV]  FastVideo PR #1350 "Add NVFP4QAT linear layer", code-review thread (_global_sf)
  *   [FI3] flashinfer PR #1774 "Masked batch nvfp4 quantization"
  *   [FI5] flashinfer docs flashinfer.gemm.mm_nvfp4_svdquant (signature, Parameters)

@@ -1,7 +1,7 @@
 // quantize.cu -- global scale (amax) reductions and the NVFP4 block quantizers.
 //
 // Sources (page title, section):
-//   TensorRT-LLM NVFP4LinearMethod.create_weights (linear.py:871-915): block size 16,
+//   TensorRT-LLM NVFP4LinearMethod.create_weights: block size 16,
 //     [out, in/2] packed weight, scale buffer pad_up(rows,128) x pad_up(in/16,4),
 //     input_scale = 448*6/amax_input, alpha = amax_in*amax_w/(448*6*448*6).
 //   FastVideo PR #1350 "Add NVFP4QAT linear layer", review thread: _global_sf

@@ -18,7 +18,7 @@
  *     arithmetic.
  *
  * Sources (cited by page title and section):
- *   [TRT]  TensorRT-LLM NVFP4LinearMethod.create_weights (linear.py:871-915): the
+ *   [TRT]  TensorRT-LLM NVFP4LinearMethod.create_weights: the
  *          [out, in/2] packed weight, the block-16 scale buffer padded to
  *          pad_up(rows,128) x pad_up(in/16,4), input_scale = 448*6/amax_input,
  *          alpha = amax_input*amax_weight/(448*6*448*6).
