@@ -74,8 +74,8 @@ def file_sha(path):
 # The CUDA kernel behind each launch name that can be a workload's dominant launch (the key of
 # its DRAM traffic in profiles/traffic.json).
 KERNEL_OF_LAUNCH = {
-    "quantize": "quantize_kernel", "quantize_masked": "quantize_kernel",
-    "silu_mul_quantize": "silu_quantize_kernel", "global_scale_quantize": "global_scale_quantize_kernel",
+    "quantize": "quantize_kernel", "quantize_masked": "persistent_quantize_kernel",
+    "silu_mul_quantize": "persistent_quantize_kernel", "global_scale_quantize": "global_scale_quantize_kernel",
     "global_scale_quantize_x": "global_scale_quantize_kernel",
     "quantize_smooth_lora_down": "svdquant_input_kernel",
 }

@@ -216,30 +216,35 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantParams p)
   chunk_store<false, kSmooth>(p, ch, nullptr, gsf, inv_tab);
 }
 
-// SiLU * up: persistent CTAs that load the SiLU table into shared memory once and walk the
-// chunks of all items (item-major) with a grid stride, so the live chunks of every item are
-// spread over all CTAs whatever the masks are.  (Issuing the next chunk's loads before the
-// current chunk's arithmetic, with one or two blocks per thread and 2-6 CTAs per SM, measured
-// 2-15% slower than this plain loop with two blocks per thread and four CTAs per SM.)
-constexpr int kSiluUnroll = 2;
-constexpr int kSiluCtasPerSm = 4;
-// The table fits the default 48 KB of dynamic shared memory (no opt-in attribute needed).
+// Persistent CTAs that walk the chunks of all items (item-major) with a grid stride, so the
+// live chunks of every item are spread over all CTAs whatever the masks are, and chunks
+// beyond an item's mask cost a few instructions instead of a CTA launch.  Used for SiLU * up
+// (which loads the SiLU table into shared memory once per CTA) and for the masked
+// quantizer.  (Issuing the next chunk's loads before the current chunk's arithmetic, with
+// one or two blocks per thread and 2-6 CTAs per SM, measured 2-15% slower for SiLU * up than
+// this plain loop with two blocks per thread and four CTAs per SM.)
+template <bool kSilu>
+constexpr int kPersistUnroll = kSilu ? 2 : 4;
+constexpr int kPersistCtasPerSm = 4;
+// The SiLU table fits the default 48 KB of dynamic shared memory (no opt-in attribute needed).
 static_assert(kSiluTableBytes <= 48 * 1024, "SiLU table exceeds the default dynamic shared memory");
-__global__ void __launch_bounds__(kThreads, kSiluCtasPerSm) silu_quantize_kernel(const QuantParams p) {
+template <bool kSilu>
+__global__ void __launch_bounds__(kThreads, kPersistCtasPerSm) persistent_quantize_kernel(const QuantParams p) {
   extern __shared__ float4 silu_smem[];
   __shared__ float inv_tab[128];
   float* tab = reinterpret_cast<float*>(silu_smem);
   pdl_launch_dependents();
   pdl_wait();
-  silu_table_load(tab, p.silu_tab, threadIdx.x, kThreads);
+  if constexpr (kSilu) silu_table_load(tab, p.silu_tab, threadIdx.x, kThreads);
+  constexpr int kUnroll = kPersistUnroll<kSilu>;
   const uint64_t total = static_cast<uint64_t>(p.chunks_per_item) * p.items;
-  Chunk<true, kSiluUnroll> ch;
+  Chunk<kSilu, kUnroll> ch;
   uint32_t table_item = 0xffffffffu;           // the item whose inverse scales inv_tab holds
   float gsf = 0.0f;
   for (uint64_t chunk = blockIdx.x; chunk < total; chunk += gridDim.x) {
     const uint32_t item = static_cast<uint32_t>(chunk / p.chunks_per_item);
     const uint32_t local = static_cast<uint32_t>(chunk - static_cast<uint64_t>(item) * p.chunks_per_item);
-    chunk_load(p, static_cast<int>(item), local * (kThreads * kSiluUnroll), ch);
+    chunk_load(p, static_cast<int>(item), local * (kThreads * kUnroll), ch);
     if (item != table_item) {                   // uniform over the CTA
       __syncthreads();                          // the previous item's table is no longer read
       gsf = __ldg(p.gsf + item);
@@ -247,7 +252,7 @@ __global__ void __launch_bounds__(kThreads, kSiluCtasPerSm) silu_quantize_kernel
       table_item = item;
       __syncthreads();                          // (also orders the SiLU table's first load)
     }
-    chunk_store<true, false>(p, ch, tab, gsf, inv_tab);
+    chunk_store<kSilu, false>(p, ch, tab, gsf, inv_tab);
   }
 }
 
@@ -525,13 +530,15 @@ int launch_quantize(const void* x, int64_t b, int64_t m, int64_t k, bool silu, c
   set_cpad_divisor(p);
   p.silu_tab = info.silu_table;
   p.items = static_cast<uint32_t>(b);
-  if (silu) {
-    constexpr int U = kSiluUnroll;
+  if (silu || mask) {
+    // persistent grid over the chunks of all items
+    const int U = silu ? kPersistUnroll<true> : kPersistUnroll<false>;
     p.chunks_per_item = (p.blocks + kThreads * U - 1) / (kThreads * U);
     const int64_t chunks = static_cast<int64_t>(p.chunks_per_item) * b;
-    const int64_t cap = static_cast<int64_t>(info.sm_count) * kSiluCtasPerSm;
-    return launch_kernel(silu_quantize_kernel, dim3(static_cast<unsigned>(chunks < cap ? chunks : cap)),
-                         dim3(kThreads), kSiluTableBytes, stream, p);
+    const int64_t cap = static_cast<int64_t>(info.sm_count) * kPersistCtasPerSm;
+    const dim3 grid(static_cast<unsigned>(chunks < cap ? chunks : cap));
+    if (silu) return launch_kernel(persistent_quantize_kernel<true>, grid, dim3(kThreads), kSiluTableBytes, stream, p);
+    if (!pqs) return launch_kernel(persistent_quantize_kernel<false>, grid, dim3(kThreads), 0, stream, p);
   }
   constexpr int U = 4;
   p.chunks_per_item = (p.blocks + kThreads * U - 1) / (kThreads * U);
