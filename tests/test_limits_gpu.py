@@ -92,3 +92,21 @@ def test_quantize_wide_rows(oracle):
     q, sf = nv.nvfp4_quantize(dev_bf16(x), dev_f32(gsf))
     q_ref, sf_ref = oracle.quantize(x, gsf)
     assert (host(q) == q_ref).all() and (host(sf) == sf_ref).all()
+
+
+@pytest.mark.parametrize("silu", [False, True])
+def test_masked_quantize_1024_items(oracle, silu):
+    # 1024 items of 5 rows: one chunk per item, so the persistent grid changes item (and
+    # rebuilds its table of inverse scales) on almost every chunk; masks 0..5
+    b, m, k = 1024, 5, 32
+    x = S.normal_with_outliers_bf16((b, m, 2 * k if silu else k), 0.01, 50.0, 46, S.TID["x"])
+    mask = S.rng(46, S.TID["mask"]).integers(0, m + 1, b).astype(np.int32)
+    mask[:2] = [0, m]
+    _, gsf = oracle.global_scale_batched(x, mask, silu_mul=silu)
+    q = torch.full((b, m, k // 2), 0xA5, dtype=torch.uint8, device="cuda")
+    sf = torch.full((b, nv.nvfp4_scale_bytes(m, k)), 0x5A, dtype=torch.uint8, device="cuda")
+    fn = nv.nvfp4_silu_mul_quantize_batched if silu else nv.nvfp4_quantize_masked_batched
+    fn(dev_bf16(x), dev_f32(gsf), dev_i32(mask), q, sf)
+    q_ref, sf_ref = (oracle.silu_mul_quantize_batched if silu else oracle.quantize_masked_batched)(
+        x, gsf, mask, q_fill=0xA5, sf_fill=0x5A)
+    assert (host(q) == q_ref).all() and (host(sf) == sf_ref).all()
