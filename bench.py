@@ -770,7 +770,7 @@ class OracleSample:
         self.unit = "GB/s" if workload.startswith("quant") else "TFLOP/s"
         w = workload
         if w == "swiglu_block":
-            self.rows = rows or 4
+            self.rows = rows or 12          # ~10 s of the oracle on 16 host threads
             d = S.swiglu_block(8192, 5120, 8192, 0)
             self.x = d["x"][:self.rows].copy()
             self.wgu, self.wd = d["w_gate_up"], d["w_down"]
