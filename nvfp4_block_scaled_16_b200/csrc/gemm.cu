@@ -33,19 +33,23 @@
 //               SFA chunk and two of the SFB chunks, each CTA from its own shared memory
 //               into its own tensor memory, then the MMA; the low-rank term follows as kind::f16 (bf16) MMAs into the same
 //               accumulator.  Commits are multicast to both CTAs.
-//   warps 2-5   epilogue (both CTAs): tcgen05.ld of the CTA's 128 x 256 fp32 accumulator
-//               (each warp owns its 32-lane TMEM quarter), alpha * acc + bias, bf16 staged
-//               in shared memory and written by TMA stores (one 32 x 64 tile at a time).
-//               The SiLU * up epilogue uses warps 2-9: two per lane quarter, each with 64
-//               of the tile's 128 h columns.
+//   warps 2-9   epilogue (both CTAs): tcgen05.ld of the CTA's 128 x 256 fp32 accumulator,
+//               two warps per 32-lane TMEM quarter (each warp can only read its own
+//               quarter), each draining two of the four 64-column subtiles: alpha * acc +
+//               bias, bf16 staged in shared memory and written by TMA stores (one 32 x 64
+//               tile at a time).  The grouped bf16 kernel keeps one warp per quarter
+//               (warps 2-5, all four subtiles).  The SiLU * up epilogue: two warps per
+//               quarter, each with 64 of the tile's 128 h columns.
 // Two accumulators of 256 columns share TMEM columns [192, 256): the epilogue drains that
 // overlap first and releases the accumulator, so the next tile's MMAs overlap the rest of
 // the epilogue.  Scale factors use columns [448, 496).
 // SiLU * up epilogue: the B half of CTA 0 is 128 rows of the gate weight and the B half of
 // CTA 1 the same 128 rows of the up weight, so accumulator columns [0, 128) hold g and
-// [128, 256) hold u for 128 columns of h.  Each thread owns 64 columns of one row: it rounds g and u to
-// bf16 exactly as the bf16 epilogue would, forms h, and quantizes each 16-value block with
-// the caller's global scale (64 code bytes and 8 scale bytes per row and tile).  Every
+// [128, 256) hold u for 128 columns of h.  Each thread owns 64 columns of one row: it rounds
+// g and u to bf16 exactly as the bf16 epilogue would, forms h with silu(g) from the SiLU table
+// (copied into shared memory by the epilogue warps at the start), and quantizes each
+// 16-value block with the caller's global scale (32 code bytes and 4 scale bytes per row,
+// warp and tile).  Every
 // epilogue warp loads all its accumulator columns before any arithmetic and releases the
 // accumulator right after, so the next tile's MMAs overlap the whole SiLU and quantization.
 // Every mbarrier wait is bounded (about one second of global time); a wait that runs out
