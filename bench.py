@@ -666,6 +666,52 @@ class SvdquantLinear(Workload):
                 "l2": L2_NOTE}
 
 
+class Bf16aLinear(Workload):
+    """The bf16-activation NVFP4 linear (nvfp4_gemm_bf16a: the pages' f16a_nvfp4weight_scaled_mm
+    in its compiled form) at the SwiGLU block's gate/up shape: x [8192, 5120] bf16, NVFP4
+    weight [16384, 5120], bf16 out."""
+    name = "bf16a_linear"
+    unit = "TFLOP/s"
+    dominant = "gemm"
+
+    def __init__(self, nv, seed=0):
+        import torch
+        self.nv = nv
+        self.M, self.K, self.N = 8192, 5120, 16384
+        d = S.swiglu_block(self.M, self.K, self.N // 2, seed)
+        self.x_host = d["x"]
+        self.x = to_dev_bf16(d["x"])
+        self.wq, self.wsf, self.amax_w = quantize_weight(nv, to_dev_bf16(d["w_gate_up"]))
+        dev = self.x.device
+        self.aq = torch.empty((self.M, self.K // 2), dtype=torch.uint8, device=dev)
+        self.asf = torch.empty(nv.nvfp4_scale_bytes(self.M, self.K), dtype=torch.uint8, device=dev)
+        self.scalars = torch.empty(3, dtype=torch.float32, device=dev)
+        self.out = torch.empty((self.M, self.N), dtype=torch.bfloat16, device=dev)
+        torch.cuda.synchronize()
+
+    def launches(self):
+        lib, s = self.nv, self
+        # nvfp4_gemm_bf16a is these two launches; they are listed separately so that the
+        # kernel pass times each
+        return [("global_scale_quantize", lambda: lib.nvfp4_global_scale_quantize(
+                    s.x, s.amax_w, s.scalars[0:1], s.scalars[1:2], s.scalars[2:3], s.aq, s.asf)),
+                ("gemm", lambda: lib.nvfp4_gemm(s.aq, s.wq, s.asf, s.wsf, s.scalars[2:3], None, s.out))]
+
+    def work(self):
+        return 2.0 * self.M * self.N * self.K
+
+    def kernel_work(self):
+        return {"global_scale_quantize": (2.5625 * self.M * self.K, "GB/s"), "gemm": (self.work(), "TFLOP/s")}
+
+    def e2e_io(self):
+        return self.x_host, self.x, self.out
+
+    def config(self):
+        return {"workload": "bf16-activation NVFP4 linear (dynamic activation scale and quantization, then the FP4 "
+                            "GEMM) x [8192,5120] ~N(0,1), W [16384,5120] ~N(0,0.02), bf16 out",
+                "l2": L2_NOTE}
+
+
 class PR1Linear(Workload):
     name = "pr1_linear"
     unit = "TFLOP/s"
@@ -711,7 +757,7 @@ def workload_config(name, rank_lr, swiglu_path="fused"):
     cls = {"swiglu_block": SwigluBlock, "quant_dense": QuantDense, "quant_dense_fused": QuantDenseFused,
            "quant_masked": QuantMasked, "quant_silu": QuantMasked, "grouped_moe": GroupedMoE,
            "grouped_swiglu": GroupedSwiglu, "lowrank": LowRank, "svdquant_linear": SvdquantLinear,
-           "pr1_linear": PR1Linear}[name]
+           "pr1_linear": PR1Linear, "bf16a_linear": Bf16aLinear}[name]
     w = cls.__new__(cls)
     w.fused = swiglu_path == "fused"
     w.M, w.H, w.I = 8192, 5120, 8192
@@ -746,6 +792,8 @@ def make_workload(name, nv, rank_lr, swiglu_path="fused"):
         return SvdquantLinear(nv, rank_lr)
     if name == "pr1_linear":
         return PR1Linear(nv)
+    if name == "bf16a_linear":
+        return Bf16aLinear(nv)
     raise SystemExit(f"unknown workload {name}")
 
 
@@ -813,6 +861,14 @@ class OracleSample:
             self.x = S.normal_bf16((self.m, self.k), 1.0, 0, S.TID["x"])
             self.w = S.normal_bf16((self.n, self.k), 0.02, 0, S.TID["w"])
             self.sample = f"{self.m} rows x N={self.n} x K={self.k}"
+        elif w == "bf16a_linear":
+            self.rows = rows or 16          # ~10 s of the oracle on 16 host threads
+            d = S.swiglu_block(8192, 5120, 8192, 0)
+            self.x = d["x"][:self.rows].copy()
+            self.w = d["w_gate_up"]
+            self.m, self.k, self.n = self.rows, 5120, 16384
+            self.sample = f"{self.rows} of 8192 activation rows (global scale of the rows, quantize, GEMM against " \
+                          f"the [16384, 5120] weight)"
         else:
             raise SystemExit(f"no oracle sample for {w}")
         self._setup()
@@ -832,7 +888,7 @@ class OracleSample:
             self.ad, gd = O.global_scale(self.wd)
             self.qd, self.sfd = O.quantize(self.wd, gd)
             self.ax, self.gx = O.global_scale(self.x)          # static activation scale (calibration)
-        elif self.workload in ("pr1_linear", "grouped_moe", "lowrank", "svdquant_linear"):
+        elif self.workload in ("pr1_linear", "grouped_moe", "lowrank", "svdquant_linear", "bf16a_linear"):
             self.aw, gw = O.global_scale(self.w)
             self.qw, self.sfw = O.quantize(self.w, gw)
 
@@ -935,7 +991,7 @@ def main():
     ap.add_argument("--impl", default="nvfp4", choices=["nvfp4", "reference"])
     ap.add_argument("--workload", default="swiglu_block",
                     choices=["swiglu_block", "quant_dense", "quant_dense_fused", "quant_masked", "quant_silu", "grouped_moe",
-                             "grouped_swiglu", "lowrank", "svdquant_linear", "pr1_linear"])
+                             "grouped_swiglu", "lowrank", "svdquant_linear", "pr1_linear", "bf16a_linear"])
     ap.add_argument("--rank-lr", type=int, default=64)
     ap.add_argument("--swiglu-path", default="fused", choices=["fused", "unfused"],
                     help="swiglu_block: SiLU*mul quantization in the gate/up GEMM epilogue, or as its own kernel")

@@ -205,6 +205,28 @@ NVFP4_API int nvfp4_gemm(const uint8_t *a, const uint8_t *b, const uint8_t *a_sf
                int64_t k, nvfp4_stream_t stream);
 
 /*
+ * bf16-activation NVFP4 linear [NVF f16a_nvfp4weight_scaled_mm: bf16 activation, NVFP4
+ * weight, bf16 [M, N] out; its compiler path quantizes the activation and runs the scaled
+ * FP4 matmul]:  out = nvfp4_gemm(quantize(a, gsf_a), b, alpha) with the activation's global
+ * scale computed on the device (dynamic), alpha = amax_a * amax_b / (448*6)^2.
+ *   a_bf16     [m, k] bf16, 16-byte aligned; k % 64 == 0, k > 0, m >= 0.
+ *   b, b_sf    the NVFP4 weight [n, k/2] and its scales, as in nvfp4_gemm.
+ *   b_amax     fp32 [1] device: the weight's amax (its global scale is 448*6 / b_amax; the
+ *              pages pass weight_global_scale, this library keeps amaxes so that alpha is
+ *              the [TRT] product formula).
+ *   bias_bf16  nullable bf16 [n]; out_bf16 bf16 [m, n] as in nvfp4_gemm.
+ *   a_q_ws     caller workspace uint8 [m, k/2] (16-byte aligned): the quantized activation.
+ *   a_sf_ws    caller workspace uint8 [nvfp4_scale_bytes(m, k)] (16-byte aligned).
+ *   scalars_ws caller workspace fp32 [3]: receives amax_a, gsf_a and alpha.
+ * Two launches on `stream` (nvfp4_global_scale_quantize, then nvfp4_gemm); allocates
+ * nothing beyond the stream's reduction workspace (allocated on its first use).  The
+ * quantized activation is left in the workspace and equals nvfp4_quantize's bit for bit.
+ */
+NVFP4_API int nvfp4_gemm_bf16a(const void *a_bf16, const uint8_t *b, const uint8_t *b_sf, const float *b_amax,
+                               const void *bias_bf16, void *out_bf16, uint8_t *a_q_ws, uint8_t *a_sf_ws,
+                               float *scalars_ws, int64_t m, int64_t n, int64_t k, nvfp4_stream_t stream);
+
+/*
  * Masked grouped GEMM for MoE experts [FI3: inputs for grouped_gemm_nt_masked; NVF
  * routed_experts GroupedLinear].  For every expert e and row i < mask[e]:
  *   out[e, i, :] = bf16(alpha[e] * a[e, i, :] @ b[e]^T)

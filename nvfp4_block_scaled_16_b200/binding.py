@@ -24,6 +24,7 @@ EXPORTED_SYMBOLS = (
     "nvfp4_quantize_masked_batched",
     "nvfp4_silu_mul_quantize_batched",
     "nvfp4_gemm",
+    "nvfp4_gemm_bf16a",
     "nvfp4_grouped_gemm_masked",
     "nvfp4_gemm_lowrank_bias",
     "nvfp4_gemm_silu_mul_quantize",
@@ -55,6 +56,7 @@ _SIGNATURES = {
     "nvfp4_quantize_masked_batched": (_INT, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P]),
     "nvfp4_silu_mul_quantize_batched": (_INT, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P]),
     "nvfp4_gemm": (_INT, [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
+    "nvfp4_gemm_bf16a": (_INT, [_P] * 9 + [_I64, _I64, _I64, _P]),
     "nvfp4_grouped_gemm_masked": (_INT, [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P]),
     "nvfp4_gemm_lowrank_bias": (_INT, [_P, _P, _P, _P, _P, _P, _P, _I64, _P, _P, _I64, _I64, _I64, _P]),
     "nvfp4_gemm_silu_mul_quantize": (_INT, [_P] * 11 + [_I64, _I64, _I64, _P]),
@@ -247,6 +249,25 @@ def nvfp4_gemm(a, b, a_sf, b_sf, alpha, bias=None, out=None, stream=None):
                                        m, n, 2 * kh, _stream(stream))
     _check("nvfp4_gemm", st)
     return out
+
+
+def nvfp4_gemm_bf16a(a, b, b_sf, b_amax, bias=None, out=None, a_q_ws=None, a_sf_ws=None, scalars_ws=None,
+                     stream=None):
+    """bf16 activation a [m, k] x NVFP4 weight b [n, k/2] -> (out [m, n] bf16, a_q [m, k/2], a_sf, scalars [3]):
+    the activation's dynamic global scale and quantization, then the FP4 GEMM."""
+    m, k = a.shape
+    n = b.shape[0]
+    dev = a.device
+    out = torch.empty((m, n), dtype=torch.bfloat16, device=dev) if out is None else out
+    a_q_ws = torch.empty((m, k // 2), dtype=torch.uint8, device=dev) if a_q_ws is None else a_q_ws
+    if a_sf_ws is None:
+        a_sf_ws = torch.empty(max(nvfp4_scale_bytes(m, k), 0), dtype=torch.uint8, device=dev)
+    scalars_ws = torch.empty(3, dtype=torch.float32, device=dev) if scalars_ws is None else scalars_ws
+    with torch.cuda.device(dev):
+        st = load_library().nvfp4_gemm_bf16a(_ptr(a), _ptr(b), _ptr(b_sf), _ptr(b_amax), _ptr(bias), _ptr(out),
+                                             _ptr(a_q_ws), _ptr(a_sf_ws), _ptr(scalars_ws), m, n, k, _stream(stream))
+    _check("nvfp4_gemm_bf16a", st)
+    return out, a_q_ws, a_sf_ws, scalars_ws
 
 
 def nvfp4_grouped_gemm_masked(a, b, a_sf, b_sf, mask, alpha, out=None, stream=None):

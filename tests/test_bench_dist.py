@@ -78,7 +78,7 @@ def test_reference_arm_config_is_computed_without_a_gpu():
     sys.path.insert(0, ROOT)
     import bench
     for name in ("swiglu_block", "quant_dense", "quant_dense_fused", "quant_masked", "quant_silu", "grouped_moe",
-                 "grouped_swiglu", "lowrank", "svdquant_linear", "pr1_linear"):
+                 "grouped_swiglu", "lowrank", "svdquant_linear", "pr1_linear", "bf16a_linear"):
         cfg = bench.workload_config(name, 64)
         assert isinstance(cfg["workload"], str) and cfg["workload"]
         assert "l2" in cfg
