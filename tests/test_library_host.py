@@ -164,3 +164,28 @@ def test_svdquant_input_argument_checks(lib):
         assert lib.nvfp4_quantize_smooth_lora_down(*bad) == INVALID, i
     assert lib.nvfp4_quantize_smooth(A16, 4, 32, None, A16, A16, A16, None) == INVALID       # pqs required
     assert lib.nvfp4_quantize_smooth(A16, 4, 32, A1, A16, A16, A16, None) == INVALID         # misaligned pqs
+
+
+def test_global_scale_quantize_argument_checks(lib):
+    # (x, m, k, amax, gsf, other_amax, alpha, q, sf, stream)
+    assert lib.nvfp4_global_scale_quantize(A16, 4, 24, None, A16, None, None, A16, A16, None) == INVALID   # k % 16
+    assert lib.nvfp4_global_scale_quantize(A16, 4, 32, None, None, None, None, A16, A16, None) == INVALID  # gsf
+    assert lib.nvfp4_global_scale_quantize(A16, 4, 32, None, A16, A16, None, A16, A16, None) == INVALID    # alpha
+    assert lib.nvfp4_global_scale_quantize(A16, 4, 32, None, A16, None, None, None, A16, None) == INVALID  # q
+    assert lib.nvfp4_global_scale_quantize(A1, 4, 32, None, A16, None, None, A16, A16, None) == INVALID    # x
+    assert lib.nvfp4_selftest_grid_barrier(A16, 4, 24, A16, A16, A16, None) == INVALID
+
+
+def test_bf16a_argument_checks(lib):
+    # (a, b, b_sf, b_amax, bias, out, a_q_ws, a_sf_ws, scalars_ws, m, n, k, stream)
+    args = [A16] * 9
+    assert lib.nvfp4_gemm_bf16a(*args, 128, 256, 96, None) == INVALID          # k % 64
+    assert lib.nvfp4_gemm_bf16a(*args, 128, 100, 256, None) == INVALID         # n % 8
+    for i in (0, 1, 2, 3, 5, 6, 7, 8):                                          # required pointers (bias is optional)
+        bad = list(args)
+        bad[i] = None
+        assert lib.nvfp4_gemm_bf16a(*bad, 128, 256, 256, None) == INVALID, i
+    for i in (0, 1, 2, 4, 5, 6, 7):                                             # 16-byte alignment
+        bad = list(args)
+        bad[i] = A1
+        assert lib.nvfp4_gemm_bf16a(*bad, 128, 256, 256, None) == INVALID, i
