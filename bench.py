@@ -818,7 +818,7 @@ class OracleSample:
         self.unit = "GB/s" if workload.startswith("quant") else "TFLOP/s"
         w = workload
         if w == "swiglu_block":
-            self.rows = rows or 12          # ~10 s of the oracle on 16 host threads
+            self.rows = rows or 48          # ~10 s of the oracle on 16 host threads
             d = S.swiglu_block(8192, 5120, 8192, 0)
             self.x = d["x"][:self.rows].copy()
             self.wgu, self.wd = d["w_gate_up"], d["w_down"]
@@ -862,7 +862,7 @@ class OracleSample:
             self.w = S.normal_bf16((self.n, self.k), 0.02, 0, S.TID["w"])
             self.sample = f"{self.m} rows x N={self.n} x K={self.k}"
         elif w == "bf16a_linear":
-            self.rows = rows or 16          # ~10 s of the oracle on 16 host threads
+            self.rows = rows or 64          # ~10 s of the oracle on 16 host threads
             d = S.swiglu_block(8192, 5120, 8192, 0)
             self.x = d["x"][:self.rows].copy()
             self.w = d["w_gate_up"]
