@@ -80,14 +80,17 @@ constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;  // 38 KB
 constexpr uint32_t kFp4TxBytes = 2u * kStageBytes;              // both CTAs
 constexpr uint32_t kLrTxBytes = 2u * (kABytes + kBBytes);
 constexpr int kMaxExperts = 1024;
-// Warps: 0 TMA producer, 1 MMA issuer, then the epilogue warps: two per TMEM lane quarter
-// (each drains half of the tile's columns, so a tile's epilogue takes about half the time of
-// one warp per quarter), except in the grouped bf16 kernel, whose expert prefix table leaves
-// shared memory for the staging tiles of one warp per quarter only.
-template <bool kGrouped, bool kSwiGLU>
-constexpr int kEpiWarps = (kGrouped && !kSwiGLU) ? 4 : 8;
-template <bool kGrouped, bool kSwiGLU>
-constexpr int kThreads = 64 + 32 * kEpiWarps<kGrouped, kSwiGLU>;
+// Warps: 0 TMA producer, 1 MMA issuer, then kQW epilogue warps per TMEM lane quarter.  Two
+// per quarter (each draining half of the tile's columns) halve a tile's epilogue, which pays
+// when the epilogue is on the critical path: short K loops, few tiles.  On long K loops the
+// epilogue hides behind the next tile's mainloop anyway, and one warp per quarter (with two
+// staging tiles) leaves more issue slots to the producer and MMA warps: measured 118.9 against
+// 122.9 us on 8192 x 5120 x 8192 and 233.5 against 247.8 us on 8192 x 16384 x 5120, but 30.7
+// against 28.7 us on 4096 x 3072 x 3072.  The SiLU * up epilogue always uses two.
+template <int kQW>
+constexpr int kEpiWarps = 4 * kQW;
+template <int kQW>
+constexpr int kThreads = 64 + 32 * kEpiWarps<kQW>;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccOverlapCol = 192;          // accumulator 1 starts here
 constexpr uint32_t kSfaCol = 448;                 // SFA: 448 + 4j, SFB: 464 + 8j (+4 upper half)
@@ -103,13 +106,15 @@ struct __align__(8) Control {
   int32_t abort;
   int32_t prefix[kMaxExperts + 1];   // grouped: prefix sums of pair tiles per expert
 };
-// bf16 epilogue: one 32-row x 64-column bf16 staging tile (4 KB, 128-byte swizzle) per
-// epilogue warp, written to global memory by TMA stores.
+// bf16 epilogue: 32-row x 64-column bf16 staging tiles (4 KB, 128-byte swizzle) per epilogue
+// warp, written to global memory by TMA stores: two per warp (one store in flight while the
+// next tile is written) with one warp per quarter, one with two (or in the grouped kernel,
+// whose expert prefix table takes the room).
 constexpr int kStoreTileBytes = 32 * 128;
-template <bool kGrouped, bool kSwiGLU>
-constexpr int kStagingBuffers = kSwiGLU ? 0 : 1;
-template <bool kGrouped, bool kSwiGLU>
-constexpr int kStagingBytes = kStagingBuffers<kGrouped, kSwiGLU> * kEpiWarps<kGrouped, kSwiGLU> * kStoreTileBytes;
+template <bool kGrouped, bool kSwiGLU, int kQW>
+constexpr int kStagingBuffers = kSwiGLU ? 0 : ((kQW == 1 && !kGrouped) ? 2 : 1);
+template <bool kGrouped, bool kSwiGLU, int kQW>
+constexpr int kStagingBytes = kStagingBuffers<kGrouped, kSwiGLU, kQW> * kEpiWarps<kQW> * kStoreTileBytes;
 // SiLU * up epilogue: the SiLU table (32 KB) after the ring.
 template <bool kSwiGLU>
 constexpr int kTableBytes = kSwiGLU ? static_cast<int>(kSiluTableBytes) : 0;
@@ -117,12 +122,13 @@ constexpr int kTableBytes = kSwiGLU ? static_cast<int>(kSiluTableBytes) : 0;
 template <bool kGrouped>
 constexpr int kControlBytes = kGrouped ? static_cast<int>(sizeof(Control))
                                        : static_cast<int>(offsetof(Control, prefix)) + 8;
-template <bool kGrouped, bool kSwiGLU>
-constexpr int kSmemBytes =
-    kStages * kStageBytes + kStagingBytes<kGrouped, kSwiGLU> + kTableBytes<kSwiGLU> + kControlBytes<kGrouped> + 1024;
+template <bool kGrouped, bool kSwiGLU, int kQW>
+constexpr int kSmemBytes = kStages * kStageBytes + kStagingBytes<kGrouped, kSwiGLU, kQW> + kTableBytes<kSwiGLU> +
+                           kControlBytes<kGrouped> + 1024;
 constexpr int kMaxDynamicSmem = 227 * 1024;      // sm_100 opt-in limit per block
-static_assert(kSmemBytes<false, false> <= kMaxDynamicSmem && kSmemBytes<true, false> <= kMaxDynamicSmem &&
-                  kSmemBytes<false, true> <= kMaxDynamicSmem && kSmemBytes<true, true> <= kMaxDynamicSmem,
+static_assert(kSmemBytes<false, false, 1> <= kMaxDynamicSmem && kSmemBytes<false, false, 2> <= kMaxDynamicSmem &&
+                  kSmemBytes<true, false, 1> <= kMaxDynamicSmem && kSmemBytes<false, true, 2> <= kMaxDynamicSmem &&
+                  kSmemBytes<true, true, 2> <= kMaxDynamicSmem,
               "shared memory layout exceeds the per-block limit");
 
 // Instruction descriptors (tcgen05 "instruction descriptor" bit fields).
@@ -266,14 +272,14 @@ struct Maps {
 
 // ---- the kernel ---------------------------------------------------------------------------------
 
-template <bool kGrouped, bool kLowRank, bool kSwiGLU>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kGrouped, kSwiGLU>, 1)
+template <bool kGrouped, bool kLowRank, bool kSwiGLU, int kQW>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kQW>, 1)
     nvfp4_gemm_kernel(const __grid_constant__ Maps maps, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* staging = smem + kStages * kStageBytes;     // 1024-byte aligned (the ring is 190 KB)
-  float* silu_tab = reinterpret_cast<float*>(staging + kStagingBytes<kGrouped, kSwiGLU>);
-  Control& ctl = *reinterpret_cast<Control*>(staging + kStagingBytes<kGrouped, kSwiGLU> + kTableBytes<kSwiGLU>);
+  float* silu_tab = reinterpret_cast<float*>(staging + kStagingBytes<kGrouped, kSwiGLU, kQW>);
+  Control& ctl = *reinterpret_cast<Control*>(staging + kStagingBytes<kGrouped, kSwiGLU, kQW> + kTableBytes<kSwiGLU>);
   volatile int32_t* abort = &ctl.abort;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -288,7 +294,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kGrouped, k
       mbar_init(&ctl.empty[s], 1);
     }
     mbar_init(&ctl.acc_full, 1);
-    mbar_init(&ctl.acc_empty, 2 * kEpiWarps<kGrouped, kSwiGLU>);   // every epilogue warp of both CTAs
+    mbar_init(&ctl.acc_empty, 2 * kEpiWarps<kQW>);   // every epilogue warp of both CTAs
     ctl.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -471,8 +477,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kGrouped, k
     const uint32_t acc_empty_leader = map_to_rank(&ctl.acc_empty, 0);
     if constexpr (kSwiGLU) {
       // the epilogue warps load the SiLU table while the first tile's mainloop runs
-      silu_table_load(silu_tab, p.silu_tab, threadIdx.x - 64, 32 * kEpiWarps<kGrouped, true>);
-      asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpiWarps<kGrouped, true>) : "memory");
+      silu_table_load(silu_tab, p.silu_tab, threadIdx.x - 64, 32 * kEpiWarps<kQW>);
+      asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpiWarps<kQW>) : "memory");
     }
     uint32_t tcount = 0;
     TileCoord t;
@@ -499,7 +505,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kGrouped, k
         uint8_t* sf_e = p.sf + static_cast<int64_t>(t.expert) * p.sf_item_stride;
         const uint32_t groups = static_cast<uint32_t>(p.n / 64);
         {
-          constexpr int kQuarterWarps = kEpiWarps<kGrouped, true> / 4;   // epilogue warps per lane quarter
+          constexpr int kQuarterWarps = kQW;                     // epilogue warps per lane quarter
           constexpr int kCols = 128 / kQuarterWarps;            // h columns of this warp
           constexpr int kBlocks = kCols / 16;                   // 16-value blocks per thread
           const int part = (warp - 2) >> 2;                     // which kCols-wide slice
@@ -560,7 +566,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kGrouped, k
         // the mask stay untouched.
         const int slab_row = t.m_tile * kTileM + static_cast<int>(rank) * kBM + quarter * 32;
         const bool use_tma = kGrouped ? slab_row + 32 <= t.valid_rows : slab_row < p.m;
-        uint8_t* stage_tile = staging + (warp - 2) * kStoreTileBytes;
+        constexpr int kBufs = kStagingBuffers<kGrouped, kSwiGLU, kQW>;
+        uint8_t* stage_warp = staging + (warp - 2) * kBufs * kStoreTileBytes;
         __nv_bfloat16* out_row = p.out + (static_cast<int64_t>(t.expert) * p.m + row) * p.n;
         // The quarter's warps split the four 64-column subtiles in drain order: accumulator 0
         // drains its last 64 columns first, accumulator 1 its first 64 (the columns the next
@@ -568,7 +575,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kGrouped, k
         // first subtile.  A warp that never reads the overlap may release it at once; the
         // tile after next reuses this accumulator only after every warp has released the
         // next tile's, which it does after finishing this one.
-        constexpr int kSubs = 16 / kEpiWarps<kGrouped, kSwiGLU>;   // subtiles per warp
+        constexpr int kSubs = 4 / kQW;                          // subtiles per warp
         const int part = (warp - 2) >> 2;
         for (int j = 0; j < kSubs; ++j) {
           const int i = part * kSubs + j;
@@ -613,8 +620,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kGrouped, k
             o[g].w = pack_bf16x2(f[6], f[7]);
           }
           if (use_tma) {
+            uint8_t* stage_tile = stage_warp + (nstore % kBufs) * kStoreTileBytes;
             const uint32_t stage_row = smem_u32(stage_tile) + lane * 128;
-            if (nstore > 0 && lane == 0) bulk_wait_read<0>();   // the previous store has read the tile
+            if (lane == 0) bulk_wait_read<kBufs - 1>();   // the store that last used this tile has read it
             __syncwarp();
             // 128-byte swizzle: 16-byte chunk g of row r sits at chunk position g ^ (r % 8)
 #pragma unroll
@@ -729,6 +737,36 @@ struct GemmArgs {
   int32_t stall_stage = -1;                // self-test only
 };
 
+// Launches the kernel instantiation with kQW epilogue warps per lane quarter: the one-time
+// set-up per instantiation (dynamic shared memory opt-in, the number of 2-CTA clusters that
+// fit on the device at once: the persistent grid size), then a grid of min(tiles, clusters)
+// pairs.
+template <bool kGrouped, bool kLowRank, bool kSwiGLU, int kQW>
+int run_gemm(const Maps& maps, const GemmParams& p, int64_t tiles, const DeviceInfo& info, cudaStream_t stream) {
+  auto kernel = nvfp4_gemm_kernel<kGrouped, kLowRank, kSwiGLU, kQW>;
+  constexpr int kSmem = kSmemBytes<kGrouped, kSwiGLU, kQW>;
+  static int max_clusters = 0;
+  if (max_clusters == 0) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess) {
+      cudaGetLastError();
+      return NVFP4_ERR_CUDA;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(info.sm_count / 2 * 2);
+    cfg.blockDim = dim3(kThreads<kQW>);
+    cfg.dynamicSmemBytes = kSmem;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg) != cudaSuccess || clusters <= 0) {
+      cudaGetLastError();
+      clusters = info.sm_count / 2;
+    }
+    max_clusters = clusters;
+  }
+  const int64_t max_pairs = max_clusters;
+  const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
+  return launch_kernel(kernel, dim3(2 * pairs), dim3(kThreads<kQW>), kSmem, stream, maps, p);
+}
+
 template <bool kGrouped, bool kLowRank, bool kSwiGLU>
 int launch_gemm(const GemmArgs& g, cudaStream_t stream) {
   const int64_t E = g.E, m = g.m, n = g.n, k = g.k;
@@ -800,34 +838,20 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream) {
     p.rows_pad = static_cast<int32_t>((m + 127) / 128 * 128);
   }
 
-  auto kernel = nvfp4_gemm_kernel<kGrouped, kLowRank, kSwiGLU>;
-  // One-time set-up per kernel instantiation: the dynamic shared memory opt-in and the
-  // number of 2-CTA clusters that fit on the device at once (the persistent grid size).
-  static int max_clusters = 0;
-  if (max_clusters == 0) {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes<kGrouped, kSwiGLU>) !=
-        cudaSuccess) {
-      cudaGetLastError();
-      return NVFP4_ERR_CUDA;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(info.sm_count / 2 * 2);
-    cfg.blockDim = dim3(kThreads<kGrouped, kSwiGLU>);
-    cfg.dynamicSmemBytes = kSmemBytes<kGrouped, kSwiGLU>;
-    int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg) != cudaSuccess || clusters <= 0) {
-      cudaGetLastError();
-      clusters = info.sm_count / 2;
-    }
-    max_clusters = clusters;
-  }
   const int64_t tiles = kGrouped ? static_cast<int64_t>(E) * p.m_tiles * p.n_tiles
                                  : static_cast<int64_t>(p.m_tiles) * p.n_tiles;
   if (tiles >= (int64_t(1) << 31)) return NVFP4_ERR_INVALID_ARGUMENT;
-  const int64_t max_pairs = max_clusters;
-  const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
-  return launch_kernel(kernel, dim3(2 * pairs), dim3(kThreads<kGrouped, kSwiGLU>), kSmemBytes<kGrouped, kSwiGLU>,
-                       stream, maps, p);
+  if constexpr (kSwiGLU) {
+    return run_gemm<kGrouped, kLowRank, kSwiGLU, 2>(maps, p, tiles, info, stream);
+  } else if constexpr (kGrouped) {
+    return run_gemm<kGrouped, kLowRank, kSwiGLU, 1>(maps, p, tiles, info, stream);
+  } else {
+    // one epilogue warp per lane quarter when the K loop hides the epilogue and there are
+    // at least two waves of tiles; two otherwise (see kEpiWarps)
+    if (k >= 4096 && tiles >= static_cast<int64_t>(info.sm_count))
+      return run_gemm<kGrouped, kLowRank, kSwiGLU, 1>(maps, p, tiles, info, stream);
+    return run_gemm<kGrouped, kLowRank, kSwiGLU, 2>(maps, p, tiles, info, stream);
+  }
 }
 
 // Self-test of the bounded wait: one thread waits for an mbarrier phase that nothing ever

@@ -198,6 +198,30 @@ def test_lowrank_full_size(oracle, r):
     assert_gemm_close(S.bf16_bits_to_f32(out[ii, jj]).astype(np.float64), ref, f"lowrank full r={r}")
 
 
+@pytest.mark.parametrize("m,n,k,r", [(4096, 2560, 4096, 64), (2048, 4864, 6144, 0)])
+def test_long_k_gemms_take_the_one_warp_epilogue(oracle, m, n, k, r):
+    # K >= 4096 and at least one tile per SM: the launcher picks the kernel with one epilogue
+    # warp per TMEM lane quarter and two staging tiles; low-rank (r > 0) and plain (r = 0)
+    xa = S.normal_bf16((m, k), 1.0, 47 + r, S.TID["x"])
+    xb = S.normal_bf16((n, k), 0.02, 47 + r, S.TID["w"])
+    qa, sfa, amax_a = quantized(oracle, xa)
+    qb, sfb, amax_b = quantized(oracle, xb)
+    alpha = np.float32(oracle.alpha(float(amax_a), float(amax_b)))
+    ii, jj = sample_positions(m, n, 4096, r + 1)
+    if r:
+        dd = S.normal_bf16((m, r), 1.0, 47, S.TID["d"])
+        l1 = S.f32_to_bf16_bits(S.rng(47, S.TID["l1"]).standard_normal((n, r), dtype=np.float32) * np.float32(0.01)
+                                / alpha)
+        bias = S.normal_bf16((n,), 0.1, 47, S.TID["bias"])
+        out = host(nv.nvfp4_gemm_lowrank_bias(dev_u8(qa), dev_u8(qb), dev_u8(sfa), dev_u8(sfb), dev_f32(alpha),
+                                              dev_bf16(dd), dev_bf16(l1), dev_bf16(bias)))
+        ref = oracle.gemm_ref_sampled(qa, qb, sfa, sfb, alpha, k, ii, jj, d=dd, l1=l1, bias=bias)
+    else:
+        out = host(nv.nvfp4_gemm(dev_u8(qa), dev_u8(qb), dev_u8(sfa), dev_u8(sfb), dev_f32(alpha)))
+        ref = oracle.gemm_ref_sampled(qa, qb, sfa, sfb, alpha, k, ii, jj)
+    assert_gemm_close(S.bf16_bits_to_f32(out[ii, jj]).astype(np.float64), ref, f"{m}x{n}x{k} r={r}")
+
+
 def test_grouped_full_size_sampled(oracle):
     d = S.grouped_moe()
     E, mmax, k, n = 16, 2048, 5120, 8192
