@@ -1,6 +1,10 @@
-"""Shared helpers of the GPU parity tests (placement and comparison only)."""
+"""Shared helpers of the parity tests (placement, comparison and fixture loading only)."""
+import os
+
 import numpy as np
 import torch
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 
 # GEMM tolerance: |out - ref| <= 1e-2*|ref| + 1e-3*max|ref|, ref in fp64 from the
 # dequantized operands.
@@ -98,3 +102,45 @@ def assert_nvfp4_close(q, s, q_ref, s_ref, gsf, what="", max_frac=1e-2):
     bad = np.abs(v - vr) > bound
     assert not bad.any(), f"{what}: {int(bad.sum())} values beyond two e2m1 steps; first {np.argwhere(bad)[:3].tolist()}"
     return scale_frac, code_frac
+
+
+def load_worked_example():
+    """The hand-worked example of tests/golden/nvfp4_worked_example.txt as arrays.
+
+    Returns a dict: rows, k, row, amax, gsf; x (uint16 bf16 bits [rows, k], zero except
+    the worked row) and x_values (that row's values, fp64); codes [k] and dq [k] (fp64)
+    of that row; scales [k/16] (codes); q ([rows, k/2] packed bytes, low nibble first) and
+    sf ([sf_bytes], the row's scales at sf_offsets, every other byte 0) as the quantizer
+    must write them; gemm_self, gemm_ones and their bf16 roundings gemm_self_bf16,
+    gemm_ones_bf16; ones_amax, ones_gsf, ones_scale, ones_code of the all-ones operand."""
+    kv = {}
+    with open(os.path.join(GOLDEN, "nvfp4_worked_example.txt")) as f:
+        for line in f:
+            line = line.split("#", 1)[0].split()
+            if line:
+                kv[line[0]] = line[1:]
+    rows, k, row = int(kv["rows"][0]), int(kv["k"][0]), int(kv["row"][0])
+    nb = k // 16
+    xs = np.concatenate([np.array(kv[f"x{j}"], np.float64) for j in range(nb)])
+    x32 = torch.from_numpy(xs.astype(np.float32))
+    bits = x32.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    if not np.array_equal(torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).double().numpy(), xs):
+        raise ValueError("worked example: an input value is not a bf16 number")
+    x = np.zeros((rows, k), np.uint16)
+    x[row] = bits
+    codes = np.concatenate([np.array([int(c, 16) for c in kv[f"codes{j}"]], np.uint8) for j in range(nb)])
+    scales = np.array([int(kv[f"scale{j}"][0], 16) for j in range(nb)], np.uint8)
+    q = np.zeros((rows, k // 2), np.uint8)
+    q[row] = codes[0::2] | (codes[1::2] << 4)
+    sf = np.zeros(int(kv["sf_bytes"][0]), np.uint8)
+    sf[np.array(kv["sf_offsets"], np.int64)] = scales
+    return {
+        "rows": rows, "k": k, "row": row, "amax": float(kv["amax"][0]), "gsf": float(kv["gsf"][0]),
+        "x": x, "x_values": xs, "codes": codes, "scales": scales, "q": q, "sf": sf,
+        "sf_offsets": np.array(kv["sf_offsets"], np.int64),
+        "dq": np.concatenate([np.array(kv[f"dq{j}"], np.float64) for j in range(nb)]),
+        "gemm_self": float(kv["gemm_self"][0]), "gemm_ones": float(kv["gemm_ones"][0]),
+        "gemm_self_bf16": float(kv["gemm_self_bf16"][0]), "gemm_ones_bf16": float(kv["gemm_ones_bf16"][0]),
+        "ones_amax": float(kv["ones_amax"][0]), "ones_gsf": float(kv["ones_gsf"][0]),
+        "ones_scale": int(kv["ones_scale"][0], 16), "ones_code": int(kv["ones_code"][0]),
+    }

@@ -1,0 +1,72 @@
+"""The CUDA path against the hand-worked example in tests/golden/nvfp4_worked_example.txt.
+
+The fixture was derived by hand from the format definitions and the pages' formulas, so
+these tests hold the kernels to values no program produced: the fused global-scale
+quantizer, the dense quantizer with a given global scale (every packed byte and every
+scale byte, padding included) and the block-scaled FP4 GEMM (exact bf16 outputs, since
+the fixture's sums lie far from any bf16 rounding midpoint)."""
+import numpy as np
+import pytest
+import torch
+
+import nvfp4_block_scaled_16_b200 as nv
+from tests.helpers import assert_gemm_close, bf16_to_f64, dev_bf16, dev_f32, host, load_worked_example
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from nvfp4_block_scaled_16_b200 import build
+    build.build()
+    nv.load_library()
+    yield
+
+
+@pytest.fixture(autouse=True)
+def _status_clean():
+    yield
+    assert nv.nvfp4_device_status(clear=True) == 0, "a device-side wait timed out"
+
+
+@pytest.fixture(scope="module")
+def ex():
+    return load_worked_example()
+
+
+def test_global_scale_quantize(ex):
+    amax, gsf, alpha, q, sf = nv.nvfp4_global_scale_quantize(dev_bf16(ex["x"]), other_amax=dev_f32(ex["amax"]))
+    assert host(amax)[0] == ex["amax"] and host(gsf)[0] == ex["gsf"]
+    assert host(alpha)[0] == np.float32(1.0)
+    assert np.array_equal(host(q), ex["q"])
+    assert np.array_equal(host(sf), ex["sf"])
+
+
+def test_quantize(ex):
+    q = torch.full((ex["rows"], ex["k"] // 2), 0xAA, dtype=torch.uint8, device="cuda")
+    sf = torch.full((ex["sf"].size,), 0xAA, dtype=torch.uint8, device="cuda")
+    nv.nvfp4_quantize(dev_bf16(ex["x"]), dev_f32(ex["gsf"]), q, sf)
+    assert np.array_equal(host(q), ex["q"])
+    assert np.array_equal(host(sf), ex["sf"])
+
+
+def test_gemm(ex):
+    rows, k, row = ex["rows"], ex["k"], ex["row"]
+    qa, sfa = nv.nvfp4_quantize(dev_bf16(ex["x"]), dev_f32(ex["gsf"]))
+    out = nv.nvfp4_gemm(qa, qa, sfa, sfa, dev_f32(1.0))
+    want = np.zeros((rows, rows))
+    want[row, row] = ex["gemm_self_bf16"]
+    assert np.array_equal(bf16_to_f64(out), want)
+
+    ones = dev_bf16(np.full((8, k), 0x3F80, np.uint16))
+    amax_b, gsf_b, alpha, qb, sfb = nv.nvfp4_global_scale_quantize(ones, other_amax=dev_f32(ex["amax"]))
+    assert host(amax_b)[0] == ex["ones_amax"] and host(gsf_b)[0] == ex["ones_gsf"]
+    assert np.all(host(qb) == ex["ones_code"] * 0x11)
+    assert host(alpha)[0] == np.float32(1.0 / 2688.0)
+    out = bf16_to_f64(nv.nvfp4_gemm(qa, qb, sfa, sfb, alpha))
+    want = np.zeros((rows, 8))
+    want[row, :] = ex["gemm_ones_bf16"]
+    assert np.array_equal(out, want)
+    ref = np.zeros((rows, 8))
+    ref[row, :] = ex["gemm_ones"]
+    assert_gemm_close(out, ref, "worked example, ones operand")

@@ -1,0 +1,75 @@
+"""The oracle against the hand-worked example in tests/golden/nvfp4_worked_example.txt.
+
+The fixture's values were derived with pencil and paper from the format definitions and
+the pages' formulas (its header gives the sources and each step), not by a program, so
+these tests pin the oracle's global scale, quantizer, scale layout, dequantization and
+GEMM reference to something other than the oracle.  The first test checks the fixture
+against itself (codes x scales = dequantized values, the padded scale size)."""
+import numpy as np
+import pytest
+import torch
+
+from tests.helpers import E2M1, e4m3_values, load_worked_example
+
+
+@pytest.fixture(scope="module")
+def ex():
+    return load_worked_example()
+
+
+def test_fixture_is_consistent(ex):
+    k = ex["k"]
+    s = np.repeat(e4m3_values(ex["scales"]), 16)
+    assert np.array_equal(E2M1[ex["codes"]] * s, ex["dq"])
+    # padded scale size pad_up(rows, 128) * pad_up(k/16, 4)
+    assert ex["sf"].size == (-(-ex["rows"] // 128) * 128) * (-(-(k // 16) // 4) * 4)
+    assert ex["amax"] == np.abs(ex["x_values"]).max()
+    assert ex["gsf"] == 448.0 * 6.0 / ex["amax"]
+    assert ex["gemm_self"] == float(np.dot(ex["dq"], ex["dq"]))
+    assert ex["gemm_ones"] == float(ex["dq"].sum())
+    for exact, rounded in [(ex["gemm_self"], ex["gemm_self_bf16"]), (ex["gemm_ones"], ex["gemm_ones_bf16"])]:
+        assert torch.tensor(exact, dtype=torch.float64).to(torch.bfloat16).item() == rounded
+
+
+def test_oracle_global_scale(oracle, ex):
+    amax, gsf = oracle.global_scale(ex["x"])
+    assert float(amax) == ex["amax"] and float(gsf) == ex["gsf"]
+    ones = np.full((8, ex["k"]), 0x3F80, np.uint16)        # bf16 1.0
+    amax_b, gsf_b = oracle.global_scale(ones)
+    assert float(amax_b) == ex["ones_amax"] and float(gsf_b) == ex["ones_gsf"]
+    assert np.float32(oracle.alpha(ex["amax"], ex["amax"])) == np.float32(1.0)
+    assert np.float32(oracle.alpha(ex["amax"], ex["ones_amax"])) == np.float32(1.0 / 2688.0)
+
+
+def test_oracle_quantize(oracle, ex):
+    q, sf = oracle.quantize(ex["x"], ex["gsf"], sf_fill=0xAA)
+    assert np.array_equal(q, ex["q"])
+    assert np.array_equal(sf, ex["sf"])
+
+
+def test_oracle_dequantize(oracle, ex):
+    q, sf = oracle.quantize(ex["x"], ex["gsf"])
+    dq = oracle.dequantize_logical(q, sf, ex["rows"], ex["k"])
+    assert np.array_equal(dq[ex["row"]], ex["dq"])
+    assert not np.any(np.delete(dq, ex["row"], axis=0))
+
+
+def test_oracle_gemm(oracle, ex):
+    rows, k, row = ex["rows"], ex["k"], ex["row"]
+    q, sf = oracle.quantize(ex["x"], ex["gsf"])
+    out = oracle.gemm_ref(q, q, sf, sf, oracle.alpha(ex["amax"], ex["amax"]), rows, rows, k)
+    want = np.zeros((rows, rows))
+    want[row, row] = ex["gemm_self"]
+    assert np.array_equal(out, want)
+    bits = torch.tensor([ex["gemm_self_bf16"]], dtype=torch.bfloat16).view(torch.int16).item() & 0xFFFF
+    assert oracle.f64_to_bf16(ex["gemm_self"]) == bits
+
+    ones = np.full((8, k), 0x3F80, np.uint16)
+    qb, sfb = oracle.quantize(ones, ex["ones_gsf"])
+    assert np.all(qb == ex["ones_code"] * 0x11)
+    assert np.all(sfb.reshape(-1)[[r * 16 + c for r in range(8) for c in range(4)]] == ex["ones_scale"])
+    alpha = np.float32(oracle.alpha(ex["amax"], ex["ones_amax"]))
+    out = oracle.gemm_ref(q, qb, sf, sfb, alpha, rows, 8, k)
+    # alpha is 1/2688 rounded to fp32; every other factor is exact
+    assert np.allclose(out[row], ex["gemm_ones"], rtol=2.0 ** -23, atol=0)
+    assert not np.any(np.delete(out, row, axis=0))
