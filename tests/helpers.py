@@ -112,7 +112,9 @@ def load_worked_example():
     of that row; scales [k/16] (codes); q ([rows, k/2] packed bytes, low nibble first) and
     sf ([sf_bytes], the row's scales at sf_offsets, every other byte 0) as the quantizer
     must write them; gemm_self, gemm_ones and their bf16 roundings gemm_self_bf16,
-    gemm_ones_bf16; ones_amax, ones_gsf, ones_scale, ones_code of the all-ones operand."""
+    gemm_ones_bf16; ones_amax, ones_gsf, ones_scale, ones_code of the all-ones operand;
+    the variants' inputs silu_gate, mask, pre_quant_scale, lowrank_r, lowrank_l1, bias and
+    the low-rank GEMM's outputs lowrank_row (row 33 off the diagonal), lowrank_other."""
     kv = {}
     with open(os.path.join(GOLDEN, "nvfp4_worked_example.txt")) as f:
         for line in f:
@@ -143,4 +145,60 @@ def load_worked_example():
         "gemm_self_bf16": float(kv["gemm_self_bf16"][0]), "gemm_ones_bf16": float(kv["gemm_ones_bf16"][0]),
         "ones_amax": float(kv["ones_amax"][0]), "ones_gsf": float(kv["ones_gsf"][0]),
         "ones_scale": int(kv["ones_scale"][0], 16), "ones_code": int(kv["ones_code"][0]),
+        "silu_gate": float(kv["silu_gate"][0]), "mask": int(kv["mask"][0]),
+        "pre_quant_scale": float(kv["pre_quant_scale"][0]), "lowrank_r": int(kv["lowrank_r"][0]),
+        "lowrank_l1": float(kv["lowrank_l1"][0]), "bias": float(kv["bias"][0]),
+        "lowrank_row": float(kv["lowrank_row"][0]), "lowrank_other": float(kv["lowrank_other"][0]),
     }
+
+
+def bf16_bits(values) -> np.ndarray:
+    """fp64 values that are bf16 numbers -> their uint16 bit patterns (raises otherwise)."""
+    v = np.asarray(values, np.float64)
+    bits = torch.from_numpy(v.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    back = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).double().numpy()
+    if not np.array_equal(back, v):
+        raise ValueError("not a bf16 number")
+    return bits
+
+
+def worked_variants(ex):
+    """Inputs of the worked example's variants as uint16 bf16 bits: the SiLU-and-mul input
+    [1, rows, 2k], the smooth-quantize input x/2 and its pre_quant_scale [k], and the
+    low-rank GEMM's d [rows, r], l1 [rows, r] and bias [rows]."""
+    rows, k, row = ex["rows"], ex["k"], ex["row"]
+    xv = np.zeros((rows, k))
+    xv[row] = ex["x_values"]
+    gu = np.zeros((1, rows, 2 * k))
+    gu[0, row, :k] = ex["silu_gate"]
+    gu[0, row, k:] = ex["x_values"] / ex["silu_gate"]
+    r = ex["lowrank_r"]
+    d = np.zeros((rows, r))
+    d[row, 0] = 1.0
+    l1 = np.zeros((rows, r))
+    l1[:, 0] = ex["lowrank_l1"]
+    return {
+        "silu_x": bf16_bits(gu), "smooth_x": bf16_bits(xv / ex["pre_quant_scale"]),
+        "pqs": bf16_bits(np.full(k, ex["pre_quant_scale"])), "d": bf16_bits(d), "l1": bf16_bits(l1),
+        "bias": bf16_bits(np.full(rows, ex["bias"])),
+    }
+
+
+def masked_expectations(ex, fill):
+    """q and sf of the masked variant: the worked bytes on rows below the mask, the
+    sentinel on the rest (row r's scales at (r%32)*16 + (r//32)*4 + c for 40 rows, k = 64)."""
+    q = np.full_like(ex["q"], fill)
+    q[:ex["mask"]] = ex["q"][:ex["mask"]]
+    sf = np.full_like(ex["sf"], fill)
+    for r in range(ex["mask"]):
+        for c in range(ex["k"] // 16):
+            sf[(r % 32) * 16 + (r // 32) * 4 + c] = ex["sf"][(r % 32) * 16 + (r // 32) * 4 + c]
+    return q, sf
+
+
+def lowrank_expectation(ex, exact=True):
+    rows, row = ex["rows"], ex["row"]
+    out = np.full((rows, rows), ex["lowrank_other"])
+    out[row, :] = ex["lowrank_row"]
+    out[row, row] = (ex["gemm_self"] + ex["lowrank_row"]) if exact else ex["gemm_self_bf16"]
+    return out

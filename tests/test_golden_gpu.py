@@ -3,14 +3,16 @@
 The fixture was derived by hand from the format definitions and the pages' formulas, so
 these tests hold the kernels to values no program produced: the fused global-scale
 quantizer, the dense quantizer with a given global scale (every packed byte and every
-scale byte, padding included) and the block-scaled FP4 GEMM (exact bf16 outputs, since
-the fixture's sums lie far from any bf16 rounding midpoint)."""
+scale byte, padding included), the block-scaled FP4 GEMM (exact bf16 outputs, since the
+fixture's sums lie far from any bf16 rounding midpoint), and the SiLU-and-mul, masked,
+smooth and low-rank variants on inputs that reduce to the same bytes."""
 import numpy as np
 import pytest
 import torch
 
 import nvfp4_block_scaled_16_b200 as nv
-from tests.helpers import assert_gemm_close, bf16_to_f64, dev_bf16, dev_f32, host, load_worked_example
+from tests.helpers import (assert_gemm_close, bf16_to_f64, dev_bf16, dev_f32, dev_i32, host, load_worked_example,
+                           lowrank_expectation, masked_expectations, worked_variants)
 
 pytestmark = pytest.mark.gpu
 
@@ -70,3 +72,37 @@ def test_gemm(ex):
     ref = np.zeros((rows, 8))
     ref[row, :] = ex["gemm_ones"]
     assert_gemm_close(out, ref, "worked example, ones operand")
+
+
+def test_silu_mul_variant(ex):
+    v = worked_variants(ex)
+    x = dev_bf16(v["silu_x"])
+    amax, gsf = nv.nvfp4_global_scale_batched(x, silu_mul=True)
+    assert host(amax)[0] == ex["amax"] and host(gsf)[0] == ex["gsf"]
+    q = torch.full((1, ex["rows"], ex["k"] // 2), 0xAA, dtype=torch.uint8, device="cuda")
+    sf = torch.full((1, ex["sf"].size), 0xAA, dtype=torch.uint8, device="cuda")
+    nv.nvfp4_silu_mul_quantize_batched(x, gsf, q_out=q, sf_out=sf)
+    assert np.array_equal(host(q)[0], ex["q"]) and np.array_equal(host(sf)[0], ex["sf"])
+
+
+def test_masked_variant(ex):
+    q = torch.full((1, ex["rows"], ex["k"] // 2), 0xAA, dtype=torch.uint8, device="cuda")
+    sf = torch.full((1, ex["sf"].size), 0xAA, dtype=torch.uint8, device="cuda")
+    nv.nvfp4_quantize_masked_batched(dev_bf16(ex["x"][None]), dev_f32(ex["gsf"]), mask=dev_i32([ex["mask"]]),
+                                     q_out=q, sf_out=sf)
+    q_want, sf_want = masked_expectations(ex, 0xAA)
+    assert np.array_equal(host(q)[0], q_want) and np.array_equal(host(sf)[0], sf_want)
+
+
+def test_smooth_variant(ex):
+    v = worked_variants(ex)
+    q, sf = nv.nvfp4_quantize_smooth(dev_bf16(v["smooth_x"]), dev_bf16(v["pqs"]), dev_f32(ex["gsf"]))
+    assert np.array_equal(host(q), ex["q"]) and np.array_equal(host(sf), ex["sf"])
+
+
+def test_lowrank_variant(ex):
+    v = worked_variants(ex)
+    qa, sfa = nv.nvfp4_quantize(dev_bf16(ex["x"]), dev_f32(ex["gsf"]))
+    out = nv.nvfp4_gemm_lowrank_bias(qa, qa, sfa, sfa, dev_f32(1.0), dev_bf16(v["d"]), dev_bf16(v["l1"]),
+                                     dev_bf16(v["bias"]))
+    assert np.array_equal(bf16_to_f64(out), lowrank_expectation(ex, exact=False))

@@ -3,13 +3,16 @@
 The fixture's values were derived with pencil and paper from the format definitions and
 the pages' formulas (its header gives the sources and each step), not by a program, so
 these tests pin the oracle's global scale, quantizer, scale layout, dequantization and
-GEMM reference to something other than the oracle.  The first test checks the fixture
-against itself (codes x scales = dequantized values, the padded scale size)."""
+GEMM reference to something other than the oracle, and its SiLU-and-mul, masked, smooth
+and low-rank variants to inputs built so that they reduce to the same bytes.  The first
+test checks the fixture against itself (codes x scales = dequantized values, the padded
+scale size, the sums)."""
 import numpy as np
 import pytest
 import torch
 
-from tests.helpers import E2M1, e4m3_values, load_worked_example
+from tests.helpers import (E2M1, e4m3_values, load_worked_example, lowrank_expectation, masked_expectations,
+                           worked_variants)
 
 
 @pytest.fixture(scope="module")
@@ -73,3 +76,32 @@ def test_oracle_gemm(oracle, ex):
     # alpha is 1/2688 rounded to fp32; every other factor is exact
     assert np.allclose(out[row], ex["gemm_ones"], rtol=2.0 ** -23, atol=0)
     assert not np.any(np.delete(out, row, axis=0))
+
+
+def test_oracle_silu_mul_variant(oracle, ex):
+    v = worked_variants(ex)
+    amax, gsf = oracle.global_scale_batched(v["silu_x"], None, silu_mul=True)
+    assert float(amax[0]) == ex["amax"] and float(gsf[0]) == ex["gsf"]
+    q, sf = oracle.silu_mul_quantize_batched(v["silu_x"], gsf, q_fill=0xAA, sf_fill=0xAA)
+    assert np.array_equal(q[0], ex["q"]) and np.array_equal(sf[0], ex["sf"])
+
+
+def test_oracle_masked_variant(oracle, ex):
+    q, sf = oracle.quantize_masked_batched(ex["x"][None], np.float32([ex["gsf"]]),
+                                           mask=np.int32([ex["mask"]]), q_fill=0xAA, sf_fill=0xAA)
+    q_want, sf_want = masked_expectations(ex, 0xAA)
+    assert np.array_equal(q[0], q_want) and np.array_equal(sf[0], sf_want)
+
+
+def test_oracle_smooth_variant(oracle, ex):
+    v = worked_variants(ex)
+    q, sf = oracle.quantize_smooth(v["smooth_x"], v["pqs"], ex["gsf"], sf_fill=0xAA)
+    assert np.array_equal(q, ex["q"]) and np.array_equal(sf, ex["sf"])
+
+
+def test_oracle_lowrank_variant(oracle, ex):
+    v = worked_variants(ex)
+    rows, k = ex["rows"], ex["k"]
+    q, sf = oracle.quantize(ex["x"], ex["gsf"])
+    out = oracle.gemm_ref(q, q, sf, sf, 1.0, rows, rows, k, d=v["d"], l1=v["l1"], bias=v["bias"])
+    assert np.array_equal(out, lowrank_expectation(ex))
