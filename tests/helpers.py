@@ -114,7 +114,9 @@ def load_worked_example():
     must write them; gemm_self, gemm_ones and their bf16 roundings gemm_self_bf16,
     gemm_ones_bf16; ones_amax, ones_gsf, ones_scale, ones_code of the all-ones operand;
     the variants' inputs silu_gate, mask, pre_quant_scale, lowrank_r, lowrank_l1, bias and
-    the low-rank GEMM's outputs lowrank_row (row 33 off the diagonal), lowrank_other."""
+    the low-rank GEMM's outputs lowrank_row (row 33 off the diagonal), lowrank_other; the
+    grouped GEMM's grouped_mask, grouped_alpha_mult (alpha[e] = mult/2688) and grouped_row;
+    and the fused gate/up SiLU-and-mul quantize case (swiglu_*)."""
     kv = {}
     with open(os.path.join(GOLDEN, "nvfp4_worked_example.txt")) as f:
         for line in f:
@@ -149,6 +151,15 @@ def load_worked_example():
         "pre_quant_scale": float(kv["pre_quant_scale"][0]), "lowrank_r": int(kv["lowrank_r"][0]),
         "lowrank_l1": float(kv["lowrank_l1"][0]), "bias": float(kv["bias"][0]),
         "lowrank_row": float(kv["lowrank_row"][0]), "lowrank_other": float(kv["lowrank_other"][0]),
+        "grouped_mask": [int(v) for v in kv["grouped_mask"]],
+        "grouped_alpha_mult": [float(v) for v in kv["grouped_alpha_mult"]],
+        "grouped_row": [float(v) for v in kv["grouped_row"]],
+        "swiglu_n": int(kv["swiglu_n"][0]), "swiglu_up_div": float(kv["swiglu_up_div"][0]),
+        "swiglu_g": float(kv["swiglu_g"][0]), "swiglu_u": float(kv["swiglu_u"][0]),
+        "swiglu_h": float(kv["swiglu_h"][0]), "swiglu_byte": int(kv["swiglu_byte"][0], 16),
+        "swiglu_scale": int(kv["swiglu_scale"][0], 16), "swiglu_sf_bytes": int(kv["swiglu_sf_bytes"][0]),
+        "swiglu_sf_offsets": np.array(kv["swiglu_sf_offsets"], np.int64),
+        "swiglu_grouped_mask": [int(v) for v in kv["swiglu_grouped_mask"]],
     }
 
 
@@ -202,3 +213,46 @@ def lowrank_expectation(ex, exact=True):
     out[row, :] = ex["lowrank_row"]
     out[row, row] = (ex["gemm_self"] + ex["lowrank_row"]) if exact else ex["gemm_self_bf16"]
     return out
+
+
+def grouped_expectation(ex, fill):
+    """out [2, rows, 8] of the grouped variant: 0 on rows below each expert's mask, the
+    expert's row value on row 33 when the mask covers it, `fill` on unwritten rows."""
+    rows, row = ex["rows"], ex["row"]
+    out = np.full((2, rows, 8), fill, np.float64)
+    for e, m in enumerate(ex["grouped_mask"]):
+        out[e, :m] = 0.0
+        if row < m:
+            out[e, row] = ex["grouped_row"][e]
+    return out
+
+
+def swiglu_expectation(ex):
+    """(q [rows, n/2], sf [swiglu_sf_bytes]) of the fused gate/up SiLU-and-mul quantize case."""
+    q = np.zeros((ex["rows"], ex["swiglu_n"] // 2), np.uint8)
+    q[ex["row"]] = ex["swiglu_byte"]
+    sf = np.zeros(ex["swiglu_sf_bytes"], np.uint8)
+    sf[ex["swiglu_sf_offsets"]] = ex["swiglu_scale"]
+    return q, sf
+
+
+def swiglu_grouped_expectation(ex, fill):
+    """The grouped form [2, ...]: the dense result on rows below each expert's mask, `fill`
+    on the rest and on their scale entries (row r, block c at
+    (c//4)*512 + (r%32)*16 + (r//32)*4 + c%4 for these 40 rows)."""
+    q1, sf1 = swiglu_expectation(ex)
+    q = np.full((2,) + q1.shape, fill, np.uint8)
+    sf = np.full((2, sf1.size), fill, np.uint8)
+    for e, m in enumerate(ex["swiglu_grouped_mask"]):
+        q[e, :m] = q1[:m]
+        for r in range(m):
+            for c in range(ex["swiglu_n"] // 16):
+                o = (c // 4) * 512 + (r % 32) * 16 + (r // 32) * 4 + c % 4
+                sf[e, o] = sf1[o]
+    return q, sf
+
+
+def ones_rows(n, k) -> np.ndarray:
+    """bf16 bits of an [n, k] tensor of ones."""
+    return np.full((n, k), 0x3F80, np.uint16)
+

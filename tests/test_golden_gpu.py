@@ -5,14 +5,16 @@ these tests hold the kernels to values no program produced: the fused global-sca
 quantizer, the dense quantizer with a given global scale (every packed byte and every
 scale byte, padding included), the block-scaled FP4 GEMM (exact bf16 outputs, since the
 fixture's sums lie far from any bf16 rounding midpoint), and the SiLU-and-mul, masked,
-smooth and low-rank variants on inputs that reduce to the same bytes."""
+smooth, low-rank, masked grouped and fused gate/up SiLU-and-mul variants on inputs whose
+results follow from the example by hand."""
 import numpy as np
 import pytest
 import torch
 
 import nvfp4_block_scaled_16_b200 as nv
-from tests.helpers import (assert_gemm_close, bf16_to_f64, dev_bf16, dev_f32, dev_i32, host, load_worked_example,
-                           lowrank_expectation, masked_expectations, worked_variants)
+from tests.helpers import (assert_gemm_close, bf16_to_f64, dev_bf16, dev_f32, dev_i32, grouped_expectation, host,
+                           load_worked_example, lowrank_expectation, masked_expectations, ones_rows,
+                           swiglu_expectation, swiglu_grouped_expectation, worked_variants)
 
 pytestmark = pytest.mark.gpu
 
@@ -60,7 +62,7 @@ def test_gemm(ex):
     want[row, row] = ex["gemm_self_bf16"]
     assert np.array_equal(bf16_to_f64(out), want)
 
-    ones = dev_bf16(np.full((8, k), 0x3F80, np.uint16))
+    ones = dev_bf16(ones_rows(8, k))
     amax_b, gsf_b, alpha, qb, sfb = nv.nvfp4_global_scale_quantize(ones, other_amax=dev_f32(ex["amax"]))
     assert host(amax_b)[0] == ex["ones_amax"] and host(gsf_b)[0] == ex["ones_gsf"]
     assert np.all(host(qb) == ex["ones_code"] * 0x11)
@@ -106,3 +108,43 @@ def test_lowrank_variant(ex):
     out = nv.nvfp4_gemm_lowrank_bias(qa, qa, sfa, sfa, dev_f32(1.0), dev_bf16(v["d"]), dev_bf16(v["l1"]),
                                      dev_bf16(v["bias"]))
     assert np.array_equal(bf16_to_f64(out), lowrank_expectation(ex, exact=False))
+
+
+def _ones_operand(ex, n):
+    _, _, alpha, qb, sfb = nv.nvfp4_global_scale_quantize(dev_bf16(ones_rows(n, ex["k"])),
+                                                          other_amax=dev_f32(ex["amax"]))
+    return qb, sfb, host(alpha)[0]
+
+
+def test_grouped_variant(ex):
+    rows = ex["rows"]
+    qa, sfa = nv.nvfp4_quantize(dev_bf16(ex["x"]), dev_f32(ex["gsf"]))
+    qb, sfb, _ = _ones_operand(ex, 8)
+    alphas = np.float32([m / 2688.0 for m in ex["grouped_alpha_mult"]])
+    out = torch.full((2, rows, 8), -1.0, dtype=torch.bfloat16, device="cuda")
+    nv.nvfp4_grouped_gemm_masked(torch.stack([qa, qa]), torch.stack([qb, qb]), torch.stack([sfa, sfa]),
+                                 torch.stack([sfb, sfb]), dev_i32(ex["grouped_mask"]), dev_f32(alphas), out=out)
+    assert np.array_equal(bf16_to_f64(out), grouped_expectation(ex, -1.0))
+
+
+def test_swiglu_variant(ex):
+    rows, n = ex["rows"], ex["swiglu_n"]
+    qa, sfa = nv.nvfp4_quantize(dev_bf16(ex["x"]), dev_f32(ex["gsf"]))
+    qb, sfb, alpha_g = _ones_operand(ex, n)
+    alpha_u = np.float32(alpha_g / np.float32(ex["swiglu_up_div"]))
+    gsf_h = np.float32(np.float32(2688.0) / np.float32(ex["swiglu_h"]))
+    q = torch.full((rows, n // 2), 0xAA, dtype=torch.uint8, device="cuda")
+    sf = torch.full((ex["swiglu_sf_bytes"],), 0xAA, dtype=torch.uint8, device="cuda")
+    nv.nvfp4_gemm_silu_mul_quantize(qa, qb, qb, sfa, sfb, sfb, dev_f32(alpha_g), dev_f32(alpha_u), dev_f32(gsf_h),
+                                    q_out=q, sf_out=sf)
+    q_want, sf_want = swiglu_expectation(ex)
+    assert np.array_equal(host(q), q_want) and np.array_equal(host(sf), sf_want)
+
+    two = lambda t: torch.stack([t, t])
+    q = torch.full((2, rows, n // 2), 0xAA, dtype=torch.uint8, device="cuda")
+    sf = torch.full((2, ex["swiglu_sf_bytes"]), 0xAA, dtype=torch.uint8, device="cuda")
+    nv.nvfp4_grouped_gemm_silu_mul_quantize_masked(two(qa), two(qb), two(qb), two(sfa), two(sfb), two(sfb),
+                                                   dev_i32(ex["swiglu_grouped_mask"]), dev_f32([alpha_g] * 2),
+                                                   dev_f32([alpha_u] * 2), dev_f32([gsf_h] * 2), q_out=q, sf_out=sf)
+    q_want, sf_want = swiglu_grouped_expectation(ex, 0xAA)
+    assert np.array_equal(host(q), q_want) and np.array_equal(host(sf), sf_want)

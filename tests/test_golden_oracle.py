@@ -3,15 +3,17 @@
 The fixture's values were derived with pencil and paper from the format definitions and
 the pages' formulas (its header gives the sources and each step), not by a program, so
 these tests pin the oracle's global scale, quantizer, scale layout, dequantization and
-GEMM reference to something other than the oracle, and its SiLU-and-mul, masked, smooth
-and low-rank variants to inputs built so that they reduce to the same bytes.  The first
+GEMM reference to something other than the oracle, and its SiLU-and-mul, masked, smooth,
+low-rank, masked grouped and fused gate/up SiLU-and-mul variants to inputs built so that
+their results follow from the example by hand.  The first
 test checks the fixture against itself (codes x scales = dequantized values, the padded
 scale size, the sums)."""
 import numpy as np
 import pytest
 import torch
 
-from tests.helpers import (E2M1, e4m3_values, load_worked_example, lowrank_expectation, masked_expectations,
+from tests.helpers import (E2M1, e4m3_values, grouped_expectation, load_worked_example, lowrank_expectation,
+                           masked_expectations, ones_rows, swiglu_expectation, swiglu_grouped_expectation,
                            worked_variants)
 
 
@@ -105,3 +107,55 @@ def test_oracle_lowrank_variant(oracle, ex):
     q, sf = oracle.quantize(ex["x"], ex["gsf"])
     out = oracle.gemm_ref(q, q, sf, sf, 1.0, rows, rows, k, d=v["d"], l1=v["l1"], bias=v["bias"])
     assert np.array_equal(out, lowrank_expectation(ex))
+
+
+def bf16_value(bits):
+    return torch.from_numpy(np.array([bits], np.uint16).view(np.int16)).view(torch.bfloat16).item()
+
+
+def _ones_operand(oracle, n, k):
+    amax, gsf = oracle.global_scale(ones_rows(n, k))
+    q, sf = oracle.quantize(ones_rows(n, k), gsf)
+    return q, sf, float(amax)
+
+
+def test_oracle_grouped_variant(oracle, ex):
+    rows, k = ex["rows"], ex["k"]
+    q, sf = oracle.quantize(ex["x"], ex["gsf"])
+    qb, sfb, _ = _ones_operand(oracle, 8, k)
+    alphas = np.float32([m / 2688.0 for m in ex["grouped_alpha_mult"]])
+    out = oracle.grouped_gemm_ref(np.stack([q, q]), np.stack([qb, qb]), np.stack([sf, sf]), np.stack([sfb, sfb]),
+                                  ex["grouped_mask"], alphas, 2, rows, 8, k)
+    want = grouped_expectation(ex, np.nan)
+    # the kernel writes bf16: round the fp64 reference once, as the oracle rounds it
+    bf = np.vectorize(lambda v: v if np.isnan(v) else bf16_value(oracle.f64_to_bf16(v)))(out)
+    assert np.array_equal(bf, want, equal_nan=True)
+
+
+def _swiglu_operands(oracle, ex):
+    q, sf = oracle.quantize(ex["x"], ex["gsf"])
+    qb, sfb, amax_b = _ones_operand(oracle, ex["swiglu_n"], ex["k"])
+    alpha_g = np.float32(oracle.alpha(ex["amax"], amax_b))
+    alpha_u = np.float32(alpha_g / np.float32(ex["swiglu_up_div"]))
+    gsf_h = np.float32(np.float32(2688.0) / np.float32(ex["swiglu_h"]))
+    return q, sf, qb, sfb, alpha_g, alpha_u, gsf_h
+
+
+def test_oracle_swiglu_variant(oracle, ex):
+    rows, k, n, row = ex["rows"], ex["k"], ex["swiglu_n"], ex["row"]
+    q, sf, qb, sfb, ag, au, gsf_h = _swiglu_operands(oracle, ex)
+    gu = oracle.gemm_gate_up_bf16(q, qb, qb, sf, sfb, sfb, ag, au, n, k, [row, 0])
+    vals = torch.from_numpy(gu.view(np.int16)).view(torch.bfloat16).double().numpy()
+    assert np.all(vals[0, :n] == ex["swiglu_g"]) and np.all(vals[0, n:] == ex["swiglu_u"])
+    assert not np.any(vals[1])
+    h = oracle.silu_mul(gu[:1])
+    assert np.all(torch.from_numpy(h.view(np.int16)).view(torch.bfloat16).double().numpy() == ex["swiglu_h"])
+    q_want, sf_want = swiglu_expectation(ex)
+    qh, sfh = oracle.gemm_silu_mul_quantize(q, qb, qb, sf, sfb, sfb, ag, au, gsf_h, rows, n, k, sf_fill=0xAA)
+    assert np.array_equal(qh, q_want) and np.array_equal(sfh, sf_want)
+    two = lambda t: np.stack([t, t])
+    qg, sfg = oracle.grouped_gemm_silu_mul_quantize(two(q), two(qb), two(qb), two(sf), two(sfb), two(sfb),
+                                                    ex["swiglu_grouped_mask"], [ag, ag], [au, au], [gsf_h, gsf_h],
+                                                    2, rows, n, k, q_fill=0xAA, sf_fill=0xAA)
+    q_want, sf_want = swiglu_grouped_expectation(ex, 0xAA)
+    assert np.array_equal(qg, q_want) and np.array_equal(sfg, sf_want)
