@@ -116,7 +116,8 @@ def load_worked_example():
     the variants' inputs silu_gate, mask, pre_quant_scale, lowrank_r, lowrank_l1, bias and
     the low-rank GEMM's outputs lowrank_row (row 33 off the diagonal), lowrank_other; the
     grouped GEMM's grouped_mask, grouped_alpha_mult (alpha[e] = mult/2688) and grouped_row;
-    and the fused gate/up SiLU-and-mul quantize case (swiglu_*)."""
+    the fused gate/up SiLU-and-mul quantize case (swiglu_*); the LoRA-down case's rank
+    lora_r and row 33's input sum row_sum with its bf16 rounding row_sum_bf16."""
     kv = {}
     with open(os.path.join(GOLDEN, "nvfp4_worked_example.txt")) as f:
         for line in f:
@@ -160,6 +161,8 @@ def load_worked_example():
         "swiglu_scale": int(kv["swiglu_scale"][0], 16), "swiglu_sf_bytes": int(kv["swiglu_sf_bytes"][0]),
         "swiglu_sf_offsets": np.array(kv["swiglu_sf_offsets"], np.int64),
         "swiglu_grouped_mask": [int(v) for v in kv["swiglu_grouped_mask"]],
+        "lora_r": int(kv["lora_r"][0]), "row_sum": float(kv["row_sum"][0]),
+        "row_sum_bf16": float(kv["row_sum_bf16"][0]),
     }
 
 
@@ -174,9 +177,10 @@ def bf16_bits(values) -> np.ndarray:
 
 
 def worked_variants(ex):
-    """Inputs of the worked example's variants as uint16 bf16 bits: the SiLU-and-mul input
-    [1, rows, 2k], the smooth-quantize input x/2 and its pre_quant_scale [k], and the
-    low-rank GEMM's d [rows, r], l1 [rows, r] and bias [rows]."""
+    """Inputs of the worked example's variants as uint16 bf16 bits: the LoRA-down weight
+    [lora_r, k] and its pre_quant_scale-scaled form, the SiLU-and-mul input [1, rows, 2k],
+    the smooth-quantize input x/2 and its pre_quant_scale [k], and the low-rank GEMM's
+    d [rows, r], l1 [rows, r] and bias [rows]."""
     rows, k, row = ex["rows"], ex["k"], ex["row"]
     xv = np.zeros((rows, k))
     xv[row] = ex["x_values"]
@@ -188,7 +192,11 @@ def worked_variants(ex):
     d[row, 0] = 1.0
     l1 = np.zeros((rows, r))
     l1[:, 0] = ex["lowrank_l1"]
+    w = np.zeros((ex["lora_r"], k))
+    w[0, :] = 1.0
+    w[1, 0] = 1.0
     return {
+        "lora_w": bf16_bits(w), "lora_w_scaled": bf16_bits(w * ex["pre_quant_scale"]),
         "silu_x": bf16_bits(gu), "smooth_x": bf16_bits(xv / ex["pre_quant_scale"]),
         "pqs": bf16_bits(np.full(k, ex["pre_quant_scale"])), "d": bf16_bits(d), "l1": bf16_bits(l1),
         "bias": bf16_bits(np.full(rows, ex["bias"])),
@@ -255,4 +263,12 @@ def swiglu_grouped_expectation(ex, fill):
 def ones_rows(n, k) -> np.ndarray:
     """bf16 bits of an [n, k] tensor of ones."""
     return np.full((n, k), 0x3F80, np.uint16)
+
+
+def lora_expectation(ex, value):
+    """d [rows, lora_r] of the LoRA-down case with `value` (exact or bf16) at (row, 0)."""
+    d = np.zeros((ex["rows"], ex["lora_r"]))
+    d[ex["row"], 0] = value
+    d[ex["row"], 1] = ex["x_values"][0]
+    return d
 

@@ -5,15 +5,15 @@ these tests hold the kernels to values no program produced: the fused global-sca
 quantizer, the dense quantizer with a given global scale (every packed byte and every
 scale byte, padding included), the block-scaled FP4 GEMM (exact bf16 outputs, since the
 fixture's sums lie far from any bf16 rounding midpoint), and the SiLU-and-mul, masked,
-smooth, low-rank, masked grouped and fused gate/up SiLU-and-mul variants on inputs whose
-results follow from the example by hand."""
+smooth, low-rank, masked grouped, fused gate/up SiLU-and-mul, LoRA-down, bf16-activation
+and SiLU-and-mul-only variants on inputs whose results follow from the example by hand."""
 import numpy as np
 import pytest
 import torch
 
 import nvfp4_block_scaled_16_b200 as nv
 from tests.helpers import (assert_gemm_close, bf16_to_f64, dev_bf16, dev_f32, dev_i32, grouped_expectation, host,
-                           load_worked_example, lowrank_expectation, masked_expectations, ones_rows,
+                           load_worked_example, lora_expectation, lowrank_expectation, masked_expectations, ones_rows,
                            swiglu_expectation, swiglu_grouped_expectation, worked_variants)
 
 pytestmark = pytest.mark.gpu
@@ -148,3 +148,30 @@ def test_swiglu_variant(ex):
                                                    dev_f32([alpha_u] * 2), dev_f32([gsf_h] * 2), q_out=q, sf_out=sf)
     q_want, sf_want = swiglu_grouped_expectation(ex, 0xAA)
     assert np.array_equal(host(q), q_want) and np.array_equal(host(sf), sf_want)
+
+
+def test_lora_down_variant(ex):
+    v = worked_variants(ex)
+    want = lora_expectation(ex, ex["row_sum_bf16"])
+    d = nv.nvfp4_lora_down(dev_bf16(ex["x"]), dev_bf16(v["lora_w"]))
+    assert np.array_equal(bf16_to_f64(d), want)
+    q, sf, d = nv.nvfp4_quantize_smooth_lora_down(dev_bf16(v["smooth_x"]), dev_bf16(v["pqs"]), dev_f32(ex["gsf"]),
+                                                  dev_bf16(v["lora_w_scaled"]))
+    assert np.array_equal(host(q), ex["q"]) and np.array_equal(host(sf), ex["sf"])
+    assert np.array_equal(bf16_to_f64(d), want)
+
+
+def test_bf16a_variant(ex):
+    qb, sfb, _ = _ones_operand(ex, 8)
+    out, a_q, a_sf, scalars = nv.nvfp4_gemm_bf16a(dev_bf16(ex["x"]), qb, sfb, dev_f32(ex["ones_amax"]))
+    assert list(host(scalars)) == [np.float32(ex["amax"]), np.float32(ex["gsf"]), np.float32(1.0 / 2688.0)]
+    assert np.array_equal(host(a_q), ex["q"]) and np.array_equal(host(a_sf), ex["sf"])
+    want = np.zeros((ex["rows"], 8))
+    want[ex["row"], :] = ex["gemm_ones_bf16"]
+    assert np.array_equal(bf16_to_f64(out), want)
+
+
+def test_silu_and_mul_variant(ex):
+    v = worked_variants(ex)
+    h = nv.nvfp4_silu_and_mul(dev_bf16(v["silu_x"][0]))
+    assert np.array_equal(host(h), ex["x"])

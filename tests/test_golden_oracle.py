@@ -4,7 +4,7 @@ The fixture's values were derived with pencil and paper from the format definiti
 the pages' formulas (its header gives the sources and each step), not by a program, so
 these tests pin the oracle's global scale, quantizer, scale layout, dequantization and
 GEMM reference to something other than the oracle, and its SiLU-and-mul, masked, smooth,
-low-rank, masked grouped and fused gate/up SiLU-and-mul variants to inputs built so that
+low-rank, masked grouped, fused gate/up SiLU-and-mul and LoRA-down variants to inputs built so that
 their results follow from the example by hand.  The first
 test checks the fixture against itself (codes x scales = dequantized values, the padded
 scale size, the sums)."""
@@ -12,8 +12,8 @@ import numpy as np
 import pytest
 import torch
 
-from tests.helpers import (E2M1, e4m3_values, grouped_expectation, load_worked_example, lowrank_expectation,
-                           masked_expectations, ones_rows, swiglu_expectation, swiglu_grouped_expectation,
+from tests.helpers import (E2M1, e4m3_values, grouped_expectation, load_worked_example, lora_expectation,
+                           lowrank_expectation, masked_expectations, ones_rows, swiglu_expectation, swiglu_grouped_expectation,
                            worked_variants)
 
 
@@ -159,3 +159,17 @@ def test_oracle_swiglu_variant(oracle, ex):
                                                     2, rows, n, k, q_fill=0xAA, sf_fill=0xAA)
     q_want, sf_want = swiglu_grouped_expectation(ex, 0xAA)
     assert np.array_equal(qg, q_want) and np.array_equal(sfg, sf_want)
+
+
+def test_oracle_lora_down_variant(oracle, ex):
+    v = worked_variants(ex)
+    d = oracle.lora_down(ex["x"], v["lora_w"])
+    assert np.array_equal(d, lora_expectation(ex, ex["row_sum"]))
+    assert bf16_value(oracle.f64_to_bf16(ex["row_sum"])) == ex["row_sum_bf16"]
+    # the unsmoothed x/2 against the scaled weight: the same products
+    assert np.array_equal(oracle.lora_down(v["smooth_x"], v["lora_w_scaled"]), d)
+
+
+def test_oracle_silu_and_mul_variant(oracle, ex):
+    v = worked_variants(ex)
+    assert np.array_equal(oracle.silu_mul(v["silu_x"][0]), ex["x"])
