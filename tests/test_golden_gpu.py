@@ -46,6 +46,17 @@ def test_global_scale_quantize(ex):
     assert np.array_equal(host(sf), ex["sf"])
 
 
+def test_global_scale(ex):
+    amax, gsf, alpha = nv.nvfp4_global_scale(dev_bf16(ex["x"]), other_amax=dev_f32(ex["ones_amax"]))
+    assert host(amax)[0] == ex["amax"] and host(gsf)[0] == ex["gsf"]
+    assert host(alpha)[0] == np.float32(1.0 / 2688.0)
+    # batched over two items with masks 34 and 33: the second item's valid rows end just
+    # before the worked row, so it sees only zeros and its amax is clamped to 1e-12
+    amax, gsf = nv.nvfp4_global_scale_batched(dev_bf16(np.stack([ex["x"], ex["x"]])), mask=dev_i32([34, 33]))
+    assert list(host(amax)) == [np.float32(ex["amax"]), np.float32(1e-12)]
+    assert list(host(gsf)) == [np.float32(ex["gsf"]), np.float32(2688.0) / np.float32(1e-12)]
+
+
 def test_quantize(ex):
     q = torch.full((ex["rows"], ex["k"] // 2), 0xAA, dtype=torch.uint8, device="cuda")
     sf = torch.full((ex["sf"].size,), 0xAA, dtype=torch.uint8, device="cuda")

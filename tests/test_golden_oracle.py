@@ -42,6 +42,11 @@ def test_oracle_global_scale(oracle, ex):
     ones = np.full((8, ex["k"]), 0x3F80, np.uint16)        # bf16 1.0
     amax_b, gsf_b = oracle.global_scale(ones)
     assert float(amax_b) == ex["ones_amax"] and float(gsf_b) == ex["ones_gsf"]
+    # two items with masks 34 and 33: the second sees only zero rows, amax clamps to 1e-12
+    # (the clamp the FastVideo review thread's global-scale helper applies)
+    amax2, gsf2 = oracle.global_scale_batched(np.stack([ex["x"], ex["x"]]), np.int32([34, 33]))
+    assert list(amax2) == [np.float32(ex["amax"]), np.float32(1e-12)]
+    assert list(gsf2) == [np.float32(ex["gsf"]), np.float32(2688.0) / np.float32(1e-12)]
     assert np.float32(oracle.alpha(ex["amax"], ex["amax"])) == np.float32(1.0)
     assert np.float32(oracle.alpha(ex["amax"], ex["ones_amax"])) == np.float32(1.0 / 2688.0)
 
