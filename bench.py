@@ -969,7 +969,7 @@ def run_reference(args, world, rank):
     wl = args.workload
     rows = 1 if wl in ("swiglu_block", "grouped_swiglu") else None
     o = OracleSample(wl, rows)
-    o.measure(min(args.warmup, 1))
+    o.measure(args.warmup)
     t0 = time.perf_counter()
     value, secs = o.measure(args.steps)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": o.unit, "n_gpus": args.gpus,

@@ -84,3 +84,30 @@ def test_reference_arm_config_is_computed_without_a_gpu():
         assert "l2" in cfg
     assert "sum 8088" in bench.workload_config("grouped_swiglu", 64)["workload"]
     assert "r=32" in bench.workload_config("lowrank", 32)["workload"]
+
+
+def test_reference_arm_prints_one_contract_line():
+    # the reference arm at N = 1 on the smallest workload: one JSON line with the contract's
+    # keys, the impl tag, and the cpu_baseline / e2e objects describing this run
+    import json
+    sys.path.insert(0, ROOT)
+    import bench
+
+    class Args:
+        workload, steps, warmup, gpus, rank_lr, swiglu_path = "pr1_linear", 2, 3, 1, 64, "fused"
+    out = io.StringIO()
+    with redirect_stdout(out):
+        bench.run_reference(Args, 1, 0)
+    lines = out.getvalue().strip().splitlines()
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["steps"] == 2 and line["warmup"] == 3
+    assert line["value"] > 0 and line["unit"] == "TFLOP/s" and line["higher_is_better"] is True
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["cpu_baseline"]["cores"] >= 1 and line["cpu_baseline"]["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+    assert line["config"] == bench.workload_config("pr1_linear", 64, "fused")
