@@ -28,10 +28,12 @@
  *    is alpha = amax_a * amax_b / (448*6)^2 [TRT alpha].  Both are fp32 DEVICE values,
  *    so every call is stream-ordered and capturable in a CUDA graph.
  *  - Every call launches on `stream` (a cudaStream_t; NULL is the legacy default
- *    stream), never synchronizes the host, and allocates nothing per call.  The first
- *    call on a device (and, for the global-scale reductions, the first on a stream)
- *    allocates a small library-owned workspace with cudaMalloc; make that first call
- *    before capturing the stream into a CUDA graph.
+ *    stream) and allocates nothing per call.  The first call on a device sets up the
+ *    library's per-device state: it allocates the status word and the 32 KB SiLU table
+ *    with cudaMalloc and fills the table with one kernel on the legacy default stream,
+ *    waiting for it (the only host synchronization outside nvfp4_device_status).  The
+ *    first global-scale reduction on a stream allocates that stream's small workspace.
+ *    Make both first calls before capturing a stream into a CUDA graph.
  *  - Arguments are validated before anything is launched: a call that returns an
  *    error has written nothing.
  *  - Return value: NVFP4_OK or one of the NVFP4_ERR_* codes below.
