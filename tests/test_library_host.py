@@ -189,3 +189,16 @@ def test_bf16a_argument_checks(lib):
         bad = list(args)
         bad[i] = A1
         assert lib.nvfp4_gemm_bf16a(*bad, 128, 256, 256, None) == INVALID, i
+
+
+def test_empty_gemms_are_noops(lib):
+    # m, n or E == 0 (with valid k): nothing to compute, no pointer read, no device needed
+    N7 = [None] * 7
+    assert lib.nvfp4_gemm(*N7, 0, 256, 256, None) == 0
+    assert lib.nvfp4_gemm(*N7, 128, 0, 256, None) == 0
+    assert lib.nvfp4_gemm_lowrank_bias(*N7, 32, None, None, 0, 256, 256, None) == 0
+    assert lib.nvfp4_grouped_gemm_masked(*N7, 0, 128, 256, 256, None) == 0
+    assert lib.nvfp4_grouped_gemm_masked(*N7, 4, 0, 256, 256, None) == 0
+    assert lib.nvfp4_gemm_silu_mul_quantize(*([None] * 11), 0, 256, 256, None) == 0
+    # an empty shape is still checked: k must be a positive multiple of 64
+    assert lib.nvfp4_gemm(*N7, 0, 256, 96, None) == INVALID
