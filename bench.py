@@ -805,6 +805,20 @@ def scale(v, unit):
 # CPU oracle timing (reference arm and cpu_baseline)
 # ---------------------------------------------------------------------------------------
 
+def host_cpu():
+    """The host's CPU model and logical CPU count, reported beside the oracle's timing."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu_model": model, "host_cpus": os.cpu_count()}
+
+
 class OracleSample:
     """The CPU oracle on a bounded sample of a workload: ``setup()`` prepares (and
     quantizes, offline) the weights once; each ``step()`` runs the sample's hot path and
@@ -977,7 +991,7 @@ def run_reference(args, world, rank):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (plain C oracle)",
             "data": "synthetic", "config": workload_config(wl, args.rank_lr, args.swiglu_path),
             "cpu_baseline": {"value": value, "unit": o.unit, "cores": o.threads, "kind": "oracle",
-                             "sample": o.sample + " per step"},
+                             "sample": o.sample + " per step", **host_cpu()},
             "e2e": {"value": value, "unit": o.unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "wall_s": round(time.perf_counter() - t0, 2)}
     print(json.dumps(line), flush=True)
@@ -1224,7 +1238,7 @@ def main():
         o = OracleSample(wl.name)
         v, secs = o.measure(1)
         cpu = {"value": v, "unit": wl.unit, "cores": o.threads, "kind": "oracle", "sample": o.sample,
-               "seconds": round(secs, 2)}
+               "seconds": round(secs, 2), **host_cpu()}
 
     if rank == 0:
         clk = clocks.summary()

@@ -108,6 +108,8 @@ def test_reference_arm_prints_one_contract_line():
     assert line["value"] > 0 and line["unit"] == "TFLOP/s" and line["higher_is_better"] is True
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
     assert line["cpu_baseline"]["cores"] >= 1 and line["cpu_baseline"]["sample"]
+    assert line["cpu_baseline"]["host_cpus"] >= line["cpu_baseline"]["cores"]
+    assert "cpu_model" in line["cpu_baseline"]
     assert line["e2e"] == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
     assert line["config"] == bench.workload_config("pr1_linear", 64, "fused")
