@@ -248,7 +248,8 @@ NVFP4_API int nvfp4_grouped_gemm_masked(const uint8_t *a, const uint8_t *b, cons
  * Low-rank-corrected GEMM (SVDQuant) [FI5 mm_nvfp4_svdquant]:
  *   out = bf16(alpha * (a @ b^T + d @ l1^T) [+ bias])
  * i.e. the FP4 K-loop and then a bf16 MMA of d @ l1^T into the same fp32 accumulator,
- * with the epilogue alpha * acc + bias; l1 is the LoRA-up weight pre-divided by alpha.
+ * with the epilogue alpha * acc + bias; l1 is the LoRA-up weight, already divided by alpha
+ * by the caller.
  *   d     bf16 [m, r] contiguous, 16-byte aligned (LoRA-down output).
  *   l1    bf16 [n, r] contiguous, 16-byte aligned.
  *   r     rank: a positive multiple of 32, at most 256.

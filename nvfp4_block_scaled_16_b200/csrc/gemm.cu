@@ -9,8 +9,8 @@
 //
 // Sources (page title, section): flashinfer docs mm_nvfp4_svdquant (signature,
 // Parameters: packed (m, k/2) and (n, k/2) operands, 128x4-swizzled ue4m3 scales,
-// alpha device scalar, rank-r bf16 correction issued as a second MMA into the same
-// accumulator after the FP4 K-loop, epilogue alpha*acc + bias); TensorRT-LLM
+// alpha device scalar; the rank-r bf16 correction is one more MMA that adds into the
+// FP4 K-loop's TMEM accumulator once that loop ends; epilogue alpha*acc + bias); TensorRT-LLM
 // NVFP4LinearMethod.create_weights (weight [out, in/2], alpha); flashinfer PR #1774
 // "Masked batch nvfp4 quantization" (masked per-expert operands for the grouped GEMM, and
 // the silu_and_mul quantizer whose input is the gate/up projection's output); the Llama4
