@@ -1052,8 +1052,8 @@ def main():
     # edges: it gives the step time (value).  The kernel graph has an event node around
     # every kernel (consecutive kernels then cannot overlap): it gives each kernel's own
     # duration (parts, roofline).  Both run inside the timed region, alternating step by step.  Should
-    # the driver refuse timing on graph event nodes, every kernel is captured into its own
-    # graph and timed by events recorded around its replay (no overlap either way).
+    # the CUDA driver refuse timing on graph event nodes, every kernel is captured into its
+    # own graph and timed by events recorded around its replay (no overlap either way).
     with torch.cuda.stream(stream):
         step()
     torch.cuda.synchronize()
