@@ -202,3 +202,15 @@ def test_empty_gemms_are_noops(lib):
     assert lib.nvfp4_gemm_silu_mul_quantize(*([None] * 11), 0, 256, 256, None) == 0
     # an empty shape is still checked: k must be a positive multiple of 64
     assert lib.nvfp4_gemm(*N7, 0, 256, 96, None) == INVALID
+
+
+def test_plain_c_client(lib, tmp_path):
+    # the C ABI from C99 alone: include/nvfp4.h, link libnvfp4.so, host-only calls
+    import subprocess
+    from nvfp4_block_scaled_16_b200 import build
+    exe = str(tmp_path / "c_abi_check")
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c_abi_check.c"), "-o", exe, "-L", build.PKG, "-lnvfp4",
+                    "-Wl,-rpath," + build.PKG], check=True)
+    run = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0 and run.stdout.strip() == "ok", run.stderr
