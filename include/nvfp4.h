@@ -26,7 +26,7 @@
  *  - The global scale is gsf = 448*6 / amax with amax = max|x| (NaN counted as 0,
  *    +-Inf as FLT_MAX, clamped below at 1e-12) [FV, TRT input_scale].  The GEMM factor
  *    is alpha = amax_a * amax_b / (448*6)^2 [TRT alpha].  Both are fp32 DEVICE values,
- *    so every call is stream-ordered and capturable in a CUDA graph.
+ *    so no call reads a scalar back to the host: calls are ordered by their stream alone.
  *  - Every call launches on `stream` (a cudaStream_t; NULL is the legacy default
  *    stream) and allocates nothing per call.  The first call on a device sets up the
  *    library's per-device state: it allocates the status word and the 32 KB SiLU table
@@ -104,19 +104,20 @@ NVFP4_API int nvfp4_global_scale_batched(const void *x_bf16, int64_t b, int64_t 
 
 /*
  * Non-allocating variant of nvfp4_global_scale_batched (same arguments, same results).
- * The pages have no counterpart of this entry point; it exists for callers that cannot
- * let the library call cudaMalloc: code being captured into a CUDA graph, hosts whose
- * device memory belongs to their own allocator or is fixed at start-up, and paths that
- * must not risk the implicit synchronization an allocation can cause.  Its reduction
- * scratch is a fixed device array inside the library (4100 bytes, held by every GPU that
- * loads the library until the process exits) instead of the per-stream workspace.
+ * The pages have no counterpart of this entry point.  It exists for callers that cannot
+ * let the library call cudaMalloc: hosts whose device memory belongs to their own
+ * allocator or is a fixed budget set at start-up (a pre-sized pool in an inference
+ * server, an embedded deployment), and latency-critical paths that must not risk the
+ * implicit device synchronization an allocation can cause.  Its reduction scratch is a
+ * fixed device array inside the library (4100 bytes, held by every GPU that loads the
+ * library until the process exits) instead of the per-stream workspace.
  *   b must be at most 1024; larger b returns NVFP4_ERR_INVALID_ARGUMENT before anything
  *   is launched.
  *   The first call on each device looks up the array's device address (no allocation);
- *   make that first call before capturing the stream into a CUDA graph.
- *   Every call clears and uses the same array: calls that overlap on the GPU (concurrent
- *   streams, or concurrently running graphs) race with each other and must be ordered by
- *   the caller.  Calls on one stream are ordered and safe.
+ *   make that first call before any stream capture.
+ *   Every call clears the words it uses and shares the same array: calls that overlap on
+ *   the GPU (concurrent streams) race with each other and must be ordered by the caller.
+ *   Calls on one stream are ordered and safe.
  * Calls no cudaMalloc, cudaFree or other allocating routine.
  */
 NVFP4_API int nvfp4_global_scale_batched_noalloc(const void *x_bf16, int64_t b, int64_t m, int64_t k,

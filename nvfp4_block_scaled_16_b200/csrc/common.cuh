@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstdint>
+#include <functional>
 #include <utility>
 
 #include "nvfp4.h"
@@ -32,6 +33,13 @@ int stream_workspace(cudaStream_t stream, uint32_t** out);
 
 // Maps the last CUDA error (launch configuration, ...) to a status code.
 int launch_status();
+
+// One-time launch set-up of `kernel` on `device` (the current device): the first call for
+// the pair runs `setup`, which may opt the kernel into dynamic shared memory and query its
+// occupancy (both are properties of the current device), and caches the value it stores;
+// later calls for the pair return the cached value.  Runs under the library lock, so
+// `setup` must not call current_device or stream_workspace.  Returns setup's status.
+int kernel_setup(const void* kernel, int device, const std::function<int(int*)>& setup, int* value);
 
 // Whether kernels are launched with programmatic dependent launch (nvfp4_set_pdl).
 bool pdl_enabled();

@@ -19,6 +19,7 @@ std::mutex g_mu;
 std::atomic<int> g_pdl{1};      // programmatic dependent launch, on by default (sm_100 supports it)
 DeviceInfo g_dev[64];
 std::map<std::pair<int, cudaStream_t>, uint32_t*> g_ws;
+std::map<std::pair<const void*, int>, int> g_kernel_cfg;   // (kernel, device) -> launch set-up value
 
 }  // namespace
 
@@ -95,6 +96,22 @@ int stream_workspace(cudaStream_t stream, uint32_t** out) {
   }
   g_ws[key] = ws;
   *out = ws;
+  return NVFP4_OK;
+}
+
+int kernel_setup(const void* kernel, int device, const std::function<int(int*)>& setup, int* value) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  const auto key = std::make_pair(kernel, device);
+  auto it = g_kernel_cfg.find(key);
+  if (it != g_kernel_cfg.end()) {
+    *value = it->second;
+    return NVFP4_OK;
+  }
+  int v = 0;
+  const int st = setup(&v);
+  if (st != NVFP4_OK) return st;
+  g_kernel_cfg[key] = v;
+  *value = v;
   return NVFP4_OK;
 }
 

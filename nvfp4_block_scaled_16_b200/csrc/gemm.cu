@@ -738,18 +738,18 @@ struct GemmArgs {
 };
 
 // Launches the kernel instantiation with kQW epilogue warps per lane quarter: the one-time
-// set-up per instantiation (dynamic shared memory opt-in, the number of 2-CTA clusters that
-// fit on the device at once: the persistent grid size), then a grid of min(tiles, clusters)
-// pairs.
+// set-up per instantiation and device (dynamic shared memory opt-in, the number of 2-CTA
+// clusters that fit on the device at once: the persistent grid size), then a grid of
+// min(tiles, clusters) pairs.
 template <bool kGrouped, bool kLowRank, bool kSwiGLU, int kQW>
 int run_gemm(const Maps& maps, const GemmParams& p, int64_t tiles, const DeviceInfo& info, cudaStream_t stream) {
   auto kernel = nvfp4_gemm_kernel<kGrouped, kLowRank, kSwiGLU, kQW>;
   constexpr int kSmem = kSmemBytes<kGrouped, kSwiGLU, kQW>;
-  static int max_clusters = 0;
-  if (max_clusters == 0) {
+  int max_clusters = 0;
+  const int st = kernel_setup(reinterpret_cast<const void*>(kernel), info.device, [&](int* clusters_out) {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess) {
       cudaGetLastError();
-      return NVFP4_ERR_CUDA;
+      return static_cast<int>(NVFP4_ERR_CUDA);
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(info.sm_count / 2 * 2);
@@ -760,8 +760,10 @@ int run_gemm(const Maps& maps, const GemmParams& p, int64_t tiles, const DeviceI
       cudaGetLastError();
       clusters = info.sm_count / 2;
     }
-    max_clusters = clusters;
-  }
+    *clusters_out = clusters;
+    return static_cast<int>(NVFP4_OK);
+  }, &max_clusters);
+  if (st != NVFP4_OK) return st;
   const int64_t max_pairs = max_clusters;
   const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
   return launch_kernel(kernel, dim3(2 * pairs), dim3(kThreads<kQW>), kSmem, stream, maps, p);

@@ -566,16 +566,18 @@ int launch_global_scale_quantize(const void* x_bf16, int64_t m, int64_t k, float
   uint32_t* ws = nullptr;
   st = stream_workspace(stream, &ws);
   if (st != NVFP4_OK) return st;
-  static int per_sm = 0;          // co-resident CTAs per SM, found once
-  if (per_sm == 0) {
+  int per_sm = 0;          // co-resident CTAs per SM, found once per device
+  st = kernel_setup(reinterpret_cast<const void*>(global_scale_quantize_kernel), info.device, [](int* out) {
     int n = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, global_scale_quantize_kernel, kThreads, 0) != cudaSuccess ||
         n <= 0) {
       cudaGetLastError();
-      return NVFP4_ERR_CUDA;
+      return static_cast<int>(NVFP4_ERR_CUDA);
     }
-    per_sm = n < kGsqCtasPerSm ? n : kGsqCtasPerSm;
-  }
+    *out = n < kGsqCtasPerSm ? n : kGsqCtasPerSm;
+    return static_cast<int>(NVFP4_OK);
+  }, &per_sm);
+  if (st != NVFP4_OK) return st;
   QuantParams p = {};
   p.x = static_cast<const uint16_t*>(x_bf16);
   p.x_row_stride = k;
@@ -699,12 +701,11 @@ int nvfp4_silu_mul_quantize_batched(const void* x_bf16, int64_t b, int64_t m, in
 
 // ---- non-allocating variant of the batched global scale ------------------------------------
 //
-// Some callers cannot let the library call cudaMalloc: code that is being captured into a
-// CUDA graph (allocation is not a capturable operation), hosts whose device memory is
-// owned by their own allocator or fixed at start-up (inference servers with a pre-sized
-// pool, embedded deployments), and latency-critical paths that must not risk the implicit
-// device synchronization cudaMalloc can cause.  nvfp4_global_scale_batched_noalloc serves
-// them: its reduction scratch is the file-scope device array below instead of the lazily
+// Some callers cannot let the library call cudaMalloc: hosts whose device memory is owned
+// by their own allocator or fixed at start-up (inference servers with a pre-sized pool,
+// embedded deployments), and latency-critical paths that must not risk the implicit device
+// synchronization cudaMalloc can cause.  nvfp4_global_scale_batched_noalloc serves them:
+// its reduction scratch is the file-scope device array below instead of the lazily
 // allocated per-stream workspace, so the call allocates nothing, ever.
 namespace nvfp4 {
 namespace {

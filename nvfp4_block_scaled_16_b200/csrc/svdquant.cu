@@ -437,14 +437,16 @@ int launch_svdquant(const void* x, int64_t m, int64_t k, const void* pqs, const 
   const int smem = svd_smem_bytes(static_cast<int>(r));
   constexpr int kOptIn = 227 * 1024 - 512;   // every ring size fits below this (static table: 512 B)
   static_assert(svd_smem_bytes(96) <= kOptIn && svd_smem_bytes(128) <= kOptIn, "ring larger than the opt-in");
-  static bool configured = false;
-  if (!configured) {
+  int configured = 0;      // the shared-memory opt-in is a per-device setting
+  const int st_cfg = kernel_setup(reinterpret_cast<const void*>(kernel), info.device, [&](int* out) {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kOptIn) != cudaSuccess) {
       cudaGetLastError();
-      return NVFP4_ERR_CUDA;
+      return static_cast<int>(NVFP4_ERR_CUDA);
     }
-    configured = true;
-  }
+    *out = 1;
+    return static_cast<int>(NVFP4_OK);
+  }, &configured);
+  if (st_cfg != NVFP4_OK) return st_cfg;
   if (smem > kOptIn) return NVFP4_ERR_INVALID_ARGUMENT;
   dim3 grid(kSvdSplit, static_cast<unsigned>((m + kSvdRows - 1) / kSvdRows));
   return launch_kernel(kernel, grid, dim3(kSvdThreads), static_cast<size_t>(smem), stream, maps, p);

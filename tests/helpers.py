@@ -82,28 +82,6 @@ def e4m3_values(codes: np.ndarray) -> np.ndarray:
     return torch.from_numpy(np.ascontiguousarray(codes, np.uint8)).view(torch.float8_e4m3fn).double().numpy()
 
 
-def assert_nvfp4_close(q, s, q_ref, s_ref, gsf, what="", max_frac=1e-2):
-    """NVFP4 outputs of the same h computed along two fp32 accumulation orders: codes and
-    scale codes may differ where h crossed a rounding boundary.  Requires at most
-    `max_frac` of scales and of codes to differ, and every dequantized value within
-    2 * max(scale) / gsf (two e2m1 steps of the larger block scale) plus 1% of the value.
-    q [rows, k/2] packed codes; s [rows, k/16] logical scale codes."""
-    c, cr = unpack_codes(q), unpack_codes(q_ref)
-    s, s_ref = np.asarray(s, np.uint8), np.asarray(s_ref, np.uint8)
-    scale_frac = float(np.mean(s != s_ref)) if s.size else 0.0
-    code_frac = float(np.mean(c != cr)) if c.size else 0.0
-    assert scale_frac <= max_frac, f"{what}: {scale_frac:.2e} of the block scales differ"
-    assert code_frac <= max_frac, f"{what}: {code_frac:.2e} of the codes differ"
-    sv = np.repeat(e4m3_values(s), 16, axis=-1)
-    svr = np.repeat(e4m3_values(s_ref), 16, axis=-1)
-    v = E2M1[c] * sv / float(gsf)
-    vr = E2M1[cr] * svr / float(gsf)
-    bound = 2.0 * np.maximum(sv, svr) / float(gsf) + 1e-2 * np.abs(vr)
-    bad = np.abs(v - vr) > bound
-    assert not bad.any(), f"{what}: {int(bad.sum())} values beyond two e2m1 steps; first {np.argwhere(bad)[:3].tolist()}"
-    return scale_frac, code_frac
-
-
 def load_worked_example():
     """The hand-worked example of tests/golden/nvfp4_worked_example.txt as arrays.
 
@@ -272,3 +250,147 @@ def lora_expectation(ex, value):
     d[ex["row"], 1] = ex["x_values"][0]
     return d
 
+
+
+# ---- full-size coverage and faithful bf16 rounding ------------------------------------------
+
+def tile_positions(m, n, tile_m, tile_n, seed, interior=2):
+    """Output positions (ii, jj) covering every tile_m x tile_n tile of an [m, n] output: the
+    tile's four corners (clipped to the output, so ragged edge tiles get their last row and
+    column) and `interior` seeded random points inside it."""
+    g = np.random.default_rng([int(seed), 977])
+    ii, jj = [], []
+    for r0 in range(0, m, tile_m):
+        r1 = min(m, r0 + tile_m) - 1
+        for c0 in range(0, n, tile_n):
+            c1 = min(n, c0 + tile_n) - 1
+            ii += [r0, r0, r1, r1]
+            jj += [c0, c1, c0, c1]
+            ii += list(g.integers(r0, r1 + 1, interior))
+            jj += list(g.integers(c0, c1 + 1, interior))
+    return np.array(ii, np.int64), np.array(jj, np.int64)
+
+
+def bf16_value(bits) -> np.ndarray:
+    u = np.asarray(bits, np.uint16).astype(np.uint32) << np.uint32(16)
+    return u.view(np.float32).astype(np.float64)
+
+
+def _bf16_order(bits) -> np.ndarray:
+    """Monotone integer key of bf16 bit patterns (adjacent finite values differ by 1; +0 and
+    -0 share the key 0)."""
+    b = np.asarray(bits, np.uint16).astype(np.int64)
+    mag = b & 0x7FFF
+    return np.where(b & 0x8000, -mag, mag)
+
+
+def fp32_accumulation_bound(k, alpha, sum_abs):
+    """Bound on |alpha * (fp32 sum of k products) - alpha * (exact sum)| for the tensor cores'
+    accumulation: one fp32 rounding (relative 2^-24) per 64-wide MMA K-step of the running sum,
+    whose magnitude never exceeds the sum of |products|, plus the alpha product, times a
+    safety factor of 4."""
+    return 4.0 * (k / 64.0 + 2.0) * 2.0 ** -24 * abs(float(alpha)) * np.asarray(sum_abs, np.float64)
+
+
+def assert_bf16_faithful(got_bits, ref_bits, exact, bound, what=""):
+    """bf16 results of a GEMM whose exact value is known: each must be `ref_bits` (the exact
+    value rounded to nearest, ties to even) or, where the exact value lies within `bound` of
+    the midpoint between `ref_bits` and an adjacent bf16 value, that adjacent value (the fp32
+    accumulation landed on the other side of the tie).  Returns (number of such differences,
+    largest |exact - midpoint| / bound among them)."""
+    got_bits = np.asarray(got_bits, np.uint16).reshape(-1)
+    ref_bits = np.asarray(ref_bits, np.uint16).reshape(-1)
+    exact = np.asarray(exact, np.float64).reshape(-1)
+    bound = np.broadcast_to(np.asarray(bound, np.float64), exact.shape)
+    vg, vr = bf16_value(got_bits), bf16_value(ref_bits)
+    diff = vg != vr
+    if not diff.any():
+        return 0, 0.0
+    adjacent = np.abs(_bf16_order(got_bits) - _bf16_order(ref_bits)) == 1
+    mid = 0.5 * (vg + vr)
+    ratio = np.abs(exact - mid) / np.maximum(bound, 1e-300)
+    bad = diff & ~(adjacent & (ratio <= 1.0))
+    if bad.any():
+        i = int(np.argwhere(bad)[0][0])
+        raise AssertionError(f"{what}: {int(bad.sum())} of {exact.size} bf16 results are not a faithful rounding; "
+                             f"first at {i}: got {vg[i]!r} ref {vr[i]!r} exact {exact[i]!r} bound {bound[i]!r}")
+    return int(diff.sum()), float(ratio[diff].max())
+
+
+def abs_codes(q) -> np.ndarray:
+    """Packed e2m1 bytes with both sign bits cleared: the GEMM of these operands (scales are
+    unsigned) is the sum of |products|."""
+    return (np.asarray(q, np.uint8) & np.uint8(0x77)).astype(np.uint8)
+
+
+def check_full_size(oracle, out, qa, sfa, qb, sfb, alpha, k, ii, jj, what, d=None, l1=None, bias=None):
+    """out (bf16 bits) at (ii, jj) against the oracle: the tolerance, and faithful rounding of
+    the exact value (the bias, when given, is added exactly by the epilogue's fma)."""
+    ref = oracle.gemm_ref_sampled(qa, qb, sfa, sfb, alpha, k, ii, jj, d=d, l1=l1, bias=bias)
+    got_bits = out[ii, jj]
+    assert_gemm_close(bf16_value(got_bits), ref, what)
+    r = 0 if d is None else d.shape[-1]
+    sum_abs = oracle.gemm_ref_sampled(abs_codes(qa), abs_codes(qb), sfa, sfb, alpha, k, ii, jj,
+                                      d=None if d is None else d & np.uint16(0x7FFF),
+                                      l1=None if l1 is None else l1 & np.uint16(0x7FFF))
+    bound = fp32_accumulation_bound(k + 4 * r, 1.0, sum_abs) + (2.0 ** -24 * np.abs(ref) if bias is not None else 0.0)
+    stats = assert_bf16_faithful(got_bits, f64_to_bf16_bits(oracle, ref), ref, bound, what)
+    print(f"{what}: {len(ii)} outputs, {stats[0]} at the other side of a near tie (worst |exact-tie|/bound "
+          f"{stats[1]:.3f})")
+
+
+# ---- the SiLU * up epilogue against the oracle ---------------------------------------------
+
+def f64_to_bf16_bits(oracle, v):
+    return np.array([oracle.f64_to_bf16(float(x)) for x in np.asarray(v).reshape(-1)], np.uint16)
+
+
+def check_projections_faithful(oracle, ops, gu_lib, ii, jj, n, k, what):
+    """g and u of the library at output positions (ii, jj): faithful roundings of the exact
+    fp64 projections (nearest, or the other side of a tie within the accumulation bound)."""
+    qa, qg, qu, sa, sg, su, al_g, al_u = ops[:8]
+    stats = []
+    for half, (qb, sb, al) in enumerate(((qg, sg, al_g), (qu, su, al_u))):
+        exact = oracle.gemm_ref_sampled(qa, qb, sa, sb, al, k, ii, jj)
+        sum_abs = oracle.gemm_ref_sampled(abs_codes(qa), abs_codes(qb), sa, sb, al, k, ii, jj)
+        got = gu_lib[ii, half * n + jj]
+        stats.append(assert_bf16_faithful(got, f64_to_bf16_bits(oracle, exact), exact,
+                                          fp32_accumulation_bound(k, 1.0, sum_abs), f"{what} {'gu'[half]}"))
+    print(f"{what}: projections differing from round-to-nearest (count, worst |exact-tie|/bound): {stats}")
+    return stats
+
+
+def check_explained_vs_composition(oracle, ops, gsf, q_rows, s_rows, gu_rows, rows, n, k, what, gu_ref=None):
+    """The fused output at `rows` (q_rows [len, n/2], logical scales s_rows [len, n/16]) against the
+    oracle's fp64 composition: every 16-value block that differs must hold a g or u value that
+    differs from the exact projection rounded to nearest, and every such value must be a
+    faithful rounding of the exact value.  `gu_ref`, when given, is the oracle's [g | u] at `rows`
+    (oracle.gemm_gate_up_bf16), which is then not recomputed."""
+    if gu_ref is None:
+        gu_ref = oracle.gemm_gate_up_bf16(*ops[:8], n, k, rows)
+    q_ref = np.zeros((len(rows), n // 2), np.uint8)
+    s_ref = np.zeros((len(rows), n // 16), np.uint8)
+    for i in range(len(rows)):
+        qi, sfi = oracle.silu_mul_quantize_batched(gu_ref[i][None, None], np.float32([gsf]))
+        q_ref[i] = qi[0, 0]
+        s_ref[i] = sf_logical(sfi[0], 1, n)[0]
+    diff = gu_rows != gu_ref
+    ri, ci = np.nonzero(diff)
+    qa, qg, qu, sa, sg, su, al_g, al_u = ops[:8]
+    for half, (qb, sb, al) in enumerate(((qg, sg, al_g), (qu, su, al_u))):
+        sel = (ci >= n) if half else (ci < n)
+        if not sel.any():
+            continue
+        ii, jj = np.asarray(rows)[ri[sel]], ci[sel] - half * n
+        exact = oracle.gemm_ref_sampled(qa, qb, sa, sb, al, k, ii, jj)
+        sum_abs = oracle.gemm_ref_sampled(abs_codes(qa), abs_codes(qb), sa, sb, al, k, ii, jj)
+        assert_bf16_faithful(gu_rows[ri[sel], ci[sel]], gu_ref[ri[sel], ci[sel]], exact,
+                             fp32_accumulation_bound(k, 1.0, sum_abs), f"{what} {'gu'[half]}")
+    nb = n // 16
+    blk = (unpack_codes(q_rows) != unpack_codes(q_ref)).reshape(len(rows), nb, 16).any(-1) | (s_rows != s_ref)
+    explained = diff[:, :n].reshape(len(rows), nb, 16).any(-1) | diff[:, n:].reshape(len(rows), nb, 16).any(-1)
+    unexplained = blk & ~explained
+    assert not unexplained.any(), f"{what}: blocks differ from the fp64 composition with every g and u exact: " \
+                                  f"{np.argwhere(unexplained)[:5].tolist()}"
+    print(f"{what}: {int(diff.sum())} of {diff.size} projections and {int(blk.sum())} of {blk.size} blocks differ "
+          f"from the fp64 composition, all at near-tie roundings")

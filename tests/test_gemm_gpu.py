@@ -4,14 +4,19 @@ on the dequantized operands, within |out - ref| <= 1e-2*|ref| + 1e-3*max|ref|.
 Operands are quantized by the oracle, so these tests pin the GEMM alone: the packing
 (low nibble = lower K index), the 128x4 scale layout read straight into tensor memory,
 the accumulator layout and the epilogue.  Sizes span several 128 x 256 tiles with ragged
-M, N and K tails; the full-size cases check sampled outputs."""
+M, N and K tails.  The full-size cases check the four corners and two interior points of
+every 256 x 256 output tile (every expert tile of the grouped GEMM): within the tolerance,
+and, more strictly, each bf16 output is a faithful rounding of the exact value (nearest, or
+the other neighbour where the exact value lies within the fp32 accumulation bound of a
+tie)."""
 import numpy as np
 import pytest
 import torch
 
 import nvfp4_block_scaled_16_b200 as nv
 import nvfp4_synth as S
-from tests.helpers import (assert_gemm_close, bf16_to_f64, dev_bf16, dev_f32, dev_i32, dev_u8, host)
+from tests.helpers import (assert_gemm_close, bf16_to_f64, check_full_size, dev_bf16, dev_f32, dev_i32, dev_u8, host,
+                           tile_positions)
 
 pytestmark = pytest.mark.gpu
 
@@ -160,27 +165,29 @@ def test_grouped_masked(oracle, E, mmax, n, k, mask):
         assert (o[e, v:] == -3.0).all(), f"expert {e}: rows beyond the mask were written"
 
 
-# ---- full sizes, sampled outputs ------------------------------------------------------------
+# ---- full sizes, every output tile ------------------------------------------------------------
 
-def sample_positions(m, n, count, seed):
-    g = S.rng(seed, S.TID["sample"])
-    ii = g.integers(0, m, count)
-    jj = g.integers(0, n, count)
-    # always include the corners of the ragged edges
-    ii[:4] = [0, m - 1, 0, m - 1]
-    jj[:4] = [0, n - 1, n - 1, 0]
-    return ii, jj
-
-
-def test_swiglu_gate_up_full_size_sampled(oracle):
+def test_swiglu_gate_up_full_size_every_tile(oracle):
     # [8192 x 5120] @ [16384 x 5120]^T, the large dense GEMM of the SwiGLU block
     m, n, k = 8192, 16384, 5120
     qa, sfa, qb, sfb, alpha = operands(oracle, m, n, k, seed=0)
     out = host(run_gemm(qa, sfa, qb, sfb, alpha))
-    ii, jj = sample_positions(m, n, 2048, 1)
-    ref = oracle.gemm_ref_sampled(qa, qb, sfa, sfb, alpha, k, ii, jj)
-    got = S.bf16_bits_to_f32(out[ii, jj]).astype(np.float64)
-    assert_gemm_close(got, ref, "gate/up 8192x16384x5120 (sampled)")
+    ii, jj = tile_positions(m, n, 256, 256, seed=1)
+    check_full_size(oracle, out, qa, sfa, qb, sfb, alpha, k, ii, jj, "gate/up 8192x16384x5120 (every tile)")
+
+
+def test_swiglu_down_full_size_every_tile(oracle):
+    # the down projection at its configuration size: [8192 x 8192] @ [5120 x 8192]^T (K = 8192,
+    # one epilogue warp per lane quarter with two staging tiles)
+    m, n, k = 8192, 5120, 8192
+    xa = S.normal_bf16((m, k), 1.0, 0, S.TID["x"])
+    xb = S.swiglu_block()["w_down"]
+    qa, sfa, amax_a = quantized(oracle, xa)
+    qb, sfb, amax_b = quantized(oracle, xb)
+    alpha = np.float32(oracle.alpha(float(amax_a), float(amax_b)))
+    out = host(run_gemm(qa, sfa, qb, sfb, alpha))
+    ii, jj = tile_positions(m, n, 256, 256, seed=2)
+    check_full_size(oracle, out, qa, sfa, qb, sfb, alpha, k, ii, jj, "down 8192x5120x8192 (every tile)")
 
 
 @pytest.mark.parametrize("r", [32, 64, 128])
@@ -193,9 +200,9 @@ def test_lowrank_full_size(oracle, r):
     l1 = S.f32_to_bf16_bits(d["l1_f32"] / alpha)
     out = host(nv.nvfp4_gemm_lowrank_bias(dev_u8(qa), dev_u8(qb), dev_u8(sfa), dev_u8(sfb), dev_f32(alpha),
                                           dev_bf16(d["d"]), dev_bf16(l1), dev_bf16(d["bias"])))
-    ii, jj = sample_positions(m, n, 4096, r)
-    ref = oracle.gemm_ref_sampled(qa, qb, sfa, sfb, alpha, k, ii, jj, d=d["d"], l1=l1, bias=d["bias"])
-    assert_gemm_close(S.bf16_bits_to_f32(out[ii, jj]).astype(np.float64), ref, f"lowrank full r={r}")
+    ii, jj = tile_positions(m, n, 256, 256, seed=r)
+    check_full_size(oracle, out, qa, sfa, qb, sfb, alpha, k, ii, jj, f"lowrank full r={r} (every tile)", d=d["d"],
+                    l1=l1, bias=d["bias"])
 
 
 @pytest.mark.parametrize("m,n,k,r", [(4096, 2560, 4096, 64), (2048, 4864, 6144, 0)])
@@ -207,7 +214,7 @@ def test_long_k_gemms_take_the_one_warp_epilogue(oracle, m, n, k, r):
     qa, sfa, amax_a = quantized(oracle, xa)
     qb, sfb, amax_b = quantized(oracle, xb)
     alpha = np.float32(oracle.alpha(float(amax_a), float(amax_b)))
-    ii, jj = sample_positions(m, n, 4096, r + 1)
+    ii, jj = tile_positions(m, n, 256, 256, seed=r + 1)
     if r:
         dd = S.normal_bf16((m, r), 1.0, 47, S.TID["d"])
         l1 = S.f32_to_bf16_bits(S.rng(47, S.TID["l1"]).standard_normal((n, r), dtype=np.float32) * np.float32(0.01)
@@ -215,14 +222,14 @@ def test_long_k_gemms_take_the_one_warp_epilogue(oracle, m, n, k, r):
         bias = S.normal_bf16((n,), 0.1, 47, S.TID["bias"])
         out = host(nv.nvfp4_gemm_lowrank_bias(dev_u8(qa), dev_u8(qb), dev_u8(sfa), dev_u8(sfb), dev_f32(alpha),
                                               dev_bf16(dd), dev_bf16(l1), dev_bf16(bias)))
-        ref = oracle.gemm_ref_sampled(qa, qb, sfa, sfb, alpha, k, ii, jj, d=dd, l1=l1, bias=bias)
+        check_full_size(oracle, out, qa, sfa, qb, sfb, alpha, k, ii, jj, f"{m}x{n}x{k} r={r}", d=dd, l1=l1,
+                        bias=bias)
     else:
         out = host(nv.nvfp4_gemm(dev_u8(qa), dev_u8(qb), dev_u8(sfa), dev_u8(sfb), dev_f32(alpha)))
-        ref = oracle.gemm_ref_sampled(qa, qb, sfa, sfb, alpha, k, ii, jj)
-    assert_gemm_close(S.bf16_bits_to_f32(out[ii, jj]).astype(np.float64), ref, f"{m}x{n}x{k} r={r}")
+        check_full_size(oracle, out, qa, sfa, qb, sfb, alpha, k, ii, jj, f"{m}x{n}x{k}")
 
 
-def test_grouped_full_size_sampled(oracle):
+def test_grouped_full_size_every_expert_tile(oracle):
     d = S.grouped_moe()
     E, mmax, k, n = 16, 2048, 5120, 8192
     mask = d["mask"]
@@ -238,9 +245,9 @@ def test_grouped_full_size_sampled(oracle):
     for e in range(E):
         v = int(mask[e])
         if v:
-            ii, jj = sample_positions(v, n, 256, e)
-            ref = oracle.gemm_ref_sampled(qa[e], qw[e], sfa[e], sfw[e], alphas[e], k, ii, jj)
-            assert_gemm_close(S.bf16_bits_to_f32(o[e, ii, jj]).astype(np.float64), ref, f"expert {e}")
+            ii, jj = tile_positions(v, n, 256, 256, seed=e)
+            check_full_size(oracle, o[e], qa[e], sfa[e], qw[e], sfw[e], alphas[e], k, ii, jj,
+                            f"expert {e} ({v} rows, every tile)")
         if v < mmax:
             tail = o[e, v:]
             assert (tail == S.f32_to_bf16_bits(np.float32([-3.0]))[0]).all()

@@ -8,7 +8,7 @@ import torch
 
 import nvfp4_block_scaled_16_b200 as nv
 import nvfp4_synth as S
-from tests.helpers import dev_bf16, dev_f32, dev_i32, dev_u8, first_diff, host
+from tests.helpers import bf16_value, dev_bf16, dev_f32, dev_i32, dev_u8, first_diff, host
 
 pytestmark = pytest.mark.gpu
 
@@ -104,6 +104,45 @@ def test_quantize_signed_zeros_and_tiny_values(oracle):
 def test_quantize_constant_and_zero_tensors(oracle):
     check_dense(oracle, np.full((128, 64), S.f32_to_bf16_bits(np.float32([-2.5]))[0], np.uint16))
     check_dense(oracle, np.zeros((5, 32), np.uint16), gsf=np.float32(2688.0 / 1e-12))
+
+
+def every_bf16_block_maximum():
+    """One 16-value block per non-negative finite bf16 value v (0x0000..0x7F7F): v at a seeded
+    position, the other 15 values seeded fractions of +-v rounded to bf16 (never above v), so
+    v is the block maximum; returns (blocks [n, 16] bf16 bits, v)."""
+    v_bits = np.arange(0, 0x7F80, dtype=np.uint16)
+    v = bf16_value(v_bits)
+    g = np.random.default_rng([5, 16])
+    frac = g.uniform(-1.0, 1.0, (v.size, 15))
+    others = S.f32_to_bf16_bits((frac * v[:, None]).astype(np.float32))
+    x = np.concatenate([v_bits[:, None], others], axis=1)
+    perm = np.argsort(g.random((v.size, 16)), axis=1)
+    return np.take_along_axis(x, perm, axis=1), v
+
+
+def test_quantize_every_bf16_block_maximum(oracle):
+    # The block scale is (vmax / 6) * gsf; the kernels form vmax / 6 as a product with fp32(1/6)
+    # and one correction step, which must equal the IEEE quotient for every bf16 vmax.  Every
+    # non-negative finite bf16 value is a block maximum here, each block with its own global
+    # scale, a power of two that puts (vmax / 6) * gsf in the e4m3 range (so the product is
+    # exact and the scale byte shows the quotient's rounding, ties included), and once more
+    # with gsf = 1 through the dense quantizer.
+    x, v = every_bf16_block_maximum()
+    n = v.size
+    j = np.where(v > 0, np.clip(np.round(np.log2(288.0 / np.maximum(v, 1e-300))), -126, 100), 0)
+    gsf = (2.0 ** j).astype(np.float32)
+    xb = np.ascontiguousarray(x.reshape(n, 1, 16))
+    for mask in (None, np.ones(n, np.int32)):       # grid over items, and the persistent masked quantizer
+        q = torch.full((n, 1, 8), 0xAB, dtype=torch.uint8, device="cuda")
+        sf = torch.full((n, nv.nvfp4_scale_bytes(1, 16)), 0xCD, dtype=torch.uint8, device="cuda")
+        nv.nvfp4_quantize_masked_batched(dev_bf16(xb), dev_f32(gsf), None if mask is None else dev_i32(mask), q, sf)
+        q_ref, sf_ref = oracle.quantize_masked_batched(xb, gsf, mask, q_fill=0xAB, sf_fill=0xCD)
+        assert first_diff(host(q), q_ref) is None, first_diff(host(q), q_ref)
+        assert first_diff(host(sf), sf_ref) is None, first_diff(host(sf), sf_ref)
+    one = np.float32([1.0])
+    q, sf = nv.nvfp4_quantize(dev_bf16(x), dev_f32(one))
+    q_ref, sf_ref = oracle.quantize(x, one[0])
+    assert first_diff(host(q), q_ref) is None and first_diff(host(sf), sf_ref) is None
 
 
 def test_quantize_full_size_with_outliers(oracle):

@@ -1,25 +1,32 @@
 """GPU parity of the gate/up GEMM whose epilogue emits SiLU(g) * u as NVFP4
 (nvfp4_gemm_silu_mul_quantize and its masked grouped form).
 
-Three comparisons:
+Comparisons:
   * unit scales and integer-friendly codes with power-of-two alphas, where the fp32
     accumulation is exact, so g, u, h and the quantized output must equal the oracle's
     composition bit for bit (codes of valid rows and the whole scale buffer);
-  * random operands: bit-exact against the unfused GPU sequence (bf16 GEMMs, then the
-    SiLU-and-mul quantizer) -- the fusion changes no rounding -- and close to the oracle's
-    composition (at most 1% of scales and codes differ, every value within two e2m1
-    steps), because the oracle's projections are exact fp64 rounded once to bf16 while
-    the tensor cores accumulate in fp32;
+  * random operands, complete and bit-exact: the library's own bf16 projections g and u
+    (nvfp4_gemm) are fed to the oracle's SiLU-and-mul quantizer with the same gsf_h, and
+    the fused kernel's codes and scales must equal the oracle's bit for bit (every row,
+    the padding rows' zero scales included); the fused kernel also equals the unfused GPU
+    sequence bit for bit;
+  * the library's g and u against the exact fp64 projections: each is the exact value
+    rounded to nearest, or, where the exact value lies within the fp32 accumulation bound
+    of a bf16 tie, the neighbour on the other side (a faithful rounding);
+  * against the oracle's fp64 composition (projections rounded once): a 16-value block of
+    the output may differ only where one of its g or u values is such a near-tie rounding;
   * masked grouped: rows at or beyond mask[e] (codes and scale entries) stay untouched.
-Sizes span several 256 x 128 output tiles with ragged M; the full-size case checks
-sampled rows of the 8192 x 8192 (hidden 5120) SwiGLU block."""
+Sizes span several 256 x 128 output tiles with ragged M; the full-size case checks every
+row of the 8192 x 8192 (hidden 5120) SwiGLU block bit for bit, the projections at points
+of every output tile, and eight whole rows against the fp64 composition."""
 import numpy as np
 import pytest
 import torch
 
 import nvfp4_block_scaled_16_b200 as nv
 import nvfp4_synth as S
-from tests.helpers import assert_nvfp4_close, dev_f32, dev_i32, dev_u8, host, sf_logical
+from tests.helpers import (check_explained_vs_composition, check_projections_faithful, dev_f32, dev_i32, dev_u8, host,
+                           sf_logical, tile_positions)
 
 pytestmark = pytest.mark.gpu
 
@@ -103,19 +110,33 @@ def test_unit_scales_bit_exact_vs_oracle(oracle, m, n, k):
     assert (sf == sf_ref).all(), np.argwhere(sf != sf_ref)[:5]     # including zeroed padding rows
 
 
+def library_gate_up(ops):
+    """[g | u] bf16 [m, 2n] from the library's plain GEMM (bf16(alpha * acc), the rounding the
+    fused epilogue applies before SiLU), on the device."""
+    qa, qg, qu, sa, sg, su, al_g, al_u = ops[:8]
+    g = nv.nvfp4_gemm(dev_u8(qa), dev_u8(qg), dev_u8(sa), dev_u8(sg), dev_f32(al_g))
+    u = nv.nvfp4_gemm(dev_u8(qa), dev_u8(qu), dev_u8(sa), dev_u8(su), dev_f32(al_u))
+    return torch.cat([g, u], dim=-1).contiguous()
+
+
 @pytest.mark.parametrize("m,n,k", [(300, 384, 320), (256, 256, 5120), (129, 640, 1024)])
-def test_random_matches_unfused_and_oracle(oracle, m, n, k):
+def test_random_bit_exact_vs_oracle_quantizer_on_library_projections(oracle, m, n, k):
     ops = real_operands(oracle, m, n, k, seed=m + k)
     gsf = ops[-1]
     q, sf = run_fused(*ops)
+    gu = library_gate_up(ops)
     q_u, sf_u = run_unfused(*ops)
     assert (q == q_u).all(), np.argwhere(q != q_u)[:5]
     assert (sf == sf_u).all(), np.argwhere(sf != sf_u)[:5]
-    q_ref, sf_ref = oracle.gemm_silu_mul_quantize(*ops[:8], gsf, m, n, k)
-    assert_nvfp4_close(q, sf_logical(sf, m, n), q_ref, sf_logical(sf_ref, m, n), gsf, f"swiglu {m}x{n}x{k}")
-    rows_pad = -(-m // 128) * 128
-    pad = sf_logical(sf, rows_pad, n)[m:]
-    assert (pad == 0).all(), "padding rows of the scale buffer must be zero"
+    gu_h = host(gu)
+    q_ref, sf_ref = oracle.silu_mul_quantize_batched(gu_h[None], np.float32([gsf]))
+    assert (q == q_ref[0]).all(), np.argwhere(q != q_ref[0])[:5]
+    assert (sf == sf_ref[0]).all(), np.argwhere(sf != sf_ref[0])[:5]     # padding rows' zero scales included
+    rows = np.arange(m)
+    ii, jj = np.repeat(rows, n), np.tile(np.arange(n), m)
+    check_projections_faithful(oracle, ops, gu_h, ii, jj, n, k, f"swiglu {m}x{n}x{k}")
+    check_explained_vs_composition(oracle, ops, gsf, q, sf_logical(sf, m, n), gu_h, rows, n, k,
+                                   f"swiglu {m}x{n}x{k}")
 
 
 def test_concatenated_gate_up_weight(oracle):
@@ -135,8 +156,11 @@ def test_concatenated_gate_up_weight(oracle):
     wq, wsf = dev_u8(qw), dev_u8(sw)
     q, sf = nv.nvfp4_gemm_silu_mul_quantize(dev_u8(qa), wq[:n], wq[n:], dev_u8(sa), wsf[:half], wsf[half:],
                                             dev_f32(al), dev_f32(al), dev_f32(gsf[0]))
-    q_ref, sf_ref = oracle.gemm_silu_mul_quantize(*ops, gsf[0], m, n, k)
-    assert_nvfp4_close(host(q), sf_logical(host(sf), m, n), q_ref, sf_logical(sf_ref, m, n), gsf[0], "concat")
+    gu_h = host(library_gate_up(ops))
+    q_ref, sf_ref = oracle.silu_mul_quantize_batched(gu_h[None], gsf)
+    assert (host(q) == q_ref[0]).all() and (host(sf) == sf_ref[0]).all()
+    check_explained_vs_composition(oracle, ops, gsf[0], host(q), sf_logical(host(sf), m, n), gu_h, np.arange(m), n,
+                                   k, "concat")
 
 
 def test_output_bounds(oracle):
@@ -208,7 +232,7 @@ def test_grouped_unit_scales_bit_exact_vs_oracle(oracle):
     assert (sf == sf_ref).all(), np.argwhere(sf != sf_ref)[:5]      # rows >= mask keep 0xCD
 
 
-def test_grouped_random_matches_unfused_and_oracle(oracle):
+def test_grouped_random_bit_exact_vs_oracle_quantizer_on_library_projections(oracle):
     E, mmax, n, k = 5, 384, 256, 512
     mask = np.array([384, 0, 257, 1, 128], np.int32)
     ops = grouped_real(oracle, E, mmax, n, k, mask, seed=13)
@@ -222,21 +246,26 @@ def test_grouped_random_matches_unfused_and_oracle(oracle):
     sx = torch.full((E, nv.nvfp4_scale_bytes(mmax, n)), 0xCD, dtype=torch.uint8, device="cuda")
     nv.nvfp4_silu_mul_quantize_batched(x, dev_f32(gsf), mask=dev_i32(mask), q_out=qx, sf_out=sx)
     assert (q == host(qx)).all() and (sf == host(sx)).all()
-    q_ref, sf_ref = oracle.grouped_gemm_silu_mul_quantize(qa, qg, qu, sa, sg, su, mask, al_g, al_u, gsf, E, mmax,
-                                                          n, k, q_fill=0xAB, sf_fill=0xCD)
+    # the oracle's quantizer on the library's projections, every valid row, bit for bit
+    gu_h = host(x)
+    q_ref, sf_ref = oracle.silu_mul_quantize_batched(gu_h, gsf, mask, q_fill=0xAB, sf_fill=0xCD)
+    assert (q == q_ref).all(), np.argwhere(q != q_ref)[:5]
+    assert (sf == sf_ref).all(), np.argwhere(sf != sf_ref)[:5]
     for e in range(E):
         v = int(mask[e])
         assert (q[e, v:] == 0xAB).all(), f"expert {e}: rows beyond the mask were written"
         rows_pad = -(-mmax // 128) * 128
         assert (sf_logical(sf[e], rows_pad, n)[v:] == 0xCD).all(), f"expert {e}: scales beyond the mask written"
         if v:
-            assert_nvfp4_close(q[e, :v], sf_logical(sf[e], v, n), q_ref[e, :v], sf_logical(sf_ref[e], v, n),
-                               gsf[e], f"expert {e}")
+            ops_e = (qa[e], qg[e], qu[e], sa[e], sg[e], su[e], al_g[e], al_u[e])
+            rows = np.arange(v)
+            check_explained_vs_composition(oracle, ops_e, gsf[e], q[e, :v], sf_logical(sf[e], v, n), gu_h[e, :v],
+                                           rows, n, k, f"expert {e}")
 
 
 # ---- full size, sampled rows ---------------------------------------------------------------------
 
-def test_swiglu_block_full_size_sampled_rows(oracle):
+def test_swiglu_block_full_size_every_row(oracle):
     # x [8192, 5120]; W_gate_up [16384, 5120] as one tensor: gate = rows [0, 8192), up = the rest
     m, k, n = 8192, 5120, 8192
     d = S.swiglu_block()
@@ -247,12 +276,20 @@ def test_swiglu_block_full_size_sampled_rows(oracle):
     al = np.float32(oracle.alpha(float(am_a), float(am_w)))
     half = nv.nvfp4_scale_bytes(n, k)
     ops = (qa, qw[:n], qw[n:], sa, sw[:half], sw[half:], al, al)
-    rows = np.array([0, 1, 127, 128, 4095, 5000, 8190, 8191])
-    x = oracle.gemm_gate_up_bf16(*ops, n, k, rows)
-    gsf = np.float32(oracle.global_scale_batched(x[None], None, silu_mul=True)[1][0])   # calibrated on samples
+    gu = library_gate_up(ops)
+    gu_h = host(gu)
+    del gu
+    # the static scale of h, calibrated on the whole h of the library's projections
+    gsf = np.float32(oracle.global_scale_batched(gu_h[None], None, silu_mul=True)[1][0])
     q, sf = run_fused(*ops, gsf)
-    q_u, sf_u = run_unfused(*ops, gsf)
-    assert (q == q_u).all() and (sf == sf_u).all()
-    q_ref, s_ref = oracle.gemm_silu_mul_quantize_rows(*ops, gsf, n, k, rows)
-    s_all = sf_logical(sf, m, n)
-    assert_nvfp4_close(q[rows], s_all[rows], q_ref, s_ref, gsf, "swiglu 8192x8192x5120 (sampled rows)")
+    # every row of the output, bit for bit, against the oracle's quantizer on the same projections
+    q_ref, sf_ref = oracle.silu_mul_quantize_batched(gu_h[None], np.float32([gsf]))
+    assert (q == q_ref[0]).all(), np.argwhere(q != q_ref[0])[:5]
+    assert (sf == sf_ref[0]).all(), np.argwhere(sf != sf_ref[0])[:5]
+    # the projections at the corners and two interior points of every 256 x 128 output tile
+    ii, jj = tile_positions(m, n, 256, 128, seed=3)
+    check_projections_faithful(oracle, ops, gu_h, ii, jj, n, k, "swiglu 8192x8192x5120 (every tile)")
+    # eight whole rows (both CTAs of a pair, the first and the last tile rows) against the fp64 composition
+    rows = np.array([0, 1, 127, 128, 4095, 5000, 8190, 8191])
+    check_explained_vs_composition(oracle, ops, gsf, q[rows], sf_logical(sf, m, n)[rows], gu_h[rows], rows, n, k,
+                                   "swiglu 8192x8192x5120 (rows)")

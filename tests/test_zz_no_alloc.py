@@ -1,11 +1,11 @@
 """The non-allocating batched global scale, called through the C ABI.
 
-Some callers cannot let the library allocate device memory: code being captured into a
-CUDA graph, hosts whose device memory belongs to their own allocator, and paths that must
+Some callers cannot let the library allocate device memory: hosts whose device memory
+belongs to their own allocator or is a fixed budget set at start-up, and paths that must
 not risk the implicit synchronization of cudaMalloc.  nvfp4_global_scale_batched_noalloc
 takes its reduction scratch from a fixed array inside the library instead; these checks
-compare it with the allocating entry point on two calls in a row (the array is reused and
-must be cleared by each call), and check its size limit.  The file name sorts last so a
+compare it with the allocating entry point and with the oracle on two calls in a row (the
+array is reused and must be cleared by each call), and check its size limit.  The file name sorts last so a
 run that stops at the first failure has run every other test first.
 """
 import ctypes
@@ -44,7 +44,7 @@ def call_noalloc(lib, x, mask, silu, amax, gsf):
 
 
 @pytest.mark.parametrize("silu", [False, True])
-def test_noalloc_matches_allocating_entry_point(lib, silu):
+def test_noalloc_matches_allocating_entry_point(lib, oracle, silu):
     b, m, k = 6, 90, 64
     for call, seed in enumerate((31, 32)):                  # two calls in a row, different data
         w = 2 * k if silu else k
@@ -57,11 +57,18 @@ def test_noalloc_matches_allocating_entry_point(lib, silu):
         torch.cuda.synchronize()
         # the reduction is a max, so the result is exact: the tolerance is zero
         assert torch.equal(amax, ref_amax) and torch.equal(gsf, ref_gsf), (call, amax, ref_amax)
+        # and both equal the oracle's per-item global scale over the valid rows
+        o_amax, o_gsf = oracle.global_scale_batched(S.normal_bf16((b, m, w), 1.0 + call, seed=seed),
+                                                    mask.cpu().numpy(), silu_mul=silu)
+        assert (amax.cpu().numpy() == o_amax).all() and (gsf.cpu().numpy() == o_gsf).all()
 
 
-def test_noalloc_without_mask_and_size_limit(lib):
-    x = to_dev(S.normal_bf16((3, 17, 48), 2.0, seed=5))
+def test_noalloc_without_mask_and_size_limit(lib, oracle):
+    x_bits = S.normal_bf16((3, 17, 48), 2.0, seed=5)
+    x = to_dev(x_bits)
     ref_amax, ref_gsf = nv.nvfp4_global_scale_batched(x, None)
+    o_amax, o_gsf = oracle.global_scale_batched(x_bits, None)
+    assert (ref_amax.cpu().numpy() == o_amax).all() and (ref_gsf.cpu().numpy() == o_gsf).all()
     amax = torch.empty(3, dtype=torch.float32, device="cuda")
     gsf = torch.empty(3, dtype=torch.float32, device="cuda")
     for _ in range(2):
