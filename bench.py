@@ -29,6 +29,13 @@ graph.  The value is whole-job throughput (sum over ranks of the work / the max 
 ranks of the device time).  With N > 1 every rank runs its own independent batch (data
 parallel, no collective on the data path): weak scaling.
 
+On one GPU the default run then times every other configuration the same way (the PR1
+linear, the quantize sweep -- dense, masked, SiLU-and-mul --, the masked grouped GEMM, the
+low-rank GEMM at r = 32, 64, 128), each reported under ``configs`` with its value, its
+dominant kernel's roofline, its parts and an oracle sample; and the headline's step graph
+is replayed back to back for at least one second (``sustained``: the power-capped regime,
+with its own clock record).  --no-configs / --no-sustained skip them.
+
 ``--impl reference`` times the CPU oracle (the plain C reference implementation) on a
 bounded sample of the same workload on this machine's host cores.
 """
@@ -158,10 +165,13 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
+    _count = 0
+
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join("/tmp", f"nvfp4_clocks_{os.getpid()}.csv")
+        ClockSampler._count += 1          # one file per sampler: a process may run several
+        self.path = os.path.join("/tmp", f"nvfp4_clocks_{os.getpid()}_{ClockSampler._count}.csv")
 
     def __enter__(self):
         try:
@@ -997,6 +1007,230 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+# The other configurations, timed by the default run after the headline (one GPU only), each
+# with its roofline and its oracle sample: (workload, low-rank r).
+EXTRA_CONFIGS = [("pr1_linear", 0), ("quant_dense", 0), ("quant_masked", 0), ("quant_silu", 0),
+                 ("grouped_moe", 0), ("lowrank", 32), ("lowrank", 64), ("lowrank", 128)]
+
+
+class Timer:
+    """CUDA-graph timing of one workload's step: a step graph (event nodes at its start and
+    end only, kernels chained by programmatic dependent launch) and a kernel graph (an event
+    node around every kernel), replayed alternately after an L2 flush."""
+
+    def __init__(self, nv, wl, stream, flush_l2):
+        import torch
+        self.nv, self.wl, self.stream, self.flush_l2 = nv, wl, stream, flush_l2
+        self.launches = launches = wl.launches()
+
+        def step(evs=None):
+            for i, (_, fn) in enumerate(launches):
+                if evs is not None:
+                    evs[i].record()
+                fn()
+            if evs is not None:
+                evs[len(launches)].record()
+
+        # One eager pass on the launch stream (allocates the library's per-stream scratch),
+        # then the two CUDA graphs.  Should the CUDA driver refuse timing on graph event nodes,
+        # every kernel is captured into its own graph and timed by events recorded around its
+        # replay (no overlap either way).
+        with torch.cuda.stream(stream):
+            step()
+        torch.cuda.synchronize()
+        self.step_events = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+        self.kernel_events = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(launches) + 1)]
+        self.graph_s, self.graph_k = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph_s, stream=stream):
+            self.step_events[0].record()
+            step()
+            self.step_events[1].record()
+        with torch.cuda.graph(self.graph_k, stream=stream):
+            step(self.kernel_events)
+        torch.cuda.synchronize()
+        self.mode = ("step: one CUDA graph per step, event nodes at its start and end (kernels chained by "
+                     "programmatic dependent launch: %s); kernels: a second pass with an event node around every "
+                     "kernel" % ("on" if nv.nvfp4_get_pdl() else "off"))
+        self.split = None
+        try:
+            with torch.cuda.stream(stream):
+                self.run_step()
+                self.run_kernels()
+        except Exception:                                      # noqa: BLE001
+            torch.cuda.synchronize()
+            self.graph_s = self.graph_k = None
+            self.split = []
+            for _, fn in launches:
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    fn()
+                self.split.append(g)
+            self.outer = [torch.cuda.Event(enable_timing=True) for _ in range(len(launches) + 1)]
+            self.mode = "one CUDA graph per kernel, events around each replay (step time = first to last event)"
+
+    def replay_step(self):
+        if self.split is None:
+            self.graph_s.replay()
+        else:
+            for g in self.split:
+                g.replay()
+
+    def run_kernels(self):
+        if self.split is None:
+            self.graph_k.replay()
+            self.stream.synchronize()
+            ev = self.kernel_events
+        else:
+            for i, g in enumerate(self.split):
+                self.outer[i].record()
+                g.replay()
+            self.outer[-1].record()
+            self.stream.synchronize()
+            ev = self.outer
+        return [ev[i].elapsed_time(ev[i + 1]) for i in range(len(self.launches))]
+
+    def run_step(self):
+        if self.split is not None:
+            self.run_kernels()
+            return self.outer[0].elapsed_time(self.outer[-1])
+        self.graph_s.replay()
+        self.stream.synchronize()
+        return self.step_events[0].elapsed_time(self.step_events[1])
+
+    def warm(self, n):
+        import torch
+        with torch.cuda.stream(self.stream):
+            for _ in range(n):
+                self.flush_l2()
+                self.replay_step()
+        torch.cuda.synchronize()
+
+    def timed(self, steps):
+        """`steps` replays of each graph, alternating step by step, so that both passes see the
+        same clocks and power state.  Returns (step times, per-step kernel times) in ms."""
+        import torch
+        step_ms, samples = [], []
+        with torch.cuda.stream(self.stream):
+            for _ in range(steps):
+                self.flush_l2()
+                step_ms.append(self.run_step())
+                self.flush_l2()
+                samples.append(self.run_kernels())
+        torch.cuda.synchronize()
+        return step_ms, samples
+
+    def release(self):
+        self.graph_s = self.graph_k = self.split = None
+
+
+def summarize(wl, step_ms, samples, launches, peaks, peak_kind, world):
+    """value / ms_per_step (whole job), per-kernel parts and the dominant kernel's roofline."""
+    per_kernel = {name: [smp[i] for smp in samples] for i, (name, _) in enumerate(launches)}
+    steps = len(step_ms)
+    work_all, total_ms_max = aggregate(world, wl.work() * steps, sum(step_ms))
+    value = scale(work_all / (total_ms_max * 1e-3), wl.unit)
+    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    hbm_peak = peaks["hbm_gbs"]
+    parts = {}
+    for name, (w, unit) in wl.kernel_work().items():
+        ms = statistics.mean(per_kernel[name])
+        ach = scale(w / (ms * 1e-3), unit)
+        peak = fp4_peak if unit == "TFLOP/s" else hbm_peak
+        parts[name] = {"ms": round(ms, 5), "achieved": round(ach, 2), "unit": unit, "frac": round(ach / peak, 4)}
+    dom = wl.dominant
+    w, unit = wl.kernel_work()[dom]
+    dom_ms = statistics.mean(per_kernel[dom])
+    achieved = scale(w / (dom_ms * 1e-3), unit)
+    peak = fp4_peak if unit == "TFLOP/s" else hbm_peak
+    kernel_name = KERNEL_OF_LAUNCH.get(dom, "nvfp4_gemm_kernel" if unit == "TFLOP/s" else "quantize_kernel")
+    roofline = {"bound": "tensor" if unit == "TFLOP/s" else "hbm", "achieved": round(achieved, 2),
+                "peak": round(peak, 1), "unit": unit, "frac": round(achieved / peak, 4),
+                "traffic": recorded_traffic(kernel_name, f"{wl.name}:{dom}"), "kernel": dom,
+                "peak_source": f"{peak_kind}: " + (
+                    f"bf16 burst {peaks['bf16_tflops']} TFLOP/s x {FP4_OVER_BF16} (nominal FP4/BF16 dense ratio)"
+                    if unit == "TFLOP/s" else f"HBM copy {peaks['hbm_gbs']} GB/s")}
+    return value, total_ms_max / steps, parts, roofline
+
+
+def measure_e2e(wl, timer, stream, flush_l2, args, world):
+    """End to end through the public API: every step uploads its input from pinned host
+    memory and downloads its result.  Uploads, compute and downloads run on three streams
+    (PCIe is full duplex), through double-buffered device staging tensors ordered by events,
+    so step i+1 uploads and step i-1 downloads while step i computes."""
+    import torch
+    x_host_bits, x_dev, y_dev = wl.e2e_io()
+    x_pinned = torch.from_numpy(np.ascontiguousarray(x_host_bits).view(np.int16)).view(x_dev.dtype).pin_memory()
+    y_pinned = [torch.empty(y_dev.shape, dtype=y_dev.dtype).pin_memory() for _ in range(2)]
+    x_stage = [torch.empty_like(x_dev) for _ in range(2)]
+    y_stage = [torch.empty_like(y_dev) for _ in range(2)]
+    h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+    total = args.warmup + args.steps
+    ev_in, ev_used, ev_out, ev_down = ([torch.cuda.Event() for _ in range(total)] for _ in range(4))
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    for i in range(total):
+        buf = i % 2
+        with torch.cuda.stream(h2d):
+            if i == args.warmup:
+                t_start.record()
+            if i >= 2:
+                h2d.wait_event(ev_used[i - 2])          # staging buffer free again
+            x_stage[buf].copy_(x_pinned, non_blocking=True)
+            ev_in[i].record()
+        with torch.cuda.stream(stream):
+            flush_l2()
+            stream.wait_event(ev_in[i])
+            x_dev.copy_(x_stage[buf], non_blocking=True)
+            ev_used[i].record()
+            timer.replay_step()
+            if i >= 2:
+                stream.wait_event(ev_down[i - 2])
+            y_stage[buf].copy_(y_dev, non_blocking=True)
+            ev_out[i].record()
+        with torch.cuda.stream(d2h):
+            d2h.wait_event(ev_out[i])
+            y_pinned[buf].copy_(y_stage[buf], non_blocking=True)
+            ev_down[i].record()
+    with torch.cuda.stream(d2h):
+        t_end.record()
+    torch.cuda.synchronize()
+    e2e_ms = t_start.elapsed_time(t_end)
+    e2e_work, e2e_ms = aggregate(world, wl.work() * args.steps, e2e_ms)
+    e2e_val = scale(e2e_work / (e2e_ms * 1e-3), wl.unit)
+    return {"value": round(e2e_val, 3), "unit": wl.unit,
+            "h2d_bytes_per_step": int(x_pinned.numel() * x_pinned.element_size()),
+            "d2h_bytes_per_step": int(y_pinned[0].numel() * y_pinned[0].element_size()),
+            "ms_per_step": round(e2e_ms / args.steps, 4),
+            "pipeline": "upload, compute and download on three streams, double-buffered device staging; time from "
+                        "the first timed upload to the last timed download"}
+
+
+def measure_sustained(timer, wl, world, local, min_seconds=1.0):
+    """The step graph replayed back to back (each replay after an L2 flush) for at least
+    `min_seconds` of wall time: the power-capped regime a long run settles in, with its own
+    clock record."""
+    import torch
+    step_ms = []
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        t0 = time.perf_counter()
+        with torch.cuda.stream(timer.stream):
+            while time.perf_counter() - t0 < min_seconds:
+                timer.flush_l2()
+                step_ms.append(timer.run_step())
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - t0
+    barrier(world)
+    work_all, total_ms_max = aggregate(world, wl.work() * len(step_ms), sum(step_ms))
+    clk = clocks.summary()
+    return {"value": round(scale(work_all / (total_ms_max * 1e-3), wl.unit), 3), "unit": wl.unit,
+            "ms_per_step": round(total_ms_max / len(step_ms), 5), "steps": len(step_ms), "wall_s": round(wall, 3),
+            "clocks": {"sm_mhz": clk.get("sm_mhz"), "sm_max_mhz": clk.get("sm_max_mhz"),
+                       "reasons": clk.get("reasons"), "power_w_max": clk.get("power_w_max")}}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -1011,6 +1245,9 @@ def main():
                     help="swiglu_block: SiLU*mul quantization in the gate/up GEMM epilogue, or as its own kernel")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="time only the chosen workload (the default run also times the other configurations)")
+    ap.add_argument("--no-sustained", action="store_true")
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch without programmatic dependent launch (the library default is on)")
     args = ap.parse_args()
@@ -1026,8 +1263,6 @@ def main():
     import nvfp4_block_scaled_16_b200 as nv
     world, rank, local = dist_setup(args.gpus)
     nv.load_library()
-    wl = make_workload(args.workload, nv, args.rank_lr, args.swiglu_path)
-    launches = wl.launches()
     if args.no_pdl:
         nv.nvfp4_set_pdl(False)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
@@ -1038,200 +1273,30 @@ def main():
         flush.zero_()
         clean.max()
 
-    def step(evs=None):
-        for i, (_, fn) in enumerate(launches):
-            if evs is not None:
-                evs[i].record()
-            fn()
-        if evs is not None:
-            evs[len(launches)].record()
-
-    # One eager pass on the launch stream (allocates the library's per-stream scratch),
-    # then two CUDA graphs of the step.  The step graph has an external event node only at
-    # its start and end, so consecutive kernels keep their programmatic-dependent-launch
-    # edges: it gives the step time (value).  The kernel graph has an event node around
-    # every kernel (consecutive kernels then cannot overlap): it gives each kernel's own
-    # duration (parts, roofline).  Both run inside the timed region, alternating step by step.  Should
-    # the CUDA driver refuse timing on graph event nodes, every kernel is captured into its
-    # own graph and timed by events recorded around its replay (no overlap either way).
-    with torch.cuda.stream(stream):
-        step()
-    torch.cuda.synchronize()
-
-    def replay_all(graphs):
-        for g in graphs:
-            g.replay()
-
-    step_events = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
-    kernel_events = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(launches) + 1)]
-    graph_s, graph_k = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph_s, stream=stream):
-        step_events[0].record()
-        step()
-        step_events[1].record()
-    with torch.cuda.graph(graph_k, stream=stream):
-        step(kernel_events)
-    torch.cuda.synchronize()
-    timing_mode = ("step: one CUDA graph per step, event nodes at its start and end (kernels chained by "
-                   "programmatic dependent launch: %s); kernels: a second pass with an event node around every "
-                   "kernel" % ("on" if nv.nvfp4_get_pdl() else "off"))
-
-    def run_step_graph():
-        graph_s.replay()
-        stream.synchronize()
-        return step_events[0].elapsed_time(step_events[1])
-
-    def run_kernels_graph():
-        graph_k.replay()
-        stream.synchronize()
-        return [kernel_events[i].elapsed_time(kernel_events[i + 1]) for i in range(len(launches))]
-
-    run_step, run_kernels = run_step_graph, run_kernels_graph
-    try:
-        with torch.cuda.stream(stream):
-            run_step()
-            run_kernels()
-    except Exception:                                      # noqa: BLE001
-        torch.cuda.synchronize()
-        graphs = []
-        for _, fn in launches:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                fn()
-            graphs.append(g)
-        outer = [torch.cuda.Event(enable_timing=True) for _ in range(len(launches) + 1)]
-        timing_mode = "one CUDA graph per kernel, events around each replay (step time = first to last event)"
-
-        def run_kernels_split():
-            for i, g in enumerate(graphs):
-                outer[i].record()
-                g.replay()
-            outer[-1].record()
-            stream.synchronize()
-            return [outer[i].elapsed_time(outer[i + 1]) for i in range(len(launches))]
-
-        def run_step_split():
-            run_kernels_split()
-            return outer[0].elapsed_time(outer[-1])
-
-        run_step, run_kernels = run_step_split, run_kernels_split
-        graph_s = None
-
-        def replay_step():
-            replay_all(graphs)
-    else:
-        def replay_step():
-            graph_s.replay()
-
-    with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
-            flush_l2()
-            replay_step()
-    torch.cuda.synchronize()
+    peaks, peak_kind = load_peaks()
+    wl = make_workload(args.workload, nv, args.rank_lr, args.swiglu_path)
+    timer = Timer(nv, wl, stream, flush_l2)
+    timer.warm(args.warmup)
     if nv.nvfp4_device_status(clear=True) != 0:
         raise SystemExit("device-side timeout during warm-up")
 
-    step_ms, samples = [], []
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
         t_wall = time.perf_counter()
-        # the two passes alternate step by step, so that both see the same clocks and power
-        # state (a long run can reach the power cap)
-        with torch.cuda.stream(stream):
-            for s in range(args.steps):
-                flush_l2()
-                step_ms.append(run_step())
-                flush_l2()
-                samples.append(run_kernels())
-        torch.cuda.synchronize()
+        step_ms, samples = timer.timed(args.steps)
         t_wall = time.perf_counter() - t_wall
+    clk = clocks.summary()
     barrier(world)
     status = nv.nvfp4_device_status(clear=True)
     if status != 0:
         raise SystemExit(f"device-side timeout in the timed region (status {status})")
+    value, ms_per_step, parts, roofline = summarize(wl, step_ms, samples, timer.launches, peaks, peak_kind, world)
 
-    per_kernel = {name: [smp[i] for smp in samples] for i, (name, _) in enumerate(launches)}
-    total_ms = sum(step_ms)
-    work_all, total_ms_max = aggregate(world, wl.work() * args.steps, total_ms)
-    value = scale(work_all / (total_ms_max * 1e-3), wl.unit)
-    ms_per_step = total_ms_max / args.steps
-
-    peaks, peak_kind = load_peaks()
-    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
-    hbm_peak = peaks["hbm_gbs"]
-    parts = {}
-    for name, (w, unit) in wl.kernel_work().items():
-        ms = statistics.mean(per_kernel[name])
-        ach = scale(w / (ms * 1e-3), unit)
-        peak = fp4_peak if unit == "TFLOP/s" else hbm_peak
-        parts[name] = {"ms": round(ms, 5), "achieved": round(ach, 2), "unit": unit,
-                       "frac": round(ach / peak, 4)}
-
-    dom = wl.dominant
-    w, unit = wl.kernel_work()[dom]
-    dom_ms = statistics.mean(per_kernel[dom])
-    achieved = scale(w / (dom_ms * 1e-3), unit)
-    peak = fp4_peak if unit == "TFLOP/s" else hbm_peak
-    kernel_name = KERNEL_OF_LAUNCH.get(dom, "nvfp4_gemm_kernel" if unit == "TFLOP/s" else "quantize_kernel")
-    traffic = recorded_traffic(kernel_name, f"{wl.name}:{dom}")
-    roofline = {"bound": "tensor" if unit == "TFLOP/s" else "hbm", "achieved": round(achieved, 2),
-                "peak": round(peak, 1), "unit": unit, "frac": round(achieved / peak, 4), "traffic": traffic,
-                "kernel": dom, "peak_source": f"{peak_kind}: " + (
-                    f"bf16 burst {peaks['bf16_tflops']} TFLOP/s x {FP4_OVER_BF16} (nominal FP4/BF16 dense ratio)"
-                    if unit == "TFLOP/s" else f"HBM copy {peaks['hbm_gbs']} GB/s")}
-
+    sustained = None if args.no_sustained else measure_sustained(timer, wl, world, local)
     e2e = None
     if not args.no_e2e and wl.e2e_io() is not None:
-        # End to end through the public API: every step uploads its input from pinned host
-        # memory and downloads its result.  Uploads, compute and downloads run on three
-        # streams (PCIe is full duplex), through double-buffered device staging tensors
-        # ordered by events, so step i+1 uploads and step i-1 downloads while step i computes.
-        x_host_bits, x_dev, y_dev = wl.e2e_io()
-        x_pinned = torch.from_numpy(np.ascontiguousarray(x_host_bits).view(np.int16)).view(x_dev.dtype).pin_memory()
-        y_pinned = [torch.empty(y_dev.shape, dtype=y_dev.dtype).pin_memory() for _ in range(2)]
-        x_stage = [torch.empty_like(x_dev) for _ in range(2)]
-        y_stage = [torch.empty_like(y_dev) for _ in range(2)]
-        h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
-        total = args.warmup + args.steps
-        ev_in, ev_used, ev_out, ev_down = ([torch.cuda.Event() for _ in range(total)] for _ in range(4))
-        t_start = torch.cuda.Event(enable_timing=True)
-        t_end = torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize()
-        for i in range(total):
-            buf = i % 2
-            with torch.cuda.stream(h2d):
-                if i == args.warmup:
-                    t_start.record()
-                if i >= 2:
-                    h2d.wait_event(ev_used[i - 2])          # staging buffer free again
-                x_stage[buf].copy_(x_pinned, non_blocking=True)
-                ev_in[i].record()
-            with torch.cuda.stream(stream):
-                flush_l2()
-                stream.wait_event(ev_in[i])
-                x_dev.copy_(x_stage[buf], non_blocking=True)
-                ev_used[i].record()
-                replay_step()
-                if i >= 2:
-                    stream.wait_event(ev_down[i - 2])
-                y_stage[buf].copy_(y_dev, non_blocking=True)
-                ev_out[i].record()
-            with torch.cuda.stream(d2h):
-                d2h.wait_event(ev_out[i])
-                y_pinned[buf].copy_(y_stage[buf], non_blocking=True)
-                ev_down[i].record()
-        with torch.cuda.stream(d2h):
-            t_end.record()
-        torch.cuda.synchronize()
-        e2e_ms = t_start.elapsed_time(t_end)
-        e2e_work, e2e_ms = aggregate(world, wl.work() * args.steps, e2e_ms)
-        e2e_val = scale(e2e_work / (e2e_ms * 1e-3), wl.unit)
-        e2e = {"value": round(e2e_val, 3), "unit": wl.unit, "h2d_bytes_per_step": int(x_pinned.numel() * x_pinned.element_size()),
-               "d2h_bytes_per_step": int(y_pinned[0].numel() * y_pinned[0].element_size()),
-               "ms_per_step": round(e2e_ms / args.steps, 4),
-               "pipeline": "upload, compute and download on three streams, double-buffered device staging; time from "
-                           "the first timed upload to the last timed download"}
+        e2e = measure_e2e(wl, timer, stream, flush_l2, args, world)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -1239,18 +1304,55 @@ def main():
         v, secs = o.measure(1)
         cpu = {"value": v, "unit": wl.unit, "cores": o.threads, "kind": "oracle", "sample": o.sample,
                "seconds": round(secs, 2), **host_cpu()}
+    n_launches = 2 * len(timer.launches) * args.steps
+    unit, config, timing_mode = wl.unit, wl.config(), timer.mode
+    timer.release()
+    del timer, wl
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+    # the other configurations (one GPU: the scaling runs time the headline only)
+    configs = None
+    if world == 1 and not args.no_configs and args.workload == "swiglu_block":
+        configs = {}
+        for name, r in EXTRA_CONFIGS:
+            key = f"{name}_r{r}" if name == "lowrank" else name
+            w = make_workload(name, nv, r or args.rank_lr)
+            t = Timer(nv, w, stream, flush_l2)
+            t.warm(args.warmup)
+            with ClockSampler(local) as ck:
+                sm, smp = t.timed(args.steps)
+            st = nv.nvfp4_device_status(clear=True)
+            if st != 0:
+                raise SystemExit(f"device-side timeout while timing {key} (status {st})")
+            v, ms, prt, rl = summarize(w, sm, smp, t.launches, peaks, peak_kind, world)
+            n_launches += 2 * len(t.launches) * args.steps
+            entry = {"value": round(v, 3), "unit": w.unit, "ms_per_step": round(ms, 5), "roofline": rl, "parts": prt,
+                     "config": w.config(), "clocks": {k: ck.summary().get(k) for k in ("sm_mhz", "reasons")}}
+            if not args.no_cpu_baseline:
+                o = OracleSample(name)
+                cv, secs = o.measure(1)
+                entry["cpu_baseline"] = {"value": cv, "unit": o.unit, "cores": o.threads, "kind": "oracle",
+                                         "sample": o.sample, "seconds": round(secs, 2)}
+            configs[key] = entry
+            t.release()
+            del t, w
+            torch.cuda.synchronize()
+            torch.cuda.empty_cache()
 
     if rank == 0:
-        clk = clocks.summary()
-        line = {"metric": METRIC, "value": round(value, 3), "unit": wl.unit, "n_gpus": world, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "e2m1 x e2m1 (ue4m3 block scales) -> f32 accumulate",
-                "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights)", "config": wl.config(),
+        line = {"metric": METRIC, "value": round(value, 3), "unit": unit, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "e2m1 x e2m1 (ue4m3 block scales) -> f32 accumulate",
+                "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights)", "config": config,
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-                # our kernels launched in the timed region: the step pass and the kernel pass
-                "gpu_launches": 2 * len(launches) * args.steps, "parts": parts,
+                # our kernels launched in the timed regions: the step pass and the kernel pass of
+                # the headline and of every other configuration
+                "gpu_launches": n_launches, "parts": parts,
                 "clocks": {"sm_mhz": clk.get("sm_mhz"), "sm_max_mhz": clk.get("sm_max_mhz"),
                            "reasons": clk.get("reasons")},
+                "sustained": sustained, "configs": configs,
                 "wall_s_timed_region": round(t_wall, 4), "timing": timing_mode}
         if world > 1:
             line["config"]["parallelism"] = f"dp{world} (independent batch per GPU, no collective)"
