@@ -106,8 +106,8 @@ struct Chunk {
 };
 
 // Blocks f = base + u * kThreads + threadIdx.x with f < end (and f < p.blocks) are this
-// chunk's.  kKeep: the loads keep x in the caches (a second pass will read it again).
-template <bool kSilu, int kUnroll, bool kKeep = false>
+// chunk's.
+template <bool kSilu, int kUnroll>
 __device__ __forceinline__ void chunk_load(const QuantParams& p, int item, uint32_t base, Chunk<kSilu, kUnroll>& ch,
                                            uint32_t end = 0xffffffffu) {
   int valid = p.m;
@@ -132,13 +132,8 @@ __device__ __forceinline__ void chunk_load(const QuantParams& p, int item, uint3
     ch.live[u] = f < p.blocks && f < end && r < static_cast<uint32_t>(valid) && c < p.nb;
     if (ch.live[u]) {
       const uint16_t* src = x + static_cast<int64_t>(r) * p.x_row_stride + c * 16;
-      if constexpr (kKeep) {
-        ch.raw[u][0] = __ldg(reinterpret_cast<const uint4*>(src));
-        ch.raw[u][1] = __ldg(reinterpret_cast<const uint4*>(src + 8));
-      } else {
-        ch.raw[u][0] = load_stream(src);
-        ch.raw[u][1] = load_stream(src + 8);
-      }
+      ch.raw[u][0] = load_stream(src);
+      ch.raw[u][1] = load_stream(src + 8);
       if constexpr (kSilu) {
         ch.raw[u][2] = load_stream(src + p.k);
         ch.raw[u][3] = load_stream(src + p.k + 8);
@@ -400,16 +395,46 @@ __global__ void __launch_bounds__(kThreads) amax_batched_kernel(const uint16_t* 
 // ---- global scale and quantize in one launch -----------------------------------------------
 //
 // The global scale needs the amax of the whole tensor before any block can be quantized.
-// One persistent grid, every CTA resident at once (a cooperative launch), does both: CTA j
-// takes the contiguous range of 16-element blocks [j B / G, (j + 1) B / G); it reduces the
-// max |x| of its range (loads that keep x in L2), folds it into the workspace with an atomic
-// max, and arrives on a grid barrier; once every CTA has arrived, each computes gsf from the
-// same maximum and quantizes its range, last chunk first, so that the lines it read most
-// recently (the ones most likely still in L2) are read again first.  Workspace words:
-// 0 = barrier arrivals, 1 = amax bits, 2 = CTAs done reading the maximum; the last of
-// those resets all three for the next call on the stream.
-constexpr int kGsqUnroll = 4;
-constexpr int kGsqCtasPerSm = 3;
+// One persistent grid, one CTA per SM, every CTA resident at once (a cooperative launch),
+// does both, for k % 64 == 0 (k / 16 blocks per row fill whole 4-block scale groups).  x is
+// viewed as rows of 128 bytes, one 4-block scale group each (group g holds blocks 4g..4g+3,
+// which are the 64 elements of x at 64 g, and its codes are the 32 bytes of q at 32 g), and
+// CTA j takes the contiguous groups [j R / G, (j + 1) R / G).  A producer warp streams the
+// CTA's groups through a ring of three 60 KB shared-memory slots with tiled TMA loads (480
+// groups per slot, 128-byte swizzle, so a compute thread reads its 16-byte chunks without
+// bank conflicts); 30 compute warps take half a group (two blocks) per thread and slot.
+//   phase 1: the slots pass through the ring once (x read from HBM once); the compute warps
+//     take max |x| of each (packed bf16 pairs, NaN dropped like fmaxf) and release it,
+//     except the last three, which stay resident; the CTA folds its max into the workspace
+//     with an atomic max and arrives on a grid barrier (bounded spin on an acquire load).
+//     Slots that phase 2 reads again are loaded with the L2 evict-last policy.
+//   phase 2: every CTA computes gsf from the same maximum, quantizes the resident slots,
+//     while the producer reloads the earlier slots from L2 into the freed ones, last first.
+//     Each pair of threads writes its group's 32 code bytes and its four scale bytes (one
+//     word of the 128x4 layout, assembled by a shuffle), and the CTA zeroes its share of the
+//     padding rows' scale words.
+// Workspace words: 0 = barrier arrivals, 1 = amax bits, 2 = CTAs done reading the maximum,
+// 3 = set by a CTA whose own bounded ring wait gave up (then no CTA writes anything); the
+// last CTA to read the maximum resets all four for the next call on the stream.
+constexpr int kGsqComputeWarps = 30;
+constexpr int kGsqCompute = 32 * kGsqComputeWarps;              // compute threads: half a group each per slot
+constexpr int kGsqThreads = kGsqCompute + 32;                   // and the producer warp (at most 1024)
+constexpr uint32_t kGsqSlotGroups = kGsqCompute / 2;            // 480 groups = 60 KB of x per slot
+constexpr uint32_t kGsqSlotBytes = kGsqSlotGroups * 128;
+constexpr uint32_t kGsqSlots = 3;
+constexpr uint32_t kGsqSmemBytes = kGsqSlots * kGsqSlotBytes + 1024;   // + alignment to 1024 bytes
+constexpr uint32_t kGsqBox = kGsqSlotGroups / 2;                // groups per TMA box (two per slot)
+static_assert(kGsqThreads <= 1024 && kGsqBox <= 256, "block size or TMA box too large");
+static_assert((kGsqBox * 128) % 1024 == 0, "every TMA box lands 1024-byte aligned (128-byte swizzle)");
+
+struct GsqParams {
+  uint8_t* q;
+  uint8_t* sf;
+  uint32_t groups_total;   // m * nb / 4
+  uint32_t nb4;            // groups per row of x: nb / 4
+  uint32_t nb4_magic, nb4_shift;   // g / nb4 = (g * magic) >> shift for g < 2^31
+  uint32_t m, rows_pad;
+};
 
 __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
   uint32_t v;
@@ -417,54 +442,169 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
   return v;
 }
 
-__global__ void __launch_bounds__(kThreads, kGsqCtasPerSm)
-    global_scale_quantize_kernel(const QuantParams p, uint32_t* ws, float* amax_out, float* gsf_out,
-                                 const float* other_amax, float* alpha_out, int* status, uint32_t withheld) {
-  __shared__ float red[kThreads / 32];
+__device__ __forceinline__ uint64_t l2_policy(bool keep) {
+  uint64_t pol;
+  if (keep)
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  else
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// Tiled TMA load of kGsqBox groups (rows of 128 bytes) starting at group `row` into this
+// CTA's shared memory, completing on `bar`, with an L2 eviction policy.
+__device__ __forceinline__ void gsq_tma_load(void* dst, const CUtensorMap* map, uint64_t* bar, int row, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%3, %4}], "
+      "[%2], %5;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(0), "r"(row), "l"(pol)
+      : "memory");
+}
+
+__device__ __forceinline__ __nv_bfloat162 as_bf162(uint32_t w) {
+  return *reinterpret_cast<const __nv_bfloat162*>(&w);
+}
+
+// Running max |x| over the 8 bf16 values of a 16-byte chunk, as packed pairs.
+__device__ __forceinline__ __nv_bfloat162 absmax_chunk(const uint4& c, __nv_bfloat162 m) {
+  m = __hmax2(m, __habs2(as_bf162(c.x)));
+  m = __hmax2(m, __habs2(as_bf162(c.y)));
+  m = __hmax2(m, __habs2(as_bf162(c.z)));
+  m = __hmax2(m, __habs2(as_bf162(c.w)));
+  return m;
+}
+__device__ __forceinline__ float bf162_max(__nv_bfloat162 m) {
+  return fmaxf(__bfloat162float(m.x), __bfloat162float(m.y));
+}
+
+// One 16-element block (two chunks) with the block maximum taken on packed bf16 pairs: the
+// same value as block_scale_code's fp32 maximum (every |x| is a bf16 value), so the result
+// equals quantize16 bit for bit.
+__device__ __forceinline__ QBlock gsq_block(const uint4& lo4, const uint4& hi4, float gsf, const float* inv_tab) {
+  const __nv_bfloat162 zero = __floats2bfloat162_rn(0.0f, 0.0f);
+  const float vmax = bf162_max(absmax_chunk(hi4, absmax_chunk(lo4, zero)));
+  const uint32_t s8 = ue4m3_encode(__fmul_rn(div6_bf16(vmax), gsf));
+  float v[16];
+  unpack_bf16x8(lo4, v);
+  unpack_bf16x8(hi4, v + 8);
+  return quantize16_codes(v, s8, inv_tab[s8]);
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+// Thread t's half of group t / 2 in a 128-byte-swizzled slot at shared address `slot`:
+// chunks 4 h .. 4 h + 3 (h = t % 2), chunk j of row g being at 16-byte position j ^ (g % 8).
+// The eight threads of a quarter warp read eight different 16-byte bank groups.
+__device__ __forceinline__ void gsq_read_half(uint32_t slot, uint32_t t, uint4 (&c)[4]) {
+  const uint32_t g = t >> 1, h = t & 1;
+  const uint32_t row = slot + g * 128;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) c[i] = lds128(row + (((4 * h + i) ^ (g & 7)) << 4));
+}
+
+__global__ void __launch_bounds__(kGsqThreads, 1)
+    global_scale_quantize_kernel(const __grid_constant__ CUtensorMap xmap, const GsqParams p, uint32_t* ws,
+                                 float* amax_out, float* gsf_out, const float* other_amax, float* alpha_out,
+                                 int* status, uint32_t withheld) {
+  extern __shared__ uint8_t gsq_raw[];
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gsq_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ uint64_t full[kGsqSlots], empty[kGsqSlots];
+  __shared__ int32_t abort_flag;
+  __shared__ float red[kGsqComputeWarps];
   __shared__ float s_amax;
   __shared__ float inv_tab[128];
   pdl_wait();
+  const int warp = threadIdx.x >> 5;
+  const uint32_t t = threadIdx.x;
+  const bool producer = warp == kGsqComputeWarps;
   const uint32_t grid = gridDim.x;
   const uint32_t expected = grid + withheld;   // self-test: arrivals that never come
-  const uint32_t lo = static_cast<uint32_t>(static_cast<uint64_t>(p.blocks) * blockIdx.x / grid);
-  const uint32_t hi = static_cast<uint32_t>(static_cast<uint64_t>(p.blocks) * (blockIdx.x + 1) / grid);
-  constexpr uint32_t kChunk = kThreads * kGsqUnroll;
+  const uint32_t g_lo = static_cast<uint32_t>(static_cast<uint64_t>(p.groups_total) * blockIdx.x / grid);
+  const uint32_t g_hi = static_cast<uint32_t>(static_cast<uint64_t>(p.groups_total) * (blockIdx.x + 1) / grid);
+  const uint32_t slots_total = (g_hi - g_lo + kGsqSlotGroups - 1) / kGsqSlotGroups;   // pieces of the range
+  const uint32_t resident = min(slots_total, kGsqSlots);     // pieces that stay in the ring after phase 1
+  if (threadIdx.x == 0) {
+    for (uint32_t i = 0; i < kGsqSlots; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kGsqComputeWarps);
+    }
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  uint32_t fpar = 0, epar = 0;      // per-slot phase parity bits of full / empty waits
 
-  // phase 1: max |x| over this CTA's blocks
+  // ---------------------------------------------------------------- phase 1
   float mx = 0.0f;
-  for (uint32_t base = lo; base < hi; base += kChunk) {
-    Chunk<false, kGsqUnroll> ch;
-    chunk_load<false, kGsqUnroll, true>(p, 0, base, ch, hi);
+  if (producer) {
+    if (elect_one()) {
+      prefetch_map(&xmap);
+      for (uint32_t piece = 0; piece < slots_total; ++piece) {
+        const uint32_t s = piece % kGsqSlots;
+        if (piece >= kGsqSlots) {
+          if (!mbar_wait_fast(&empty[s], (epar >> s) & 1u, &abort_flag, status)) break;
+          epar ^= 1u << s;
+        }
+        const uint64_t pol = l2_policy(piece + resident < slots_total);   // read again in phase 2
+        uint8_t* dst = ring + s * kGsqSlotBytes;
+        const int row = static_cast<int>(g_lo + piece * kGsqSlotGroups);
+        mbar_arrive_expect_tx(&full[s], kGsqSlotBytes);
+        gsq_tma_load(dst, &xmap, &full[s], row, pol);
+        gsq_tma_load(dst + kGsqBox * 128, &xmap, &full[s], row + static_cast<int>(kGsqBox), pol);
+      }
+    }
+    __syncwarp();
+  } else {
+    const __nv_bfloat162 zero = __floats2bfloat162_rn(0.0f, 0.0f);
+    __nv_bfloat162 m2 = zero;
+    for (uint32_t piece = 0; piece < slots_total; ++piece) {
+      const uint32_t s = piece % kGsqSlots;
+      // warp-uniform outcome, so that the warp's lanes leave the loop together
+      if (!__all_sync(0xffffffffu, mbar_wait_fast(&full[s], (fpar >> s) & 1u, &abort_flag, status))) break;
+      fpar ^= 1u << s;
+      if (g_lo + piece * kGsqSlotGroups + (t >> 1) < g_hi) {
+        uint4 c[4];
+        gsq_read_half(smem_u32(ring) + s * kGsqSlotBytes, t, c);
 #pragma unroll
-    for (int u = 0; u < kGsqUnroll; ++u)
-      if (ch.live[u]) mx = absmax8(ch.raw[u][1], absmax8(ch.raw[u][0], mx));   // fmaxf drops NaN
+        for (int j = 0; j < 4; ++j) m2 = absmax_chunk(c[j], m2);
+      }
+      __syncwarp();
+      if (piece + resident < slots_total && (t & 31) == 0) mbar_arrive(&empty[s]);
+    }
+    mx = bf162_max(m2);
   }
   mx = warp_max(mx);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+  if ((threadIdx.x & 31) == 0 && !producer) red[warp] = mx;
   __syncthreads();
   if (threadIdx.x == 0) {
     float v = red[0];
 #pragma unroll
-    for (int w = 1; w < kThreads / 32; ++w) v = fmaxf(v, red[w]);
+    for (int w = 1; w < kGsqComputeWarps; ++w) v = fmaxf(v, red[w]);
+    if (abort_flag) atomicExch(ws + 3, 1u);            // a ring wait gave up: nobody writes
     atomicMax(ws + 1, __float_as_uint(v));
-    __threadfence();
-    atomicAdd(ws, 1u);
+    // arrive, ordered after the atomic max (and ws[3]) by release semantics
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ws) : "memory");
     // grid barrier, bounded: every CTA is resident, so only a fault elsewhere can stall it
     const uint64_t t0 = global_ns();
     bool ok = true;
-    while (ld_acquire_gpu(ws) < expected) {
-      if (global_ns() - t0 > kWaitLimitNs) {
+    for (uint32_t i = 1; ld_acquire_gpu(ws) < expected; ++i) {
+      if ((i & 63u) == 0 && global_ns() - t0 > kWaitLimitNs) {
         ok = false;
         atomicExch(status, NVFP4_ERR_DEVICE_TIMEOUT);
         break;
       }
-      __nanosleep(100);
     }
     float a = -1.0f;                                   // -1: give up, write nothing
     if (ok) {
-      a = fmaxf(fminf(__uint_as_float(ld_acquire_gpu(ws + 1)), FLT_MAX), 1e-12f);
+      if (ld_acquire_gpu(ws + 3) == 0u)
+        a = fmaxf(fminf(__uint_as_float(ld_acquire_gpu(ws + 1)), FLT_MAX), 1e-12f);
       if (atomicAdd(ws + 2, 1u) == grid - 1) {         // every CTA has read the maximum
         atomicExch(ws + 1, 0u);
+        atomicExch(ws + 3, 0u);
         atomicExch(ws + 2, 0u);
         atomicExch(ws, 0u);
       }
@@ -473,7 +613,16 @@ __global__ void __launch_bounds__(kThreads, kGsqCtasPerSm)
   }
   __syncthreads();
   const float amax = s_amax;
-  if (amax < 0.0f) return;
+  if (amax < 0.0f) {
+    if (abort_flag) {
+      // a ring wait gave up: give outstanding TMA loads a bounded time to land before the
+      // CTA's shared memory is released
+      const uint64_t t0 = global_ns();
+      while (global_ns() - t0 < 2000000ull) {
+      }
+    }
+    return;
+  }
   pdl_launch_dependents();            // every CTA of this grid is past the barrier
   const float gsf = __fdiv_rn(2688.0f, amax);
   if (blockIdx.x == 0 && threadIdx.x == 0) {
@@ -481,19 +630,86 @@ __global__ void __launch_bounds__(kThreads, kGsqCtasPerSm)
     *gsf_out = gsf;
     if (other_amax) *alpha_out = __fdiv_rn(__fmul_rn(amax, *other_amax), 7225344.0f);
   }
-
-  // phase 2: quantize this CTA's blocks, last chunk first
-  inv_table_build(inv_tab, gsf);
+  if (threadIdx.x < 128) inv_tab[threadIdx.x] = inv_scale(threadIdx.x, gsf);
   __syncthreads();
-  const uint32_t chunks = (hi - lo + kChunk - 1) / kChunk;
-  for (uint32_t j = chunks; j-- > 0;) {
-    Chunk<false, kGsqUnroll> ch;
-    chunk_load<false, kGsqUnroll, false>(p, 0, lo + j * kChunk, ch, hi);
-    chunk_store<false, false>(p, ch, nullptr, gsf, inv_tab);
+
+  // ---------------------------------------------------------------- phase 2: last piece first
+  if (producer) {
+    if (elect_one()) {
+      const uint64_t pol = l2_policy(false);
+      for (uint32_t i = resident; i < slots_total; ++i) {
+        const uint32_t piece = slots_total - 1 - i;
+        const uint32_t s = piece % kGsqSlots;
+        if (!mbar_wait_fast(&empty[s], (epar >> s) & 1u, &abort_flag, status)) break;
+        epar ^= 1u << s;
+        uint8_t* dst = ring + s * kGsqSlotBytes;
+        const int row = static_cast<int>(g_lo + piece * kGsqSlotGroups);
+        mbar_arrive_expect_tx(&full[s], kGsqSlotBytes);
+        gsq_tma_load(dst, &xmap, &full[s], row, pol);
+        gsq_tma_load(dst + kGsqBox * 128, &xmap, &full[s], row + static_cast<int>(kGsqBox), pol);
+      }
+    }
+    __syncwarp();
+  } else {
+    const uint32_t groups4 = p.nb4;           // 4-block groups per row of the scale layout
+    for (uint32_t i = 0; i < slots_total; ++i) {
+      const uint32_t piece = slots_total - 1 - i;
+      const uint32_t s = piece % kGsqSlots;
+      if (i >= resident) {                     // reloaded from L2
+        if (!__all_sync(0xffffffffu, mbar_wait_fast(&full[s], (fpar >> s) & 1u, &abort_flag, status))) break;
+        fpar ^= 1u << s;
+      }
+      const uint32_t g = g_lo + piece * kGsqSlotGroups + (t >> 1);
+      uint32_t scales = 0;                     // this thread's two scale bytes
+      if (g < g_hi) {                          // the same for both threads of a group
+        uint4 c[4];
+        gsq_read_half(smem_u32(ring) + s * kGsqSlotBytes, t, c);
+        const QBlock b0 = gsq_block(c[0], c[1], gsf, inv_tab);
+        const QBlock b1 = gsq_block(c[2], c[3], gsf, inv_tab);
+        *reinterpret_cast<uint4*>(p.q + static_cast<int64_t>(g) * 32 + (t & 1) * 16) =
+            make_uint4(b0.lo, b0.hi, b1.lo, b1.hi);
+        scales = b0.s8 | (b1.s8 << 8);
+      }
+      const uint32_t other = __shfl_xor_sync(0xffffffffu, scales, 1);
+      if (g < g_hi && (t & 1) == 0) {
+        const uint32_t r = static_cast<uint32_t>((static_cast<uint64_t>(g) * p.nb4_magic) >> p.nb4_shift);
+        const uint32_t c0 = (g - r * groups4) * 4;
+        *reinterpret_cast<uint32_t*>(p.sf + sf_offset(r, c0, groups4)) = scales | (other << 16);
+      }
+      __syncwarp();
+      if ((t & 31) == 0) mbar_arrive(&empty[s]);
+    }
+    // padding rows [m, rows_pad): their scale words are zero
+    const uint32_t pad_words = (p.rows_pad - p.m) * groups4;
+    for (uint32_t i = blockIdx.x * kGsqCompute + t; i < pad_words; i += grid * kGsqCompute) {
+      const uint32_t r = p.m + i / groups4;
+      *reinterpret_cast<uint32_t*>(p.sf + sf_offset(r, (i % groups4) * 4, groups4)) = 0u;
+    }
   }
 }
 
 // ---- host helpers -------------------------------------------------------------------------
+
+// nvfp4_global_scale: one launch of amax_dense_kernel.
+int launch_amax_dense(const void* x_bf16, int64_t numel, float* amax_out, float* gsf_out, const float* other_amax,
+                      float* alpha_out, cudaStream_t stream) {
+  if (numel < 0 || !gsf_out || (numel > 0 && !x_bf16)) return NVFP4_ERR_INVALID_ARGUMENT;
+  if ((other_amax == nullptr) != (alpha_out == nullptr)) return NVFP4_ERR_INVALID_ARGUMENT;
+  if ((x_bf16 && !aligned(x_bf16, 16)) || !aligned(gsf_out, 4) || (amax_out && !aligned(amax_out, 4)) ||
+      (other_amax && (!aligned(other_amax, 4) || !aligned(alpha_out, 4))))
+    return NVFP4_ERR_INVALID_ARGUMENT;
+  DeviceInfo info;
+  int st = current_device(&info);
+  if (st != NVFP4_OK) return st;
+  uint32_t* ws = nullptr;
+  st = stream_workspace(stream, &ws);
+  if (st != NVFP4_OK) return st;
+  const int64_t nvec = numel / 8;
+  int64_t blocks = (nvec + kThreads * 4 - 1) / (kThreads * 4);
+  blocks = blocks < 1 ? 1 : (blocks > info.sm_count * 8 ? info.sm_count * 8 : blocks);
+  return launch_kernel(amax_dense_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), 0, stream,
+                       static_cast<const uint16_t*>(x_bf16), numel, ws, amax_out, gsf_out, other_amax, alpha_out);
+}
 
 int launch_quantize(const void* x, int64_t b, int64_t m, int64_t k, bool silu, const int32_t* mask,
                     const float* gsf, uint8_t* q, uint8_t* sf, cudaStream_t stream, const void* pqs = nullptr) {
@@ -548,7 +764,8 @@ int launch_quantize(const void* x, int64_t b, int64_t m, int64_t k, bool silu, c
 }
 
 // nvfp4_global_scale_quantize; `withheld` > 0 (self-test only) makes the grid barrier wait
-// for arrivals that never come.
+// for arrivals that never come.  k % 64 == 0 and m > 0 take the one-launch kernel; other
+// shapes take the amax kernel and then the dense quantizer (the same results).
 int launch_global_scale_quantize(const void* x_bf16, int64_t m, int64_t k, float* amax_out, float* gsf_out,
                                  const float* other_amax, float* alpha_out, uint8_t* q_out, uint8_t* sf_out,
                                  cudaStream_t stream, uint32_t withheld) {
@@ -559,43 +776,68 @@ int launch_global_scale_quantize(const void* x_bf16, int64_t m, int64_t k, float
       (amax_out && !aligned(amax_out, 4)) || (other_amax && (!aligned(other_amax, 4) || !aligned(alpha_out, 4))))
     return NVFP4_ERR_INVALID_ARGUMENT;
   const int64_t nb = k / 16, cpad = (nb + 3) / 4 * 4, rows_pad = (m + 127) / 128 * 128;
-  if (rows_pad * cpad >= (int64_t(1) << 31) - 4096) return NVFP4_ERR_INVALID_ARGUMENT;   // f < 2^31
+  if (rows_pad * cpad >= (int64_t(1) << 31) - 4096) return NVFP4_ERR_INVALID_ARGUMENT;   // indices < 2^31
+  if (k % 64 != 0 || m == 0) {
+    if (withheld) return NVFP4_ERR_INVALID_ARGUMENT;   // the self-test needs the one-launch kernel
+    int st = launch_amax_dense(x_bf16, m * k, amax_out, gsf_out, other_amax, alpha_out, stream);
+    if (st != NVFP4_OK) return st;
+    return launch_quantize(x_bf16, 1, m, k, false, nullptr, gsf_out, q_out, sf_out, stream);
+  }
+  if (!aligned(q_out, 16) || !aligned(sf_out, 4)) return NVFP4_ERR_INVALID_ARGUMENT;
   DeviceInfo info;
   int st = current_device(&info);
   if (st != NVFP4_OK) return st;
   uint32_t* ws = nullptr;
   st = stream_workspace(stream, &ws);
   if (st != NVFP4_OK) return st;
-  int per_sm = 0;          // co-resident CTAs per SM, found once per device
-  st = kernel_setup(reinterpret_cast<const void*>(global_scale_quantize_kernel), info.device, [](int* out) {
+  const int smem = static_cast<int>(kGsqSmemBytes);
+  int per_sm = 0;          // co-resident CTAs per SM (the grid must be resident at once), per device
+  st = kernel_setup(reinterpret_cast<const void*>(global_scale_quantize_kernel), info.device, [&](int* out) {
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, global_scale_quantize_kernel, kThreads, 0) != cudaSuccess ||
+    if (cudaFuncSetAttribute(global_scale_quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, global_scale_quantize_kernel, kGsqThreads, smem) !=
+            cudaSuccess ||
         n <= 0) {
       cudaGetLastError();
       return static_cast<int>(NVFP4_ERR_CUDA);
     }
-    *out = n < kGsqCtasPerSm ? n : kGsqCtasPerSm;
+    *out = n;
     return static_cast<int>(NVFP4_OK);
   }, &per_sm);
   if (st != NVFP4_OK) return st;
-  QuantParams p = {};
-  p.x = static_cast<const uint16_t*>(x_bf16);
-  p.x_row_stride = k;
+  GsqParams p = {};
   p.q = q_out;
   p.sf = sf_out;
-  p.m = static_cast<int32_t>(m);
-  p.k = static_cast<int32_t>(k);
-  p.nb = static_cast<uint32_t>(nb);
-  p.cpad = static_cast<uint32_t>(cpad);
+  p.m = static_cast<uint32_t>(m);
   p.rows_pad = static_cast<uint32_t>(rows_pad);
-  p.blocks = static_cast<uint32_t>(rows_pad * cpad);
-  set_cpad_divisor(p);
-  p.items = 1;
-  const int64_t chunks = (p.blocks + kThreads * kGsqUnroll - 1) / (kThreads * kGsqUnroll);
+  p.nb4 = static_cast<uint32_t>(nb / 4);
+  p.groups_total = static_cast<uint32_t>(m * (nb / 4));
+  // Granlund-Montgomery: with l = ceil(log2 nb4) and magic = ceil(2^(31 + l) / nb4),
+  // floor(g / nb4) = floor(g * magic / 2^(31 + l)) for every g < 2^31 (magic < 2^32).
+  uint32_t l = 0;
+  while ((uint64_t(1) << l) < p.nb4) ++l;
+  p.nb4_magic = static_cast<uint32_t>(((uint64_t(1) << (31 + l)) + p.nb4 - 1) / p.nb4);
+  p.nb4_shift = 31 + l;
+  // x as rows of 128 bytes (one 4-block group each), boxes of 256 rows, 128-byte swizzle;
+  // rows beyond the tensor read as zeros
+  CUtensorMap xmap;
+  EncodeTiledFn encode = encode_tiled_fn();
+  if (!encode) return NVFP4_ERR_CUDA;
+  const cuuint64_t dims[2] = {128, p.groups_total};
+  const cuuint64_t strides[1] = {128};
+  const cuuint32_t box[2] = {128, kGsqBox};
+  const cuuint32_t elem_strides[2] = {1, 1};
+  if (encode(&xmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(x_bf16), dims, strides, box, elem_strides,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return NVFP4_ERR_INVALID_ARGUMENT;
+  const int64_t want = (static_cast<int64_t>(p.groups_total) + kGsqSlotGroups - 1) / kGsqSlotGroups;
   const int64_t cap = static_cast<int64_t>(info.sm_count) * per_sm;
-  const unsigned grid = static_cast<unsigned>(chunks < 1 ? 1 : (chunks < cap ? chunks : cap));
-  return launch_kernel_cooperative(global_scale_quantize_kernel, dim3(grid), dim3(kThreads), 0, stream, p, ws, amax_out,
-                                   gsf_out, other_amax, alpha_out, info.status, withheld);
+  const unsigned grid = static_cast<unsigned>(want < 1 ? 1 : (want < cap ? want : cap));
+  return launch_kernel_cooperative(global_scale_quantize_kernel, dim3(grid), dim3(kGsqThreads),
+                                   static_cast<size_t>(smem), stream, xmap, p, ws, amax_out, gsf_out, other_amax,
+                                   alpha_out, info.status, withheld);
 }
 
 }  // namespace
@@ -607,22 +849,7 @@ extern "C" {
 
 int nvfp4_global_scale(const void* x_bf16, int64_t numel, float* amax_out, float* gsf_out,
                        const float* other_amax, float* alpha_out, nvfp4_stream_t stream) {
-  if (numel < 0 || !gsf_out || (numel > 0 && !x_bf16)) return NVFP4_ERR_INVALID_ARGUMENT;
-  if ((other_amax == nullptr) != (alpha_out == nullptr)) return NVFP4_ERR_INVALID_ARGUMENT;
-  if ((x_bf16 && !aligned(x_bf16, 16)) || !aligned(gsf_out, 4) || (amax_out && !aligned(amax_out, 4)) ||
-      (other_amax && (!aligned(other_amax, 4) || !aligned(alpha_out, 4))))
-    return NVFP4_ERR_INVALID_ARGUMENT;
-  DeviceInfo info;
-  int st = current_device(&info);
-  if (st != NVFP4_OK) return st;
-  uint32_t* ws = nullptr;
-  st = stream_workspace(stream, &ws);
-  if (st != NVFP4_OK) return st;
-  const int64_t nvec = numel / 8;
-  int64_t blocks = (nvec + kThreads * 4 - 1) / (kThreads * 4);
-  blocks = blocks < 1 ? 1 : (blocks > info.sm_count * 8 ? info.sm_count * 8 : blocks);
-  return launch_kernel(amax_dense_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), 0, stream,
-                       static_cast<const uint16_t*>(x_bf16), numel, ws, amax_out, gsf_out, other_amax, alpha_out);
+  return launch_amax_dense(x_bf16, numel, amax_out, gsf_out, other_amax, alpha_out, stream);
 }
 
 int nvfp4_global_scale_batched(const void* x_bf16, int64_t b, int64_t m, int64_t k, const int32_t* mask,
