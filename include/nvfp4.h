@@ -62,7 +62,8 @@ enum nvfp4_status {
   NVFP4_ERR_UNSUPPORTED_DEVICE = 2, /* the current device is not compute capability 10.0 */
   NVFP4_ERR_CUDA = 3,             /* a CUDA runtime/driver call or a launch failed */
   NVFP4_ERR_DEVICE_TIMEOUT = 4,   /* a bounded device-side wait gave up (see nvfp4_device_status) */
-  NVFP4_ERR_OUT_OF_MEMORY = 5     /* the one-time workspace allocation failed */
+  NVFP4_ERR_OUT_OF_MEMORY = 5,    /* the one-time workspace allocation failed */
+  NVFP4_ERR_INDEX = 6             /* debug builds: a kernel computed an index outside its operand */
 };
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -399,6 +400,20 @@ NVFP4_API int nvfp4_device_status(int *status_out, int clear);
  * nvfp4_device_status (which re-zeroes it); the next call then computes correctly.
  */
 NVFP4_API int nvfp4_selftest_bounded_wait(nvfp4_stream_t stream);
+
+/*
+ * Debug builds (libnvfp4_debug.so, built with `python -m nvfp4_block_scaled_16_b200.build
+ * --debug`) check every global-memory index a kernel computes for a plain load or store (TMA
+ * transfers are bounded by their tensor maps) against the extent the call's arguments give the
+ * operand; an index out of range is not accessed and NVFP4_ERR_INDEX is recorded in the device
+ * status word (read it with nvfp4_device_status).  Release builds compile the checks away.
+ * nvfp4_debug_index_checks returns 1 in a debug build, 0 otherwise.
+ * nvfp4_selftest_index_check launches one thread that submits an index equal to its extent to
+ * the check: a debug build records NVFP4_ERR_INDEX, a release build records nothing.  No
+ * memory is accessed either way.  (The pages have no counterpart of these two calls.)
+ */
+NVFP4_API int nvfp4_debug_index_checks(void);
+NVFP4_API int nvfp4_selftest_index_check(nvfp4_stream_t stream);
 NVFP4_API int nvfp4_selftest_gemm_stall(const uint8_t *a, const uint8_t *b, const uint8_t *a_sf,
                                         const uint8_t *b_sf, const float *alpha, void *out_bf16, int64_t m,
                                         int64_t n, int64_t k, nvfp4_stream_t stream);

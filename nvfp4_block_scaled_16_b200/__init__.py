@@ -37,5 +37,7 @@ from .binding import (  # noqa: F401
     nvfp4_selftest_bounded_wait,
     nvfp4_selftest_gemm_stall,
     nvfp4_selftest_grid_barrier,
+    nvfp4_selftest_index_check,
+    nvfp4_debug_index_checks,
     nvfp4_device_status,
 )

@@ -38,6 +38,8 @@ EXPORTED_SYMBOLS = (
     "nvfp4_selftest_bounded_wait",
     "nvfp4_selftest_gemm_stall",
     "nvfp4_selftest_grid_barrier",
+    "nvfp4_debug_index_checks",
+    "nvfp4_selftest_index_check",
     "nvfp4_device_status",
 )
 
@@ -70,6 +72,8 @@ _SIGNATURES = {
     "nvfp4_selftest_bounded_wait": (_INT, [_P]),
     "nvfp4_selftest_gemm_stall": (_INT, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "nvfp4_selftest_grid_barrier": (_INT, [_P, _I64, _I64, _P, _P, _P, _P]),
+    "nvfp4_debug_index_checks": (_INT, []),
+    "nvfp4_selftest_index_check": (_INT, [_P]),
     "nvfp4_device_status": (_INT, [ctypes.POINTER(_INT), _INT]),
 }
 
@@ -81,7 +85,9 @@ class NVFP4Error(RuntimeError):
 
 
 def library_path() -> str:
-    return os.path.join(_HERE, "libnvfp4.so")
+    """libnvfp4.so, or with NVFP4_LIBRARY=debug the index-checking libnvfp4_debug.so."""
+    name = "libnvfp4_debug.so" if os.environ.get("NVFP4_LIBRARY") == "debug" else "libnvfp4.so"
+    return os.path.join(_HERE, name)
 
 
 def load_library():
@@ -90,7 +96,8 @@ def load_library():
     if _LIB is None:
         path = library_path()
         if not os.path.exists(path):
-            raise ImportError(f"{path} is missing; build it with `python -m nvfp4_block_scaled_16_b200.build`")
+            raise ImportError(f"{path} is missing; build it with `python -m nvfp4_block_scaled_16_b200.build`"
+                              + (" --debug" if path.endswith("_debug.so") else ""))
         lib = ctypes.CDLL(path)
         for name, (res, args) in _SIGNATURES.items():
             fn = getattr(lib, name)
@@ -431,6 +438,16 @@ def nvfp4_selftest_grid_barrier(x, stream=None):
         st = load_library().nvfp4_selftest_grid_barrier(_ptr(x), m, k, _ptr(gsf), _ptr(q), _ptr(sf), _stream(stream))
     _check("nvfp4_selftest_grid_barrier", st)
     return gsf, q, sf
+
+
+def nvfp4_debug_index_checks() -> bool:
+    """Whether the loaded library checks kernel indices (the debug build)."""
+    return bool(load_library().nvfp4_debug_index_checks())
+
+
+def nvfp4_selftest_index_check(stream=None):
+    """Submit one out-of-range index to the debug-build check (nothing is accessed)."""
+    _check("nvfp4_selftest_index_check", load_library().nvfp4_selftest_index_check(_stream(stream)))
 
 
 def nvfp4_device_status(clear: bool = True) -> int:

@@ -105,6 +105,21 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// Index checks of plain global loads and stores: in debug builds (-DNVFP4_DEBUG_INDEX) an
+// index at or beyond the operand's extent is reported as NVFP4_ERR_INDEX in the device status
+// word and the caller skips the access; release builds compile the check to `true`.
+#ifdef NVFP4_DEBUG_INDEX
+constexpr bool kDebugIndex = true;
+__device__ __forceinline__ bool index_ok(uint64_t index, uint64_t extent, int* status) {
+  if (index < extent) return true;
+  if (status) atomicExch(status, NVFP4_ERR_INDEX);   // (a kernel without a status word passes null)
+  return false;
+}
+#else
+constexpr bool kDebugIndex = false;
+__device__ __forceinline__ bool index_ok(uint64_t, uint64_t, int*) { return true; }
+#endif
+
 // cuTensorMapEncodeTiled, fetched from the driver through the runtime (no -lcuda).
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,

@@ -10,6 +10,11 @@
 namespace nvfp4 {
 namespace {
 
+// One index equal to its extent, submitted to the debug-build check (nothing is accessed).
+__global__ void index_check_selftest_kernel(int* status) {
+  if (threadIdx.x == 0) (void)index_ok(1, 1, status);
+}
+
 __global__ void silu_table_kernel(float* tab) {
   const uint32_t i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < kSiluEntries) tab[i] = silu_table_entry(i);
@@ -148,6 +153,7 @@ const char* nvfp4_status_string(int status) {
     case NVFP4_ERR_CUDA: return "NVFP4_ERR_CUDA";
     case NVFP4_ERR_DEVICE_TIMEOUT: return "NVFP4_ERR_DEVICE_TIMEOUT";
     case NVFP4_ERR_OUT_OF_MEMORY: return "NVFP4_ERR_OUT_OF_MEMORY";
+    case NVFP4_ERR_INDEX: return "NVFP4_ERR_INDEX";
     default: return "NVFP4_ERR_UNKNOWN";
   }
 }
@@ -157,6 +163,15 @@ int64_t nvfp4_scale_bytes(int64_t rows, int64_t k) {
   const int64_t rp = (rows + 127) / 128 * 128;
   const int64_t cp = (k / 16 + 3) / 4 * 4;
   return rp * cp;
+}
+
+int nvfp4_debug_index_checks(void) { return nvfp4::kDebugIndex ? 1 : 0; }
+
+int nvfp4_selftest_index_check(nvfp4_stream_t stream) {
+  nvfp4::DeviceInfo info;
+  int st = nvfp4::current_device(&info);
+  if (st != NVFP4_OK) return st;
+  return nvfp4::launch_kernel(nvfp4::index_check_selftest_kernel, dim3(1), dim3(32), 0, stream, info.status);
 }
 
 int nvfp4_set_pdl(int enable) {

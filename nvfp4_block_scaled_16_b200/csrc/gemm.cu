@@ -542,7 +542,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kQW>, 1)
             }
             uint4* dst = reinterpret_cast<uint4*>(q_row + part * (kCols / 2));
             uint8_t* sdst = sf_e + sf_offset(static_cast<uint32_t>(row), c0, groups);
-            if constexpr (kBlocks == 4) {
+            const bool in_range =
+                index_ok(static_cast<uint64_t>(reinterpret_cast<uint8_t*>(dst) - p.q) + kCols / 2 - 1,
+                         static_cast<uint64_t>(p.experts) * p.m * (p.n / 2), p.status) &&
+                index_ok(static_cast<uint64_t>(sdst - p.sf) + kBlocks - 1,
+                         static_cast<uint64_t>(p.experts) * p.sf_item_stride, p.status);
+            if (!in_range) {
+            } else if constexpr (kBlocks == 4) {
               dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
               dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
               *reinterpret_cast<uint32_t*>(sdst) = scales;
@@ -552,7 +558,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kQW>, 1)
             }
           } else if (pad_row) {
             uint8_t* sdst = sf_e + sf_offset(static_cast<uint32_t>(row), c0, groups);
-            if constexpr (kBlocks == 4) {
+            if (!index_ok(static_cast<uint64_t>(sdst - p.sf) + kBlocks - 1,
+                          static_cast<uint64_t>(p.experts) * p.sf_item_stride, p.status)) {
+            } else if constexpr (kBlocks == 4) {
               *reinterpret_cast<uint32_t*>(sdst) = 0u;
             } else {
               *reinterpret_cast<uint16_t*>(sdst) = 0;
@@ -584,7 +592,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kQW>, 1)
           uint4 bias8[8];                      // issued before the TMEM load to hide its latency
 #pragma unroll
           for (int g = 0; g < 8; ++g)
-            bias8[g] = (p.bias && col_base + 8 * g < p.n)
+            bias8[g] = (p.bias && col_base + 8 * g < p.n &&
+                        index_ok(static_cast<uint64_t>(col_base + 8 * g + 7), static_cast<uint64_t>(p.n), p.status))
                            ? __ldg(reinterpret_cast<const uint4*>(p.bias + col_base + 8 * g))
                            : make_uint4(0u, 0u, 0u, 0u);
           uint32_t v[64];
@@ -641,7 +650,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kQW>, 1)
           } else {
 #pragma unroll
             for (int g = 0; g < 8; ++g)
-              if (col_base + 8 * g < p.n) *reinterpret_cast<uint4*>(out_row + col_base + 8 * g) = o[g];
+              if (col_base + 8 * g < p.n &&
+                  index_ok(static_cast<uint64_t>(out_row + col_base + 8 * g - p.out) + 7,
+                           static_cast<uint64_t>(p.experts) * p.m * p.n, p.status))
+                *reinterpret_cast<uint4*>(out_row + col_base + 8 * g) = o[g];
           }
         }
       }

@@ -68,6 +68,7 @@ struct QuantParams {
   const float* silu_tab;   // SiLU table in global memory (SiLU variant)
   uint32_t chunks_per_item;
   uint32_t items;
+  int* status;             // device status word (debug-build index checks)
 };
 
 // Division by cpad (a multiple of 4) with the Granlund-Montgomery multiplier of 31-bit
@@ -130,6 +131,9 @@ __device__ __forceinline__ void chunk_load(const QuantParams& p, int item, uint3
     ch.r[u] = r;
     ch.c[u] = c;
     ch.live[u] = f < p.blocks && f < end && r < static_cast<uint32_t>(valid) && c < p.nb;
+    if (kDebugIndex && ch.live[u])    // the block's last element (of the up half with SiLU) lies in the item
+      ch.live[u] = index_ok(static_cast<uint64_t>(r) * p.x_row_stride + c * 16 + (kSilu ? p.k : 0) + 15,
+                            static_cast<uint64_t>(p.x_item_stride), p.status);
     if (ch.live[u]) {
       const uint16_t* src = x + static_cast<int64_t>(r) * p.x_row_stride + c * 16;
       ch.raw[u][0] = load_stream(src);
@@ -171,9 +175,11 @@ __device__ __forceinline__ void chunk_store(const QuantParams& p, const Chunk<kS
       if constexpr (kSmooth) {
         // x_hat = bf16(x * pre_quant_scale) for the block's 16 columns (the scale vector is
         // the same for every row: these loads hit in L1 / L2)
-        float sc[16];
-        unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(p.pqs + c * 16)), sc);
-        unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(p.pqs + c * 16 + 8)), sc + 8);
+        float sc[16] = {};
+        if (index_ok(c * 16 + 15, static_cast<uint64_t>(p.k), p.status)) {
+          unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(p.pqs + c * 16)), sc);
+          unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(p.pqs + c * 16 + 8)), sc + 8);
+        }
 #pragma unroll
         for (int i = 0; i < 16; i += 2) {
           float a, b;
@@ -185,14 +191,17 @@ __device__ __forceinline__ void chunk_store(const QuantParams& p, const Chunk<kS
         }
       }
       const QBlock b = quantize16(v, gsf, inv_tab);
-      *reinterpret_cast<uint2*>(q + static_cast<int64_t>(r) * (p.k / 2) + c * 8) = make_uint2(b.lo, b.hi);
-      sf[sf_offset(r, c, groups)] = static_cast<uint8_t>(b.s8);
+      const int64_t qo = static_cast<int64_t>(r) * (p.k / 2) + c * 8, so = sf_offset(r, c, groups);
+      if (index_ok(qo + 7, static_cast<uint64_t>(p.q_item_stride), p.status))
+        *reinterpret_cast<uint2*>(q + qo) = make_uint2(b.lo, b.hi);
+      if (index_ok(so, static_cast<uint64_t>(p.sf_item_stride), p.status)) sf[so] = static_cast<uint8_t>(b.s8);
     } else if (ch.base + u * kThreads + threadIdx.x < min(p.blocks, ch.end)) {
       // Padding scale entries: a column beyond the last block of a valid row, or (no mask)
       // a padding row below m.
       const bool pad_col = r < static_cast<uint32_t>(ch.valid) && c >= p.nb;
       const bool pad_row = p.mask == nullptr && r >= static_cast<uint32_t>(p.m);
-      if (pad_col || pad_row) sf[sf_offset(r, c, groups)] = 0;
+      if ((pad_col || pad_row) && index_ok(sf_offset(r, c, groups), static_cast<uint64_t>(p.sf_item_stride), p.status))
+        sf[sf_offset(r, c, groups)] = 0;
     }
   }
 }
@@ -255,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, kPersistCtasPerSm) persistent_quanti
 
 // h[r, c] = bf16(silu(x[r, c]) * x[r, k + c]) for rows of width 2k; 8 outputs per thread.
 __global__ void __launch_bounds__(kThreads) silu_and_mul_kernel(const uint16_t* x, int64_t rows, int32_t k,
-                                                                uint16_t* h, const float* silu_tab) {
+                                                                uint16_t* h, const float* silu_tab, int* status) {
   extern __shared__ float4 silu_smem[];
   float* tab = reinterpret_cast<float*>(silu_smem);
   pdl_launch_dependents();
@@ -268,6 +277,9 @@ __global__ void __launch_bounds__(kThreads) silu_and_mul_kernel(const uint16_t* 
        i += static_cast<int64_t>(gridDim.x) * kThreads) {
     const int64_t r = i / per_row;
     const int64_t c = (i - r * per_row) * 8;
+    if (!index_ok(r * 2 * k + k + c + 7, static_cast<uint64_t>(rows) * 2 * k, status) ||
+        !index_ok(r * k + c + 7, static_cast<uint64_t>(rows) * k, status))
+      continue;
     float u[8], o[8];
     const uint4 g = load_stream(x + r * 2 * k + c);
     unpack_bf16x8(load_stream(x + r * 2 * k + k + c), u);
@@ -336,7 +348,7 @@ __device__ void reduce_and_finalize(float local, uint32_t* ws, int item, int ite
 
 __global__ void __launch_bounds__(kThreads) amax_dense_kernel(const uint16_t* x, int64_t numel, uint32_t* ws,
                                                               float* amax_out, float* gsf_out,
-                                                              const float* other_amax, float* alpha_out) {
+                                                              const float* other_amax, float* alpha_out, int* status) {
   pdl_launch_dependents();
   pdl_wait();
   float m = 0.0f;
@@ -344,13 +356,15 @@ __global__ void __launch_bounds__(kThreads) amax_dense_kernel(const uint16_t* x,
   const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
   int64_t i = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
   for (; i + 3 * stride < nvec; i += 4 * stride) {
+    if (!index_ok(8 * (i + 3 * stride) + 7, static_cast<uint64_t>(numel), status)) break;
     const uint4 a = load_stream(x + 8 * i);
     const uint4 b = load_stream(x + 8 * (i + stride));
     const uint4 c = load_stream(x + 8 * (i + 2 * stride));
     const uint4 d = load_stream(x + 8 * (i + 3 * stride));
     m = absmax8(a, m); m = absmax8(b, m); m = absmax8(c, m); m = absmax8(d, m);
   }
-  for (; i < nvec; i += stride) m = absmax8(load_stream(x + 8 * i), m);
+  for (; i < nvec; i += stride)
+    if (index_ok(8 * i + 7, static_cast<uint64_t>(numel), status)) m = absmax8(load_stream(x + 8 * i), m);
   if (blockIdx.x == 0 && threadIdx.x < numel - 8 * nvec) {
     const float t = __uint_as_float(static_cast<uint32_t>(x[8 * nvec + threadIdx.x]) << 16);
     m = fmaxf(m, fabsf(t));
@@ -363,7 +377,7 @@ __global__ void __launch_bounds__(kThreads) amax_dense_kernel(const uint16_t* x,
 template <bool kSilu>
 __global__ void __launch_bounds__(kThreads) amax_batched_kernel(const uint16_t* x, int32_t m, int32_t k,
                                                                 const int32_t* mask, uint32_t* ws,
-                                                                float* amax_out, float* gsf_out) {
+                                                                float* amax_out, float* gsf_out, int* status) {
   pdl_launch_dependents();
   pdl_wait();
   const int item = blockIdx.y;
@@ -378,6 +392,7 @@ __global__ void __launch_bounds__(kThreads) amax_batched_kernel(const uint16_t* 
     if constexpr (kSilu) {
       const int64_t r = i / per_row;
       const int64_t c = (i - r * per_row) * 8;
+      if (!index_ok(r * width + k + c + 7, static_cast<uint64_t>(m) * width, status)) continue;
       const uint4 g = load_stream(xi + r * width + c);
       const uint4 u = load_stream(xi + r * width + k + c);
       float gf[8], uf[8];
@@ -385,7 +400,7 @@ __global__ void __launch_bounds__(kThreads) amax_batched_kernel(const uint16_t* 
       unpack_bf16x8(u, uf);
 #pragma unroll
       for (int j = 0; j < 8; ++j) mx = fmaxf(mx, fabsf(silu_mul_bf16(gf[j], uf[j])));
-    } else {
+    } else if (index_ok(8 * i + 7, static_cast<uint64_t>(m) * width, status)) {
       mx = absmax8(load_stream(xi + 8 * i), mx);
     }
   }
@@ -666,15 +681,18 @@ __global__ void __launch_bounds__(kGsqThreads, 1)
         gsq_read_half(smem_u32(ring) + s * kGsqSlotBytes, t, c);
         const QBlock b0 = gsq_block(c[0], c[1], gsf, inv_tab);
         const QBlock b1 = gsq_block(c[2], c[3], gsf, inv_tab);
-        *reinterpret_cast<uint4*>(p.q + static_cast<int64_t>(g) * 32 + (t & 1) * 16) =
-            make_uint4(b0.lo, b0.hi, b1.lo, b1.hi);
+        if (index_ok(static_cast<uint64_t>(g) * 32 + (t & 1) * 16 + 15, static_cast<uint64_t>(p.groups_total) * 32,
+                     status))
+          *reinterpret_cast<uint4*>(p.q + static_cast<int64_t>(g) * 32 + (t & 1) * 16) =
+              make_uint4(b0.lo, b0.hi, b1.lo, b1.hi);
         scales = b0.s8 | (b1.s8 << 8);
       }
       const uint32_t other = __shfl_xor_sync(0xffffffffu, scales, 1);
       if (g < g_hi && (t & 1) == 0) {
         const uint32_t r = static_cast<uint32_t>((static_cast<uint64_t>(g) * p.nb4_magic) >> p.nb4_shift);
         const uint32_t c0 = (g - r * groups4) * 4;
-        *reinterpret_cast<uint32_t*>(p.sf + sf_offset(r, c0, groups4)) = scales | (other << 16);
+        if (index_ok(sf_offset(r, c0, groups4) + 3, static_cast<uint64_t>(p.rows_pad) * groups4 * 4, status))
+          *reinterpret_cast<uint32_t*>(p.sf + sf_offset(r, c0, groups4)) = scales | (other << 16);
       }
       __syncwarp();
       if ((t & 31) == 0) mbar_arrive(&empty[s]);
@@ -683,7 +701,8 @@ __global__ void __launch_bounds__(kGsqThreads, 1)
     const uint32_t pad_words = (p.rows_pad - p.m) * groups4;
     for (uint32_t i = blockIdx.x * kGsqCompute + t; i < pad_words; i += grid * kGsqCompute) {
       const uint32_t r = p.m + i / groups4;
-      *reinterpret_cast<uint32_t*>(p.sf + sf_offset(r, (i % groups4) * 4, groups4)) = 0u;
+      if (index_ok(sf_offset(r, (i % groups4) * 4, groups4) + 3, static_cast<uint64_t>(p.rows_pad) * groups4 * 4, status))
+        *reinterpret_cast<uint32_t*>(p.sf + sf_offset(r, (i % groups4) * 4, groups4)) = 0u;
     }
   }
 }
@@ -708,7 +727,8 @@ int launch_amax_dense(const void* x_bf16, int64_t numel, float* amax_out, float*
   int64_t blocks = (nvec + kThreads * 4 - 1) / (kThreads * 4);
   blocks = blocks < 1 ? 1 : (blocks > info.sm_count * 8 ? info.sm_count * 8 : blocks);
   return launch_kernel(amax_dense_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), 0, stream,
-                       static_cast<const uint16_t*>(x_bf16), numel, ws, amax_out, gsf_out, other_amax, alpha_out);
+                       static_cast<const uint16_t*>(x_bf16), numel, ws, amax_out, gsf_out, other_amax, alpha_out,
+                       info.status);
 }
 
 int launch_quantize(const void* x, int64_t b, int64_t m, int64_t k, bool silu, const int32_t* mask,
@@ -746,6 +766,7 @@ int launch_quantize(const void* x, int64_t b, int64_t m, int64_t k, bool silu, c
   set_cpad_divisor(p);
   p.silu_tab = info.silu_table;
   p.items = static_cast<uint32_t>(b);
+  p.status = info.status;
   if (silu || mask) {
     // persistent grid over the chunks of all items
     const int U = silu ? kPersistUnroll<true> : kPersistUnroll<false>;
@@ -874,7 +895,8 @@ int nvfp4_global_scale_batched(const void* x_bf16, int64_t b, int64_t m, int64_t
   dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(b));
   const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
   return launch_kernel(silu_mul ? amax_batched_kernel<true> : amax_batched_kernel<false>, grid, dim3(kThreads), 0,
-                       stream, x, static_cast<int32_t>(m), static_cast<int32_t>(k), mask, ws, amax_out, gsf_out);
+                       stream, x, static_cast<int32_t>(m), static_cast<int32_t>(k), mask, ws, amax_out, gsf_out,
+                       info.status);
 }
 
 int nvfp4_quantize(const void* x_bf16, int64_t m, int64_t k, const float* gsf, uint8_t* q_out, uint8_t* sf_out,
@@ -894,7 +916,7 @@ int nvfp4_silu_and_mul(const void* x_bf16, int64_t rows, int64_t k, void* h_bf16
   blocks = blocks > info.sm_count * 4 ? info.sm_count * 4 : blocks;
   return launch_kernel(silu_and_mul_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), kSiluTableBytes,
                        stream, static_cast<const uint16_t*>(x_bf16), rows, static_cast<int32_t>(k),
-                       static_cast<uint16_t*>(h_bf16), info.silu_table);
+                       static_cast<uint16_t*>(h_bf16), info.silu_table, info.status);
 }
 
 int nvfp4_quantize_smooth(const void* x_bf16, int64_t m, int64_t k, const void* pre_quant_scale_bf16,
@@ -1009,5 +1031,6 @@ extern "C" int nvfp4_global_scale_batched_noalloc(const void* x_bf16, int64_t b,
   dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(b));
   const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
   return launch_kernel(silu_mul ? amax_batched_kernel<true> : amax_batched_kernel<false>, grid, dim3(kThreads), 0,
-                       stream, x, static_cast<int32_t>(m), static_cast<int32_t>(k), mask, scratch, amax_out, gsf_out);
+                       stream, x, static_cast<int32_t>(m), static_cast<int32_t>(k), mask, scratch, amax_out, gsf_out,
+                       static_cast<int*>(nullptr));
 }

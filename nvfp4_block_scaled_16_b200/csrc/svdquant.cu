@@ -293,7 +293,12 @@ __global__ void __cluster_dims__(kSvdSplit, 1, 1) __launch_bounds__(kSvdThreads,
             scales |= qb.s8 << (8 * blk);
           }
           uint8_t* qdst = p.q + static_cast<int64_t>(grow) * (p.k / 2) + kc / 2 + 8 * b0;
-          if constexpr (kSvdBlocksPerThread == 4) {
+          const bool in_range =
+              index_ok(static_cast<uint64_t>(qdst - p.q) + 8 * kSvdBlocksPerThread - 1,
+                       static_cast<uint64_t>(p.m) * (p.k / 2), p.status) &&
+              index_ok(sf_word + kSvdBlocksPerThread - 1, static_cast<uint64_t>(p.rows_pad) * (p.k / 16), p.status);
+          if (!in_range) {
+          } else if constexpr (kSvdBlocksPerThread == 4) {
             reinterpret_cast<uint4*>(qdst)[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
             reinterpret_cast<uint4*>(qdst)[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
             *reinterpret_cast<uint32_t*>(p.sf + sf_word) = scales;
@@ -305,7 +310,8 @@ __global__ void __cluster_dims__(kSvdSplit, 1, 1) __launch_bounds__(kSvdThreads,
             p.sf[sf_word] = static_cast<uint8_t>(scales);
           }
         } else if (grow < p.rows_pad) {
-          if constexpr (kSvdBlocksPerThread == 4) {
+          if (!index_ok(sf_word + kSvdBlocksPerThread - 1, static_cast<uint64_t>(p.rows_pad) * (p.k / 16), p.status)) {
+          } else if constexpr (kSvdBlocksPerThread == 4) {
             *reinterpret_cast<uint32_t*>(p.sf + sf_word) = 0u;
           } else if constexpr (kSvdBlocksPerThread == 2) {
             *reinterpret_cast<uint16_t*>(p.sf + sf_word) = 0;
@@ -364,6 +370,7 @@ __global__ void __cluster_dims__(kSvdSplit, 1, 1) __launch_bounds__(kSvdThreads,
     if (grow < p.m) {
       __nv_bfloat16* drow = p.d + static_cast<int64_t>(grow) * p.r + col0;
       for (int j = 0; j < cols; j += 4) {
+        if (!index_ok(static_cast<uint64_t>(drow + j - p.d) + 3, static_cast<uint64_t>(p.m) * p.r, p.status)) continue;
         float acc[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {

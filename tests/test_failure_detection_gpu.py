@@ -14,6 +14,7 @@ from tests.helpers import assert_gemm_close, bf16_to_f64, dev_bf16, dev_f32, dev
 pytestmark = pytest.mark.gpu
 
 NVFP4_ERR_DEVICE_TIMEOUT = 4
+NVFP4_ERR_INDEX = 6
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -65,3 +66,13 @@ def test_grid_barrier_timeout_writes_nothing_and_recovers(oracle):
     assert nv.nvfp4_device_status(clear=True) == 0
     assert host(g2)[0] == gsf_o
     assert (host(q2) == q_o).all() and (host(s2) == sf_o).all()
+
+
+def test_index_check_records_an_error_in_debug_builds_only():
+    # One index equal to its extent goes through the check (nothing is accessed): the debug
+    # build (NVFP4_LIBRARY=debug) records NVFP4_ERR_INDEX, the release build compiles the
+    # check away and records nothing.
+    assert nv.nvfp4_device_status(clear=True) == 0
+    nv.nvfp4_selftest_index_check()
+    want = NVFP4_ERR_INDEX if nv.nvfp4_debug_index_checks() else 0
+    assert nv.nvfp4_device_status(clear=True) == want

@@ -51,7 +51,13 @@ def test_status_strings(lib):
     assert nv.nvfp4_status_string(0) == "NVFP4_OK"
     assert nv.nvfp4_status_string(1) == "NVFP4_ERR_INVALID_ARGUMENT"
     assert nv.nvfp4_status_string(4) == "NVFP4_ERR_DEVICE_TIMEOUT"
+    assert nv.nvfp4_status_string(6) == "NVFP4_ERR_INDEX"
     assert nv.nvfp4_status_string(99) == "NVFP4_ERR_UNKNOWN"
+
+
+def test_release_library_has_no_index_checks(lib):
+    # the default library is the release build; the debug build reports its checks
+    assert nv.nvfp4_debug_index_checks() is (nv.library_path().endswith("_debug.so"))
 
 
 P = ctypes.c_void_p
