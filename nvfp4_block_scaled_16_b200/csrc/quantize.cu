@@ -68,8 +68,16 @@ struct QuantParams {
   const float* silu_tab;   // SiLU table in global memory (SiLU variant)
   uint32_t chunks_per_item;
   uint32_t items;
-  int* status;             // device status word (debug-build index checks)
+#ifdef NVFP4_DEBUG_INDEX
+  int* status;             // device status word (debug-build index checks; the member alone
+                           // costs the persistent quantizer a register spill in release builds)
+#endif
 };
+#ifdef NVFP4_DEBUG_INDEX
+#define QSTATUS(p) ((p).status)
+#else
+#define QSTATUS(p) static_cast<int*>(nullptr)
+#endif
 
 // Division by cpad (a multiple of 4) with the Granlund-Montgomery multiplier of 31-bit
 // dividends: with l = ceil(log2 cpad) and m = ceil(2^(31+l) / cpad), floor(f / cpad) =
@@ -133,7 +141,7 @@ __device__ __forceinline__ void chunk_load(const QuantParams& p, int item, uint3
     ch.live[u] = f < p.blocks && f < end && r < static_cast<uint32_t>(valid) && c < p.nb;
     if (kDebugIndex && ch.live[u])    // the block's last element (of the up half with SiLU) lies in the item
       ch.live[u] = index_ok(static_cast<uint64_t>(r) * p.x_row_stride + c * 16 + (kSilu ? p.k : 0) + 15,
-                            static_cast<uint64_t>(p.x_item_stride), p.status);
+                            static_cast<uint64_t>(p.x_item_stride), QSTATUS(p));
     if (ch.live[u]) {
       const uint16_t* src = x + static_cast<int64_t>(r) * p.x_row_stride + c * 16;
       ch.raw[u][0] = load_stream(src);
@@ -176,7 +184,7 @@ __device__ __forceinline__ void chunk_store(const QuantParams& p, const Chunk<kS
         // x_hat = bf16(x * pre_quant_scale) for the block's 16 columns (the scale vector is
         // the same for every row: these loads hit in L1 / L2)
         float sc[16] = {};
-        if (index_ok(c * 16 + 15, static_cast<uint64_t>(p.k), p.status)) {
+        if (index_ok(c * 16 + 15, static_cast<uint64_t>(p.k), QSTATUS(p))) {
           unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(p.pqs + c * 16)), sc);
           unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(p.pqs + c * 16 + 8)), sc + 8);
         }
@@ -192,15 +200,15 @@ __device__ __forceinline__ void chunk_store(const QuantParams& p, const Chunk<kS
       }
       const QBlock b = quantize16(v, gsf, inv_tab);
       const int64_t qo = static_cast<int64_t>(r) * (p.k / 2) + c * 8, so = sf_offset(r, c, groups);
-      if (index_ok(qo + 7, static_cast<uint64_t>(p.q_item_stride), p.status))
+      if (index_ok(qo + 7, static_cast<uint64_t>(p.q_item_stride), QSTATUS(p)))
         *reinterpret_cast<uint2*>(q + qo) = make_uint2(b.lo, b.hi);
-      if (index_ok(so, static_cast<uint64_t>(p.sf_item_stride), p.status)) sf[so] = static_cast<uint8_t>(b.s8);
+      if (index_ok(so, static_cast<uint64_t>(p.sf_item_stride), QSTATUS(p))) sf[so] = static_cast<uint8_t>(b.s8);
     } else if (ch.base + u * kThreads + threadIdx.x < min(p.blocks, ch.end)) {
       // Padding scale entries: a column beyond the last block of a valid row, or (no mask)
       // a padding row below m.
       const bool pad_col = r < static_cast<uint32_t>(ch.valid) && c >= p.nb;
       const bool pad_row = p.mask == nullptr && r >= static_cast<uint32_t>(p.m);
-      if ((pad_col || pad_row) && index_ok(sf_offset(r, c, groups), static_cast<uint64_t>(p.sf_item_stride), p.status))
+      if ((pad_col || pad_row) && index_ok(sf_offset(r, c, groups), static_cast<uint64_t>(p.sf_item_stride), QSTATUS(p)))
         sf[sf_offset(r, c, groups)] = 0;
     }
   }
@@ -766,7 +774,9 @@ int launch_quantize(const void* x, int64_t b, int64_t m, int64_t k, bool silu, c
   set_cpad_divisor(p);
   p.silu_tab = info.silu_table;
   p.items = static_cast<uint32_t>(b);
+#ifdef NVFP4_DEBUG_INDEX
   p.status = info.status;
+#endif
   if (silu || mask) {
     // persistent grid over the chunks of all items
     const int U = silu ? kPersistUnroll<true> : kPersistUnroll<false>;
