@@ -231,6 +231,38 @@ NVFP4_API int nvfp4_gemm_bf16a(const void *a_bf16, const uint8_t *b, const uint8
                                float *scalars_ws, int64_t m, int64_t n, int64_t k, nvfp4_stream_t stream);
 
 /*
+ * bf16-activation NVFP4 linear with a static activation scale [NVF
+ * f16a_nvfp4weight_scaled_mm: bf16 activation, NVFP4 weight, bf16 [M, N] out, which the
+ * compiler path runs as the activation's block quantization and the scaled FP4 matmul; TRT
+ * create_weights: a calibrated input_scale for the activation]:
+ *   out = nvfp4_gemm(quantize(a, a_gsf), b, alpha)
+ *   a_bf16     [m, k] bf16, 16-byte aligned; k % 64 == 0, n % 8 == 0.
+ *   b, b_sf    the NVFP4 weight [n, k/2] and its scales, as in nvfp4_gemm.
+ *   a_gsf      fp32 [1] device: the activation's static global scale (448*6 / calibrated amax).
+ *   alpha      fp32 [1] device: calibrated amax_a * amax_b / (448*6)^2.
+ *   bias_bf16  nullable bf16 [n]; out_bf16 bf16 [m, n] as in nvfp4_gemm.
+ *   a_q_ws     caller workspace uint8 [m, k/2] (16-byte aligned): receives the quantized
+ *              activation, equal to nvfp4_quantize(a_bf16, a_gsf) bit for bit.
+ *   a_sf_ws    caller workspace uint8 [nvfp4_scale_bytes(m, k)] (16-byte aligned), likewise.
+ *   one_launch 0: nvfp4_quantize then nvfp4_gemm on `stream` (the faster form on B200).
+ *              1: one GEMM launch whose epilogue warps, before draining any accumulator,
+ *              quantize a share of the activation (128-row slab x 256-column K chunk units,
+ *              K chunks first) into the workspace and count each finished chunk; a CTA's TMA
+ *              producer loads chunk c of A only after every slab's chunk c is counted.  Needs
+ *              k <= 16384; uses the stream's reduction workspace (allocated on its first use)
+ *              for the chunk counters and leaves it zeroed.  Every CTA of the grid (one 2-CTA
+ *              cluster per pair of SMs) must be resident at once, as the persistent GEMM's
+ *              grid is when nothing else holds the SMs; a counter wait that runs out (1 s)
+ *              records NVFP4_ERR_DEVICE_TIMEOUT.
+ * Both forms give the same bytes.  With n = 0 only the workspace is written (nvfp4_quantize);
+ * every argument is checked before anything is launched, so an invalid call writes nothing.
+ */
+NVFP4_API int nvfp4_gemm_bf16a_static(const void *a_bf16, const uint8_t *b, const uint8_t *b_sf, const float *a_gsf,
+                                      const float *alpha, const void *bias_bf16, void *out_bf16, uint8_t *a_q_ws,
+                                      uint8_t *a_sf_ws, int64_t m, int64_t n, int64_t k, int one_launch,
+                                      nvfp4_stream_t stream);
+
+/*
  * Masked grouped GEMM for MoE experts [FI3: inputs for grouped_gemm_nt_masked; NVF
  * routed_experts GroupedLinear].  For every expert e and row i < mask[e]:
  *   out[e, i, :] = bf16(alpha[e] * a[e, i, :] @ b[e]^T)

@@ -24,6 +24,7 @@ from .binding import (  # noqa: F401
     nvfp4_silu_mul_quantize_batched,
     nvfp4_gemm,
     nvfp4_gemm_bf16a,
+    nvfp4_gemm_bf16a_static,
     nvfp4_grouped_gemm_masked,
     nvfp4_gemm_lowrank_bias,
     nvfp4_gemm_silu_mul_quantize,

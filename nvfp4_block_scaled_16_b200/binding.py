@@ -25,6 +25,7 @@ EXPORTED_SYMBOLS = (
     "nvfp4_silu_mul_quantize_batched",
     "nvfp4_gemm",
     "nvfp4_gemm_bf16a",
+    "nvfp4_gemm_bf16a_static",
     "nvfp4_grouped_gemm_masked",
     "nvfp4_gemm_lowrank_bias",
     "nvfp4_gemm_silu_mul_quantize",
@@ -59,6 +60,7 @@ _SIGNATURES = {
     "nvfp4_silu_mul_quantize_batched": (_INT, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P]),
     "nvfp4_gemm": (_INT, [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "nvfp4_gemm_bf16a": (_INT, [_P] * 9 + [_I64, _I64, _I64, _P]),
+    "nvfp4_gemm_bf16a_static": (_INT, [_P] * 9 + [_I64, _I64, _I64, _INT, _P]),
     "nvfp4_grouped_gemm_masked": (_INT, [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P]),
     "nvfp4_gemm_lowrank_bias": (_INT, [_P, _P, _P, _P, _P, _P, _P, _I64, _P, _P, _I64, _I64, _I64, _P]),
     "nvfp4_gemm_silu_mul_quantize": (_INT, [_P] * 11 + [_I64, _I64, _I64, _P]),
@@ -275,6 +277,25 @@ def nvfp4_gemm_bf16a(a, b, b_sf, b_amax, bias=None, out=None, a_q_ws=None, a_sf_
                                              _ptr(a_q_ws), _ptr(a_sf_ws), _ptr(scalars_ws), m, n, k, _stream(stream))
     _check("nvfp4_gemm_bf16a", st)
     return out, a_q_ws, a_sf_ws, scalars_ws
+
+
+def nvfp4_gemm_bf16a_static(a, b, b_sf, a_gsf, alpha, bias=None, out=None, a_q_ws=None, a_sf_ws=None, one_launch=False,
+                            stream=None):
+    """bf16 activation a [m, k] x NVFP4 weight b [n, k/2] with a static activation scale a_gsf [1]
+    -> (out [m, n] bf16, a_q [m, k/2], a_sf); one_launch picks the fused single-kernel form."""
+    m, k = a.shape
+    n = b.shape[0]
+    dev = a.device
+    out = torch.empty((m, n), dtype=torch.bfloat16, device=dev) if out is None else out
+    a_q_ws = torch.empty((m, k // 2), dtype=torch.uint8, device=dev) if a_q_ws is None else a_q_ws
+    if a_sf_ws is None:
+        a_sf_ws = torch.empty(max(nvfp4_scale_bytes(m, k), 0), dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        st = load_library().nvfp4_gemm_bf16a_static(_ptr(a), _ptr(b), _ptr(b_sf), _ptr(a_gsf), _ptr(alpha), _ptr(bias),
+                                                    _ptr(out), _ptr(a_q_ws), _ptr(a_sf_ws), m, n, k, int(one_launch),
+                                                    _stream(stream))
+    _check("nvfp4_gemm_bf16a_static", st)
+    return out, a_q_ws, a_sf_ws
 
 
 def nvfp4_grouped_gemm_masked(a, b, a_sf, b_sf, mask, alpha, out=None, stream=None):

@@ -44,6 +44,13 @@ int kernel_setup(const void* kernel, int device, const std::function<int(int*)>&
 // Whether kernels are launched with programmatic dependent launch (nvfp4_set_pdl).
 bool pdl_enabled();
 
+// The dense GEMM whose epilogue warps first quantize the bf16 activation a_bf16 [m, k] with
+// the static global scale a_gsf into a_q_ws / a_sf_ws, from which its producers load A chunk
+// by chunk (gemm.cu).  Checks its own arguments; k <= 16384.
+int gemm_quantize_a(const void* a_bf16, const uint8_t* b, const uint8_t* b_sf, const float* a_gsf, const float* alpha,
+                    const void* bias_bf16, void* out_bf16, uint8_t* a_q_ws, uint8_t* a_sf_ws, int64_t m, int64_t n,
+                    int64_t k, cudaStream_t stream);
+
 // Launches `kernel` on `stream`, with the programmatic-stream-serialization attribute when
 // PDL is enabled: the kernel may then start while its predecessor in the stream finishes,
 // and every kernel of this library waits (griddepcontrol.wait) before its first global

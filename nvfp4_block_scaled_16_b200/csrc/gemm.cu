@@ -118,18 +118,22 @@ constexpr int kStagingBytes = kStagingBuffers<kGrouped, kSwiGLU, kQW> * kEpiWarp
 // SiLU * up epilogue: the SiLU table (32 KB) after the ring.
 template <bool kSwiGLU>
 constexpr int kTableBytes = kSwiGLU ? static_cast<int>(kSiluTableBytes) : 0;
-// The expert prefix table (the last member of Control) is only allocated for grouped kernels.
-template <bool kGrouped>
-constexpr int kControlBytes = kGrouped ? static_cast<int>(sizeof(Control))
-                                       : static_cast<int>(offsetof(Control, prefix)) + 8;
-template <bool kGrouped, bool kSwiGLU, int kQW>
+// The expert prefix table (the last member of Control) is only allocated for grouped kernels;
+// the fused activation quantizer keeps its 128 inverse block scales in its first 512 bytes.
+template <bool kGrouped, bool kQuantA = false>
+constexpr int kControlBytes = kGrouped  ? static_cast<int>(sizeof(Control))
+                              : kQuantA ? static_cast<int>(offsetof(Control, prefix)) + 512
+                                        : static_cast<int>(offsetof(Control, prefix)) + 8;
+template <bool kGrouped, bool kSwiGLU, int kQW, bool kQuantA = false>
 constexpr int kSmemBytes = kStages * kStageBytes + kStagingBytes<kGrouped, kSwiGLU, kQW> + kTableBytes<kSwiGLU> +
-                           kControlBytes<kGrouped> + 1024;
+                           kControlBytes<kGrouped, kQuantA> + 1024;
 constexpr int kMaxDynamicSmem = 227 * 1024;      // sm_100 opt-in limit per block
 static_assert(kSmemBytes<false, false, 1> <= kMaxDynamicSmem && kSmemBytes<false, false, 2> <= kMaxDynamicSmem &&
                   kSmemBytes<true, false, 1> <= kMaxDynamicSmem && kSmemBytes<false, true, 2> <= kMaxDynamicSmem &&
-                  kSmemBytes<true, true, 2> <= kMaxDynamicSmem,
+                  kSmemBytes<true, true, 2> <= kMaxDynamicSmem && kSmemBytes<false, false, 1, true> <= kMaxDynamicSmem &&
+                  kSmemBytes<false, false, 2, true> <= kMaxDynamicSmem,
               "shared memory layout exceeds the per-block limit");
+constexpr int kQuantAMaxChunks = 64;             // fused activation quantizer: k <= 64 * 256
 
 // Instruction descriptors (tcgen05 "instruction descriptor" bit fields).
 //   kind::mxf4nvf4: A/B format E2M1 (1) at bits 7..9 / 10..12, both K-major, N>>3 at
@@ -235,6 +239,14 @@ struct GemmParams {
   int32_t stall_stage;        // self-test only: K stage of each pair's first tile whose loads
                               // are withheld, so a bounded wait runs out (-1: none)
   const float* silu_tab;      // SiLU * up epilogue: the SiLU table in global memory
+  // fused activation quantizer (the bf16-activation linear with a static activation scale):
+  // A is x quantized with qa_gsf into qa_q / qa_sf (which the A and SFA tensor maps read)
+  const uint16_t* qa_x;       // [m, k] bf16
+  const float* qa_gsf;        // [1] static global scale of x
+  uint8_t* qa_q;              // [m, k/2]
+  uint8_t* qa_sf;             // [nvfp4_scale_bytes(m, k)]
+  uint32_t* qa_ws;            // stream workspace: [0] CTAs finished, [1 + c] 128-row slabs of K chunk c done
+  int32_t qa_slabs;           // ceil(m / 128)
 };
 
 struct TileCoord {
@@ -270,11 +282,99 @@ struct Maps {
   CUtensorMap out;            // bf16 output [E, mmax, n], boxes of 32 rows x 64 columns
 };
 
+// ---- fused activation quantizer ------------------------------------------------------------------
+// The work is split into units of one 128-row slab x one 256-column K chunk of x (2048 blocks
+// of 16 values), numbered chunk-major (u = c * slabs + s), so that every slab's early chunks are
+// ready first; CTA j quantizes units j, j + grid, ... with its epilogue warps before they drain
+// any accumulator, and counts each finished unit in qa_ws[1 + c] with release semantics.  A
+// producer loads chunk c of a slab only after it has seen qa_ws[1 + c] == slabs (acquire), and
+// remembers the chunks it has seen.
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+// orders this thread's generic-proxy global accesses with its async-proxy (TMA) ones
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
+// Quantizes this CTA's units with the kEpi epilogue threads (t = thread index among them):
+// item i = it * kEpi + t of a unit is row i / 16, block i % 16 of the chunk, so a warp reads
+// two rows' 512 contiguous bytes and writes their 128 contiguous code bytes; the four blocks
+// of a scale group sit in adjacent lanes and one of them writes the group's 4-byte word.
+template <int kEpi>
+__device__ void quantize_a_units(const GemmParams& p, int t, float* inv_tab) {
+  constexpr int kItems = 2048 / kEpi;            // items per thread and unit
+  constexpr int kBatch = kItems < 8 ? kItems : 8; // loads in flight per thread
+  const float gsf = __ldg(p.qa_gsf);
+  if (t < 128) inv_tab[t] = inv_scale(static_cast<uint32_t>(t), gsf);
+  asm volatile("bar.sync 1, %0;" ::"n"(kEpi) : "memory");
+  const int nb = p.k / 16;
+  const uint32_t groups = static_cast<uint32_t>(p.sf_groups);
+  const int units = p.qa_slabs * p.k_stages;
+  const int lane = t & 31;
+  for (int u = blockIdx.x; u < units; u += gridDim.x) {
+    const int c = u / p.qa_slabs, slab = u - c * p.qa_slabs;
+    const int nblk = min(16, nb - 16 * c);       // blocks of this chunk in a row (a multiple of 4)
+    for (int it0 = 0; it0 < kItems; it0 += kBatch) {
+      uint4 raw[kBatch][2];
+#pragma unroll
+      for (int b = 0; b < kBatch; ++b) {
+        const int i = (it0 + b) * kEpi + t;
+        const int row = slab * 128 + i / 16, blk = i % 16;
+        if (row < p.m && blk < nblk &&
+            index_ok(static_cast<uint64_t>(row) * p.k + (16 * c + blk) * 16 + 15, static_cast<uint64_t>(p.m) * p.k,
+                     p.status)) {
+          const uint16_t* src = p.qa_x + static_cast<int64_t>(row) * p.k + (16 * c + blk) * 16;
+          raw[b][0] = __ldg(reinterpret_cast<const uint4*>(src));
+          raw[b][1] = __ldg(reinterpret_cast<const uint4*>(src + 8));
+        } else {
+          raw[b][0] = raw[b][1] = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < kBatch; ++b) {
+        const int i = (it0 + b) * kEpi + t;
+        const int row = slab * 128 + i / 16, blk = i % 16;
+        float v[16];
+        const uint32_t w[8] = {raw[b][0].x, raw[b][0].y, raw[b][0].z, raw[b][0].w,
+                               raw[b][1].x, raw[b][1].y, raw[b][1].z, raw[b][1].w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          v[2 * e] = bf16_lo(w[e]);
+          v[2 * e + 1] = bf16_hi(w[e]);
+        }
+        const QBlock qb = quantize16(v, gsf, inv_tab);
+        // the scale group's four bytes, from the lanes of blocks 4g .. 4g + 3 (lane = i % 32)
+        const uint32_t s1 = __shfl_down_sync(0xffffffffu, qb.s8, 1);
+        const uint32_t s2 = __shfl_down_sync(0xffffffffu, qb.s8, 2);
+        const uint32_t s3 = __shfl_down_sync(0xffffffffu, qb.s8, 3);
+        if (blk < nblk && row < p.m) {
+          const int64_t qo = static_cast<int64_t>(row) * (p.k / 2) + (16 * c + blk) * 8;
+          if (index_ok(qo + 7, static_cast<uint64_t>(p.m) * (p.k / 2), p.status))
+            *reinterpret_cast<uint2*>(p.qa_q + qo) = make_uint2(qb.lo, qb.hi);
+        }
+        if (blk < nblk && (lane & 3) == 0 && row < slab * 128 + 128) {
+          // rows of the slab beyond m are padding: their scale words are zero
+          const uint32_t word = row < p.m ? (qb.s8 | (s1 << 8) | (s2 << 16) | (s3 << 24)) : 0u;
+          const int64_t so = sf_offset(static_cast<uint32_t>(row), static_cast<uint32_t>(16 * c + blk), groups);
+          if (index_ok(so + 3, static_cast<uint64_t>(p.qa_slabs) * 128 * groups * 4, p.status))
+            *reinterpret_cast<uint32_t*>(p.qa_sf + so) = word;
+        }
+      }
+    }
+    fence_proxy_async_global();                  // the producers read these bytes with TMA
+    asm volatile("bar.sync 1, %0;" ::"n"(kEpi) : "memory");
+    if (t == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(p.qa_ws + 1 + c) : "memory");
+  }
+}
+
 // ---- the kernel ---------------------------------------------------------------------------------
 
-template <bool kGrouped, bool kLowRank, bool kSwiGLU, int kQW>
+template <bool kGrouped, bool kLowRank, bool kSwiGLU, int kQW, bool kQuantA = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kQW>, 1)
     nvfp4_gemm_kernel(const __grid_constant__ Maps maps, const GemmParams p) {
+  static_assert(!kQuantA || (!kGrouped && !kLowRank && !kSwiGLU), "the fused activation quantizer is dense only");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* staging = smem + kStages * kStageBytes;     // 1024-byte aligned (the ring is 190 KB)
@@ -349,6 +449,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kQW>, 1)
     uint32_t s = 0, phase = 0;
     bool wrapped = false;      // the ring has been filled once: every later stage waits for its slot
     bool ok = true;
+    uint64_t chunks_ready = 0;   // fused activation quantizer: K chunks seen complete for every slab
     TileCoord t;
     for (int tile = pair; ok && tile_coord<kGrouped>(p, ctl, tile, t); tile += pairs) {
       const int a_row = t.m_tile * kTileM + static_cast<int>(rank) * kBM;
@@ -368,6 +469,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kQW>, 1)
         uint8_t* st = smem + s * kStageBytes;
         const uint32_t full_bar = map_to_rank(&ctl.full[s], 0);
         const bool withheld = ks == p.stall_stage && tile == pair;   // self-test: nothing completes it
+        if constexpr (kQuantA) {
+          if (ks < p.k_stages && !((chunks_ready >> ks) & 1ull)) {
+            // wait (bounded) until every slab's chunk ks is quantized: each poll reads the
+            // counters of all chunks not yet seen (lane l: chunks l and l + 32) in one round
+            // trip, and the chunks found complete are remembered
+            const uint64_t t0 = global_ns();
+            for (uint32_t i = 0;; ++i) {
+              uint32_t lo = 0, hi = 0;
+              if (lane < p.k_stages && !((chunks_ready >> lane) & 1ull))
+                lo = ld_acquire_u32(p.qa_ws + 1 + lane) >= static_cast<uint32_t>(p.qa_slabs);
+              if (lane + 32 < p.k_stages && !((chunks_ready >> (lane + 32)) & 1ull))
+                hi = ld_acquire_u32(p.qa_ws + 33 + lane) >= static_cast<uint32_t>(p.qa_slabs);
+              chunks_ready |= static_cast<uint64_t>(__ballot_sync(0xffffffffu, lo)) |
+                              (static_cast<uint64_t>(__ballot_sync(0xffffffffu, hi)) << 32);
+              if ((chunks_ready >> ks) & 1ull) break;
+              if ((i & 15u) == 15u) {
+                bool give_up = *abort != 0;
+                if (!give_up && global_ns() - t0 > kWaitLimitNs) {
+                  give_up = true;
+                  if (lane == 0) {
+                    *abort = 1;
+                    atomicExch(p.status, NVFP4_ERR_DEVICE_TIMEOUT);
+                  }
+                }
+                if (__any_sync(0xffffffffu, give_up)) break;
+              }
+            }
+            if (!(ok = ((chunks_ready >> ks) & 1ull) != 0)) break;
+            fence_proxy_async_global();   // the TMA loads below read what other CTAs stored
+          }
+        }
         if (!withheld && elect_one()) {
           if (ks < p.k_stages) {
             if (leader) mbar_arrive_expect_tx(&ctl.full[s], kFp4TxBytes);
@@ -480,6 +612,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kQW>, 1)
       silu_table_load(silu_tab, p.silu_tab, threadIdx.x - 64, 32 * kEpiWarps<kQW>);
       asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpiWarps<kQW>) : "memory");
     }
+    if constexpr (kQuantA) quantize_a_units<32 * kEpiWarps<kQW>>(p, threadIdx.x - 64, reinterpret_cast<float*>(ctl.prefix));
     uint32_t tcount = 0;
     TileCoord t;
     uint32_t nstore = 0;                       // TMA stores issued by this warp (bf16 epilogue)
@@ -679,6 +812,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<kQW>, 1)
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
   }
+  if constexpr (kQuantA) {
+    // the last CTA to finish (every producer has read its counters, every unit is counted)
+    // re-zeroes the workspace words for the next call on the stream
+    if (threadIdx.x == 0) {
+      __threadfence();
+      if (atomicAdd(p.qa_ws, 1u) == gridDim.x - 1) {
+        for (int c = 0; c < p.k_stages; ++c) atomicExch(p.qa_ws + 1 + c, 0u);
+        atomicExch(p.qa_ws, 0u);
+      }
+    }
+  }
 }
 
 // ---- host side ------------------------------------------------------------------------------------
@@ -745,6 +889,8 @@ struct GemmArgs {
   const uint8_t *b2 = nullptr, *b2_sf = nullptr;  // SiLU * up: up weight (b: gate weight)
   const float *alpha2 = nullptr, *gsf_h = nullptr;
   uint8_t *q = nullptr, *sf = nullptr;
+  const void* qa_x = nullptr;              // fused activation quantizer: bf16 x (a, a_sf: its workspace)
+  const float* qa_gsf = nullptr;
   int64_t E = 1, m = 0, n = 0, k = 0;      // n: output width (the width of h for SiLU * up)
   int32_t stall_stage = -1;                // self-test only
 };
@@ -753,10 +899,10 @@ struct GemmArgs {
 // set-up per instantiation and device (dynamic shared memory opt-in, the number of 2-CTA
 // clusters that fit on the device at once: the persistent grid size), then a grid of
 // min(tiles, clusters) pairs.
-template <bool kGrouped, bool kLowRank, bool kSwiGLU, int kQW>
+template <bool kGrouped, bool kLowRank, bool kSwiGLU, int kQW, bool kQuantA = false>
 int run_gemm(const Maps& maps, const GemmParams& p, int64_t tiles, const DeviceInfo& info, cudaStream_t stream) {
-  auto kernel = nvfp4_gemm_kernel<kGrouped, kLowRank, kSwiGLU, kQW>;
-  constexpr int kSmem = kSmemBytes<kGrouped, kSwiGLU, kQW>;
+  auto kernel = nvfp4_gemm_kernel<kGrouped, kLowRank, kSwiGLU, kQW, kQuantA>;
+  constexpr int kSmem = kSmemBytes<kGrouped, kSwiGLU, kQW, kQuantA>;
   int max_clusters = 0;
   const int st = kernel_setup(reinterpret_cast<const void*>(kernel), info.device, [&](int* clusters_out) {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess) {
@@ -781,7 +927,7 @@ int run_gemm(const Maps& maps, const GemmParams& p, int64_t tiles, const DeviceI
   return launch_kernel(kernel, dim3(2 * pairs), dim3(kThreads<kQW>), kSmem, stream, maps, p);
 }
 
-template <bool kGrouped, bool kLowRank, bool kSwiGLU>
+template <bool kGrouped, bool kLowRank, bool kSwiGLU, bool kQuantA = false>
 int launch_gemm(const GemmArgs& g, cudaStream_t stream) {
   const int64_t E = g.E, m = g.m, n = g.n, k = g.k;
   if (E < 0 || m < 0 || n < 0 || k <= 0 || k % 64 != 0 || n % 8 != 0) return NVFP4_ERR_INVALID_ARGUMENT;
@@ -802,6 +948,9 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream) {
   }
   if (kGrouped && (!g.mask || !aligned(g.mask, 4))) return NVFP4_ERR_INVALID_ARGUMENT;
   if (kLowRank && (!g.d || !g.l1 || !aligned(g.d, 16) || !aligned(g.l1, 16))) return NVFP4_ERR_INVALID_ARGUMENT;
+  if (kQuantA && (!g.qa_x || !g.qa_gsf || !aligned(g.qa_x, 16) || !aligned(g.qa_gsf, 4) ||
+                  (k + kStageK - 1) / kStageK > kQuantAMaxChunks))
+    return NVFP4_ERR_INVALID_ARGUMENT;
 
   DeviceInfo info;
   int st = current_device(&info);
@@ -843,6 +992,16 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream) {
   p.k_steps = static_cast<int32_t>(k / 64);
   p.sf_groups = static_cast<int32_t>(k / 64);
   p.stall_stage = g.stall_stage;
+  uint32_t* qa_ws = nullptr;
+  if (kQuantA) {
+    if ((st = stream_workspace(stream, &qa_ws)) != NVFP4_OK) return st;
+    p.qa_x = static_cast<const uint16_t*>(g.qa_x);
+    p.qa_gsf = g.qa_gsf;
+    p.qa_q = const_cast<uint8_t*>(g.a);
+    p.qa_sf = const_cast<uint8_t*>(g.a_sf);
+    p.qa_ws = qa_ws;
+    p.qa_slabs = static_cast<int32_t>((m + 127) / 128);
+  }
   if (kSwiGLU) {
     p.alpha_up = g.alpha2;
     p.gsf_h = g.gsf_h;
@@ -855,7 +1014,11 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream) {
   const int64_t tiles = kGrouped ? static_cast<int64_t>(E) * p.m_tiles * p.n_tiles
                                  : static_cast<int64_t>(p.m_tiles) * p.n_tiles;
   if (tiles >= (int64_t(1) << 31)) return NVFP4_ERR_INVALID_ARGUMENT;
-  if constexpr (kSwiGLU) {
+  if constexpr (kQuantA) {
+    if (k >= 4096 && tiles >= static_cast<int64_t>(info.sm_count))
+      return run_gemm<false, false, false, 1, true>(maps, p, tiles, info, stream);
+    return run_gemm<false, false, false, 2, true>(maps, p, tiles, info, stream);
+  } else if constexpr (kSwiGLU) {
     return run_gemm<kGrouped, kLowRank, kSwiGLU, 2>(maps, p, tiles, info, stream);
   } else if constexpr (kGrouped) {
     return run_gemm<kGrouped, kLowRank, kSwiGLU, 1>(maps, p, tiles, info, stream);
@@ -882,6 +1045,17 @@ __global__ void bounded_wait_selftest_kernel(int* status) {
 }
 
 }  // namespace
+
+int gemm_quantize_a(const void* a_bf16, const uint8_t* b, const uint8_t* b_sf, const float* a_gsf, const float* alpha,
+                    const void* bias_bf16, void* out_bf16, uint8_t* a_q_ws, uint8_t* a_sf_ws, int64_t m, int64_t n,
+                    int64_t k, cudaStream_t stream) {
+  GemmArgs g;
+  g.a = a_q_ws; g.b = b; g.a_sf = a_sf_ws; g.b_sf = b_sf; g.alpha = alpha; g.bias = bias_bf16; g.out = out_bf16;
+  g.qa_x = a_bf16; g.qa_gsf = a_gsf;
+  g.m = m; g.n = n; g.k = k;
+  return launch_gemm<false, false, false, true>(g, stream);
+}
+
 }  // namespace nvfp4
 
 using namespace nvfp4;
