@@ -436,7 +436,7 @@ __global__ void __launch_bounds__(kThreads) amax_batched_kernel(const uint16_t* 
 //     Each pair of threads writes its group's 32 code bytes and its four scale bytes (one
 //     word of the 128x4 layout, assembled by a shuffle), and the CTA zeroes its share of the
 //     padding rows' scale words.
-// Workspace words: 0 = barrier arrivals, 1 = amax bits, 2 = CTAs done reading the maximum,
+// Workspace words: 0 = barrier arrivals, 1 = CTAs done reading the maximum, 2 = amax bits,
 // 3 = set by a CTA whose own bounded ring wait gave up (then no CTA writes anything); the
 // last CTA to read the maximum resets all four for the next call on the stream.
 constexpr int kGsqComputeWarps = 30;
@@ -462,6 +462,11 @@ struct GsqParams {
 __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
   uint32_t v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint2 ld_relaxed_gpu_v2(const uint32_t* p) {
+  uint2 v;
+  asm volatile("ld.relaxed.gpu.global.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p) : "memory");
   return v;
 }
 
@@ -603,12 +608,13 @@ __global__ void __launch_bounds__(kGsqThreads, 1)
   mx = warp_max(mx);
   if ((threadIdx.x & 31) == 0 && !producer) red[warp] = mx;
   __syncthreads();
+  bool passed = false;                                 // thread 0: passed the barrier (takes a ticket)
   if (threadIdx.x == 0) {
     float v = red[0];
 #pragma unroll
     for (int w = 1; w < kGsqComputeWarps; ++w) v = fmaxf(v, red[w]);
     if (abort_flag) atomicExch(ws + 3, 1u);            // a ring wait gave up: nobody writes
-    atomicMax(ws + 1, __float_as_uint(v));
+    atomicMax(ws + 2, __float_as_uint(v));
     // arrive, ordered after the atomic max (and ws[3]) by release semantics
     asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ws) : "memory");
     // grid barrier, bounded: every CTA is resident, so only a fault elsewhere can stall it
@@ -623,18 +629,21 @@ __global__ void __launch_bounds__(kGsqThreads, 1)
     }
     float a = -1.0f;                                   // -1: give up, write nothing
     if (ok) {
-      if (ld_acquire_gpu(ws + 3) == 0u)
-        a = fmaxf(fminf(__uint_as_float(ld_acquire_gpu(ws + 1)), FLT_MAX), 1e-12f);
-      if (atomicAdd(ws + 2, 1u) == grid - 1) {         // every CTA has read the maximum
-        atomicExch(ws + 1, 0u);
-        atomicExch(ws + 3, 0u);
-        atomicExch(ws + 2, 0u);
-        atomicExch(ws, 0u);
-      }
+      // the maximum and the abort word in one load, ordered after the acquire load that saw
+      // every arrival (each CTA wrote both before its release)
+      const uint2 ma = ld_relaxed_gpu_v2(ws + 2);
+      if (ma.y == 0u) a = fmaxf(fminf(__uint_as_float(ma.x), FLT_MAX), 1e-12f);
     }
     s_amax = a;
+    passed = ok;
   }
   __syncthreads();
+  if (passed && atomicAdd(ws + 1, 1u) == grid - 1) {   // every CTA has read the maximum
+    atomicExch(ws + 2, 0u);
+    atomicExch(ws + 3, 0u);
+    atomicExch(ws + 1, 0u);
+    atomicExch(ws, 0u);
+  }
   const float amax = s_amax;
   if (amax < 0.0f) {
     if (abort_flag) {
