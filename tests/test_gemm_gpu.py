@@ -73,6 +73,32 @@ def test_unit_scales_integer_codes_bit_exact(oracle):
         assert (host(out) == expect).all(), np.argwhere(host(out) != expect)[:5]
 
 
+@pytest.mark.parametrize("m,n,k", [(128, 576, 128), (300, 392, 256), (256, 968, 64), (130, 200, 192)])
+def test_per_row_scales_bit_exact(oracle, m, n, k):
+    # Power-of-two scales of A and B that change every 32 rows and every block: a scale read
+    # from the wrong 32-row group, chunk or K step multiplies a row or column by another
+    # scale.  Codes of at most 6 and scales of at most 2 keep every fp32 sum exact, so the
+    # output equals the exact result rounded to bf16 once.
+    g = np.random.default_rng(m * n + k)
+    ca = g.integers(0, 16, size=(m, k)).astype(np.uint8)
+    cb = g.integers(0, 16, size=(n, k)).astype(np.uint8)
+    qa = (ca[:, 0::2] | (ca[:, 1::2] << 4)).astype(np.uint8)
+    qb = (cb[:, 0::2] | (cb[:, 1::2] << 4)).astype(np.uint8)
+    sfa = np.zeros(nv.nvfp4_scale_bytes(m, k), np.uint8)
+    sfb = np.zeros(nv.nvfp4_scale_bytes(n, k), np.uint8)
+    codes = (0x30, 0x38, 0x40)                                  # 0.5, 1, 2
+    for r in range(m):
+        for c in range(k // 16):
+            sfa[oracle.sf_offset(r, c, k)] = codes[(r // 32 + 2 * c + 1) % 3]
+    for r in range(n):
+        for c in range(k // 16):
+            sfb[oracle.sf_offset(r, c, k)] = codes[(r // 32 + c) % 3]
+    ref = oracle.gemm_ref(qa, qb, sfa, sfb, 1.0, m, n, k)
+    out = host(run_gemm(qa, sfa, qb, sfb, np.float32(1.0)))
+    expect = S.f32_to_bf16_bits(ref.astype(np.float32))
+    assert (out == expect).all(), np.argwhere(out != expect)[:5]
+
+
 def test_pr1_linear(oracle):
     d = S.pr1_linear()
     qa, sfa, amax_a = quantized(oracle, d["x"])
